@@ -1,0 +1,403 @@
+// CPU oracle for the weight-only quantized matmul  y = x . dequant(Wq)^T.
+//
+// TEST INFRASTRUCTURE ONLY.  Only the tests, the smoke check and the CPU
+// baseline of the benchmark may load this library.  It shares no code, header,
+// table or constant with the CUDA library; the two meet only at the byte
+// layout that both implement from its written definition.
+//
+// Plain, slow and direct on purpose: one element at a time, the steps in the
+// order the sources give them, double precision for the matmul sums.
+//
+// Sources (web pages on weight-only low-bit quantization):
+//  [MZ]  "Does Marlin support zero-point quantization?" (githubissues.com,
+//        IST-DASLab/marlin issue 5), reply by efrantar: a general fp16 x int4
+//        matmul with symmetric linear quantization, column-wise or groupsize 128,
+//        fp16 scales; zero-point fixed to 8; fp16 zero-points as the natural
+//        extension.
+//  [FL]  FLUTE project summary (sourcepulse.org, project 1846613), "How It
+//        Works": a lookup table maps each code to a de-quantized value, which a
+//        scale factor multiplies; 2/3/4-bit codes; NF4-style tables.
+//  [GT]  GPTQ-Triton project summary (sourcepulse.org, project 1838626),
+//        "How It Works" / "Highlighted Details": weights decoded on the fly
+//        before the matmul; group size -1 (one group per output column).
+//  [EX]  exllama discussion 24, "Regarding comment on benchmark memory
+//        bandwidth speeds" (quoting the GPTQ paper): activations are not
+//        quantized; only the weights are, and are de-quantized when needed.
+//
+// Readings where the sources are silent (each also listed in the design notes):
+//  R1 round() is round-half-to-even (rintf in the default rounding mode).
+//  R2 the scale is rounded to fp16 first; codes are computed with that fp16
+//     scale, so encode and decode agree.  An fp16 overflow saturates to 65504.
+//  R3 true IEEE fp32 division w / s (no reciprocal multiply, no FMA contraction).
+//  R4 asymmetric zero-point z = clamp(rint(-min / s), 0, 15), an integer held
+//     in fp16.
+//  R5 a group whose fp16 scale is 0 encodes every value as 0: SYM q = 8,
+//     ASYM z = 0 and q = 0, LUT q = index of the entry nearest 0.
+//  R6 LUT encode: q = argmin_i |w/s - T[i]| in fp32, the lowest index on ties.
+//  R7 group = -1 means one group spanning the whole row (all of K).
+//
+// Packed layout (the library's documented format, restated here from its
+// definition; see the functions code_place and scale_index):
+//  * codes: row blocks of 16 rows; per row block, K/KC chunks of KC columns
+//    (KC = 64 for 4-bit, 128 for 2-bit), each chunk 512 bytes.  Inside a chunk
+//    lane l = 4g + t (g = 0..7, t = 0..3) owns bytes [16 l, 16 l + 16): rows g
+//    and g + 8 of the block, and in every 16-column tile j of the chunk the
+//    four columns 16 j + 4 t + c, c = 0..3.  The eight codes of one tile for one
+//    lane form four pairs p = 0..3: p = h + 2 (c / 2) where h = 0 for row g and
+//    1 for row g + 8, and (c % 2) selects the low or high member of the pair.
+//      4-bit SYM/ASYM: word j of the lane; pair p low -> nibble p, high ->
+//                      nibble p + 4.
+//      4-bit LUT:      word j of the lane; pair p low -> nibble 2p, high ->
+//                      nibble 2p + 1.
+//      2-bit LUT:      word j/2 of the lane, byte 2 (j % 2) + p / 2; inside the
+//                      byte the 2-bit field 2 (p % 2) + (c % 2).
+//    Words are little-endian uint32; nibble/field f occupies bits [b f, b f + b).
+//  * scales (and ASYM zeros): fp16, [N/16][G][16]; inside the 16 the row r of
+//    the block sits at 2 (r % 8) + r / 8.
+//  * LUT: 2^bits fp16 entries, plain order.
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <cstddef>
+
+namespace {
+
+enum { MODE_SYM = 0, MODE_ASYM = 1, MODE_LUT = 2 };
+enum { DT_F16 = 0, DT_BF16 = 1 };
+enum { OK = 0, ERR_ARG = -1 };
+
+// ---------------------------------------------------------------- conversions
+
+// fp16 bits -> exact value.
+double half_value(uint16_t h) {
+  int sign = (h >> 15) & 1;
+  int e = (h >> 10) & 0x1f;
+  int m = h & 0x3ff;
+  double v;
+  if (e == 0)
+    v = std::ldexp((double)m, -24);                  // subnormal: m * 2^-24
+  else if (e == 31)
+    v = m ? NAN : INFINITY;
+  else
+    v = std::ldexp((double)(1024 + m), e - 25);      // (1 + m/1024) * 2^(e-15)
+  return sign ? -v : v;
+}
+
+// bf16 bits -> exact value (the upper half of an fp32).
+double bf16_value(uint16_t b) {
+  uint32_t u = (uint32_t)b << 16;
+  float f;
+  std::memcpy(&f, &u, 4);
+  return (double)f;
+}
+
+// Round a finite double to the nearest multiple of `quantum`, ties to even
+// multiple.  `quantum` is a power of two, so v / quantum is exact.
+double round_to_quantum(double v, double quantum) {
+  double q = v / quantum;
+  double f = std::floor(q);
+  double d = q - f;
+  if (d > 0.5 || (d == 0.5 && std::fmod(f, 2.0) != 0.0)) f += 1.0;
+  return f * quantum;
+}
+
+// Value -> fp16 bits, round to nearest even (IEEE binary16: 10 fraction bits,
+// exponent -14..15, subnormal quantum 2^-24, overflow to infinity).
+uint16_t half_bits(double v) {
+  if (std::isnan(v)) return 0x7e00;
+  uint16_t sign = std::signbit(v) ? 0x8000 : 0;
+  double a = std::fabs(v);
+  if (a == 0.0) return sign;
+  int e;
+  std::frexp(a, &e);                       // a in [2^(e-1), 2^e)
+  int exp = e - 1;                         // a in [2^exp, 2^(exp+1))
+  if (exp < -14) exp = -14;                // subnormal range shares 2^-24 quantum
+  double r = round_to_quantum(a, std::ldexp(1.0, exp - 10));
+  if (r >= 65536.0) return sign | 0x7c00;  // rounded past the largest finite
+  if (r < std::ldexp(1.0, -14))            // subnormal (or zero)
+    return sign | (uint16_t)(r / std::ldexp(1.0, -24));
+  std::frexp(r, &e);
+  exp = e - 1;                             // rounding may have bumped the binade
+  uint16_t frac = (uint16_t)(r / std::ldexp(1.0, exp - 10) - 1024.0);
+  return sign | (uint16_t)((exp + 15) << 10) | frac;
+}
+
+// Value -> bf16 bits, round to nearest even (8 significant bits, fp32 range).
+uint16_t bf16_bits(double v) {
+  if (std::isnan(v)) return 0x7fc0;
+  uint16_t sign = std::signbit(v) ? 0x8000 : 0;
+  double a = std::fabs(v);
+  if (a == 0.0) return sign;
+  int e;
+  std::frexp(a, &e);
+  int exp = e - 1;
+  if (exp < -126) exp = -126;
+  double r = round_to_quantum(a, std::ldexp(1.0, exp - 7));
+  if (r >= std::ldexp(1.0, 128)) return sign | 0x7f80;
+  if (r < std::ldexp(1.0, -126))
+    return sign | (uint16_t)(r / std::ldexp(1.0, -133));
+  std::frexp(r, &e);
+  exp = e - 1;
+  uint16_t frac = (uint16_t)(r / std::ldexp(1.0, exp - 7) - 128.0);
+  return sign | (uint16_t)((exp + 127) << 7) | frac;
+}
+
+// R2: fp16 scale, saturated to the largest finite fp16 instead of infinity.
+uint16_t scale_bits(float s32) {
+  uint16_t h = half_bits((double)s32);
+  if ((h & 0x7fff) == 0x7c00) h = (h & 0x8000) | 0x7bff;
+  return h;
+}
+
+// ------------------------------------------------------------------- layout
+
+int n_groups(int K, int group) { return group == -1 ? 1 : K / group; }
+int group_len(int K, int group) { return group == -1 ? K : group; }
+int chunk_cols(int bits) { return bits == 4 ? 64 : 128; }
+
+// Shapes the quantizer and the logical decode accept: any N, K > 0 with the
+// group dividing K.
+bool logical_ok(int N, int K, int mode, int bits, int group) {
+  if (N <= 0 || K <= 0) return false;
+  if (mode != MODE_SYM && mode != MODE_ASYM && mode != MODE_LUT) return false;
+  if (bits != 4 && !(bits == 2 && mode == MODE_LUT)) return false;
+  if (group != -1 && (group <= 0 || K % group != 0)) return false;
+  return true;
+}
+
+// Shapes the packed layout is defined for: whole row blocks and chunks, groups
+// made of whole 16-column tiles.
+bool shape_ok(int N, int K, int mode, int bits, int group) {
+  if (!logical_ok(N, K, mode, bits, group)) return false;
+  if (N % 16 != 0 || K % chunk_cols(bits) != 0) return false;
+  if (group != -1 && group % 16 != 0) return false;
+  return true;
+}
+
+// Byte offset and bit shift of code (n, k) in the packed code buffer.
+void code_place(int n, int k, int K, int mode, int bits, size_t* byte, int* shift) {
+  int kc_cols = chunk_cols(bits);
+  int rb = n / 16, r = n % 16;
+  int g = r % 8, h = r / 8;
+  int chunk = k / kc_cols, kk = k % kc_cols;
+  int j = kk / 16, t = (kk % 16) / 4, c = kk % 4;
+  int lane = 4 * g + t;
+  int p = h + 2 * (c / 2);
+  int hi = c % 2;
+  size_t chunk_base = ((size_t)rb * (K / kc_cols) + chunk) * 512 + (size_t)lane * 16;
+  if (bits == 4) {
+    int nib = (mode == MODE_LUT) ? (2 * p + hi) : (p + 4 * hi);
+    *byte = chunk_base + (size_t)j * 4 + nib / 2;
+    *shift = 4 * (nib % 2);
+  } else {
+    int byte_in_word = 2 * (j % 2) + p / 2;
+    int field = 2 * (p % 2) + hi;
+    *byte = chunk_base + (size_t)(j / 2) * 4 + byte_in_word;
+    *shift = 2 * field;
+  }
+}
+
+// Index of (row n, group gi) in the packed scale / zero buffers.
+size_t scale_index(int n, int gi, int G) {
+  int rb = n / 16, r = n % 16;
+  return ((size_t)rb * G + gi) * 16 + 2 * (r % 8) + r / 8;
+}
+
+// ------------------------------------------------------------------- quantize
+
+// Clamp-and-truncate for a float that rint() has already made integral.
+int clamp_code(float v, int qmax) {
+  if (!(v > 0.0f)) return 0;               // also catches -inf
+  if (v > (float)qmax) return qmax;
+  return (int)v;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t oracle_packed_bytes(int N, int K, int bits) { return (size_t)N * K * bits / 8; }
+
+// Per group of `group` weights along K in each row n ([MZ], [FL], [GT]):
+//   SYM  s = absmax / 7,            q = clamp(rint(w / s) + 8, 0, 15)
+//   ASYM s = (max - min) / 15,      z = clamp(rint(-min / s), 0, 15),
+//                                   q = clamp(rint(w / s) + z, 0, 15)
+//   LUT  s = absmax,                q = argmin_i |w / s - T[i]|
+// with s rounded to fp16 before use (R2) and the readings R1, R3-R7.
+// Outputs are logical (unpacked): codes[N*K], scales[N*G], zeros[N*G] (ASYM).
+int oracle_quantize(const float* W, int N, int K, int mode, int bits, int group,
+                    const uint16_t* lut, uint8_t* codes, uint16_t* scales, uint16_t* zeros) {
+  if (!W || !codes || !scales || !logical_ok(N, K, mode, bits, group)) return ERR_ARG;
+  if (mode == MODE_ASYM && !zeros) return ERR_ARG;
+  if (mode == MODE_LUT && !lut) return ERR_ARG;
+  const int G = n_groups(K, group), L = group_len(K, group);
+  const int qmax = (1 << bits) - 1;
+  const int nlut = 1 << bits;
+  for (int n = 0; n < N; ++n) {
+    for (int gi = 0; gi < G; ++gi) {
+      const float* w = W + (size_t)n * K + (size_t)gi * L;
+      uint8_t* q = codes + (size_t)n * K + (size_t)gi * L;
+      // (i) reduce the group in fp32 (max and min are exact)
+      float amax = 0.0f, mn = w[0], mx = w[0];
+      for (int i = 0; i < L; ++i) {
+        float a = std::fabs(w[i]);
+        if (a > amax) amax = a;
+        if (w[i] < mn) mn = w[i];
+        if (w[i] > mx) mx = w[i];
+      }
+      // (ii) the fp32 scale, (iii) rounded to fp16
+      float s32;
+      if (mode == MODE_SYM) s32 = amax / 7.0f;
+      else if (mode == MODE_ASYM) s32 = (mx - mn) / 15.0f;
+      else s32 = amax;
+      uint16_t s16 = scale_bits(s32);
+      float s = (float)half_value(s16);
+      scales[(size_t)n * G + gi] = s16;
+      if (mode == MODE_SYM) {
+        for (int i = 0; i < L; ++i)
+          q[i] = (uint8_t)(s == 0.0f ? 8 : clamp_code(std::rint(w[i] / s) + 8.0f, qmax));
+      } else if (mode == MODE_ASYM) {
+        int z = (s == 0.0f) ? 0 : clamp_code(std::rint(-mn / s), qmax);
+        zeros[(size_t)n * G + gi] = half_bits((double)z);
+        for (int i = 0; i < L; ++i)
+          q[i] = (uint8_t)(s == 0.0f ? 0 : clamp_code(std::rint(w[i] / s) + (float)z, qmax));
+      } else {
+        for (int i = 0; i < L; ++i) {
+          float u = (s == 0.0f) ? 0.0f : w[i] / s;
+          int best = 0;
+          float bd = std::fabs(u - (float)half_value(lut[0]));
+          for (int e = 1; e < nlut; ++e) {
+            float d = std::fabs(u - (float)half_value(lut[e]));
+            if (d < bd) { bd = d; best = e; }
+          }
+          q[i] = (uint8_t)best;
+        }
+      }
+    }
+  }
+  return OK;
+}
+
+// Logical codes/scales/zeros -> packed buffers (layout in the header comment).
+int oracle_pack(const uint8_t* codes, const uint16_t* scales, const uint16_t* zeros,
+                int N, int K, int mode, int bits, int group,
+                uint8_t* qweight, uint16_t* scales_p, uint16_t* zeros_p) {
+  if (!codes || !scales || !qweight || !scales_p || !shape_ok(N, K, mode, bits, group))
+    return ERR_ARG;
+  if (mode == MODE_ASYM && (!zeros || !zeros_p)) return ERR_ARG;
+  const int G = n_groups(K, group);
+  std::memset(qweight, 0, oracle_packed_bytes(N, K, bits));
+  for (int n = 0; n < N; ++n)
+    for (int k = 0; k < K; ++k) {
+      size_t byte;
+      int shift;
+      code_place(n, k, K, mode, bits, &byte, &shift);
+      qweight[byte] |= (uint8_t)((codes[(size_t)n * K + k] & ((1 << bits) - 1)) << shift);
+    }
+  for (int n = 0; n < N; ++n)
+    for (int gi = 0; gi < G; ++gi) {
+      scales_p[scale_index(n, gi, G)] = scales[(size_t)n * G + gi];
+      if (mode == MODE_ASYM) zeros_p[scale_index(n, gi, G)] = zeros[(size_t)n * G + gi];
+    }
+  return OK;
+}
+
+// Packed buffers -> logical codes/scales/zeros (inverse of oracle_pack).
+int oracle_unpack(const uint8_t* qweight, const uint16_t* scales_p, const uint16_t* zeros_p,
+                  int N, int K, int mode, int bits, int group,
+                  uint8_t* codes, uint16_t* scales, uint16_t* zeros) {
+  if (!qweight || !codes || !shape_ok(N, K, mode, bits, group)) return ERR_ARG;
+  const int G = n_groups(K, group);
+  for (int n = 0; n < N; ++n)
+    for (int k = 0; k < K; ++k) {
+      size_t byte;
+      int shift;
+      code_place(n, k, K, mode, bits, &byte, &shift);
+      codes[(size_t)n * K + k] = (uint8_t)((qweight[byte] >> shift) & ((1 << bits) - 1));
+    }
+  for (int n = 0; n < N; ++n)
+    for (int gi = 0; gi < G; ++gi) {
+      if (scales && scales_p) scales[(size_t)n * G + gi] = scales_p[scale_index(n, gi, G)];
+      if (mode == MODE_ASYM && zeros && zeros_p)
+        zeros[(size_t)n * G + gi] = zeros_p[scale_index(n, gi, G)];
+    }
+  return OK;
+}
+
+// Decoded weight of one code ([MZ] symmetric / fp16 zero-point, [FL] table):
+//   SYM (q - 8) s,  ASYM (q - z) s,  LUT T[q] s.  Exact in double (and in fp32).
+static double decode(int q, double s, double z, const uint16_t* lut, int mode) {
+  if (mode == MODE_SYM) return ((double)q - 8.0) * s;
+  if (mode == MODE_ASYM) return ((double)q - z) * s;
+  return half_value(lut[q]) * s;
+}
+
+// Logical codes -> W~[N*K] as exact doubles.
+int oracle_dequant(const uint8_t* codes, const uint16_t* scales, const uint16_t* zeros_or_lut,
+                   int N, int K, int mode, int bits, int group, double* out) {
+  if (!codes || !scales || !out || !logical_ok(N, K, mode, bits, group)) return ERR_ARG;
+  if (mode != MODE_SYM && !zeros_or_lut) return ERR_ARG;
+  const int G = n_groups(K, group), L = group_len(K, group);
+  for (int n = 0; n < N; ++n)
+    for (int k = 0; k < K; ++k) {
+      int gi = k / L;
+      double s = half_value(scales[(size_t)n * G + gi]);
+      double z = (mode == MODE_ASYM) ? half_value(zeros_or_lut[(size_t)n * G + gi]) : 0.0;
+      out[(size_t)n * K + k] = decode(codes[(size_t)n * K + k], s, z, zeros_or_lut, mode);
+    }
+  return OK;
+}
+
+// Values -> fp16 (dtype 0) or bf16 (dtype 1) bits, round to nearest even.
+int oracle_round(const double* in, size_t n, int dtype, uint16_t* out) {
+  if (!in || !out || (dtype != DT_F16 && dtype != DT_BF16)) return ERR_ARG;
+  for (size_t i = 0; i < n; ++i) out[i] = dtype == DT_F16 ? half_bits(in[i]) : bf16_bits(in[i]);
+  return OK;
+}
+
+// fp16 / bf16 bits -> exact values.
+int oracle_widen(const uint16_t* in, size_t n, int dtype, double* out) {
+  if (!in || !out || (dtype != DT_F16 && dtype != DT_BF16)) return ERR_ARG;
+  for (size_t i = 0; i < n; ++i) out[i] = dtype == DT_F16 ? half_value(in[i]) : bf16_value(in[i]);
+  return OK;
+}
+
+// y[m, n] = sum_k x[m, k] * W~[n, k] for output columns n in [n0, n1), read
+// straight from the packed buffers ([GT] decode-then-multiply, [EX] the
+// activations stay in their fp16/bf16 input precision).  The sum runs over k in
+// ascending order in double; y is [M, n1 - n0] row-major doubles.
+int oracle_qmm(const uint16_t* x, int xdtype, const uint8_t* qweight, const uint16_t* scales_p,
+               const uint16_t* zeros_or_lut, int M, int N, int K, int mode, int bits, int group,
+               int n0, int n1, double* y) {
+  if (!x || !qweight || !scales_p || !y || M < 0 || n0 < 0 || n1 > N || n0 > n1) return ERR_ARG;
+  if (!shape_ok(N, K, mode, bits, group)) return ERR_ARG;
+  if (mode != MODE_SYM && !zeros_or_lut) return ERR_ARG;
+  const int G = n_groups(K, group), L = group_len(K, group);
+  double* xv = new double[(size_t)M * K];
+  double* w = new double[(size_t)K];
+  for (size_t i = 0; i < (size_t)M * K; ++i)
+    xv[i] = xdtype == DT_BF16 ? bf16_value(x[i]) : half_value(x[i]);
+  for (int n = n0; n < n1; ++n) {
+    for (int k = 0; k < K; ++k) {
+      size_t byte;
+      int shift;
+      code_place(n, k, K, mode, bits, &byte, &shift);
+      int q = (qweight[byte] >> shift) & ((1 << bits) - 1);
+      int gi = k / L;
+      double s = half_value(scales_p[scale_index(n, gi, G)]);
+      double z = (mode == MODE_ASYM) ? half_value(zeros_or_lut[scale_index(n, gi, G)]) : 0.0;
+      w[k] = decode(q, s, z, zeros_or_lut, mode);
+    }
+    for (int m = 0; m < M; ++m) {
+      double acc = 0.0;
+      for (int k = 0; k < K; ++k) acc += xv[(size_t)m * K + k] * w[k];
+      y[(size_t)m * (n1 - n0) + (n - n0)] = acc;
+    }
+  }
+  delete[] xv;
+  delete[] w;
+  return OK;
+}
+
+}  // extern "C"
