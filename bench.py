@@ -1,0 +1,436 @@
+"""Benchmark of the weight-only quantized matmul on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload NAME]
+
+Default workload (the metric's headline case): the four LLaMA-7B linear-layer
+shapes of one decoder layer -- fused QKV (K 4096, N 12288), O (4096, 4096),
+fused gate/up (4096, 22016), down (11008, 4096) -- at M = 1, 2, 4, 8 and 16
+tokens: 20 qmm calls per step, symmetric int4, group 128, fp16 activations.
+Each call has its own weights (522 MB in all, over 4x the 126 MB L2), so every
+call streams its codes from HBM.  The 20 launches are captured once in a CUDA
+graph and a step is one replay.
+
+Prints one JSON line (rank 0).  `value` is HBM throughput in GB/s: algorithmic
+bytes (codes + scales + x + y) of all calls on all ranks / max-over-ranks
+device time.  With --gpus N (under torchrun) every rank runs the same
+workload on its own GPU: independent replicas, weak scaling.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "W4A16 qmm: HBM GB/s (M<=16), TFLOP/s (M>=256), % of roofline"
+
+WORKLOADS = {
+    # name: (mode, bits, group, xdtype, [(K, N)], [M])
+    "llama7b_decode": ("sym", 4, 128, "f16",
+                       [(4096, 12288), (4096, 4096), (4096, 22016), (11008, 4096)],
+                       [1, 2, 4, 8, 16]),
+    "decode_4096sq": ("sym", 4, 128, "f16", [(4096, 4096)], [1]),
+    "llama70b_asym_bf16": ("asym", 4, 128, "bf16",
+                           [(8192, 10240), (8192, 57344), (28672, 8192)], [1, 16]),
+    "lut4_nf4": ("lut", 4, 64, "f16", [(4096, 14336)], [1, 8]),
+    "lut2": ("lut", 2, 64, "f16", [(4096, 14336)], [1, 8]),
+}
+SIGMA = {"sym": 0.02, "asym": 0.015, "lut": 0.02}
+SKINNY_SOURCES = ("weight_only_quantized_int4_b200/csrc/skinny.cu",
+                  "weight_only_quantized_int4_b200/csrc/common.cuh")
+
+
+def alg_bytes(mode, bits, group, M, K, N):
+    """Bytes a call must move at least once: codes, scales (+ zeros), x, y."""
+    G = 1 if group == -1 else K // group
+    meta = N * G * 2 * (2 if mode == "asym" else 1)
+    return N * K * bits // 8 + meta + M * K * 2 + M * N * 2
+
+
+def problems(name):
+    mode, bits, group, xdt, shapes, Ms = WORKLOADS[name]
+    return [(mode, bits, group, xdt, M, K, N) for M in Ms for (K, N) in shapes]
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+def sources_hash():
+    h = hashlib.sha256()
+    for s in SKINNY_SOURCES:
+        with open(os.path.join(ROOT, s), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_per_byte():
+    """DRAM bytes per algorithmic byte from the committed ncu summary, if it was
+    taken on the current kernel source (else None)."""
+    path = os.path.join(ROOT, "profiles", "skinny_llama7b_decode_traffic.txt")
+    try:
+        kv = {}
+        with open(path) as f:
+            for line in f:
+                if ":" in line and not line.startswith("#"):
+                    k, v = line.split(":", 1)
+                    kv[k.strip()] = v.strip()
+        if kv.get("source_hash") != sources_hash():
+            return None
+        return float(kv["dram_bytes_per_algorithmic_byte"])
+    except Exception:
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi samples (every 100 ms) of SM clock and throttle reasons."""
+
+    Q = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+         "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx = float(parts[1])
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[3:7]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# --------------------------------------------------------------------------- ours
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import weight_only_quantized_int4_b200 as q
+
+    torch.cuda.set_device(local_rank)
+    q.load()
+    dev = torch.device("cuda", local_rank)
+    probs = problems(args.workload)
+    gen = torch.Generator(device=dev).manual_seed(1234 + rank)
+    calls = []
+    for i, (mode, bits, group, xdt, M, K, N) in enumerate(probs):
+        W = torch.randn(N, K, generator=gen, device=dev) * SIGMA[mode]
+        lut = None
+        if mode == "lut":
+            from weight_only_quantized_int4_b200 import synth
+            t = synth.nf4_table() if bits == 4 else synth.lut2_table(0)
+            lut = torch.from_numpy(t.view(np.int16)).to(dev)
+        qw, sc, ze = q.pack(W, mode, bits, group, lut=lut)
+        del W
+        tdt = torch.float16 if xdt == "f16" else torch.bfloat16
+        x = torch.randn(M, K, generator=gen, device=dev).to(tdt)
+        y = torch.empty(M, N, dtype=tdt, device=dev)
+        ws = q.workspace(M, N, K, mode, bits, group, device=dev)
+        zl = ze if mode == "asym" else lut
+        calls.append(dict(x=x, qw=qw, sc=sc, zl=zl, y=y, ws=ws, M=M, N=N, K=K, mode=mode,
+                          bits=bits, group=group, bytes=alg_bytes(mode, bits, group, M, K, N)))
+    torch.cuda.synchronize()
+    step_bytes = sum(c["bytes"] for c in calls)
+
+    def step():
+        for c in calls:
+            q.qmm(c["x"], c["qw"], c["sc"], c["zl"], c["N"], c["K"], c["mode"], c["bits"],
+                  c["group"], y=c["y"], ws=c["ws"])
+
+    # warm-up outside the graph (first calls set kernel attributes), then capture
+    step()
+    torch.cuda.synchronize()
+    stream = torch.cuda.Stream(device=dev)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(stream):
+        step()
+        torch.cuda.synchronize()
+        with torch.cuda.graph(graph, stream=stream):
+            step()
+    torch.cuda.synchronize()
+
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    clock = ClockSampler(local_rank)
+    clock.start()
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            graph.replay()
+        # keep the GPU busy ~0.3 s so the clock samples see it under load
+        t_end = time.time() + 0.3
+        while time.time() < t_end:
+            for _ in range(50):
+                graph.replay()
+            torch.cuda.synchronize()
+        torch.cuda.synchronize()
+        barrier()
+        torch.cuda.synchronize()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            graph.replay()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        torch.cuda.synchronize()
+    clocks = clock.stop()
+    ms = e0.elapsed_time(e1)
+    if dist is not None:
+        t = torch.tensor([ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    ms_per_step = ms / args.steps
+    value = world * step_bytes * args.steps / (ms / 1e3) / 1e9
+
+    # ---- end to end through the public API: pinned host x in, y out, per step
+    hx = [c["x"].cpu().pin_memory() for c in calls]
+    hy = [torch.empty_like(c["y"], device="cpu").pin_memory() for c in calls]
+    h2d = sum(t.numel() * t.element_size() for t in hx)
+    d2h = sum(t.numel() * t.element_size() for t in hy)
+    e2e_steps = max(3, min(args.steps, 50))
+    with torch.cuda.stream(stream):
+        for _ in range(2):
+            for c, h in zip(calls, hx):
+                c["x"].copy_(h, non_blocking=True)
+            step()
+        torch.cuda.synchronize()
+        barrier()
+        torch.cuda.synchronize()
+        a0 = torch.cuda.Event(enable_timing=True)
+        a1 = torch.cuda.Event(enable_timing=True)
+        a0.record(stream)
+        for _ in range(e2e_steps):
+            for c, h in zip(calls, hx):
+                c["x"].copy_(h, non_blocking=True)
+            step()
+            for c, h in zip(calls, hy):
+                h.copy_(c["y"], non_blocking=True)
+        a1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+    e2e_ms = a0.elapsed_time(a1)
+    if dist is not None:
+        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e_value = world * step_bytes * e2e_steps / (e2e_ms / 1e3) / 1e9
+
+    peak, peak_kind = peaks()
+    achieved = step_bytes / (ms_per_step / 1e3) / 1e9      # one GPU, the skinny kernel only
+    tpb = traffic_per_byte()
+    roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                "frac": round(achieved / peak, 4), "peak_source": peak_kind,
+                "traffic": None if tpb is None else round(tpb * step_bytes / len(calls)),
+                "kernel": "skinny_kernel (all launches of the step)",
+                "algorithmic_bytes_per_launch": round(step_bytes / len(calls))}
+    out = {"metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world,
+           "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5),
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f16",
+           "data": "synthetic (seeded torch.randn weights and activations)",
+           "config": {"workload": args.workload, "calls_per_step": len(calls),
+                      "shapes_KN": WORKLOADS[args.workload][4], "M": WORKLOADS[args.workload][5],
+                      "mode": WORKLOADS[args.workload][0], "group": WORKLOADS[args.workload][2],
+                      "l2": "inputs larger than L2: every call has its own weights "
+                            f"({sum(c['qw'].numel() for c in calls) / 1e6:.0f} MB of codes)",
+                      "launch": "CUDA graph of the step, programmatic dependent launch",
+                      "parallelism": f"replicas x{world}"},
+           "roofline": roofline,
+           "e2e": {"value": round(e2e_value, 1), "unit": "GB/s", "h2d_bytes_per_step": h2d,
+                   "d2h_bytes_per_step": d2h, "steps": e2e_steps,
+                   "how": "per step: pinned x -> device, the 20 qmm calls through the Python "
+                          "API, y -> pinned host; CUDA events on the stream"},
+           "gpu_launches": len(calls) * args.steps,
+           "clocks": clocks}
+    if rank == 0 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline(args.workload, args.cpu_seconds)
+    del graph
+    return out
+
+
+# ------------------------------------------------------------------ CPU oracle
+
+def _oracle_sample(workload, rows_per_problem, seed=0):
+    """Host inputs of a sample: for every call, `rows_per_problem` rows of W."""
+    import oracle
+    from weight_only_quantized_int4_b200 import synth
+    items = []
+    for i, (mode, bits, group, xdt, M, K, N) in enumerate(problems(workload)):
+        rows = np.arange(rows_per_problem)
+        W = synth.weights(seed + i, "W", N, K, SIGMA[mode], rows=rows)
+        lut = None
+        if mode == "lut":
+            lut = synth.nf4_table() if bits == 4 else synth.lut2_table(0)
+        codes, scales, zeros = oracle.quantize(W, mode, bits, group, lut=lut)
+        qw, sp, zp = oracle.pack(codes, scales, zeros, mode, bits, group)
+        x = synth.activations(seed + i, "x", M, K, xdt)
+        zl = zp if mode == "asym" else lut
+        frac = rows_per_problem / N
+        items.append((x, xdt, qw, sp, zl, M, rows_per_problem, K, mode, bits, group,
+                      frac * alg_bytes(mode, bits, group, M, K, N)))
+    return items
+
+
+def _run_oracle(items, threads):
+    import oracle
+    t0 = time.perf_counter()
+    total = 0.0
+    for (x, xdt, qw, sp, zl, M, n, K, mode, bits, group, b) in items:
+        oracle.qmm_threaded(x, xdt, qw, sp, zl, M, n, K, mode, bits, group, 0, n, threads)
+        total += b
+    return time.perf_counter() - t0, total
+
+
+def cpu_threads():
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def cpu_baseline(workload, seconds):
+    """The oracle (plain C++, double sums) on a bounded sample of the workload:
+    the same 20 calls restricted to their first R rows of W (whole 16-row
+    blocks), R chosen so the timed run takes about `seconds`."""
+    threads = cpu_threads()
+    probe = _oracle_sample(workload, 16)
+    dt, _ = _run_oracle(probe, threads)
+    rows = int(16 * max(1, round(seconds / max(dt, 1e-3))))
+    rows = max(16, min(rows // 16 * 16, 4096))
+    items = _oracle_sample(workload, rows)
+    dt, nbytes = _run_oracle(items, threads)
+    return {"value": round(nbytes / dt / 1e9, 4), "unit": "GB/s", "cores": threads,
+            "kind": "oracle", "seconds": round(dt, 2),
+            "sample": f"every call of the step on its first {rows} rows of W "
+                      f"({nbytes / 1e6:.1f} MB of algorithmic bytes), columns split over "
+                      f"{threads} threads"}
+
+
+def run_reference(args):
+    """The oracle as the reference arm: each step is the bounded CPU sample."""
+    threads = cpu_threads()
+    probe = _oracle_sample(args.workload, 16)
+    dt, _ = _run_oracle(probe, threads)
+    budget = max(2.0, 120.0 / max(1, args.steps + args.warmup))   # whole run ~2 minutes
+    rows = max(16, min(int(16 * round(budget / max(dt, 1e-3))) // 16 * 16, 4096))
+    items = _oracle_sample(args.workload, rows)
+    for _ in range(args.warmup):
+        _run_oracle(items, threads)
+    tot_t, tot_b = 0.0, 0.0
+    for _ in range(args.steps):
+        t, b = _run_oracle(items, threads)
+        tot_t += t
+        tot_b += b
+    value = tot_b / tot_t / 1e9
+    sample = (f"every call of the step on its first {rows} rows of W, columns split over "
+              f"{threads} threads")
+    return {"impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s",
+            "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(1e3 * tot_t / args.steps, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": args.workload, "calls_per_step": len(items)},
+            "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": threads,
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=list(WORKLOADS), default="llama7b_decode")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args)), flush=True)
+        return
+
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local_rank))
+    out = run_ours(args, rank, world, local_rank)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,168 @@
+/* qmm -- weight-only quantized matrix multiply for NVIDIA B200 (sm_100a).
+ *
+ *   y[M, N] = x[M, K] . dequant(Wq)[N, K]^T
+ *
+ * x and y are fp16 or bf16; Wq holds 4-bit (or 2-bit, LUT mode) codes, decoded
+ * on the fly inside the kernels as
+ *   QMM_SYM   (q - 8) * s           symmetric, zero-point fixed at 8
+ *   QMM_ASYM  (q - z) * s           fp16 zero-point per group
+ *   QMM_LUT   T[q] * s              fp16 table of 2^bits entries
+ * with one fp16 scale s (and zero z) per group of `group` weights along K, or
+ * one per output row when group == -1.
+ *
+ * Sources for the operation:
+ *  - "Does Marlin support zero-point quantization?" (IST-DASLab/marlin issue 5),
+ *    reply by efrantar: fp16 x int4 matmul, symmetric linear quantization with
+ *    the zero-point fixed at 8, column-wise or groupsize 128, fp16 scales; fp16
+ *    zero-points as the asymmetric extension.
+ *  - FLUTE project summary (sourcepulse.org), "How It Works": lookup-table
+ *    quantization, value = table entry times a scale factor; 2- and 4-bit codes.
+ *  - GPTQ-Triton project summary (sourcepulse.org), "How It Works": the
+ *    quantized weights are decoded on the fly right before the multiply.
+ *  - exllama discussion 24 (quoting the GPTQ paper): activations stay in
+ *    floating point; the small-M product is bound by memory bandwidth.
+ *
+ * Conventions for every entry point:
+ *  - Pointers named as device pointers must point to memory of the current CUDA
+ *    device.  The caller allocates and owns every buffer; the library keeps no
+ *    reference after the call returns.
+ *  - `stream` is a cudaStream_t (NULL = the legacy default stream).  Every call
+ *    is asynchronous on that stream and never synchronizes the device.
+ *  - The return value is a qmm_status.  Argument errors are detected on the
+ *    host before anything is launched; launch errors come from
+ *    cudaGetLastError right after the launch.  Errors raised later by a kernel
+ *    (a bounded wait that ran out) are reported by qmm_check_error.
+ *  - Shapes the GPU kernels accept: N % 16 == 0; K % 64 == 0 (4-bit) or
+ *    K % 128 == 0 (2-bit); group == -1 or group a multiple of 16 that divides K;
+ *    M >= 0.  Other shapes return QMM_ERR_UNSUPPORTED.
+ *
+ * Packed layout (written by qmm_pack, read by qmm and qmm_dequant):
+ *  - qweight: N*K*bits/8 bytes.  Rows are taken in blocks of 16; each block is
+ *    a run of K/KC chunks of 512 bytes (KC = 64 columns for 4-bit, 128 for
+ *    2-bit).  Inside a chunk, lane l = 4g + t (g = 0..7, t = 0..3) owns bytes
+ *    [16 l, 16 l + 16): rows g and g + 8 of the block and, in every 16-column
+ *    tile j of the chunk, columns 16 j + 4 t + c (c = 0..3).  Those eight codes
+ *    of a tile form four pairs p = h + 2 (c / 2) (h = 0 for row g, 1 for row
+ *    g + 8) with member c % 2.  4-bit SYM/ASYM: tile j is 32-bit word j of the
+ *    lane, pair p's members at nibbles p and p + 4.  4-bit LUT: word j, nibbles
+ *    2p and 2p + 1.  2-bit LUT: word j / 2, byte 2 (j % 2) + p / 2, 2-bit field
+ *    2 (p % 2) + (c % 2).  Words are little-endian; field f holds bits
+ *    [bits*f, bits*f + bits).
+ *  - scales (and zeros): fp16, G = K/group groups (1 for group -1), stored as
+ *    [N/16][G][16] with row r of a block at position 2 (r % 8) + r / 8, i.e.
+ *    rows g and g + 8 side by side.
+ *  - LUT (zeros_or_lut in QMM_LUT mode): 2^bits fp16 entries in code order.
+ */
+#ifndef QMM_H
+#define QMM_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum { QMM_SYM = 0, QMM_ASYM = 1, QMM_LUT = 2 } qmm_mode;
+typedef enum { QMM_F16 = 0, QMM_BF16 = 1 } qmm_dtype;
+typedef enum {
+  QMM_OK = 0,
+  QMM_ERR_ARG = -1,          /* null pointer, negative size, bad enum value      */
+  QMM_ERR_UNSUPPORTED = -2,  /* shape / mode / bits combination not implemented  */
+  QMM_ERR_ALIGN = -3,        /* pointer not aligned as documented                */
+  QMM_ERR_CUDA = -4,         /* a CUDA runtime call failed                       */
+  QMM_ERR_TIMEOUT = -5,      /* a kernel gave up a bounded wait (qmm_check_error) */
+  QMM_ERR_WORKSPACE = -6     /* workspace smaller than qmm_workspace_size        */
+} qmm_status;
+
+/* Paths for qmm_with_path. */
+enum { QMM_PATH_AUTO = 0, QMM_PATH_SKINNY = 1, QMM_PATH_TENSOR = 2 };
+
+/* Byte sizes of the packed buffers for an [N, K] weight.  Returns the size of
+ * qweight (N*K*bits/8) and writes the scale and zero buffer sizes (zeros: 0
+ * unless QMM_ASYM) when the pointers are non-NULL.  Returns 0 for shapes the
+ * packed layout does not cover. */
+size_t qmm_packed_size(int N, int K, int bits, int group, int mode,
+                       size_t* scales_bytes, size_t* zeros_bytes);
+
+/* Quantize and pack fp32 weights (round to nearest, per group along K):
+ *   SYM  s = absmax / 7,       q = clamp(rint(w / s) + 8, 0, 15)
+ *   ASYM s = (max - min) / 15, z = clamp(rint(-min / s), 0, 15),
+ *                              q = clamp(rint(w / s) + z, 0, 15)
+ *   LUT  s = absmax,           q = argmin_i |w / s - T[i]| (lowest i on ties)
+ * s is rounded to fp16 (saturating at 65504) before the codes are computed; all
+ * divisions are IEEE fp32 and rint rounds half to even.  A group whose fp16
+ * scale is 0 encodes every weight as 0 (SYM q = 8; ASYM z = q = 0; LUT the
+ * entry nearest 0).
+ *   W        device, fp32 [N, K] row-major, finite values.
+ *   lut      device, 2^bits fp16 entries (QMM_LUT), else NULL.
+ *   qweight  device, qmm_packed_size bytes, 16-byte aligned (written).
+ *   scales   device, fp16, scales_bytes (written).
+ *   zeros    device, fp16, zeros_bytes (QMM_ASYM, written), else NULL.
+ * bits: 4 for SYM/ASYM; 4 or 2 for LUT. */
+int qmm_pack(const float* W, int N, int K, int mode, int bits, int group,
+             const uint16_t* lut, void* qweight, uint16_t* scales, uint16_t* zeros,
+             void* stream);
+
+/* Bytes of workspace qmm needs for this problem (any path).  The workspace
+ * holds split-K partial sums and per-tile arrival counters.  It must be zero
+ * filled once before its first use; every completed call leaves the counters
+ * at zero again, so it can be reused by later calls on the same stream.  Calls
+ * that run at the same time (other streams) need separate workspaces.
+ * 0 means the problem needs none. */
+size_t qmm_workspace_size(int M, int N, int K, int bits, int group, int mode);
+
+/* Workspace bytes for a call that takes path `path` (QMM_PATH_*); with
+ * QMM_PATH_AUTO this is qmm_workspace_size. */
+size_t qmm_workspace_size_for(int M, int N, int K, int bits, int group, int mode, int path);
+
+/* y = x . dequant(Wq)^T.
+ *   x             device, [M, K] row-major, xdtype (fp16 or bf16), 16-byte aligned.
+ *   qweight, scales, zeros_or_lut
+ *                 device, as written by qmm_pack (zeros for ASYM, the table
+ *                 for LUT, NULL for SYM).  ASYM zeros are exact for integer
+ *                 zero-points; a fractional zero is applied with one fp16 rounding.
+ *   y             device, [M, N] row-major, same dtype as x, must not overlap x.
+ *   workspace     device, workspace_bytes >= qmm_workspace_size(...), zero
+ *                 filled before first use (see above); may be NULL with
+ *                 workspace_bytes 0, in which case no cross-CTA split-K is used.
+ * The accumulation is fp32.  M <= 16 runs the bandwidth-bound decode path,
+ * larger M the tcgen05 tensor-core path (4-bit codes; 2-bit codes stay on the
+ * decode path); qmm_path tells which.  The tensor path reads x through a TMA
+ * tensor map, so x's row pitch (K * 2 bytes) must be a multiple of 16 -- true
+ * for every K the packed layout allows. */
+int qmm(const void* x, int xdtype, const void* qweight, const uint16_t* scales,
+        const uint16_t* zeros_or_lut, int M, int N, int K, int bits, int group, int mode,
+        void* y, void* workspace, size_t workspace_bytes, void* stream);
+
+/* qmm with the path chosen by the caller (QMM_PATH_*); QMM_PATH_AUTO is qmm. */
+int qmm_with_path(const void* x, int xdtype, const void* qweight, const uint16_t* scales,
+                  const uint16_t* zeros_or_lut, int M, int N, int K, int bits, int group,
+                  int mode, void* y, void* workspace, size_t workspace_bytes, void* stream,
+                  int path);
+
+/* The path qmm picks for this problem (QMM_PATH_SKINNY or QMM_PATH_TENSOR),
+ * or a negative qmm_status for an unsupported problem. */
+int qmm_path(int M, int N, int K, int bits, int group, int mode);
+
+/* Decode the packed weights into W_out[N, K] row-major (fp16 or bf16 by
+ * out_dtype): W_out = round_to_nearest_even((q - z) * s) (SYM z = 8) or
+ * round(T[q] * s), the product taken exactly in fp32 (exact for integer
+ * zero-points).  For tests and inspection; not on the matmul path. */
+int qmm_dequant(const void* qweight, const uint16_t* scales, const uint16_t* zeros_or_lut,
+                int N, int K, int bits, int group, int mode, int out_dtype, void* W_out,
+                void* stream);
+
+/* Synchronizes `stream`, then reads and clears the library's device error word
+ * on the current device: QMM_OK, or QMM_ERR_TIMEOUT if a kernel abandoned a
+ * bounded wait since the last check. */
+int qmm_check_error(void* stream);
+
+/* Static description of a status code. */
+const char* qmm_strerror(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QMM_H */

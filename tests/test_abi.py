@@ -1,0 +1,96 @@
+"""The C-ABI library: it loads, exports every symbol include/qmm.h declares,
+and rejects bad arguments on the host (no GPU needed for any of this)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import weight_only_quantized_int4_b200 as q
+from weight_only_quantized_int4_b200 import build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    src = open(os.path.join(ROOT, "include", "qmm.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?[\w]+\**\s+\**(qmm\w*)\s*\(", src, re.M)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return q.load()
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for must in ("qmm_pack", "qmm", "qmm_packed_size", "qmm_workspace_size", "qmm_dequant",
+                 "qmm_strerror"):
+        assert must in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+    assert set(declared_functions()) <= set(q.SYMBOLS)
+
+
+def test_sizes_and_paths(lib):
+    assert q.packed_size(4096, 4096, "sym", 4, 128) == (4096 * 2048, 4096 * 32 * 2, 0)
+    assert q.packed_size(64, 256, "asym", 4, -1) == (64 * 128, 64 * 2, 64 * 2)
+    assert q.packed_size(16, 128, "lut", 2, 64) == (16 * 32, 16 * 2 * 2, 0)
+    assert q.path(1, 4096, 4096, "sym") == "skinny"
+    assert q.path(16, 4096, 4096, "sym") == "skinny"
+    assert q.path(64, 4096, 4096, "sym") == "tensor"
+
+
+@pytest.mark.parametrize("N,K,bits,group,mode,status", [
+    (100, 4096, 4, 128, "sym", -2),     # N % 16
+    (4096, 4000, 4, 128, "sym", -2),    # K % 64
+    (4096, 4096, 2, 64, "sym", -2),     # 2-bit needs LUT
+    (4096, 4160, 2, 64, "lut", -2),     # 2-bit needs K % 128
+    (4096, 4096, 4, 100, "sym", -2),    # group not a multiple of 16
+    (4096, 4096, 4, 384, "sym", -2),    # group does not divide K
+    (0, 4096, 4, 128, "sym", -1),
+    (4096, 4096, 3, 128, "lut", -1),
+])
+def test_bad_shapes_are_rejected(lib, N, K, bits, group, mode, status):
+    assert lib.qmm_path(1, N, K, bits, group, q.MODES[mode]) == status
+    assert lib.qmm_packed_size(N, K, bits, group, q.MODES[mode], None, None) == 0
+
+
+def test_bad_arguments_return_status_without_launching(lib):
+    P = ctypes.c_void_p
+    fake = P(0x1000)                      # never dereferenced: checks fail first
+    # null x
+    assert lib.qmm(None, 0, fake, fake, None, 1, 64, 64, 4, 64, 0, fake, None, 0, None) == -1
+    # bad dtype, bad mode, negative M
+    assert lib.qmm(fake, 7, fake, fake, None, 1, 64, 64, 4, 64, 0, fake, None, 0, None) == -1
+    assert lib.qmm(fake, 0, fake, fake, None, 1, 64, 64, 4, 64, 9, fake, None, 0, None) == -1
+    assert lib.qmm(fake, 0, fake, fake, None, -1, 64, 64, 4, 64, 0, fake, None, 0, None) == -1
+    # M == 0 is a no-op
+    assert lib.qmm(fake, 0, fake, fake, None, 0, 64, 64, 4, 64, 0, fake, None, 0, None) == 0
+    # ASYM / LUT need their buffer
+    assert lib.qmm(fake, 0, fake, fake, None, 1, 64, 64, 4, 64, 1, fake, None, 0, None) == -1
+    # misaligned x
+    assert lib.qmm(P(0x1002), 0, fake, fake, None, 1, 64, 64, 4, 64, 0, P(0x90000), None, 0,
+                   None) == -3
+    # y overlapping x
+    assert lib.qmm(fake, 0, P(0x200000), fake, None, 2, 64, 64, 4, 64, 0, P(0x1040), None, 0,
+                   None) == -1
+    # bad path
+    assert lib.qmm_with_path(fake, 0, fake, fake, None, 1, 64, 64, 4, 64, 0, P(0x90000), None,
+                             0, None, 5) == -1
+    # pack: null W, misaligned W
+    assert lib.qmm_pack(None, 64, 64, 0, 4, 64, None, fake, fake, None, None) == -1
+    assert lib.qmm_pack(P(0x1004), 64, 64, 0, 4, 64, None, fake, fake, None, None) == -3
+    assert lib.qmm_pack(fake, 64, 64, 2, 4, 64, None, fake, fake, None, None) == -1  # LUT, no table
+    assert lib.qmm_dequant(fake, fake, None, 64, 64, 4, 64, 0, 3, fake, None) == -1
+
+
+def test_strerror_covers_every_status(lib):
+    for s in (0, -1, -2, -3, -4, -5, -6):
+        assert q.strerror(s) != "unknown status"
+    assert q.strerror(-99) == "unknown status"

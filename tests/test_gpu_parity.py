@@ -1,0 +1,254 @@
+"""Parity of the CUDA path against the CPU oracle (needs a B200).
+
+Packing and decoding are compared byte for byte; the matmul element by element
+against the oracle's double-precision result, with |err| <= 4e-3 sum|x||w~|
+per element and relative L2 error <= 2e-3 per output.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import weight_only_quantized_int4_b200 as q
+from tests import cases
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    if not torch.cuda.is_available():
+        pytest.fail("CUDA device required for -m gpu tests")
+    from weight_only_quantized_int4_b200 import build
+    build.build()
+    q.load()
+
+
+def dev(a):
+    a = np.ascontiguousarray(a)
+    if a.dtype == np.uint16:
+        a = a.view(np.int16)
+    return torch.from_numpy(a).cuda()
+
+
+def host16(t):
+    return t.cpu().numpy().view(np.uint16)
+
+
+def to_f64(y, xdtype):
+    return y.float().cpu().numpy().astype(np.float64)
+
+
+def upload(p):
+    tdt = torch.float16 if p.xdtype == "f16" else torch.bfloat16
+    x = dev(p.x).view(tdt)
+    return x, dev(p.qw), dev(p.sp), (None if p.zl is None else dev(p.zl))
+
+
+MODES = [("sym", 4, 128), ("sym", 4, -1), ("sym", 4, 64), ("sym", 4, 32), ("asym", 4, 128),
+         ("asym", 4, 64), ("lut", 4, 64), ("lut", 4, 128), ("lut", 2, 64), ("lut", 2, 128),
+         ("lut", 2, 32), ("sym", 4, 16)]
+
+
+# ------------------------------------------------------------------ packing
+
+@pytest.mark.parametrize("mode,bits,group", MODES)
+@pytest.mark.parametrize("N,K", [(48, 256), (176, 768)])
+def test_pack_bit_exact(mode, bits, group, N, K):
+    p = cases.make(mode, bits, group, 1, N, K)
+    W = torch.from_numpy(p.W_rows).cuda()
+    lut = None if p.lut is None else dev(p.lut)
+    qw, sc, ze = q.pack(W, mode, bits, group, lut=lut)
+    torch.cuda.synchronize()
+    assert np.array_equal(qw.cpu().numpy(), p.qw)
+    assert np.array_equal(host16(sc), p.sp)
+    if mode == "asym":
+        assert np.array_equal(host16(ze), p.zp)
+
+
+def test_pack_degenerate_groups():
+    """All-zero groups, a constant group, tiny (fp16-subnormal) and huge scales."""
+    N, K = 32, 256
+    rng = np.random.default_rng(5)
+    W = (rng.standard_normal((N, K)) * 0.02).astype(np.float32)
+    W[0, :] = 0.0
+    W[1, :128] = 0.37
+    W[2, :] = W[2, :] * 1e-6
+    W[3, :] = W[3, :] * 1e7
+    W[4, 5] = 2.5 * 7 * 2.0 ** -10       # values landing exactly on x.5 grid points
+    for mode, bits, group in [("sym", 4, 128), ("asym", 4, 128), ("lut", 4, 64), ("lut", 2, 64)]:
+        lut = cases.table(mode, bits)
+        codes, scales, zeros = oracle.quantize(W, mode, bits, group, lut=lut)
+        qw_o, sp_o, zp_o = oracle.pack(codes, scales, zeros, mode, bits, group)
+        qw, sc, ze = q.pack(torch.from_numpy(W).cuda(), mode, bits, group,
+                            lut=None if lut is None else dev(lut))
+        torch.cuda.synchronize()
+        assert np.array_equal(qw.cpu().numpy(), qw_o), mode
+        assert np.array_equal(host16(sc), sp_o), mode
+        if mode == "asym":
+            assert np.array_equal(host16(ze), zp_o)
+
+
+# ------------------------------------------------------------------ decoding
+
+@pytest.mark.parametrize("mode,bits,group", MODES)
+@pytest.mark.parametrize("dtype", ["f16", "bf16"])
+def test_dequant_bit_exact(mode, bits, group, dtype):
+    p = cases.make(mode, bits, group, 1, 48, 512, seed=3)
+    tdt = torch.float16 if dtype == "f16" else torch.bfloat16
+    out = q.dequant(dev(p.qw), dev(p.sp), None if p.zl is None else dev(p.zl), p.N, p.K, mode,
+                    bits, group, dtype=tdt)
+    torch.cuda.synchronize()
+    zl = p.zeros if mode == "asym" else p.lut
+    ref = oracle.round_to(oracle.dequant(p.codes, p.scales, zl, mode, bits, group), dtype)
+    assert np.array_equal(host16(out.view(torch.int16)), ref)
+
+
+# ------------------------------------------------------------------ matmul
+
+SMALL_M = [1, 2, 3, 8, 9, 16, 17, 40]
+
+
+@pytest.mark.parametrize("mode,bits,group", MODES)
+@pytest.mark.parametrize("xdtype", ["f16", "bf16"])
+def test_qmm_small(mode, bits, group, xdtype):
+    """Several row tiles, K chunks and groups; ragged N (11 row blocks) and M."""
+    N, K = 176, 1024
+    for M in SMALL_M:
+        p = cases.make(mode, bits, group, M, N, K, xdtype, seed=M)
+        y_ref, bound = cases.expected(p)
+        x, qw, sp, zl = upload(p)
+        for path in ("auto", "skinny"):
+            ws = q.workspace(M, N, K, mode, bits, group)
+            y = q.qmm(x, qw, sp, zl, N, K, mode, bits, group, ws=ws, path=path)
+            torch.cuda.synchronize()
+            cases.compare(to_f64(y, xdtype), y_ref, bound, f"{mode}{bits} g{group} M{M} {path}")
+
+
+@pytest.mark.parametrize("ws_kind", ["none", "sized"])
+def test_qmm_workspace_modes(ws_kind):
+    """With no workspace every CTA owns whole tiles; with one, stream-K split
+    partials are reduced by the last CTA.  Both give the same y."""
+    M, N, K = 5, 2048, 4096
+    p = cases.make("sym", 4, 128, M, N, K, seed=21)
+    y_ref, bound = cases.expected(p)
+    x, qw, sp, _ = upload(p)
+    ws = q.workspace(M, N, K, "sym") if ws_kind == "sized" else None
+    y1 = q.qmm(x, qw, sp, None, N, K, "sym", 4, 128, ws=ws)
+    y2 = q.qmm(x, qw, sp, None, N, K, "sym", 4, 128, ws=ws)
+    torch.cuda.synchronize()
+    cases.compare(to_f64(y1, "f16"), y_ref, bound, ws_kind)
+    assert torch.equal(y1, y2), "repeated calls must be bit-identical (deterministic split-K)"
+    if ws is not None:
+        tiles = (N // 16 + 1) // 2          # per-tile arrival counters lead the workspace
+        assert int(ws[: tiles * 4].view(torch.int32).abs().sum()) == 0, "counters not reset"
+
+
+def test_qmm_rejects_small_workspace():
+    M, N, K = 5, 2048, 4096
+    need = q.workspace_size(M, N, K, "sym")
+    if need == 0:
+        pytest.skip("this device plan needs no workspace")
+    p = cases.make("sym", 4, 128, M, N, K, seed=22)
+    x, qw, sp, _ = upload(p)
+    small = torch.zeros(need - 256, dtype=torch.uint8, device="cuda")
+    with pytest.raises(q.QmmError) as e:
+        q.qmm(x, qw, sp, None, N, K, "sym", 4, 128, ws=small)
+    assert e.value.status == -6
+
+
+def test_qmm_writes_only_y():
+    """Guard bands around y stay untouched (no out-of-bounds stores)."""
+    M, N, K = 13, 176, 512
+    p = cases.make("asym", 4, 128, M, N, K, "bf16", seed=4)
+    y_ref, bound = cases.expected(p)
+    x, qw, sp, zl = upload(p)
+    pad = 4096
+    buf = torch.full((M * N + 2 * pad,), -12345, dtype=torch.int16, device="cuda")
+    y = buf[pad:pad + M * N].view(torch.bfloat16).view(M, N)
+    q.qmm(x, qw, sp, zl, N, K, "asym", 4, 128, y=y, ws=q.workspace(M, N, K, "asym"))
+    torch.cuda.synchronize()
+    assert torch.all(buf[:pad] == -12345) and torch.all(buf[pad + M * N:] == -12345)
+    cases.compare(to_f64(y, "bf16"), y_ref, bound, "guard")
+
+
+@pytest.mark.parametrize("mode", ["sym", "asym"])
+def test_qmm_zero_point_codes_give_exact_zero(mode):
+    M, N, K, g = 7, 64, 512, 128
+    G = K // g
+    codes = np.full((N, K), 8, np.uint8)
+    scales = oracle.round_to(np.random.default_rng(1).uniform(0.001, 0.1, (N, G)), "f16")
+    zeros = None
+    if mode == "asym":
+        z = np.random.default_rng(2).integers(0, 16, (N, G))
+        codes = np.repeat(z, g, axis=1).astype(np.uint8)
+        zeros = oracle.round_to(z.astype(np.float64), "f16")
+    qw, sp, zp = oracle.pack(codes, scales, zeros, mode, 4, g)
+    from weight_only_quantized_int4_b200 import synth
+    x = dev(synth.activations(0, "x", M, K, "f16")).view(torch.float16)
+    y = q.qmm(x, dev(qw), dev(sp), None if zp is None else dev(zp), N, K, mode, 4, g,
+              ws=q.workspace(M, N, K, mode))
+    torch.cuda.synchronize()
+    assert torch.all(y == 0)
+
+
+def test_qmm_scale_linearity_is_exact():
+    """Scaling every scale by 4 scales y by 4 exactly (the group scale is
+    applied to fp32 partial sums, so no rounding changes)."""
+    M, N, K = 6, 176, 1024
+    p = cases.make("sym", 4, 128, M, N, K, seed=8)
+    x, qw, sp, _ = upload(p)
+    s4 = dev(oracle.round_to(oracle.widen(p.sp, "f16") * 4.0, "f16"))
+    ws = q.workspace(M, N, K, "sym")
+    y1 = q.qmm(x, qw, sp, None, N, K, "sym", 4, 128, ws=ws)
+    y4 = q.qmm(x, qw, s4, None, N, K, "sym", 4, 128, ws=ws)
+    torch.cuda.synchronize()
+    assert torch.equal(y4, y1 * 4)
+
+
+def test_lut_with_integer_table_matches_sym():
+    """LUT mode with T[i] = i - 8 on the SYM codes reproduces SYM bit for bit."""
+    M, N, K = 9, 176, 1024
+    p = cases.make("sym", 4, 64, M, N, K, seed=9)
+    qw_l, sp_l, _ = oracle.pack(p.codes, p.scales, None, "lut", 4, 64)
+    T = dev(np.arange(-8, 8).astype(np.float16).view(np.uint16))
+    x, qw, sp, _ = upload(p)
+    ys = q.qmm(x, qw, sp, None, N, K, "sym", 4, 64, ws=q.workspace(M, N, K, "sym", 4, 64))
+    yl = q.qmm(x, dev(qw_l), dev(sp_l), T, N, K, "lut", 4, 64,
+               ws=q.workspace(M, N, K, "lut", 4, 64))
+    torch.cuda.synchronize()
+    assert torch.equal(ys, yl)
+
+
+def test_matches_torch_on_decoded_weights():
+    """Second opinion from a library routine: torch fp32 matmul on the weights
+    the library itself decodes (qmm_dequant)."""
+    M, N, K = 16, 512, 2048
+    p = cases.make("lut", 4, 64, M, N, K, seed=12)
+    x, qw, sp, zl = upload(p)
+    y = q.qmm(x, qw, sp, zl, N, K, "lut", 4, 64, ws=q.workspace(M, N, K, "lut", 4, 64))
+    Wt = q.dequant(qw, sp, zl, N, K, "lut", 4, 64, dtype=torch.float16)
+    ref = x.float() @ Wt.float().T
+    torch.cuda.synchronize()
+    rel = (y.float() - ref).norm() / ref.norm()
+    assert rel < 2e-3
+
+
+def test_pdl_chain_of_dependent_calls():
+    """Back-to-back calls where each consumes the previous output: every call
+    waits for its predecessor before reading x (programmatic dependent launch)."""
+    M, N, K = 4, 1024, 1024
+    p = cases.make("sym", 4, 128, M, N, K, seed=30)
+    x, qw, sp, _ = upload(p)
+    ws = q.workspace(M, N, K, "sym")
+    ys = [x]
+    for _ in range(6):
+        ys.append(q.qmm(ys[-1], qw, sp, None, N, K, "sym", 4, 128, ws=ws))
+    torch.cuda.synchronize()
+    # replay step by step with a synchronize between calls
+    zs = [x]
+    for _ in range(6):
+        zs.append(q.qmm(zs[-1], qw, sp, None, N, K, "sym", 4, 128, ws=ws))
+        torch.cuda.synchronize()
+    for a, b in zip(ys, zs):
+        assert torch.equal(a, b)

@@ -1,0 +1,166 @@
+"""Python binding of libqmm, the weight-only quantized matmul for B200.
+
+Argument marshalling only: torch tensors are passed to the C ABI
+(include/qmm.h) as raw device pointers together with the current CUDA
+stream; every step of the computation runs in the library's CUDA kernels.
+There is no fallback: if libqmm.so is missing or cannot be loaded, every call
+raises.
+
+    import weight_only_quantized_int4_b200 as q
+    qw, s, z = q.pack(W, "sym", bits=4, group=128)          # W: fp32 [N, K] on cuda
+    y = q.qmm(x, qw, s, None, N=N, K=K, mode="sym", bits=4, group=128)
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libqmm.so")
+
+MODES = {"sym": 0, "asym": 1, "lut": 2}
+DTYPES = {torch.float16: 0, torch.bfloat16: 1}
+PATHS = {"auto": 0, "skinny": 1, "tensor": 2}
+PATH_NAMES = {1: "skinny", 2: "tensor"}
+
+SYMBOLS = ("qmm_packed_size", "qmm_pack", "qmm_workspace_size", "qmm_workspace_size_for", "qmm",
+           "qmm_with_path",
+           "qmm_path", "qmm_dequant", "qmm_check_error", "qmm_strerror")
+
+_lib = None
+_lock = threading.Lock()
+
+
+class QmmError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        super().__init__(f"{what} failed: {strerror(status)} (status {status})")
+        self.status = status
+
+
+def load(path: str = LIB_PATH):
+    """Load libqmm.so (raises OSError if it is absent: build it first)."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(path):
+                raise OSError(f"{path} not found; build it with "
+                              "`python -m weight_only_quantized_int4_b200.build`")
+            lib = ctypes.CDLL(path)
+            P, I, S = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+            lib.qmm_packed_size.argtypes = [I, I, I, I, I, P, P]
+            lib.qmm_packed_size.restype = S
+            lib.qmm_pack.argtypes = [P, I, I, I, I, I, P, P, P, P, P]
+            lib.qmm_workspace_size.argtypes = [I, I, I, I, I, I]
+            lib.qmm_workspace_size.restype = S
+            lib.qmm.argtypes = [P, I, P, P, P, I, I, I, I, I, I, P, P, S, P]
+            lib.qmm_with_path.argtypes = [P, I, P, P, P, I, I, I, I, I, I, P, P, S, P, I]
+            lib.qmm_path.argtypes = [I, I, I, I, I, I]
+            lib.qmm_dequant.argtypes = [P, P, P, I, I, I, I, I, I, P, P]
+            lib.qmm_check_error.argtypes = [P]
+            lib.qmm_strerror.argtypes = [I]
+            lib.qmm_strerror.restype = ctypes.c_char_p
+            _lib = lib
+    return _lib
+
+
+def strerror(status: int) -> str:
+    return load().qmm_strerror(status).decode()
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream():
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _check(status: int, what: str):
+    if status != 0:
+        raise QmmError(status, what)
+
+
+def _dev(t, name):
+    if t is not None and not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t is not None and not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def packed_size(N, K, mode, bits=4, group=128):
+    """(qweight bytes, scale bytes, zero bytes) for an [N, K] weight."""
+    sb, zb = ctypes.c_size_t(0), ctypes.c_size_t(0)
+    q = load().qmm_packed_size(N, K, bits, group, MODES[mode], ctypes.byref(sb), ctypes.byref(zb))
+    if q == 0:
+        raise QmmError(-2, "qmm_packed_size")
+    return q, sb.value, zb.value
+
+
+def pack(W, mode, bits=4, group=128, lut=None, out=None):
+    """Quantize fp32 W[N, K] (CUDA) -> (qweight uint8, scales fp16-bits int16, zeros or None)."""
+    _dev(W, "W")
+    N, K = W.shape
+    qb, sb, zb = packed_size(N, K, mode, bits, group)
+    if out is None:
+        qw = torch.empty(qb, dtype=torch.uint8, device=W.device)
+        sc = torch.empty(sb // 2, dtype=torch.int16, device=W.device)
+        ze = torch.empty(zb // 2, dtype=torch.int16, device=W.device) if zb else None
+    else:
+        qw, sc, ze = out
+    _check(load().qmm_pack(_ptr(W), N, K, MODES[mode], bits, group, _ptr(lut), _ptr(qw),
+                           _ptr(sc), _ptr(ze), _stream()), "qmm_pack")
+    return qw, sc, ze
+
+
+def workspace_size(M, N, K, mode, bits=4, group=128):
+    return load().qmm_workspace_size(M, N, K, bits, group, MODES[mode])
+
+
+def workspace(M, N, K, mode, bits=4, group=128, device="cuda"):
+    """A zero-filled workspace for this problem (None if it needs none)."""
+    n = workspace_size(M, N, K, mode, bits, group)
+    return torch.zeros(n, dtype=torch.uint8, device=device) if n else None
+
+
+def path(M, N, K, mode, bits=4, group=128):
+    st = load().qmm_path(M, N, K, bits, group, MODES[mode])
+    if st < 0:
+        raise QmmError(st, "qmm_path")
+    return PATH_NAMES[st]
+
+
+def qmm(x, qweight, scales, zeros_or_lut, N, K, mode, bits=4, group=128, y=None, ws=None,
+        path="auto"):
+    """y[M, N] = x[M, K] . dequant(qweight)^T on x's device and current stream."""
+    _dev(x, "x")
+    if x.dtype not in DTYPES:
+        raise ValueError("x must be fp16 or bf16")
+    M = x.shape[0]
+    if x.shape[1] != K:
+        raise ValueError("x.shape[1] != K")
+    if y is None:
+        y = torch.empty(M, N, dtype=x.dtype, device=x.device)
+    nbytes = 0 if ws is None else ws.numel() * ws.element_size()
+    _check(load().qmm_with_path(_ptr(x), DTYPES[x.dtype], _ptr(qweight), _ptr(scales),
+                                _ptr(zeros_or_lut), M, N, K, bits, group, MODES[mode], _ptr(y),
+                                _ptr(ws), nbytes, _stream(), PATHS[path]), "qmm")
+    return y
+
+
+def dequant(qweight, scales, zeros_or_lut, N, K, mode, bits=4, group=128, dtype=torch.float16,
+            out=None):
+    """Decoded weights W~[N, K] (fp16 or bf16), for checks and inspection."""
+    if out is None:
+        out = torch.empty(N, K, dtype=dtype, device=qweight.device)
+    _check(load().qmm_dequant(_ptr(qweight), _ptr(scales), _ptr(zeros_or_lut), N, K, bits, group,
+                              MODES[mode], DTYPES[out.dtype], _ptr(out), _stream()),
+           "qmm_dequant")
+    return out
+
+
+def check_error():
+    """Raise if a kernel abandoned a bounded wait since the last check."""
+    _check(load().qmm_check_error(_stream()), "qmm_check_error")

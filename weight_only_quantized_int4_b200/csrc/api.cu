@@ -1,0 +1,195 @@
+// C-ABI of libqmm: argument checks, path choice (M-based dispatch) and launch.
+// The declarations, their meaning and the packed layout are in include/qmm.h.
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <algorithm>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace qk {
+
+int device_sms() {
+  static int sms[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (!sms[dev]) {
+    int v = 0;
+    cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
+    sms[dev] = v > 0 ? v : 148;
+  }
+  return sms[dev];
+}
+
+namespace {
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+int check_shape(int N, int K, int bits, int group, int mode) {
+  if (N <= 0 || K <= 0) return QMM_ERR_ARG;
+  if (mode != QMM_SYM && mode != QMM_ASYM && mode != QMM_LUT) return QMM_ERR_ARG;
+  if (bits != 4 && bits != 2) return QMM_ERR_ARG;
+  if (bits == 2 && mode != QMM_LUT) return QMM_ERR_UNSUPPORTED;
+  if (N % 16 != 0 || K % chunk_cols(bits) != 0) return QMM_ERR_UNSUPPORTED;
+  if (group != -1 && (group <= 0 || group % 16 != 0 || K % group != 0)) return QMM_ERR_UNSUPPORTED;
+  return QMM_OK;
+}
+
+int status_of(cudaError_t e) { return e == cudaSuccess ? QMM_OK : QMM_ERR_CUDA; }
+
+// Decode path while the product is bandwidth-bound (few tokens), tensor-core
+// path once it becomes a dense contraction.  2-bit codes always take the
+// decode path (in slabs of 16 tokens).
+int choose_path(int M, int bits) {
+  if (M <= 16 || !tc_supported(bits)) return QMM_PATH_SKINNY;
+  return QMM_PATH_TENSOR;
+}
+
+// The plan a call runs with; `ws_bytes` is what it needs from the workspace.
+struct Plan {
+  int path;
+  SkinnyPlan sk;
+  TcPlan tc;
+  size_t ws_bytes() const { return path == QMM_PATH_TENSOR ? tc.ws_bytes : sk.ws_bytes; }
+};
+
+Plan make_plan(int M, int N, int K, int bits, int group, int path) {
+  Plan p{};
+  p.path = path == QMM_PATH_AUTO ? choose_path(M, bits) : path;
+  if (p.path == QMM_PATH_TENSOR && !tc_supported(bits)) p.path = QMM_PATH_SKINNY;
+  if (p.path == QMM_PATH_TENSOR) p.tc = plan_tc(M, N, K, device_sms());
+  else p.sk = plan_skinny(M, N, K, bits, group, device_sms());
+  return p;
+}
+
+}  // namespace
+}  // namespace qk
+
+using namespace qk;
+
+extern "C" {
+
+size_t qmm_packed_size(int N, int K, int bits, int group, int mode, size_t* scales_bytes,
+                       size_t* zeros_bytes) {
+  if (check_shape(N, K, bits, group, mode) != QMM_OK) return 0;
+  const size_t G = group == -1 ? 1 : (size_t)(K / group);
+  if (scales_bytes) *scales_bytes = (size_t)N * G * 2;
+  if (zeros_bytes) *zeros_bytes = mode == QMM_ASYM ? (size_t)N * G * 2 : 0;
+  return (size_t)N * K * bits / 8;
+}
+
+int qmm_pack(const float* W, int N, int K, int mode, int bits, int group, const uint16_t* lut,
+             void* qweight, uint16_t* scales, uint16_t* zeros, void* stream) {
+  int st = check_shape(N, K, bits, group, mode);
+  if (st != QMM_OK) return st;
+  if (!W || !qweight || !scales) return QMM_ERR_ARG;
+  if (mode == QMM_ASYM && !zeros) return QMM_ERR_ARG;
+  if (mode == QMM_LUT && !lut) return QMM_ERR_ARG;
+  if (!aligned(W, 16) || !aligned(qweight, 16) || !aligned(scales, 4) ||
+      (zeros && !aligned(zeros, 4)))
+    return QMM_ERR_ALIGN;
+  return status_of(launch_pack(W, N, K, mode, bits, group, lut, qweight, scales, zeros,
+                               static_cast<cudaStream_t>(stream)));
+}
+
+int qmm_path(int M, int N, int K, int bits, int group, int mode) {
+  if (M < 0) return QMM_ERR_ARG;
+  int st = check_shape(N, K, bits, group, mode);
+  if (st != QMM_OK) return st;
+  return choose_path(M, bits);
+}
+
+size_t qmm_workspace_size_for(int M, int N, int K, int bits, int group, int mode, int path) {
+  if (M <= 0 || check_shape(N, K, bits, group, mode) != QMM_OK) return 0;
+  if (path != QMM_PATH_AUTO && path != QMM_PATH_SKINNY && path != QMM_PATH_TENSOR) return 0;
+  return make_plan(M, N, K, bits, group, path).ws_bytes();
+}
+
+size_t qmm_workspace_size(int M, int N, int K, int bits, int group, int mode) {
+  return qmm_workspace_size_for(M, N, K, bits, group, mode, QMM_PATH_AUTO);
+}
+
+int qmm_with_path(const void* x, int xdtype, const void* qweight, const uint16_t* scales,
+                  const uint16_t* zeros_or_lut, int M, int N, int K, int bits, int group,
+                  int mode, void* y, void* workspace, size_t workspace_bytes, void* stream,
+                  int path) {
+  if (M < 0) return QMM_ERR_ARG;
+  int st = check_shape(N, K, bits, group, mode);
+  if (st != QMM_OK) return st;
+  if (xdtype != QMM_F16 && xdtype != QMM_BF16) return QMM_ERR_ARG;
+  if (path != QMM_PATH_AUTO && path != QMM_PATH_SKINNY && path != QMM_PATH_TENSOR)
+    return QMM_ERR_ARG;
+  if (M == 0) return QMM_OK;
+  if (!x || !qweight || !scales || !y) return QMM_ERR_ARG;
+  if (mode != QMM_SYM && !zeros_or_lut) return QMM_ERR_ARG;
+  if (!aligned(x, 16) || !aligned(qweight, 16) || !aligned(scales, 4) || !aligned(y, 2) ||
+      (mode == QMM_ASYM && !aligned(zeros_or_lut, 4)) || (workspace && !aligned(workspace, 256)))
+    return QMM_ERR_ALIGN;
+  {
+    const char* xb = static_cast<const char*>(x);
+    const char* yb = static_cast<const char*>(y);
+    const size_t xs = (size_t)M * K * 2, ys = (size_t)M * N * 2;
+    if (xb < yb + ys && yb < xb + xs) return QMM_ERR_ARG;   // y overlaps x
+  }
+  Problem p{x, xdtype == QMM_BF16, qweight, scales, zeros_or_lut, M, N, K, bits, group, mode, y};
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  Plan plan = make_plan(M, N, K, bits, group, path);
+  if (plan.ws_bytes()) {
+    if (!workspace) {
+      // no workspace: every CTA owns whole tiles over all of K, no partial sums
+      if (plan.path == QMM_PATH_TENSOR) {
+        plan.tc.ctas = plan.tc.tiles_n * plan.tc.tiles_m;
+        plan.tc.ws_bytes = 0;
+      } else {
+        plan.sk.splits = plan.sk.tiles_n;
+        plan.sk.ws_bytes = 0;
+      }
+    } else if (workspace_bytes < plan.ws_bytes()) {
+      return QMM_ERR_WORKSPACE;
+    }
+  }
+  if (plan.path == QMM_PATH_TENSOR) return status_of(launch_tc(p, plan.tc, workspace, s));
+  return status_of(launch_skinny(p, plan.sk, workspace, s));
+}
+
+int qmm(const void* x, int xdtype, const void* qweight, const uint16_t* scales,
+        const uint16_t* zeros_or_lut, int M, int N, int K, int bits, int group, int mode, void* y,
+        void* workspace, size_t workspace_bytes, void* stream) {
+  return qmm_with_path(x, xdtype, qweight, scales, zeros_or_lut, M, N, K, bits, group, mode, y,
+                       workspace, workspace_bytes, stream, QMM_PATH_AUTO);
+}
+
+int qmm_dequant(const void* qweight, const uint16_t* scales, const uint16_t* zeros_or_lut, int N,
+                int K, int bits, int group, int mode, int out_dtype, void* W_out, void* stream) {
+  int st = check_shape(N, K, bits, group, mode);
+  if (st != QMM_OK) return st;
+  if (out_dtype != QMM_F16 && out_dtype != QMM_BF16) return QMM_ERR_ARG;
+  if (!qweight || !scales || !W_out) return QMM_ERR_ARG;
+  if (mode != QMM_SYM && !zeros_or_lut) return QMM_ERR_ARG;
+  if (!aligned(qweight, 16) || !aligned(W_out, 8)) return QMM_ERR_ALIGN;
+  return status_of(launch_dequant(qweight, scales, zeros_or_lut, N, K, bits, group, mode,
+                                  out_dtype, W_out, static_cast<cudaStream_t>(stream)));
+}
+
+int qmm_check_error(void* stream) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return QMM_ERR_CUDA;
+  const unsigned v = tc_read_and_clear_error();
+  if (v == 0xFFFFFFFFu) return QMM_ERR_CUDA;
+  return v ? QMM_ERR_TIMEOUT : QMM_OK;
+}
+
+const char* qmm_strerror(int status) {
+  switch (status) {
+    case QMM_OK: return "ok";
+    case QMM_ERR_ARG: return "invalid argument (null pointer, negative size or bad enum value)";
+    case QMM_ERR_UNSUPPORTED: return "unsupported shape, mode or bit width";
+    case QMM_ERR_ALIGN: return "pointer not aligned as required";
+    case QMM_ERR_CUDA: return "CUDA runtime error";
+    case QMM_ERR_TIMEOUT: return "a kernel abandoned a bounded wait";
+    case QMM_ERR_WORKSPACE: return "workspace smaller than qmm_workspace_size";
+    default: return "unknown status";
+  }
+}
+
+}  // extern "C"

@@ -1,0 +1,56 @@
+// Internal launch interface between the C-ABI layer (api.cu) and the kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace qk {
+
+struct Problem {
+  const void* x;
+  bool bf16;
+  const void* qweight;
+  const uint16_t* scales;
+  const uint16_t* zl;     // zeros (ASYM) or table (LUT)
+  int M, N, K, bits, group, mode;
+  void* y;
+};
+
+// Split-K plan of the skinny (M <= 16 per slab) decode path.
+struct SkinnyPlan {
+  int nt;          // token tiles of 8 per slab (1 or 2)
+  int rows;        // rows per CTA tile (16 * row blocks)
+  int tiles_n;     // CTA tiles along N
+  int slabs;       // token slabs (ceil(M / (8 nt)))
+  int splits;      // CTAs along K per tile
+  int cps;         // chunks per split
+  size_t ws_bytes; // workspace needed (0 if splits == 1)
+};
+
+SkinnyPlan plan_skinny(int M, int N, int K, int bits, int group, int sms);
+cudaError_t launch_skinny(const Problem& p, const SkinnyPlan& plan, void* workspace,
+                          cudaStream_t stream);
+
+// Stream-K plan of the tensor-core path (tcgen05, 4-bit codes).
+struct TcPlan {
+  int bn;          // tokens per tile (UMMA N)
+  int tiles_n, tiles_m, nkb, ctas;
+  size_t ws_bytes;
+};
+
+bool tc_supported(int bits);
+TcPlan plan_tc(int M, int N, int K, int sms);
+cudaError_t launch_tc(const Problem& p, const TcPlan& plan, void* workspace, cudaStream_t stream);
+unsigned tc_read_and_clear_error();
+
+cudaError_t launch_pack(const float* W, int N, int K, int mode, int bits, int group,
+                        const uint16_t* lut, void* qweight, uint16_t* scales, uint16_t* zeros,
+                        cudaStream_t stream);
+cudaError_t launch_dequant(const void* qweight, const uint16_t* scales,
+                           const uint16_t* zeros_or_lut, int N, int K, int bits, int group,
+                           int mode, int out_dtype, void* W_out, cudaStream_t stream);
+
+int device_sms();
+
+}  // namespace qk

@@ -1,0 +1,244 @@
+// Quantize/pack and debug-decode kernels.
+//
+// Quantization follows efrantar's reply in "Does Marlin support zero-point
+// quantization?" (IST-DASLab/marlin issue 5: symmetric int4 with the zero fixed
+// at 8 and fp16 scales; fp16 zero-points for the asymmetric variant) and the
+// FLUTE summary's "How It Works" (nearest table entry, times a scale).  The
+// arithmetic is the one documented for qmm_pack in qmm.h: fp32 group
+// reductions, IEEE fp32 division, fp16 scale rounded before use, rint half to
+// even.  This file is compiled with --fmad=false so that no product and sum is
+// ever fused.
+#include <cuda_fp16.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace qk {
+namespace {
+
+// rint() result -> code in [0, qmax]; anything not above 0 (incl. NaN) -> 0.
+__device__ __forceinline__ int clamp_code(float v, int qmax) {
+  if (!(v > 0.0f)) return 0;
+  if (v > (float)qmax) return qmax;
+  return (int)v;
+}
+
+__device__ __forceinline__ uint16_t scale_to_half(float s32) {
+  __half h = __float2half_rn(s32);
+  uint16_t b = __half_as_ushort(h);
+  if ((b & 0x7fff) == 0x7c00) b = (b & 0x8000) | 0x7bff;   // saturate, never inf
+  return b;
+}
+
+// One warp per (row n, group gi): reduce |w| or (min, max) over the group,
+// write the fp16 scale (and zero) at the packed position.
+__global__ void __launch_bounds__(256) pack_scales_kernel(const float* __restrict__ W, int N, int K,
+                                                          int mode, int L, int G,
+                                                          uint16_t* __restrict__ scales,
+                                                          uint16_t* __restrict__ zeros) {
+  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (warp >= N * G) return;
+  const int n = warp / G, gi = warp % G;
+  const float* w = W + (size_t)n * K + (size_t)gi * L;
+  float amax = 0.0f, mn = INFINITY, mx = -INFINITY;
+  for (int i = lane; i < L; i += 32) {
+    float v = w[i];
+    amax = fmaxf(amax, fabsf(v));
+    mn = fminf(mn, v);
+    mx = fmaxf(mx, v);
+  }
+  for (int o = 16; o; o >>= 1) {
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  }
+  if (lane) return;
+  float s32;
+  if (mode == kSYM) s32 = __fdiv_rn(amax, 7.0f);
+  else if (mode == kASYM) s32 = __fdiv_rn(__fsub_rn(mx, mn), 15.0f);
+  else s32 = amax;
+  const uint16_t s16 = scale_to_half(s32);
+  const size_t idx = ((size_t)(n >> 4) * G + gi) * 16 + scale_slot(n & 15);
+  scales[idx] = s16;
+  if (mode == kASYM) {
+    const float s = __half2float(__ushort_as_half(s16));
+    const int z = (s == 0.0f) ? 0 : clamp_code(rintf(__fdiv_rn(-mn, s)), 15);
+    zeros[idx] = __half_as_ushort(__int2half_rn(z));
+  }
+}
+
+struct CodeCtx {
+  const float* W;
+  int K, mode, bits, L, G, nchunks;
+  const uint16_t* scales;
+  const uint16_t* zeros;
+  const uint16_t* lut;   // 2^bits fp16 entries (LUT mode)
+  int nlut;
+};
+
+__device__ __forceinline__ int encode(float w, float s, float z, const CodeCtx& c,
+                                     const float (&lut)[16]) {
+  if (c.mode == kSYM) return s == 0.0f ? 8 : clamp_code(__fadd_rn(rintf(__fdiv_rn(w, s)), 8.0f), 15);
+  if (c.mode == kASYM) return s == 0.0f ? 0 : clamp_code(__fadd_rn(rintf(__fdiv_rn(w, s)), z), 15);
+  const float u = (s == 0.0f) ? 0.0f : __fdiv_rn(w, s);
+  int best = 0;
+  float bd = fabsf(__fsub_rn(u, lut[0]));
+  for (int e = 1; e < c.nlut; ++e) {
+    const float d = fabsf(__fsub_rn(u, lut[e]));
+    if (d < bd) { bd = d; best = e; }
+  }
+  return best;
+}
+
+// One thread per 32-bit word of the packed codes.  Word id -> (row block,
+// chunk, lane, word); the word's codes are gathered from W and placed at the
+// nibble / 2-bit field the layout assigns them.
+__global__ void __launch_bounds__(256) pack_codes_kernel(CodeCtx c, uint32_t* __restrict__ out,
+                                                         size_t nwords) {
+  const size_t wid = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (wid >= nwords) return;
+  const int word = wid & 3;
+  const int lane = (wid >> 2) & 31;
+  const size_t blk = wid >> 7;                       // 128 words per 512-byte chunk
+  const int chunk = (int)(blk % c.nchunks);
+  const int rb = (int)(blk / c.nchunks);
+  const int g = lane >> 2, t = lane & 3;
+  const int KC = chunk_cols(c.bits);
+  float lut[16];
+  for (int e = 0; e < 16; ++e)
+    lut[e] = (c.mode == kLUT && e < c.nlut) ? __half2float(__ushort_as_half(c.lut[e])) : 0.0f;
+  uint32_t v = 0;
+  const int tiles_per_word = c.bits == 4 ? 1 : 2;
+  for (int sub = 0; sub < tiles_per_word; ++sub) {
+    const int j = word * tiles_per_word + sub;                   // 16-column tile
+    const int k0 = chunk * KC + 16 * j + 4 * t;
+    const int gi = k0 / c.L;
+    for (int h = 0; h < 2; ++h) {
+      const int n = rb * 16 + g + 8 * h;
+      const size_t sidx = ((size_t)rb * c.G + gi) * 16 + scale_slot(g + 8 * h);
+      const float s = __half2float(__ushort_as_half(c.scales[sidx]));
+      const float z = c.mode == kASYM ? __half2float(__ushort_as_half(c.zeros[sidx])) : 0.0f;
+      const float4 wv = *reinterpret_cast<const float4*>(c.W + (size_t)n * c.K + k0);
+      const float wc[4] = {wv.x, wv.y, wv.z, wv.w};
+      for (int cc = 0; cc < 4; ++cc) {
+        const uint32_t q = (uint32_t)encode(wc[cc], s, z, c, lut);
+        const int p = h + 2 * (cc >> 1), hi = cc & 1;
+        int shift;
+        if (c.bits == 4) {
+          const int nib = (c.mode == kLUT) ? (2 * p + hi) : (p + 4 * hi);
+          shift = 4 * nib;
+        } else {
+          shift = 8 * (2 * sub + (p >> 1)) + 2 * (2 * (p & 1) + hi);
+        }
+        v |= q << shift;
+      }
+    }
+  }
+  out[wid] = v;
+  __threadfence();   // codes visible before this block retires (see qmm_pack)
+}
+
+// ---------------------------------------------------------------- dequant
+
+// One thread per packed word: decode its codes to (q - z) * s (or T[q] * s),
+// exact in fp32 for integer zero-points, then round once to fp16 / bf16.
+__global__ void __launch_bounds__(256) dequant_kernel(const uint32_t* __restrict__ qw,
+                                                      const uint16_t* __restrict__ scales,
+                                                      const uint16_t* __restrict__ zl, int K,
+                                                      int bits, int mode, int L, int G,
+                                                      int nchunks, bool bf16, void* out,
+                                                      size_t nwords) {
+  const size_t wid = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (wid >= nwords) return;
+  const int word = wid & 3;
+  const int lane = (wid >> 2) & 31;
+  const size_t blk = wid >> 7;
+  const int chunk = (int)(blk % nchunks);
+  const int rb = (int)(blk / nchunks);
+  const int g = lane >> 2, t = lane & 3;
+  const int KC = chunk_cols(bits);
+  const uint32_t v = qw[wid];
+  const int tiles_per_word = bits == 4 ? 1 : 2;
+  for (int sub = 0; sub < tiles_per_word; ++sub) {
+    const int j = word * tiles_per_word + sub;
+    const int k0 = chunk * KC + 16 * j + 4 * t;
+    const int gi = k0 / L;
+    for (int h = 0; h < 2; ++h) {
+      const int n = rb * 16 + g + 8 * h;
+      const size_t sidx = ((size_t)rb * G + gi) * 16 + scale_slot(g + 8 * h);
+      const float s = __half2float(__ushort_as_half(scales[sidx]));
+      const float z = mode == kSYM ? 8.0f
+                      : mode == kASYM ? __half2float(__ushort_as_half(zl[sidx])) : 0.0f;
+      float r[4];
+      for (int cc = 0; cc < 4; ++cc) {
+        const int p = h + 2 * (cc >> 1), hi = cc & 1;
+        uint32_t q;
+        if (bits == 4) {
+          const int nib = (mode == kLUT) ? (2 * p + hi) : (p + 4 * hi);
+          q = (v >> (4 * nib)) & 15u;
+        } else {
+          q = (v >> (8 * (2 * sub + (p >> 1)) + 2 * (2 * (p & 1) + hi))) & 3u;
+        }
+        if (mode == kLUT) r[cc] = __fmul_rn(__half2float(__ushort_as_half(zl[q])), s);
+        else r[cc] = __fmul_rn(__fsub_rn((float)q, z), s);
+      }
+      const size_t o = (size_t)n * K + k0;
+      if (bf16) {
+        __nv_bfloat16* p = reinterpret_cast<__nv_bfloat16*>(out) + o;
+        for (int cc = 0; cc < 4; ++cc) p[cc] = __float2bfloat16_rn(r[cc]);
+      } else {
+        __half* p = reinterpret_cast<__half*>(out) + o;
+        for (int cc = 0; cc < 4; ++cc) p[cc] = __float2half_rn(r[cc]);
+      }
+    }
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_pack(const float* W, int N, int K, int mode, int bits, int group,
+                        const uint16_t* lut, void* qweight, uint16_t* scales, uint16_t* zeros,
+                        cudaStream_t stream) {
+  const int L = group == -1 ? K : group;
+  const int G = K / L;
+  const int warps = N * G;
+  pack_scales_kernel<<<(warps * 32 + 255) / 256, 256, 0, stream>>>(W, N, K, mode, L, G, scales,
+                                                                   zeros);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  CodeCtx c;
+  c.W = W;
+  c.K = K;
+  c.mode = mode;
+  c.bits = bits;
+  c.L = L;
+  c.G = G;
+  c.nchunks = K / chunk_cols(bits);
+  c.scales = scales;
+  c.zeros = zeros;
+  c.lut = lut;
+  c.nlut = 1 << bits;
+  const size_t nwords = (size_t)N * K * bits / 32;
+  const unsigned blocks = (unsigned)((nwords + 255) / 256);
+  pack_codes_kernel<<<blocks, 256, 0, stream>>>(c, reinterpret_cast<uint32_t*>(qweight), nwords);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_dequant(const void* qweight, const uint16_t* scales,
+                           const uint16_t* zeros_or_lut, int N, int K, int bits, int group,
+                           int mode, int out_dtype, void* W_out, cudaStream_t stream) {
+  const int L = group == -1 ? K : group;
+  const int G = K / L;
+  const size_t nwords = (size_t)N * K * bits / 32;
+  const unsigned blocks = (unsigned)((nwords + 255) / 256);
+  dequant_kernel<<<blocks, 256, 0, stream>>>(reinterpret_cast<const uint32_t*>(qweight), scales,
+                                             zeros_or_lut, K, bits, mode, L, G,
+                                             K / chunk_cols(bits), out_dtype == QMM_BF16, W_out,
+                                             nwords);
+  return cudaGetLastError();
+}
+
+}  // namespace qk

@@ -1,0 +1,684 @@
+// Tensor-core path (tcgen05 + TMEM + TMA) for many tokens.
+//
+// Once M is large the product stops being bandwidth-bound and becomes a dense
+// contraction; the decode-then-multiply order of the GPTQ-Triton summary ("How
+// It Works": quantized weights decoded on the fly before the matmul) is kept,
+// but the multiply runs on the 5th-generation tensor cores:
+//
+//   D[128 weight rows, BN tokens] (fp32, TMEM) += A[128, 64] . B[BN, 64]^T
+//
+// per 64-column K block, with A = decoded weights (fp16/bf16, written into
+// shared memory in the 128-byte-swizzled K-major layout by decode warps) and
+// B = a TMA-loaded tile of x.  Warp roles (10 warps):
+//   warp 0      TMA producer: code tiles (4 KB, 8 row blocks) and x tiles
+//   warp 1      TMEM owner and MMA issuer (one elected thread)
+//   warps 2-5   decode: codes (smem) -> (q - z) s, T[q] s -> A tile (smem)
+//   warps 6-9   epilogue: TMEM -> registers -> y (or split-K partials)
+// Work is split stream-K over (tile, K block) units across a grid of one CTA
+// per SM, like the decode path; partial tiles are reduced deterministically by
+// the last CTA that finishes them.  Every mbarrier wait is bounded: a wait
+// that runs out sets the device error word (qmm_check_error) and the CTA
+// drains and exits instead of hanging.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace qk {
+
+__device__ unsigned g_tc_error = 0;
+
+namespace {
+
+constexpr int kTcThreads = 320;
+constexpr int kKB = 64;             // K columns per stage (one 128-byte swizzle row of fp16)
+constexpr int kRowsTile = 128;      // weight rows per tile (UMMA M)
+constexpr int kCodeStages = 8;
+constexpr int kCodeBytes = 8 * 512; // 8 row blocks x one 512-byte chunk
+constexpr int kATileBytes = kRowsTile * kKB * 2;   // 16 KB
+constexpr long long kWaitCycles = 4000000000ll; // ~2 s at 1.9 GHz
+
+template <int BN>
+struct TcCfg {
+  static constexpr int STAGES = BN == 256 ? 3 : 4;
+  static constexpr int B_BYTES = BN * kKB * 2;
+  static constexpr int TMEM_COLS = 2 * BN;     // two accumulator buffers
+};
+
+// ------------------------------------------------------------------ PTX helpers
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+               "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded wait for phase `parity` of `bar`.  Returns false (and raises the
+// CTA's abort flag and the device error word) if it runs out, or if another
+// thread of the CTA has already aborted.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
+  if (mbar_try(bar, parity)) return true;
+  const long long t0 = clock64();
+  while (true) {
+    if (mbar_try(bar, parity)) return true;
+    if (*abort) return false;
+    if (clock64() - t0 > kWaitCycles) {
+      *abort = 1;
+      atomicOr(&g_tc_error, 1u);
+      return false;
+    }
+  }
+}
+
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar,
+                                            int x, int y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes "
+      "[%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y)
+      : "memory");
+}
+
+__device__ __forceinline__ void fence_proxy_async() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// Shared-memory matrix descriptor: K-major, 128-byte swizzle, 8-row groups
+// 1024 bytes apart (tile bases are 1024-byte aligned).
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr >> 4) & 0x3FFF);
+  d |= (uint64_t)1 << 16;              // leading byte offset (unused for swizzled K-major)
+  d |= (uint64_t)(1024 >> 4) << 32;    // stride byte offset
+  d |= (uint64_t)1 << 46;              // descriptor version
+  d |= (uint64_t)2 << 61;              // 128-byte swizzle
+  return d;
+}
+
+__device__ __forceinline__ void umma_f16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc,
+                                         uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a), "l"(b), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ void umma_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   smem_u32(bar))
+               : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
+  uint32_t r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
+      "%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+__device__ __forceinline__ void named_bar(int id, int threads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
+// ------------------------------------------------------------------ kernel
+
+struct TcArgs {
+  const uint16_t* scales;
+  const uint16_t* zl;
+  uint16_t* y;
+  int M, N, K, L, G, nrb, nkb;
+  int tiles_n, tiles_m, tiles;
+  long long units;          // tiles * nkb
+  int ctas;
+  float* slots;             // [2 * ctas][BN][128]: a CTA's first / last partial tile
+  unsigned* counters;       // [tiles]
+};
+
+__device__ __forceinline__ int owner_of_tc(long long u, long long U, int C) {
+  return (int)(((u + 1) * (long long)C - 1) / U);
+}
+
+// Scaled decoded pair (row of the pair, two k) -> packed fp16 / bf16.
+template <bool BF16>
+__device__ __forceinline__ uint32_t scale_pair(uint32_t v, float s) {
+  if constexpr (BF16) {
+    const float lo = __uint_as_float(v << 16), hi = __uint_as_float(v & 0xFFFF0000u);
+    return pack2<true>(lo * s, hi * s);
+  } else {
+    const __half2 sh = __float2half2_rn(s);
+    const __half2 r = __hmul2(*reinterpret_cast<const __half2*>(&v), sh);
+    return *reinterpret_cast<const uint32_t*>(&r);
+  }
+}
+
+// fp16 table pair -> A operand pair: T s rounded once (fp16: one HMUL2; bf16:
+// product in fp32, then rounded); with per-row scales (group -1) the scale is
+// applied in the epilogue and T alone is converted.
+template <bool BF16, bool GM1>
+__device__ __forceinline__ uint32_t lut_pair(uint32_t t16, float s) {
+  if constexpr (!BF16) {
+    return GM1 ? t16 : scale_pair<false>(t16, s);
+  } else {
+    const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&t16));
+    return GM1 ? pack2<true>(f.x, f.y) : pack2<true>(f.x * s, f.y * s);
+  }
+}
+
+template <int MODE, bool BF16, int BN, bool GM1>
+__global__ void __launch_bounds__(kTcThreads, 1)
+    tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_w,
+              const TcArgs a) {
+  using Cfg = TcCfg<BN>;
+  constexpr int S = Cfg::STAGES;
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  // carve: A stages | B stages | code stages | LUT table | barriers
+  unsigned char* base = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  unsigned char* sA = base;
+  unsigned char* sB = sA + S * kATileBytes;
+  unsigned char* sC = sB + S * Cfg::B_BYTES;
+  unsigned char* sT = sC + kCodeStages * kCodeBytes;
+  constexpr int TAB = MODE == kLUT ? 256 * 32 * 4 : 0;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sT + TAB);
+  uint64_t* code_full = bars;
+  uint64_t* code_empty = code_full + kCodeStages;
+  uint64_t* b_full = code_empty + kCodeStages;
+  uint64_t* a_full = b_full + S;
+  uint64_t* ab_empty = a_full + S;
+  uint64_t* acc_full = ab_empty + S;      // [2]
+  uint64_t* acc_empty = acc_full + 2;     // [2]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  int* last_flag = const_cast<int*>(abort_flag) + 1;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int b = blockIdx.x;
+  const long long u_begin = (long long)b * a.units / a.ctas;
+  const long long u_end = (long long)(b + 1) * a.units / a.ctas;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kCodeStages; ++i) {
+      mbar_init(&code_full[i], 1);
+      mbar_init(&code_empty[i], 4);
+    }
+    for (int i = 0; i < S; ++i) {
+      mbar_init(&b_full[i], 1);
+      mbar_init(&a_full[i], 4);
+      mbar_init(&ab_empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&acc_full[i], 1);
+      mbar_init(&acc_empty[i], 4);
+    }
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 0 && lane == 0) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&map_x)) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&map_w)) : "memory");
+  }
+  pdl_wait();                 // inputs may come from the previous grid; TMEM taken after this
+  pdl_launch_dependents();
+
+  if constexpr (MODE == kLUT) {
+    // 4-bit pair table replicated per bank (see the decode path): fp16
+    // entries; with bf16 activations the scaled product is rounded per weight.
+    uint32_t* tab = reinterpret_cast<uint32_t*>(sT);
+    for (int i = threadIdx.x; i < 256 * 32; i += kTcThreads) {
+      const int e = i >> 5;
+      tab[i] = (uint32_t)a.zl[e & 15] | ((uint32_t)a.zl[e >> 4] << 16);
+    }
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(tmem_slot)),
+                 "r"(Cfg::TMEM_COLS)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  // Segments of this CTA: [u, u + len) within one tile.
+  auto seg_of = [&](long long u, int& tile, int& kb0, int& kb1) {
+    tile = (int)(u / a.nkb);
+    kb0 = (int)(u % a.nkb);
+    kb1 = (int)std::min<long long>(a.nkb, kb0 + (u_end - u));
+  };
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int kc = 0, ks = 0;     // running k-block counters for the code / A-B rings
+      for (long long u = u_begin; u < u_end && !*abort_flag;) {
+        int tile, kb0, kb1;
+        seg_of(u, tile, kb0, kb1);
+        const int tn = tile % a.tiles_n, tm = tile / a.tiles_n;
+        for (int kb = kb0; kb < kb1; ++kb, ++kc, ++ks) {
+          const int c = kc % kCodeStages, s = ks % S;
+          if (!mbar_wait(&code_empty[c], ((kc / kCodeStages) & 1) ^ 1, abort_flag)) break;
+          mbar_expect_tx(&code_full[c], kCodeBytes);
+          tma_load_2d(sC + c * kCodeBytes, &map_w, &code_full[c], kb * 128, tn * 8);
+          if (!mbar_wait(&ab_empty[s], ((ks / S) & 1) ^ 1, abort_flag)) break;
+          mbar_expect_tx(&b_full[s], Cfg::B_BYTES);
+          tma_load_2d(sB + s * Cfg::B_BYTES, &map_x, &b_full[s], kb * kKB, tm * BN);
+        }
+        u += kb1 - kb0;
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = (1u << 4) | (BF16 ? (1u << 7) | (1u << 10) : 0u) |
+                                 ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(kRowsTile >> 4) << 24);
+      int ks = 0, seg = 0;
+      for (long long u = u_begin; u < u_end && !*abort_flag; ++seg) {
+        int tile, kb0, kb1;
+        seg_of(u, tile, kb0, kb1);
+        const int buf = seg & 1;
+        if (!mbar_wait(&acc_empty[buf], ((seg >> 1) & 1) ^ 1, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t d = tmem_base + (uint32_t)(buf * BN);
+        bool ok = true;
+        for (int kb = kb0; kb < kb1; ++kb, ++ks) {
+          const int s = ks % S;
+          const uint32_t ph = (ks / S) & 1;
+          if (!mbar_wait(&a_full[s], ph, abort_flag) || !mbar_wait(&b_full[s], ph, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sa = smem_u32(sA + s * kATileBytes);
+          const uint32_t sb = smem_u32(sB + s * Cfg::B_BYTES);
+#pragma unroll
+          for (int k = 0; k < kKB / 16; ++k)
+            umma_f16(d, sw128_desc(sa + 32 * k), sw128_desc(sb + 32 * k), idesc,
+                     (kb > kb0 || k > 0) ? 1u : 0u);
+          umma_commit(&ab_empty[s]);
+        }
+        if (!ok) break;
+        umma_commit(&acc_full[buf]);
+        u += kb1 - kb0;
+      }
+    }
+  } else if (warp < 6) {
+    // ------------------------------------------------------------ decode warps
+    const int dw = warp - 2;                 // row blocks 2dw, 2dw + 1 of the tile
+    const int g = lane >> 2, t = lane & 3;
+    const unsigned char* tabp = sT;
+    int kc = 0, ks = 0;
+    for (long long u = u_begin; u < u_end && !*abort_flag;) {
+      int tile, kb0, kb1;
+      seg_of(u, tile, kb0, kb1);
+      const int tn = tile % a.tiles_n;
+      bool ok = true;
+      for (int kb = kb0; kb < kb1; ++kb, ++kc, ++ks) {
+        const int c = kc % kCodeStages, s = ks % S;
+        if (!mbar_wait(&code_full[c], (kc / kCodeStages) & 1, abort_flag) ||
+            !mbar_wait(&ab_empty[s], ((ks / S) & 1) ^ 1, abort_flag)) {
+          ok = false;
+          break;
+        }
+        unsigned char* At = sA + s * kATileBytes;
+#pragma unroll
+        for (int rr = 0; rr < 2; ++rr) {
+          const int rbl = 2 * dw + rr;                       // row block in the tile
+          const int rb = tn * 8 + rbl;
+          const uint4 wv = *reinterpret_cast<const uint4*>(sC + c * kCodeBytes + rbl * 512 + lane * 16);
+          const int R0 = rbl * 16 + g, R1 = R0 + 8;
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const uint32_t w = (&wv.x)[j];
+            uint32_t af[4];
+            if constexpr (MODE == kSYM) {
+              decode_int4<BF16, 8>(w, af);
+            } else if constexpr (MODE == kASYM) {
+              decode_int4<BF16, 0>(w, af);
+              const int gi = (kb * kKB + 16 * j) / a.L;
+              uint32_t zw = 0;
+              if (rb < a.nrb)
+                zw = *reinterpret_cast<const uint32_t*>(a.zl + ((size_t)rb * a.G + gi) * 16 + 2 * g);
+              if constexpr (BF16) {
+                const float2 zf = __half22float2(*reinterpret_cast<const __half2*>(&zw));
+                zw = pack2<true>(zf.x, zf.y);
+              }
+              sub_zero<BF16>(__byte_perm(zw, 0, 0x1010), __byte_perm(zw, 0, 0x3232), af);
+            } else {
+              const uint32_t l4 = (uint32_t)lane << 2;
+              af[0] = *reinterpret_cast<const uint32_t*>(tabp + lop3_and_or(w << 7, 0x7F80u, l4));
+              af[1] = *reinterpret_cast<const uint32_t*>(tabp + lop3_and_or(w >> 1, 0x7F80u, l4));
+              af[2] = *reinterpret_cast<const uint32_t*>(tabp + lop3_and_or(w >> 9, 0x7F80u, l4));
+              af[3] = *reinterpret_cast<const uint32_t*>(tabp + lop3_and_or(w >> 17, 0x7F80u, l4));
+            }
+            float2 sc = make_float2(1.f, 1.f);
+            if constexpr (!GM1) {
+              const int gi = (kb * kKB + 16 * j) / a.L;
+              sc = make_float2(0.f, 0.f);
+              if (rb < a.nrb) {
+                const uint32_t sw = *reinterpret_cast<const uint32_t*>(
+                    a.scales + ((size_t)rb * a.G + gi) * 16 + 2 * g);
+                sc = __half22float2(*reinterpret_cast<const __half2*>(&sw));
+              }
+            }
+            if constexpr (MODE == kLUT) {
+              af[0] = lut_pair<BF16, GM1>(af[0], sc.x);
+              af[2] = lut_pair<BF16, GM1>(af[2], sc.x);
+              af[1] = lut_pair<BF16, GM1>(af[1], sc.y);
+              af[3] = lut_pair<BF16, GM1>(af[3], sc.y);
+            } else if constexpr (!GM1) {
+              af[0] = scale_pair<BF16>(af[0], sc.x);
+              af[2] = scale_pair<BF16>(af[2], sc.x);
+              af[1] = scale_pair<BF16>(af[1], sc.y);
+              af[3] = scale_pair<BF16>(af[3], sc.y);
+            }
+            // k_local = 16 j + 4 t: 16-byte chunk 2j + t/2, offset 8 (t & 1)
+            const int ch = 2 * j + (t >> 1);
+            const int off = 8 * (t & 1);
+            *reinterpret_cast<uint2*>(At + R0 * 128 + ((ch ^ (R0 & 7)) << 4) + off) =
+                make_uint2(af[0], af[2]);
+            *reinterpret_cast<uint2*>(At + R1 * 128 + ((ch ^ (R1 & 7)) << 4) + off) =
+                make_uint2(af[1], af[3]);
+          }
+        }
+        fence_proxy_async();
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(&code_empty[c]);
+          mbar_arrive(&a_full[s]);
+        }
+      }
+      if (!ok) break;
+      u += kb1 - kb0;
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue warps
+    const int q = warp & 3;                  // TMEM lane quadrant of this warp
+    const int row_l = q * 32 + lane;         // weight row within the tile
+    int seg = 0;
+    for (long long u = u_begin; u < u_end && !*abort_flag; ++seg) {
+      int tile, kb0, kb1;
+      seg_of(u, tile, kb0, kb1);
+      const int tn = tile % a.tiles_n, tm = tile / a.tiles_n;
+      const int buf = seg & 1;
+      if (!mbar_wait(&acc_full[buf], (seg >> 1) & 1, abort_flag)) break;
+      tc_fence_after();
+      const int row = tn * kRowsTile + row_l;
+      float s_row = 1.0f;
+      if constexpr (GM1) {
+        if (row < a.N) s_row = __half2float(__ushort_as_half(a.scales[(size_t)(row >> 4) * 16 +
+                                                                      scale_slot(row & 15)]));
+      }
+      const long long t_first = (long long)tile * a.nkb;
+      const bool whole = (u == t_first) && (kb1 == a.nkb);
+      int first = 0, nb = 1;
+      float* slot = nullptr;
+      if (!whole) {
+        first = owner_of_tc(t_first, a.units, a.ctas);
+        nb = owner_of_tc(t_first + a.nkb - 1, a.units, a.ctas) - first + 1;
+        const int e = (tile == (int)(u_begin / a.nkb)) ? 0 : 1;
+        slot = a.slots + (size_t)(2 * b + e) * (size_t)(BN * kRowsTile);
+      }
+#pragma unroll 1
+      for (int c0 = 0; c0 < BN; c0 += 32) {
+        float v[32];
+        tmem_ld32(tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * BN + c0), v);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const int m = tm * BN + c0 + i;
+          if (whole) {
+            if (row < a.N && m < a.M) {
+              const float o = v[i] * s_row;
+              a.y[(size_t)m * a.N + row] = BF16 ? __bfloat16_as_ushort(__float2bfloat16_rn(o))
+                                                : __half_as_ushort(__float2half_rn(o));
+            }
+          } else {
+            slot[(size_t)(c0 + i) * kRowsTile + row_l] = v[i];
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty[buf]);
+      if (!whole) {
+        __threadfence();
+        named_bar(1, 128);
+        if (threadIdx.x == 192) *last_flag = (atomicAdd(&a.counters[tile], 1u) == (unsigned)(nb - 1));
+        named_bar(1, 128);
+        if (*last_flag) {
+          __threadfence();
+          for (int cc = 0; cc < BN; ++cc) {
+            const int m = tm * BN + cc;
+            float acc = 0.0f;
+            for (int k = 0; k < nb; ++k) {
+              const int bb = first + k;
+              const int ee = ((long long)bb * a.units / a.ctas < t_first) ? 1 : 0;
+              acc += __ldcg(a.slots + (size_t)(2 * bb + ee) * (BN * kRowsTile) +
+                            (size_t)cc * kRowsTile + row_l);
+            }
+            if (row < a.N && m < a.M) {
+              const float o = acc * s_row;
+              a.y[(size_t)m * a.N + row] = BF16 ? __bfloat16_as_ushort(__float2bfloat16_rn(o))
+                                                : __half_as_ushort(__float2half_rn(o));
+            }
+          }
+          if (threadIdx.x == 192) a.counters[tile] = 0u;
+        }
+        named_bar(1, 128);
+      }
+      u += kb1 - kb0;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
+                 "r"(Cfg::TMEM_COLS)
+                 : "memory");
+  }
+}
+
+}  // namespace
+}  // namespace qk
+
+namespace qk {
+namespace {
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+template <int MODE, int BN>
+constexpr size_t tc_smem_bytes() {
+  using Cfg = TcCfg<BN>;
+  return 1024 + (size_t)Cfg::STAGES * (kATileBytes + Cfg::B_BYTES) +
+         (size_t)kCodeStages * kCodeBytes + (MODE == kLUT ? 256 * 32 * 4 : 0) +
+         (2 * kCodeStages + 3 * Cfg::STAGES + 4) * 8 + 16;
+}
+
+template <int MODE, bool BF16, int BN, bool GM1>
+cudaError_t launch_tc_t(const CUtensorMap& mx, const CUtensorMap& mw, const TcArgs& args,
+                        cudaStream_t stream) {
+  auto k = tc_kernel<MODE, BF16, BN, GM1>;
+  constexpr size_t smem = tc_smem_bytes<MODE, BN>();
+  static bool attr_set[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev >= 0 && dev < 64 && !attr_set[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    attr_set[dev] = true;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(args.ctas, 1, 1);
+  cfg.blockDim = dim3(kTcThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, k, mx, mw, args);
+}
+
+template <int MODE, bool BF16, bool GM1>
+cudaError_t launch_bn(int bn, const CUtensorMap& mx, const CUtensorMap& mw, const TcArgs& args,
+                      cudaStream_t s) {
+  if (bn == 64) return launch_tc_t<MODE, BF16, 64, GM1>(mx, mw, args, s);
+  if (bn == 128) return launch_tc_t<MODE, BF16, 128, GM1>(mx, mw, args, s);
+  return launch_tc_t<MODE, BF16, 256, GM1>(mx, mw, args, s);
+}
+
+template <int MODE>
+cudaError_t launch_mode(bool bf16, bool gm1, int bn, const CUtensorMap& mx, const CUtensorMap& mw,
+                        const TcArgs& args, cudaStream_t s) {
+  if (bf16) return gm1 ? launch_bn<MODE, true, true>(bn, mx, mw, args, s)
+                       : launch_bn<MODE, true, false>(bn, mx, mw, args, s);
+  return gm1 ? launch_bn<MODE, false, true>(bn, mx, mw, args, s)
+             : launch_bn<MODE, false, false>(bn, mx, mw, args, s);
+}
+
+}  // namespace
+
+bool tc_supported(int bits) { return bits == 4; }
+
+TcPlan plan_tc(int M, int N, int K, int sms) {
+  TcPlan p{};
+  p.bn = M <= 64 ? 64 : (M <= 128 ? 128 : 256);
+  p.tiles_n = (N + kRowsTile - 1) / kRowsTile;
+  p.tiles_m = (M + p.bn - 1) / p.bn;
+  p.nkb = K / kKB;
+  const long long units = (long long)p.tiles_n * p.tiles_m * p.nkb;
+  long long ctas = sms;   // one CTA per SM (shared memory bound)
+  if (ctas > units) ctas = units;
+  p.ctas = (int)ctas;
+  const int tiles = p.tiles_n * p.tiles_m;
+  const bool split = !(units % ctas == 0 && (units / ctas) % p.nkb == 0);
+  p.ws_bytes = split ? ((size_t)tiles * 4 + 255) / 256 * 256 +
+                           (size_t)2 * p.ctas * p.bn * kRowsTile * sizeof(float)
+                     : 0;
+  return p;
+}
+
+cudaError_t launch_tc(const Problem& pr, const TcPlan& plan, void* workspace,
+                      cudaStream_t stream) {
+  auto encode = encode_fn();
+  if (!encode) return cudaErrorNotSupported;
+  CUtensorMap mx, mw;
+  {
+    const cuuint64_t dims[2] = {(cuuint64_t)pr.K, (cuuint64_t)pr.M};
+    const cuuint64_t strides[1] = {(cuuint64_t)pr.K * 2};
+    const cuuint32_t box[2] = {(cuuint32_t)kKB, (cuuint32_t)plan.bn};
+    const cuuint32_t es[2] = {1, 1};
+    if (encode(&mx, pr.bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2,
+               const_cast<void*>(pr.x), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+               CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
+  {
+    const int nchunks = pr.K / 64;
+    const cuuint64_t dims[2] = {(cuuint64_t)nchunks * 128, (cuuint64_t)(pr.N / 16)};
+    const cuuint64_t strides[1] = {(cuuint64_t)nchunks * 512};
+    const cuuint32_t box[2] = {128, 8};
+    const cuuint32_t es[2] = {1, 1};
+    if (encode(&mw, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<void*>(pr.qweight), dims, strides,
+               box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
+  TcArgs a{};
+  a.scales = pr.scales;
+  a.zl = pr.zl;
+  a.y = reinterpret_cast<uint16_t*>(pr.y);
+  a.M = pr.M;
+  a.N = pr.N;
+  a.K = pr.K;
+  a.L = pr.group == -1 ? pr.K : pr.group;
+  a.G = pr.K / a.L;
+  a.nrb = pr.N / 16;
+  a.nkb = plan.nkb;
+  a.tiles_n = plan.tiles_n;
+  a.tiles_m = plan.tiles_m;
+  a.tiles = plan.tiles_n * plan.tiles_m;
+  a.units = (long long)a.tiles * plan.nkb;
+  a.ctas = plan.ctas;
+  if (plan.ws_bytes) {
+    const size_t cbytes = ((size_t)a.tiles * 4 + 255) / 256 * 256;
+    a.counters = reinterpret_cast<unsigned*>(workspace);
+    a.slots = reinterpret_cast<float*>(reinterpret_cast<char*>(workspace) + cbytes);
+  }
+  const bool gm1 = pr.group == -1;
+  switch (pr.mode) {
+    case kSYM: return launch_mode<kSYM>(pr.bf16, gm1, plan.bn, mx, mw, a, stream);
+    case kASYM: return launch_mode<kASYM>(pr.bf16, gm1, plan.bn, mx, mw, a, stream);
+    default: return launch_mode<kLUT>(pr.bf16, gm1, plan.bn, mx, mw, a, stream);
+  }
+}
+
+unsigned tc_read_and_clear_error() {
+  unsigned v = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&v, g_tc_error, sizeof(v)) != cudaSuccess) return 0xFFFFFFFFu;
+  if (v) cudaMemcpyToSymbol(g_tc_error, &zero, sizeof(zero));
+  return v;
+}
+
+}  // namespace qk
