@@ -33,7 +33,7 @@
  *    cudaGetLastError right after the launch.  Errors raised later by a kernel
  *    (a bounded wait that ran out) are reported by qmm_check_error.
  *  - Shapes the GPU kernels accept: N % 16 == 0; K % 64 == 0 (4-bit) or
- *    K % 128 == 0 (2-bit); group == -1 or group a multiple of 16 that divides K;
+ *    K % 128 == 0 (2-bit); group == -1 or a power of two >= 16 that divides K;
  *    M >= 0.  Other shapes return QMM_ERR_UNSUPPORTED.
  *
  * Packed layout (written by qmm_pack, read by qmm and qmm_dequant):
@@ -127,8 +127,9 @@ size_t qmm_workspace_size_for(int M, int N, int K, int bits, int group, int mode
  *                 filled before first use (see above); may be NULL with
  *                 workspace_bytes 0, in which case no cross-CTA split-K is used.
  * The accumulation is fp32.  M <= 16 runs the bandwidth-bound decode path,
- * larger M the tcgen05 tensor-core path (4-bit codes; 2-bit codes stay on the
- * decode path); qmm_path tells which.  The tensor path reads x through a TMA
+ * larger M the tcgen05 tensor-core path for 4-bit codes with fp16 activations
+ * or with bf16 activations and per-row scales (group -1, SYM/ASYM); the other
+ * combinations stay on the decode path.  qmm_path tells which.  The tensor path reads x through a TMA
  * tensor map, so x's row pitch (K * 2 bytes) must be a multiple of 16 -- true
  * for every K the packed layout allows. */
 int qmm(const void* x, int xdtype, const void* qweight, const uint16_t* scales,
@@ -141,8 +142,8 @@ int qmm_with_path(const void* x, int xdtype, const void* qweight, const uint16_t
                   int mode, void* y, void* workspace, size_t workspace_bytes, void* stream,
                   int path);
 
-/* The path qmm picks for this problem (QMM_PATH_SKINNY or QMM_PATH_TENSOR),
- * or a negative qmm_status for an unsupported problem. */
+/* The path qmm picks for this problem with fp16 activations (QMM_PATH_SKINNY
+ * or QMM_PATH_TENSOR), or a negative qmm_status for an unsupported problem. */
 int qmm_path(int M, int N, int K, int bits, int group, int mode);
 
 /* Decode the packed weights into W_out[N, K] row-major (fp16 or bf16 by

@@ -52,6 +52,7 @@ def test_sizes_and_paths(lib):
     (4096, 4096, 2, 64, "sym", -2),     # 2-bit needs LUT
     (4096, 4160, 2, 64, "lut", -2),     # 2-bit needs K % 128
     (4096, 4096, 4, 100, "sym", -2),    # group not a multiple of 16
+    (4608, 4608, 4, 48, "sym", -2),     # group not a power of two
     (4096, 4096, 4, 384, "sym", -2),    # group does not divide K
     (0, 4096, 4, 128, "sym", -1),
     (4096, 4096, 3, 128, "lut", -1),

@@ -118,11 +118,35 @@ def test_qmm_small(mode, bits, group, xdtype):
         p = cases.make(mode, bits, group, M, N, K, xdtype, seed=M)
         y_ref, bound = cases.expected(p)
         x, qw, sp, zl = upload(p)
-        for path in ("auto", "skinny"):
-            ws = q.workspace(M, N, K, mode, bits, group)
+        for path in ("auto", "skinny", "tensor"):
+            ws = q.workspace(M, N, K, mode, bits, group, path=path)
             y = q.qmm(x, qw, sp, zl, N, K, mode, bits, group, ws=ws, path=path)
             torch.cuda.synchronize()
             cases.compare(to_f64(y, xdtype), y_ref, bound, f"{mode}{bits} g{group} M{M} {path}")
+
+
+TC_CASES = [("sym", 4, 128, "f16"), ("sym", 4, -1, "f16"), ("asym", 4, 128, "f16"),
+            ("lut", 4, 64, "f16"), ("lut", 4, -1, "f16"), ("sym", 4, 32, "f16"),
+            ("sym", 4, -1, "bf16"), ("asym", 4, -1, "bf16")]
+
+
+@pytest.mark.parametrize("mode,bits,group,xdtype", TC_CASES)
+def test_qmm_tensor_path(mode, bits, group, xdtype):
+    """tcgen05 path: two full 128-row tiles plus a ragged 16-row one, token tiles
+    of 64/128/256 with ragged M, stream-K split (workspace) and whole tiles
+    (no workspace)."""
+    N, K = 272, 1024
+    for M in (17, 64, 65, 130, 300):
+        p = cases.make(mode, bits, group, M, N, K, xdtype, seed=100 + M)
+        y_ref, bound = cases.expected(p)
+        x, qw, sp, zl = upload(p)
+        assert q.path(M, N, K, mode, bits, group) == "tensor"
+        for with_ws in (True, False):
+            ws = q.workspace(M, N, K, mode, bits, group, path="tensor") if with_ws else None
+            y = q.qmm(x, qw, sp, zl, N, K, mode, bits, group, ws=ws, path="tensor")
+            torch.cuda.synchronize()
+            cases.compare(to_f64(y, xdtype), y_ref, bound, f"tc {mode} g{group} M{M} ws={with_ws}")
+    q.check_error()
 
 
 @pytest.mark.parametrize("ws_kind", ["none", "sized"])

@@ -55,6 +55,8 @@ def load(path: str = LIB_PATH):
             lib.qmm_pack.argtypes = [P, I, I, I, I, I, P, P, P, P, P]
             lib.qmm_workspace_size.argtypes = [I, I, I, I, I, I]
             lib.qmm_workspace_size.restype = S
+            lib.qmm_workspace_size_for.argtypes = [I, I, I, I, I, I, I]
+            lib.qmm_workspace_size_for.restype = S
             lib.qmm.argtypes = [P, I, P, P, P, I, I, I, I, I, I, P, P, S, P]
             lib.qmm_with_path.argtypes = [P, I, P, P, P, I, I, I, I, I, I, P, P, S, P, I]
             lib.qmm_path.argtypes = [I, I, I, I, I, I]
@@ -115,13 +117,13 @@ def pack(W, mode, bits=4, group=128, lut=None, out=None):
     return qw, sc, ze
 
 
-def workspace_size(M, N, K, mode, bits=4, group=128):
-    return load().qmm_workspace_size(M, N, K, bits, group, MODES[mode])
+def workspace_size(M, N, K, mode, bits=4, group=128, path="auto"):
+    return load().qmm_workspace_size_for(M, N, K, bits, group, MODES[mode], PATHS[path])
 
 
-def workspace(M, N, K, mode, bits=4, group=128, device="cuda"):
+def workspace(M, N, K, mode, bits=4, group=128, device="cuda", path="auto"):
     """A zero-filled workspace for this problem (None if it needs none)."""
-    n = workspace_size(M, N, K, mode, bits, group)
+    n = workspace_size(M, N, K, mode, bits, group, path)
     return torch.zeros(n, dtype=torch.uint8, device=device) if n else None
 
 

@@ -32,17 +32,20 @@ int check_shape(int N, int K, int bits, int group, int mode) {
   if (bits != 4 && bits != 2) return QMM_ERR_ARG;
   if (bits == 2 && mode != QMM_LUT) return QMM_ERR_UNSUPPORTED;
   if (N % 16 != 0 || K % chunk_cols(bits) != 0) return QMM_ERR_UNSUPPORTED;
-  if (group != -1 && (group <= 0 || group % 16 != 0 || K % group != 0)) return QMM_ERR_UNSUPPORTED;
+  // groups: one per row (-1) or a power of two >= 16 dividing K
+  if (group != -1 && (group < 16 || (group & (group - 1)) != 0 || K % group != 0))
+    return QMM_ERR_UNSUPPORTED;
   return QMM_OK;
 }
 
 int status_of(cudaError_t e) { return e == cudaSuccess ? QMM_OK : QMM_ERR_CUDA; }
 
 // Decode path while the product is bandwidth-bound (few tokens), tensor-core
-// path once it becomes a dense contraction.  2-bit codes always take the
-// decode path (in slabs of 16 tokens).
-int choose_path(int M, int bits) {
-  if (M <= 16 || !tc_supported(bits)) return QMM_PATH_SKINNY;
+// path once it becomes a dense contraction.  Combinations the tensor path does
+// not cover (2-bit codes; bf16 with group scales or a table) take the decode
+// path, in slabs of 16 tokens.
+int choose_path(int M, int bits, int mode, bool bf16, int group) {
+  if (M <= 16 || !tc_supported(bits, mode, bf16, group)) return QMM_PATH_SKINNY;
   return QMM_PATH_TENSOR;
 }
 
@@ -54,12 +57,12 @@ struct Plan {
   size_t ws_bytes() const { return path == QMM_PATH_TENSOR ? tc.ws_bytes : sk.ws_bytes; }
 };
 
-Plan make_plan(int M, int N, int K, int bits, int group, int path) {
+Plan make_plan(int M, int N, int K, int bits, int group, int mode, bool bf16, int path) {
   Plan p{};
-  p.path = path == QMM_PATH_AUTO ? choose_path(M, bits) : path;
-  if (p.path == QMM_PATH_TENSOR && !tc_supported(bits)) p.path = QMM_PATH_SKINNY;
+  p.path = path == QMM_PATH_AUTO ? choose_path(M, bits, mode, bf16, group) : path;
+  if (p.path == QMM_PATH_TENSOR && !tc_supported(bits, mode, bf16, group)) p.path = QMM_PATH_SKINNY;
   if (p.path == QMM_PATH_TENSOR) p.tc = plan_tc(M, N, K, device_sms());
-  else p.sk = plan_skinny(M, N, K, bits, group, device_sms());
+  else p.sk = plan_skinny(M, N, K, bits, group, mode, bf16, device_sms());
   return p;
 }
 
@@ -97,13 +100,15 @@ int qmm_path(int M, int N, int K, int bits, int group, int mode) {
   if (M < 0) return QMM_ERR_ARG;
   int st = check_shape(N, K, bits, group, mode);
   if (st != QMM_OK) return st;
-  return choose_path(M, bits);
+  return choose_path(M, bits, mode, false, group);
 }
 
 size_t qmm_workspace_size_for(int M, int N, int K, int bits, int group, int mode, int path) {
   if (M <= 0 || check_shape(N, K, bits, group, mode) != QMM_OK) return 0;
   if (path != QMM_PATH_AUTO && path != QMM_PATH_SKINNY && path != QMM_PATH_TENSOR) return 0;
-  return make_plan(M, N, K, bits, group, path).ws_bytes();
+  // the activation dtype is not an argument here: size for the larger of the two
+  return std::max(make_plan(M, N, K, bits, group, mode, false, path).ws_bytes(),
+                  make_plan(M, N, K, bits, group, mode, true, path).ws_bytes());
 }
 
 size_t qmm_workspace_size(int M, int N, int K, int bits, int group, int mode) {
@@ -134,7 +139,7 @@ int qmm_with_path(const void* x, int xdtype, const void* qweight, const uint16_t
   }
   Problem p{x, xdtype == QMM_BF16, qweight, scales, zeros_or_lut, M, N, K, bits, group, mode, y};
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  Plan plan = make_plan(M, N, K, bits, group, path);
+  Plan plan = make_plan(M, N, K, bits, group, mode, xdtype == QMM_BF16, path);
   if (plan.ws_bytes()) {
     if (!workspace) {
       // no workspace: every CTA owns whole tiles over all of K, no partial sums
@@ -142,7 +147,8 @@ int qmm_with_path(const void* x, int xdtype, const void* qweight, const uint16_t
         plan.tc.ctas = plan.tc.tiles_n * plan.tc.tiles_m;
         plan.tc.ws_bytes = 0;
       } else {
-        plan.sk.splits = plan.sk.tiles_n;
+        plan.sk.warps = plan.sk.tiles_n;
+        plan.sk.splits = (plan.sk.tiles_n + 7) / 8;
         plan.sk.ws_bytes = 0;
       }
     } else if (workspace_bytes < plan.ws_bytes()) {

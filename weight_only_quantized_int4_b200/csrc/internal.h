@@ -23,12 +23,13 @@ struct SkinnyPlan {
   int rows;        // rows per CTA tile (16 * row blocks)
   int tiles_n;     // CTA tiles along N
   int slabs;       // token slabs (ceil(M / (8 nt)))
-  int splits;      // CTAs along K per tile
-  int cps;         // chunks per split
-  size_t ws_bytes; // workspace needed (0 if splits == 1)
+  int splits;      // CTAs per slab
+  int warps;       // stream-K workers (warps) per slab
+  size_t smem;     // dynamic shared memory per CTA
+  size_t ws_bytes; // workspace needed (0 when every CTA owns whole tiles)
 };
 
-SkinnyPlan plan_skinny(int M, int N, int K, int bits, int group, int sms);
+SkinnyPlan plan_skinny(int M, int N, int K, int bits, int group, int mode, bool bf16, int sms);
 cudaError_t launch_skinny(const Problem& p, const SkinnyPlan& plan, void* workspace,
                           cudaStream_t stream);
 
@@ -39,7 +40,7 @@ struct TcPlan {
   size_t ws_bytes;
 };
 
-bool tc_supported(int bits);
+bool tc_supported(int bits, int mode, bool bf16, int group);
 TcPlan plan_tc(int M, int N, int K, int sms);
 cudaError_t launch_tc(const Problem& p, const TcPlan& plan, void* workspace, cudaStream_t stream);
 unsigned tc_read_and_clear_error();

@@ -1,21 +1,26 @@
 // Bandwidth-bound decode path for few tokens (M <= 16 per launch slab).
 //
 // The product here is the quantized-matrix x full-precision-vector product the
-// exllama discussion quotes from the GPTQ paper: "primarily limited by memory
-// bandwidth", with weights de-quantized on the fly and activations left
-// unquantized.  The kernel streams the packed codes exactly once with 128-bit
-// L2-only loads, decodes them in registers (bit tricks for SYM/ASYM, a
-// bank-replicated shared-memory pair table for LUT), and hands the exact
-// small-integer (or table) values to the tensor cores as the A operand of
-// m16n8k16 MMAs with the tokens as the N dimension.  Group scales are applied
-// to the fp32 partial sums after each group, so the MMA sees exact operands.
+// exllama discussion quotes from the GPTQ paper: limited by memory bandwidth,
+// with weights de-quantized when needed and activations left unquantized.
+// The kernel streams the packed codes exactly once, decodes them in registers
+// (bit tricks for SYM/ASYM, a bank-replicated shared-memory pair table for
+// LUT) and hands the exact small-integer (or table) values to the tensor cores
+// as the A operand of m16n8k16 MMAs, the tokens being the N dimension.  Group
+// scales multiply the fp32 partial sums after each group, so the MMA operands
+// are exact.
 //
-// Work split (stream-K): the (row tile, K chunk) units are divided evenly
-// among a grid sized to the resident-CTA capacity of the GPU.  A CTA's warps
-// take interleaved chunks of each tile segment, reduce through shared memory,
-// and either store y (whole tile) or leave an fp32 partial in the workspace;
-// the last CTA to finish a tile adds the partials in a fixed order
-// (deterministic) and stores y.  No CTA ever waits on another.
+// Memory pipeline: every warp owns a ring of kStages shared-memory stages and
+// keeps kStages - 1 chunks in flight with cp.async (codes of R row blocks, the
+// x slice of the chunk, the chunk's scales and zeros), so an SM has tens of KB
+// of HBM reads outstanding without spending registers on them.
+//
+// Work split (stream-K): the (row tile, K chunk) units are divided evenly over
+// a grid of exactly the resident CTAs.  A CTA's warps take interleaved chunks
+// of each tile segment, reduce through shared memory, and either store y
+// (whole tile) or leave an fp32 partial in the workspace; the last CTA to
+// finish a tile adds the partials in CTA order (deterministic) and stores y.
+// No CTA waits for another.
 #include <algorithm>
 
 #include "common.cuh"
@@ -26,8 +31,19 @@ namespace {
 
 constexpr int kWarps = 8;
 constexpr int kThreads = kWarps * 32;
-constexpr int kRB = 2;                  // row blocks (of 16 rows) per tile
 constexpr int kMaxDevices = 64;
+constexpr int kSC = 128;                 // K columns per stage (a "super-chunk"): 8 tiles of 16
+constexpr int kTiles = kSC / 16;
+
+// Row blocks (16 rows) per tile: 2 for one token tile, 4 for two (keeps the
+// x bytes read per code byte at or below one).
+template <int NT>
+constexpr int rb_per_tile() { return NT == 1 ? 2 : 4; }
+
+// Ring depth per warp (stages in flight = depth - 1), sized so that one token
+// tile fits two CTAs per SM and two token tiles one CTA per SM.
+template <int MODE, int NT>
+constexpr int ring_stages() { return (NT == 1 && MODE != kLUT) ? 3 : 2; }
 
 struct SkinnyArgs {
   const uint16_t* x;
@@ -35,9 +51,12 @@ struct SkinnyArgs {
   const uint16_t* scales;
   const uint16_t* zl;
   uint16_t* y;
-  int M, N, K, L, G, nchunks, nrb, tiles;
-  long long units;     // tiles * nchunks
+  int M, N, K, G, nchunks, nrb, tiles, nsc;
+  int lg;              // log2 of the group length; -1 for one group per row
+  int stage_bytes;     // bytes of one ring stage
+  long long units;     // tiles * nsc
   int ctas;            // CTAs per slab
+  int warps;           // stream-K workers per slab (<= 8 ctas)
   float* slots;        // [slabs][2 * ctas][rows * tokens]: a CTA's first / last partial tile
   unsigned* counters;  // [slabs][tiles]
 };
@@ -45,39 +64,208 @@ struct SkinnyArgs {
 template <int MODE>
 constexpr size_t kTabBytes = MODE == kLUT ? 256 * 32 * 4 : 0;
 
-template <int BITS>
-struct Geo {
-  static constexpr int KC = chunk_cols(BITS);
-  static constexpr int TILES = KC / 16;
+// Stage layout of one warp's ring slot: codes [R][CPS][512] | x [TOK][256 B]
+// (16-byte pieces swizzled by row) | scales [R][GPS][32 B] | zeros (ASYM).
+template <int BITS, int MODE, int NT, int TPG>
+struct Stage {
+  static constexpr int R = rb_per_tile<NT>();
+  static constexpr int TOK = 8 * NT;
+  static constexpr int CPS = kSC / chunk_cols(BITS);   // chunks per stage
+  static constexpr int GPS = kTiles / TPG;             // groups per stage
+  static constexpr int X_OFF = R * CPS * 512;
+  static constexpr int S_OFF = X_OFF + TOK * kSC * 2;
+  static constexpr int Z_OFF = S_OFF + R * GPS * 32;
+  static constexpr int BYTES = Z_OFF + (MODE == kASYM ? R * GPS * 32 : 0);
+  static constexpr int XPL = TOK * 16 / 32;           // x pieces per lane
+  static constexpr int SPL = (R * GPS * 2 + 31) / 32; // scale pieces per lane (upper bound)
 };
 
-// CTA index of the stream-K range that holds unit u: ranges start at
-// floor(b * U / C).
+// CTA index of the stream-K range that holds unit u (ranges start at
+// floor(b * U / C)).
 __device__ __forceinline__ int owner_of(long long u, long long U, int C) {
   return (int)(((u + 1) * (long long)C - 1) / U);
 }
 
-template <int BITS, int MODE, bool BF16, int NT>
-__global__ void __launch_bounds__(kThreads, 2) skinny_kernel(const SkinnyArgs a) {
-  constexpr int KC = Geo<BITS>::KC;
-  constexpr int TILES = Geo<BITS>::TILES;
-  constexpr int ROWS = 16 * kRB;
-  constexpr int TOK = 8 * NT;
-  constexpr int NACC = kRB * NT * 4;
+__device__ __forceinline__ void cp_async16(uint32_t saddr, const void* src, bool valid) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(saddr), "l"(src),
+               "r"(valid ? 16 : 0)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+// D = A . B with a zero accumulator (first tile of a group).
+template <bool BF16>
+__device__ __forceinline__ void mma_16816_first(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                                uint32_t b1) {
+  const float z = 0.0f;
+  if constexpr (BF16) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%10,%10,%10,%10};"
+        : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "f"(z));
+  } else {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%10,%10,%10,%10};"
+        : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "f"(z));
+  }
+}
+
+// The CTA's unit range as tiles and super-chunks (computed once, 64-bit).
+struct Range {
+  int tb, sb;   // first tile, its first super-chunk
+  int te, se;   // tile holding the end, super-chunk where it ends (exclusive)
+  __device__ __forceinline__ int s0(int t) const { return t == tb ? sb : 0; }
+  __device__ __forceinline__ int s1(int t, int n) const { return t == te ? se : n; }
+  __device__ __forceinline__ bool has(int t) const { return t < te || (t == te && se > 0); }
+};
+
+// The super-chunks a warp processes, in order: in every tile segment
+// [s0, s1) of the CTA, s0 + w, s0 + w + 8, ...
+struct Seq {
+  int t, s;
+  __device__ __forceinline__ void norm(const Range& r, int n, int w) {
+    while (r.has(t) && s >= r.s1(t, n)) {
+      ++t;
+      s = r.s0(t) + w;
+    }
+  }
+  __device__ __forceinline__ void start(const Range& r, int n, int w) {
+    t = r.tb;
+    s = r.s0(t) + w;
+    norm(r, n, w);
+  }
+  __device__ __forceinline__ void next(const Range& r, int n, int w) {
+    s += kWarps;
+    norm(r, n, w);
+  }
+};
+
+template <int BITS, int MODE, bool BF16, int NT, int TPG>
+__global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1) skinny_kernel(const SkinnyArgs a) {
+  using St = Stage<BITS, MODE, NT, TPG>;
+  constexpr int kStages = ring_stages<MODE, NT>();
+  constexpr int R = St::R;
+  constexpr int TOK = St::TOK;
+  constexpr int NACC = R * NT * 4;        // fp32 values per lane per tile
+  constexpr int CPS = St::CPS;
 
   extern __shared__ __align__(16) unsigned char smem[];
-  __shared__ int s_last;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, t = lane & 3;
   const int slab = blockIdx.y;
   const int m_base = slab * TOK;
-  const int b = blockIdx.x;
-  const long long u_begin = (long long)b * a.units / a.ctas;
-  const long long u_end = (long long)(b + 1) * a.units / a.ctas;
+  const int n = a.nsc;
+  // this warp's stream-K range of (tile, super-chunk) units (64-bit, once)
+  const int gw = blockIdx.x * kWarps + warp;
+  const long long W = a.warps;
+  Range rg;
+  {
+    const long long ub = (long long)gw * a.units / W;
+    const long long ue = (long long)(gw + 1) * a.units / W;
+    rg.tb = (int)(ub / n);
+    rg.sb = (int)(ub - (long long)rg.tb * n);
+    rg.te = (int)(ue / n);
+    rg.se = (int)(ue - (long long)rg.te * n);
+  }
+  const int lg = a.lg;
+
+  unsigned char* tabp = smem;
+  unsigned char* ring = smem + kTabBytes<MODE> + (size_t)warp * kStages * St::BYTES;
+  const uint32_t ring_s = static_cast<uint32_t>(__cvta_generic_to_shared(ring));
+
+  // ---- lane-constant parts of the copies
+  const uint16_t* xsrc[St::XPL];
+  uint32_t xdst[St::XPL];
+  int xcol[St::XPL];
+  bool xrow_ok[St::XPL];
+#pragma unroll
+  for (int i = 0; i < St::XPL; ++i) {
+    const int q = lane + 32 * i, row = q >> 4, p = q & 15;
+    const int m = m_base + row;
+    xrow_ok[i] = m < a.M;
+    xcol[i] = p * 8;
+    xsrc[i] = a.x + (size_t)(xrow_ok[i] ? m : 0) * a.K + p * 8;
+    xdst[i] = St::X_OFF + row * (kSC * 2) + (((p & 8) | ((p ^ row) & 7)) << 4);
+  }
+  // scale / zero pieces: piece q = (r * GPS + k) * 2 + h
+  int sc_r[St::SPL], sc_k[St::SPL];
+  bool sc_on[St::SPL];
+  size_t sc_h8[St::SPL];
+#pragma unroll
+  for (int i = 0; i < St::SPL; ++i) {
+    const int q = lane + 32 * i;
+    sc_on[i] = q < R * St::GPS * 2;
+    sc_h8[i] = (size_t)(q & 1) * 8;
+    sc_k[i] = (q >> 1) % St::GPS;
+    sc_r[i] = (q >> 1) / St::GPS;
+  }
+  const int nsc_full = a.K / kSC;         // super-chunks with no column past K
 
   pdl_wait();                 // inputs of this call may come from the previous grid
   pdl_launch_dependents();    // let the next grid get resident while this one runs
+
+  // ---- prefetch state: per-tile base pointers, refreshed when the tile changes
+  const uint8_t* cbase[R];
+  bool rok[R];
+  const uint16_t* sbase[St::SPL];
+  bool srok[St::SPL];
+  int pf_tile = -1;
+  auto set_tile = [&](int tile) {
+    pf_tile = tile;
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      const int rb = tile * R + r;
+      rok[r] = rb < a.nrb;
+      cbase[r] = a.qw + (rok[r] ? (size_t)rb * a.nchunks * 512 : 0) + lane * 16;
+    }
+#pragma unroll
+    for (int i = 0; i < St::SPL; ++i) {
+      const int rb = tile * R + sc_r[i];
+      srok[i] = sc_on[i] && rb < a.nrb;
+      sbase[i] = a.scales + (srok[i] ? (size_t)rb * a.G * 16 : 0) + sc_h8[i];
+    }
+  };
+  // ---- issue the loads of super-chunk (tile, sc) into ring stage `st`
+  auto issue = [&](int tile, int sc, int st) {
+    if (tile != pf_tile) set_tile(tile);
+    const uint32_t base = ring_s + st * St::BYTES;
+    const bool full = sc < nsc_full;
+#pragma unroll
+    for (int r = 0; r < R; ++r)
+#pragma unroll
+      for (int cc = 0; cc < CPS; ++cc) {
+        const int c = sc * CPS + cc;
+        cp_async16(base + (r * CPS + cc) * 512 + lane * 16, cbase[r] + (size_t)c * 512,
+                   rok[r] && (full || c < a.nchunks));
+      }
+    const int k0 = sc * kSC;
+#pragma unroll
+    for (int i = 0; i < St::XPL; ++i)
+      cp_async16(base + xdst[i], xsrc[i] + k0, xrow_ok[i] && (full || k0 + xcol[i] < a.K));
+    const int gi0 = lg < 0 ? 0 : (k0 >> lg);
+#pragma unroll
+    for (int i = 0; i < St::SPL; ++i) {
+      if (sc_on[i]) {
+        const int gi = gi0 + sc_k[i];
+        const bool ok = srok[i] && gi < a.G;
+        const size_t off = ok ? (size_t)gi * 16 : 0;
+        const int q = lane + 32 * i;
+        cp_async16(base + St::S_OFF + q * 16, sbase[i] + off, ok);
+        if constexpr (MODE == kASYM)
+          cp_async16(base + St::Z_OFF + q * 16, (sbase[i] - a.scales) + a.zl + off, ok);
+      }
+    }
+  };
 
   if constexpr (MODE == kLUT) {
     // Pair table, replicated so that every lane reads its own bank.
@@ -117,96 +305,92 @@ __global__ void __launch_bounds__(kThreads, 2) skinny_kernel(const SkinnyArgs a)
     }
     __syncthreads();
   }
-  const unsigned char* tabp = smem;
-  float* red = reinterpret_cast<float*>(smem + kTabBytes<MODE>);
 
-  // token rows this lane feeds into the B fragments
-  const uint16_t* xrow[NT];
-  bool xok[NT];
+  if (gw >= W) return;   // spare warps of the last CTA (plans with fewer workers)
+  if (rg.tb == rg.te && rg.sb == rg.se) return;   // no units (never planned)
+
+  // ---- prologue: kStages - 1 super-chunks in flight (the warp's own units,
+  // in order: consecutive super-chunks, then the next tile)
+  int pf_t = rg.tb, pf_s = rg.sb;
+  auto pf_valid = [&]() { return pf_t < rg.te || (pf_t == rg.te && pf_s < rg.se); };
+  auto pf_next = [&]() {
+    if (++pf_s == n) {
+      pf_s = 0;
+      ++pf_t;
+    }
+  };
 #pragma unroll
-  for (int nt = 0; nt < NT; ++nt) {
-    const int m = m_base + nt * 8 + g;
-    xok[nt] = m < a.M;
-    xrow[nt] = a.x + (size_t)(xok[nt] ? m : 0) * a.K;
+  for (int s = 0; s < kStages - 1; ++s) {
+    if (pf_valid()) {
+      issue(pf_t, pf_s, s);
+      pf_next();
+    }
+    cp_async_commit();
   }
 
-  long long u = u_begin;
-  while (u < u_end) {
-    const int tile = (int)(u / a.nchunks);
-    const int c0 = (int)(u % a.nchunks);
-    const int c1 = (int)std::min<long long>(a.nchunks, c0 + (u_end - u));
-    const int rb0 = tile * kRB;
+  int st_c = 0;                          // ring stage being computed
+  int st_f = kStages - 1;                // ring stage being filled
+  for (int tile = rg.tb; rg.has(tile); ++tile) {
+    const int s0 = rg.s0(tile), s1 = rg.s1(tile, n);
 
-    float acc[kRB][NT][4];
+    float acc[R][NT][4];
 #pragma unroll
-    for (int r = 0; r < kRB; ++r)
+    for (int r = 0; r < R; ++r)
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
         for (int i = 0; i < 4; ++i) acc[r][nt][i] = 0.0f;
 
-    for (int c = c0 + warp; c < c1; c += kWarps) {
-      // ---- loads: codes of kRB row blocks, x fragments, group scales/zeros
-      uint4 code[kRB];
-#pragma unroll
-      for (int r = 0; r < kRB; ++r) {
-        const int rb = rb0 + r;
-        if (rb < a.nrb)
-          code[r] = ld_stream_u4(a.qw + ((size_t)rb * a.nchunks + c) * 512 + lane * 16);
-        else
-          code[r] = make_uint4(0, 0, 0, 0);
+    for (int sc = s0; sc < s1; ++sc) {
+      // keep the ring full: the stage refilled here was drained last iteration
+      if (pf_valid()) {
+        issue(pf_t, pf_s, st_f);
+        pf_next();
       }
-      uint2 xf[NT][TILES];
-#pragma unroll
-      for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-        for (int j = 0; j < TILES; ++j)
-          xf[nt][j] = xok[nt] ? ld_u2(xrow[nt] + c * KC + 16 * j + 4 * t) : make_uint2(0, 0);
+      cp_async_commit();
+      cp_async_wait<kStages - 1>();
+      __syncwarp();
 
-      float gacc[kRB][NT][4];
-#pragma unroll
-      for (int r = 0; r < kRB; ++r)
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-          for (int i = 0; i < 4; ++i) gacc[r][nt][i] = 0.0f;
-
-      uint32_t zw[kRB];   // ASYM zero words (z_g, z_g8) of the current group
-      int cur_gi = -1;
+      const unsigned char* st = ring + st_c * St::BYTES;
+      float gacc[R][NT][4];
+      uint4 cw[R];
 
 #pragma unroll
-      for (int j = 0; j < TILES; ++j) {
-        const int k_tile = c * KC + 16 * j;
-        const int gi = k_tile / a.L;
-        if constexpr (MODE == kASYM) {
-          if (gi != cur_gi) {
+      for (int j = 0; j < kTiles; ++j) {
+        uint2 xf[NT];
 #pragma unroll
-            for (int r = 0; r < kRB; ++r) {
-              const int rb = rb0 + r;
-              zw[r] = rb < a.nrb ? *reinterpret_cast<const uint32_t*>(
-                                       a.zl + ((size_t)rb * a.G + gi) * 16 + 2 * g)
-                                 : 0u;
-              if constexpr (BF16) {
-                const __half2 zh = *reinterpret_cast<const __half2*>(&zw[r]);
-                const float2 zf = __half22float2(zh);
-                zw[r] = pack2<true>(zf.x, zf.y);
-              }
-            }
-          }
+        for (int nt = 0; nt < NT; ++nt) {
+          const int row = g + 8 * nt;
+          const int p = 2 * j + (t >> 1);
+          const int phys = (p & 8) | ((p ^ g) & 7);
+          xf[nt] = *reinterpret_cast<const uint2*>(st + St::X_OFF + row * (kSC * 2) + phys * 16 +
+                                                   8 * (t & 1));
         }
-        cur_gi = gi;
+        const int grp = j / TPG;            // group within the stage (compile-time)
+        // the lane's 16 code bytes of chunk j / 4 (4-bit) or of the stage (2-bit)
+        if ((BITS == 4 && (j & 3) == 0) || j == 0) {
 #pragma unroll
-        for (int r = 0; r < kRB; ++r) {
+          for (int r = 0; r < R; ++r)
+            cw[r] = *reinterpret_cast<const uint4*>(st + (r * CPS + (BITS == 4 ? (j >> 2) : 0)) * 512 +
+                                                    lane * 16);
+        }
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
           uint32_t af[4], aflo[4];
           if constexpr (BITS == 4) {
-            const uint32_t w = (&code[r].x)[j];
+            // tile j: chunk j / 4 of the stage, word j % 4 of the lane
+            const uint32_t w = (&cw[r].x)[j & 3];
             if constexpr (MODE == kSYM) {
               decode_int4<BF16, 8>(w, af);
             } else if constexpr (MODE == kASYM) {
               decode_int4<BF16, 0>(w, af);
-              const uint32_t zlo = __byte_perm(zw[r], 0, 0x1010);   // (z_g, z_g)
-              const uint32_t zhi = __byte_perm(zw[r], 0, 0x3232);   // (z_g8, z_g8)
-              sub_zero<BF16>(zlo, zhi, af);
+              uint32_t zw = *reinterpret_cast<const uint32_t*>(st + St::Z_OFF +
+                                                               (r * St::GPS + grp) * 32 + 4 * g);
+              if constexpr (BF16) {
+                const float2 zf = __half22float2(*reinterpret_cast<const __half2*>(&zw));
+                zw = pack2<true>(zf.x, zf.y);
+              }
+              sub_zero<BF16>(__byte_perm(zw, 0, 0x1010), __byte_perm(zw, 0, 0x3232), af);
             } else if constexpr (!BF16) {
               const uint32_t l4 = (uint32_t)lane << 2;
               af[0] = *reinterpret_cast<const uint32_t*>(tabp + lop3_and_or(w << 7, 0x7F80u, l4));
@@ -224,215 +408,229 @@ __global__ void __launch_bounds__(kThreads, 2) skinny_kernel(const SkinnyArgs a)
               aflo[0] = e0.y; aflo[1] = e1.y; aflo[2] = e2.y; aflo[3] = e3.y;
             }
           } else {
-            // 2-bit LUT: word j/2, bytes 2 (j % 2) and 2 (j % 2) + 1
-            const uint32_t w = (&code[r].x)[j >> 1];
+            // 2-bit LUT: word j/2 of the lane, bytes 2 (j % 2) and 2 (j % 2) + 1
+            const uint32_t w = (&cw[r].x)[j >> 1];
             const int sh = 16 * (j & 1);
-            const uint32_t s0 = sh >= 7 ? (w >> (sh - 7)) : (w << 7);
-            const uint32_t s1 = w >> (sh + 1);
+            const uint32_t s0w = sh >= 7 ? (w >> (sh - 7)) : (w << 7);
+            const uint32_t s1w = w >> (sh + 1);
             if constexpr (!BF16) {
               const uint32_t l8 = (uint32_t)(lane & 15) << 3;
-              const uint2 e0 = *reinterpret_cast<const uint2*>(tabp + lop3_and_or(s0, 0x7F80u, l8));
-              const uint2 e1 = *reinterpret_cast<const uint2*>(tabp + lop3_and_or(s1, 0x7F80u, l8));
+              const uint2 e0 = *reinterpret_cast<const uint2*>(tabp + lop3_and_or(s0w, 0x7F80u, l8));
+              const uint2 e1 = *reinterpret_cast<const uint2*>(tabp + lop3_and_or(s1w, 0x7F80u, l8));
               af[0] = e0.x; af[1] = e0.y; af[2] = e1.x; af[3] = e1.y;
             } else {
               // (hi hi, lo lo) per byte: 16-byte entries, 8 copies
               const uint32_t l16 = (uint32_t)(lane & 7) << 4;
-              const uint4 e0 = *reinterpret_cast<const uint4*>(tabp + lop3_and_or(s0, 0x7F80u, l16));
-              const uint4 e1 = *reinterpret_cast<const uint4*>(tabp + lop3_and_or(s1, 0x7F80u, l16));
+              const uint4 e0 = *reinterpret_cast<const uint4*>(tabp + lop3_and_or(s0w, 0x7F80u, l16));
+              const uint4 e1 = *reinterpret_cast<const uint4*>(tabp + lop3_and_or(s1w, 0x7F80u, l16));
               af[0] = e0.x; af[1] = e0.y; af[2] = e1.x; af[3] = e1.y;
               aflo[0] = e0.z; aflo[1] = e0.w; aflo[2] = e1.z; aflo[3] = e1.w;
             }
           }
 #pragma unroll
           for (int nt = 0; nt < NT; ++nt) {
-            mma_16816<BF16>(gacc[r][nt], af, xf[nt][j].x, xf[nt][j].y);
-            if constexpr (MODE == kLUT && BF16)
-              mma_16816<BF16>(gacc[r][nt], aflo, xf[nt][j].x, xf[nt][j].y);
+            if (j % TPG == 0)
+              mma_16816_first<BF16>(gacc[r][nt], af, xf[nt].x, xf[nt].y);
+            else
+              mma_16816<BF16>(gacc[r][nt], af, xf[nt].x, xf[nt].y);
+            if constexpr (MODE == kLUT && BF16) mma_16816<BF16>(gacc[r][nt], aflo, xf[nt].x, xf[nt].y);
           }
         }
-        // group ends after this tile (or the chunk ends): apply the scales
-        if (j == TILES - 1 || ((k_tile + 16) % a.L) == 0) {
+        // the group ends after this tile (position fixed at compile time):
+        // fold the group's sums into acc with its scales
+        if ((j + 1) % TPG == 0) {
 #pragma unroll
-          for (int r = 0; r < kRB; ++r) {
-            const int rb = rb0 + r;
-            float2 s = make_float2(0.0f, 0.0f);
-            if (rb < a.nrb) {
-              const uint32_t sw = *reinterpret_cast<const uint32_t*>(
-                  a.scales + ((size_t)rb * a.G + gi) * 16 + 2 * g);
-              s = __half22float2(*reinterpret_cast<const __half2*>(&sw));
-            }
+          for (int r = 0; r < R; ++r) {
+            const uint32_t sw = *reinterpret_cast<const uint32_t*>(st + St::S_OFF +
+                                                                   (r * St::GPS + grp) * 32 + 4 * g);
+            const float2 s = __half22float2(*reinterpret_cast<const __half2*>(&sw));
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) {
               acc[r][nt][0] = fmaf(s.x, gacc[r][nt][0], acc[r][nt][0]);
               acc[r][nt][1] = fmaf(s.x, gacc[r][nt][1], acc[r][nt][1]);
               acc[r][nt][2] = fmaf(s.y, gacc[r][nt][2], acc[r][nt][2]);
               acc[r][nt][3] = fmaf(s.y, gacc[r][nt][3], acc[r][nt][3]);
-#pragma unroll
-              for (int i = 0; i < 4; ++i) gacc[r][nt][i] = 0.0f;
             }
           }
         }
       }
+      __syncwarp();   // every lane is done with this stage before it is refilled
+      st_c = st_c + 1 == kStages ? 0 : st_c + 1;
+      st_f = st_f + 1 == kStages ? 0 : st_f + 1;
     }
 
-    // ---- CTA reduction over the warps: red[warp][e][lane]
-    __syncthreads();   // table reads (LUT) / previous segment's reads are done
+    // ---- this warp's result for the tile segment: store y (whole tile) or
+    // hand a partial to the last warp that finishes the tile
+    const bool whole = s0 == 0 && s1 == n;
+    float* outv = &acc[0][0][0];
+    if (!whole) {
+      const long long t_first = (long long)tile * n;
+      const int first = owner_of(t_first, a.units, (int)W);
+      const int nb = owner_of(t_first + n - 1, a.units, (int)W) - first + 1;
+      const int first_e = ((long long)first * a.units / W < t_first) ? 1 : 0;
+      // slot 2 gw + e, e = 1 when the tile is not the warp's first; of the
+      // contributors only `first` can have e = 1
+      const int e = (tile == rg.tb) ? 0 : 1;
+      float* slots = a.slots + (size_t)slab * 2 * W * (NACC * 32);
+      float4* mine = reinterpret_cast<float4*>(slots + (size_t)(2 * gw + e) * (NACC * 32) + lane * NACC);
 #pragma unroll
-    for (int r = 0; r < kRB; ++r)
+      for (int i = 0; i < NACC / 4; ++i)
+        mine[i] = make_float4(outv[4 * i], outv[4 * i + 1], outv[4 * i + 2], outv[4 * i + 3]);
+      __threadfence();
+      __syncwarp();
+      unsigned* counter = a.counters + (size_t)slab * a.tiles + tile;
+      unsigned prev = 0;
+      if (lane == 0) prev = atomicAdd(counter, 1u);
+      prev = __shfl_sync(0xffffffffu, prev, 0);
+      if (prev != (unsigned)(nb - 1)) continue;     // not the last: the tile is someone's
+      __threadfence();
+      // last warp: add the contributions in order (deterministic)
+#pragma unroll
+      for (int i = 0; i < NACC; ++i) outv[i] = 0.0f;
+      for (int k = 0; k < nb; ++k) {
+        const float4* src = reinterpret_cast<const float4*>(
+            slots + (size_t)(2 * (first + k) + (k == 0 ? first_e : 0)) * (NACC * 32) + lane * NACC);
+#pragma unroll
+        for (int i = 0; i < NACC / 4; ++i) {
+          const float4 v = __ldcg(src + i);
+          outv[4 * i] += v.x;
+          outv[4 * i + 1] += v.y;
+          outv[4 * i + 2] += v.z;
+          outv[4 * i + 3] += v.w;
+        }
+      }
+      if (lane == 0) *counter = 0u;   // ready for the next call
+    }
+    // fragment (r, nt, i) of this lane: row (tile R + r) 16 + g + 8 (i / 2),
+    // token m_base + 8 nt + 2 t + (i % 2)
+#pragma unroll
+    for (int r = 0; r < R; ++r)
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
-          red[(warp * NACC + (r * NT + nt) * 4 + i) * 32 + lane] = acc[r][nt][i];
-    __syncthreads();
-
-    const long long t_first = (long long)tile * a.nchunks;
-    const bool whole = (u == t_first) && (c1 == a.nchunks);
-    float* slot = nullptr;
-    unsigned* counter = a.counters ? a.counters + (size_t)slab * a.tiles + tile : nullptr;
-    int nb = 1, first = 0;
-    if (!whole) {
-      first = owner_of(t_first, a.units, a.ctas);
-      nb = owner_of(t_first + a.nchunks - 1, a.units, a.ctas) - first + 1;
-      const int e = (tile == (int)(u_begin / a.nchunks)) ? 0 : 1;
-      slot = a.slots + ((size_t)slab * 2 * a.ctas + 2 * b + e) * (ROWS * TOK);
-    }
-    // element e = tok_l * ROWS + row_l: rows fastest, so y stores coalesce
-    for (int e = threadIdx.x; e < ROWS * TOK; e += kThreads) {
-      const int row_l = e % ROWS, tok_l = e / ROWS;
-      const int r = row_l >> 4, rr = row_l & 15;
-      const int nt = tok_l >> 3, tt = tok_l & 7;
-      const int src_lane = 4 * (rr & 7) + (tt >> 1);
-      const int i = 2 * (rr >> 3) + (tt & 1);
-      float v = 0.0f;
-#pragma unroll
-      for (int w = 0; w < kWarps; ++w) v += red[(w * NACC + (r * NT + nt) * 4 + i) * 32 + src_lane];
-      const int row = tile * ROWS + row_l, m = m_base + tok_l;
-      if (whole) {
-        if (row < a.N && m < a.M) {
-          if constexpr (BF16)
-            a.y[(size_t)m * a.N + row] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
-          else
-            a.y[(size_t)m * a.N + row] = __half_as_ushort(__float2half_rn(v));
-        }
-      } else {
-        slot[e] = v;
-      }
-    }
-    if (!whole) {
-      __threadfence();
-      __syncthreads();
-      if (threadIdx.x == 0) s_last = (atomicAdd(counter, 1u) == (unsigned)(nb - 1));
-      __syncthreads();
-      if (s_last) {
-        __threadfence();
-        const float* base = a.slots + (size_t)slab * 2 * a.ctas * (ROWS * TOK);
-        for (int e = threadIdx.x; e < ROWS * TOK; e += kThreads) {
-          float v = 0.0f;
-          for (int k = 0; k < nb; ++k) {
-            const int bb = first + k;
-            const int ee = ((long long)bb * a.units / a.ctas < t_first) ? 1 : 0;
-            v += __ldcg(base + (size_t)(2 * bb + ee) * (ROWS * TOK) + e);
-          }
-          const int row = tile * ROWS + e % ROWS, m = m_base + e / ROWS;
+        for (int i = 0; i < 4; ++i) {
+          const int row = (tile * R + r) * 16 + g + 8 * (i >> 1);
+          const int m = m_base + 8 * nt + 2 * t + (i & 1);
           if (row < a.N && m < a.M) {
+            const float v = acc[r][nt][i];
             if constexpr (BF16)
               a.y[(size_t)m * a.N + row] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
             else
               a.y[(size_t)m * a.N + row] = __half_as_ushort(__float2half_rn(v));
           }
         }
-        if (threadIdx.x == 0) *counter = 0u;   // ready for the next call
-      }
-    }
-    __syncthreads();   // red / s_last reused by the next segment
-    u += c1 - c0;
   }
+  cp_async_wait<0>();   // nothing may still land in shared memory after exit
 }
 
-template <int BITS, int MODE, bool BF16, int NT>
+template <int BITS, int MODE, int NT, int TPG>
 constexpr size_t smem_bytes() {
-  // pair table (LUT) followed by the cross-warp reduction buffer
-  return kTabBytes<MODE> + (size_t)kWarps * kRB * NT * 4 * 32 * sizeof(float);
+  using St = Stage<BITS, MODE, NT, TPG>;
+  return kTabBytes<MODE> + (size_t)kWarps * ring_stages<MODE, NT>() * St::BYTES;
 }
 
-// Resident CTAs per SM of one instantiation; also opts the kernel into its
-// dynamic shared memory size.  Cached per device.
-template <int BITS, int MODE, bool BF16, int NT>
+// Opts the kernel into `smem` bytes of dynamic shared memory (once per device)
+// and returns its resident CTAs per SM, or 0 if the size cannot be granted.
+template <int BITS, int MODE, bool BF16, int NT, int TPG>
 int occupancy() {
   static int occ[kMaxDevices] = {};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 0 || dev >= kMaxDevices) dev = 0;
-  if (!occ[dev]) {
-    auto k = skinny_kernel<BITS, MODE, BF16, NT>;
-    int o = 0;
-    cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         (int)smem_bytes<BITS, MODE, BF16, NT>());
-    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&o, k, kThreads,
-                                                  smem_bytes<BITS, MODE, BF16, NT>());
-    occ[dev] = o < 1 ? 1 : o;
+  if (occ[dev]) return occ[dev];
+  auto k = skinny_kernel<BITS, MODE, BF16, NT, TPG>;
+  constexpr size_t smem = smem_bytes<BITS, MODE, NT, TPG>();
+  if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+      cudaSuccess) {
+    cudaGetLastError();   // do not leave the failure behind as a sticky error
+    return 0;
   }
-  return occ[dev];
+  int o = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&o, k, kThreads, smem) != cudaSuccess) {
+    cudaGetLastError();
+    return 0;
+  }
+  occ[dev] = o;
+  return o;
 }
 
-template <int BITS, int MODE, bool BF16, int NT>
+template <int BITS, int MODE, bool BF16, int NT, int TPG>
 cudaError_t launch(const SkinnyArgs& args, int slabs, cudaStream_t stream) {
-  auto k = skinny_kernel<BITS, MODE, BF16, NT>;
-  occupancy<BITS, MODE, BF16, NT>();   // sets the shared-memory attribute once
+  auto k = skinny_kernel<BITS, MODE, BF16, NT, TPG>;
+  if (occupancy<BITS, MODE, BF16, NT, TPG>() < 1) return cudaErrorInvalidConfiguration;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(args.ctas, slabs, 1);
   cfg.blockDim = dim3(kThreads, 1, 1);
-  cfg.dynamicSmemBytes = smem_bytes<BITS, MODE, BF16, NT>();
+  cfg.dynamicSmemBytes = smem_bytes<BITS, MODE, NT, TPG>();
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, k, args);
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, k, args);
+  if (e != cudaSuccess) cudaGetLastError();   // report it once, here
+  return e;
 }
 
-template <int BITS, int MODE, bool BF16>
-cudaError_t launch_nt(const SkinnyArgs& args, int nt, int slabs, cudaStream_t s) {
-  return nt == 1 ? launch<BITS, MODE, BF16, 1>(args, slabs, s)
-                 : launch<BITS, MODE, BF16, 2>(args, slabs, s);
+// Calls f.template operator()<BITS, MODE, BF16, NT, TPG>() for the runtime values.
+template <int B, int MO, bool BF, int T, class F>
+auto dispatch_tpg(int tpg, F&& f) {
+  switch (tpg) {
+    case 1: return f.template operator()<B, MO, BF, T, 1>();
+    case 2: return f.template operator()<B, MO, BF, T, 2>();
+    case 4: return f.template operator()<B, MO, BF, T, 4>();
+    default: return f.template operator()<B, MO, BF, T, 8>();
+  }
 }
 
-int occupancy_for(int bits, int mode, bool bf16, int nt) {
-#define QMM_OCC(B, MO, BF)                                                   \
-  if (bits == B && mode == MO && bf16 == BF)                                 \
-    return nt == 1 ? occupancy<B, MO, BF, 1>() : occupancy<B, MO, BF, 2>();
-  QMM_OCC(4, kSYM, false) QMM_OCC(4, kSYM, true) QMM_OCC(4, kASYM, false)
-  QMM_OCC(4, kASYM, true) QMM_OCC(4, kLUT, false) QMM_OCC(4, kLUT, true)
-  QMM_OCC(2, kLUT, false) QMM_OCC(2, kLUT, true)
-#undef QMM_OCC
-  return 1;
+template <class F>
+auto dispatch(int bits, int mode, bool bf16, int nt, int tpg, F&& f) {
+#define QMM_CASE(B, MO, BF, T) \
+  if (bits == B && mode == MO && bf16 == BF && nt == T) return dispatch_tpg<B, MO, BF, T>(tpg, f);
+  QMM_CASE(4, kSYM, false, 1) QMM_CASE(4, kSYM, false, 2) QMM_CASE(4, kSYM, true, 1)
+  QMM_CASE(4, kSYM, true, 2) QMM_CASE(4, kASYM, false, 1) QMM_CASE(4, kASYM, false, 2)
+  QMM_CASE(4, kASYM, true, 1) QMM_CASE(4, kASYM, true, 2) QMM_CASE(4, kLUT, false, 1)
+  QMM_CASE(4, kLUT, false, 2) QMM_CASE(4, kLUT, true, 1) QMM_CASE(4, kLUT, true, 2)
+  QMM_CASE(2, kLUT, false, 1) QMM_CASE(2, kLUT, false, 2) QMM_CASE(2, kLUT, true, 1)
+  QMM_CASE(2, kLUT, true, 2)
+#undef QMM_CASE
+  return dispatch_tpg<4, kSYM, false, 1>(tpg, f);
 }
+
+// Tiles (of 16 columns) per group inside a 128-column stage: 8 for groups of
+// 128 columns or more (and for one group per row), else group / 16.
+int tiles_per_group(int group) { return (group == -1 || group >= kSC) ? 8 : group / 16; }
 
 }  // namespace
 
-SkinnyPlan plan_skinny(int M, int N, int K, int bits, int group, int sms) {
-  (void)group;
+SkinnyPlan plan_skinny(int M, int N, int K, int bits, int group, int mode, bool bf16, int sms) {
   SkinnyPlan p{};
   p.nt = M <= 8 ? 1 : 2;
-  p.rows = 16 * kRB;
+  const int R = p.nt == 1 ? 2 : 4;
+  p.rows = 16 * R;
   const int nrb = N / 16;
-  p.tiles_n = (nrb + kRB - 1) / kRB;
+  p.tiles_n = (nrb + R - 1) / R;
   p.slabs = std::max(1, (M + 8 * p.nt - 1) / (8 * p.nt));
-  const int nchunks = K / chunk_cols(bits);
-  const long long units = (long long)p.tiles_n * nchunks;
-  // one resident wave; the occupancy does not depend on mode/dtype enough to
-  // matter for sizing, so the SYM fp16 kernel's figure is used
-  const int occ = occupancy_for(bits, bits == 4 ? kSYM : kLUT, false, p.nt);
-  long long ctas = (long long)sms * occ;
-  if (ctas > units) ctas = units;
-  p.splits = (int)ctas;   // CTAs per slab (stream-K)
-  p.cps = (int)((units + ctas - 1) / ctas);
-  const bool split = (units % ctas) != 0 || (units / ctas) != nchunks;
+  const int nsc = (K + kSC - 1) / kSC;
+  const long long units = (long long)p.tiles_n * nsc;
+  const int tpg = tiles_per_group(group);
+  p.smem = dispatch(bits, mode, bf16, p.nt, tpg, [&]<int B, int MO, bool BF, int T, int TP>() {
+    return smem_bytes<B, MO, T, TP>();
+  });
+  const int occ = dispatch(bits, mode, bf16, p.nt, tpg, [&]<int B, int MO, bool BF, int T, int TP>() {
+    return occupancy<B, MO, BF, T, TP>();
+  });
+  // one resident wave of CTAs; every warp is a stream-K worker with >= 1 unit
+  long long warps = (long long)sms * (occ > 0 ? occ : 1) * kWarps;
+  if (warps > units) warps = units;
+  const long long ctas = (warps + kWarps - 1) / kWarps;
+  p.splits = (int)ctas;
+  p.warps = (int)warps;
+  const bool split = !(units % warps == 0 && (units / warps) % nsc == 0);
   if (split) {
     const size_t counters = ((size_t)p.slabs * p.tiles_n * sizeof(unsigned) + 255) / 256 * 256;
-    const size_t slots = (size_t)p.slabs * 2 * ctas * p.rows * 8 * p.nt * sizeof(float);
+    const size_t slots = (size_t)p.slabs * 2 * warps * p.rows * 8 * p.nt * sizeof(float);
     p.ws_bytes = counters + slots;
   } else {
     p.ws_bytes = 0;
@@ -451,32 +649,26 @@ cudaError_t launch_skinny(const Problem& pr, const SkinnyPlan& plan, void* works
   a.M = pr.M;
   a.N = pr.N;
   a.K = pr.K;
-  a.L = pr.group == -1 ? pr.K : pr.group;
-  a.G = pr.K / a.L;
+  const int L = pr.group == -1 ? pr.K : pr.group;
+  a.G = pr.K / L;
+  a.lg = pr.group == -1 ? -1 : __builtin_ctz((unsigned)pr.group);
   a.nchunks = pr.K / chunk_cols(pr.bits);
+  a.nsc = (pr.K + kSC - 1) / kSC;
   a.nrb = pr.N / 16;
   a.tiles = plan.tiles_n;
-  a.units = (long long)plan.tiles_n * a.nchunks;
+  a.units = (long long)plan.tiles_n * a.nsc;
   a.ctas = plan.splits;
+  a.warps = plan.warps;
   if (plan.ws_bytes) {
     const size_t counters = ((size_t)plan.slabs * plan.tiles_n * sizeof(unsigned) + 255) / 256 * 256;
     a.counters = reinterpret_cast<unsigned*>(workspace);
     a.slots = reinterpret_cast<float*>(reinterpret_cast<char*>(workspace) + counters);
   }
-  const bool bf = pr.bf16;
-  if (pr.bits == 4 && pr.mode == kSYM)
-    return bf ? launch_nt<4, kSYM, true>(a, plan.nt, plan.slabs, stream)
-              : launch_nt<4, kSYM, false>(a, plan.nt, plan.slabs, stream);
-  if (pr.bits == 4 && pr.mode == kASYM)
-    return bf ? launch_nt<4, kASYM, true>(a, plan.nt, plan.slabs, stream)
-              : launch_nt<4, kASYM, false>(a, plan.nt, plan.slabs, stream);
-  if (pr.bits == 4 && pr.mode == kLUT)
-    return bf ? launch_nt<4, kLUT, true>(a, plan.nt, plan.slabs, stream)
-              : launch_nt<4, kLUT, false>(a, plan.nt, plan.slabs, stream);
-  if (pr.bits == 2 && pr.mode == kLUT)
-    return bf ? launch_nt<2, kLUT, true>(a, plan.nt, plan.slabs, stream)
-              : launch_nt<2, kLUT, false>(a, plan.nt, plan.slabs, stream);
-  return cudaErrorInvalidValue;
+  return dispatch(pr.bits, pr.mode, pr.bf16, plan.nt, tiles_per_group(pr.group),
+                  [&]<int B, int MO, bool BF, int T, int TP>() {
+                    a.stage_bytes = Stage<B, MO, T, TP>::BYTES;
+                    return launch<B, MO, BF, T, TP>(a, plan.slabs, stream);
+                  });
 }
 
 }  // namespace qk

@@ -562,7 +562,10 @@ cudaError_t launch_tc_t(const CUtensorMap& mx, const CUtensorMap& mw, const TcAr
   cudaGetDevice(&dev);
   if (dev >= 0 && dev < 64 && !attr_set[dev]) {
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
+    if (e != cudaSuccess) {
+      cudaGetLastError();
+      return e;
+    }
     attr_set[dev] = true;
   }
   cudaLaunchConfig_t cfg = {};
@@ -575,7 +578,9 @@ cudaError_t launch_tc_t(const CUtensorMap& mx, const CUtensorMap& mw, const TcAr
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, k, mx, mw, args);
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, k, mx, mw, args);
+  if (e != cudaSuccess) cudaGetLastError();   // report it once, here
+  return e;
 }
 
 template <int MODE, bool BF16, bool GM1>
@@ -597,7 +602,17 @@ cudaError_t launch_mode(bool bf16, bool gm1, int bn, const CUtensorMap& mx, cons
 
 }  // namespace
 
-bool tc_supported(int bits) { return bits == 4; }
+// Combinations the tensor path computes within tolerance: 4-bit codes with
+// fp16 activations (the operand is fp16((q - z) s) or fp16(T s), one rounding
+// of 2^-11), or with bf16 activations when the scale is per row (the operand
+// is the exact integer q - z and the scale multiplies the fp32 result).  Group
+// scales with bf16 would round every weight to 8 bits, which together with the
+// bf16 output exceeds the error budget; those run on the decode path.
+bool tc_supported(int bits, int mode, bool bf16, int group) {
+  if (bits != 4) return false;
+  if (!bf16) return true;
+  return group == -1 && mode != kLUT;
+}
 
 TcPlan plan_tc(int M, int N, int K, int sms) {
   TcPlan p{};
