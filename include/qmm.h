@@ -72,7 +72,8 @@ typedef enum {
   QMM_ERR_ALIGN = -3,        /* pointer not aligned as documented                */
   QMM_ERR_CUDA = -4,         /* a CUDA runtime call failed                       */
   QMM_ERR_TIMEOUT = -5,      /* a kernel gave up a bounded wait (qmm_check_error) */
-  QMM_ERR_WORKSPACE = -6     /* workspace smaller than qmm_workspace_size        */
+  QMM_ERR_WORKSPACE = -6,    /* workspace smaller than qmm_workspace_size        */
+  QMM_ERR_TOO_LARGE = -7     /* qmm_noalloc: problem exceeds the static scratch  */
 } qmm_status;
 
 /* Paths for qmm_with_path. */
@@ -145,6 +146,35 @@ int qmm_with_path(const void* x, int xdtype, const void* qweight, const uint16_t
 /* The path qmm picks for this problem with fp16 activations (QMM_PATH_SKINNY
  * or QMM_PATH_TENSOR), or a negative qmm_status for an unsupported problem. */
 int qmm_path(int M, int N, int K, int bits, int group, int mode);
+
+/* qmm for callers that cannot allocate device memory.  (This entry point is
+ * an addition of this library; the sources describe no counterpart.)
+ *
+ * Some callers cannot call cudaMalloc: code that records work into a CUDA
+ * graph under stream capture (allocation is not a capturable operation), or an
+ * engine whose device memory is planned once at start-up and may not grow.
+ * qmm needs a caller-provided workspace for its split-K partial sums; this
+ * variant runs the same decode-path kernel on a scratch buffer the library
+ * owns instead: a static device array of 8 MiB that every GPU which loads
+ * the library holds until the process exits.  No call allocates: nothing here
+ * calls cudaMalloc, cudaFree or an allocating library routine.
+ *
+ * Arguments are those of qmm without the workspace.  M must be at most 16
+ * (one token slab of the decode path) and the problem's arrival counters must
+ * fit the buffer; otherwise the call returns QMM_ERR_TOO_LARGE without
+ * launching.  When the partial-sum slots of the usual plan do not fit, the
+ * call uses fewer stream-K workers (slower, same result within rounding).
+ *
+ * The first call on a device looks up the buffer's device address
+ * (cudaGetSymbolAddress, once per device, with that device current); make
+ * that first call outside any stream capture.  Every call clears the buffer's
+ * arrival counters (cudaMemsetAsync on `stream`) and then reuses the buffer,
+ * which keeps the previous call's partial sums.  All calls share the one
+ * buffer: calls that can run at the same time on the GPU (different streams
+ * without ordering between them) race and may return wrong results. */
+int qmm_noalloc(const void* x, int xdtype, const void* qweight, const uint16_t* scales,
+                const uint16_t* zeros_or_lut, int M, int N, int K, int bits, int group, int mode,
+                void* y, void* stream);
 
 /* Decode the packed weights into W_out[N, K] row-major (fp16 or bf16 by
  * out_dtype): W_out = round_to_nearest_even((q - z) * s) (SYM z = 8) or

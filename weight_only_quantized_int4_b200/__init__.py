@@ -28,7 +28,7 @@ PATH_NAMES = {1: "skinny", 2: "tensor"}
 
 SYMBOLS = ("qmm_packed_size", "qmm_pack", "qmm_workspace_size", "qmm_workspace_size_for", "qmm",
            "qmm_with_path",
-           "qmm_path", "qmm_dequant", "qmm_check_error", "qmm_strerror")
+           "qmm_path", "qmm_dequant", "qmm_check_error", "qmm_strerror", "qmm_noalloc")
 
 _lib = None
 _lock = threading.Lock()
@@ -60,6 +60,7 @@ def load(path: str = LIB_PATH):
             lib.qmm.argtypes = [P, I, P, P, P, I, I, I, I, I, I, P, P, S, P]
             lib.qmm_with_path.argtypes = [P, I, P, P, P, I, I, I, I, I, I, P, P, S, P, I]
             lib.qmm_path.argtypes = [I, I, I, I, I, I]
+            lib.qmm_noalloc.argtypes = [P, I, P, P, P, I, I, I, I, I, I, P, P]
             lib.qmm_dequant.argtypes = [P, P, P, I, I, I, I, I, I, P, P]
             lib.qmm_check_error.argtypes = [P]
             lib.qmm_strerror.argtypes = [I]
@@ -149,6 +150,21 @@ def qmm(x, qweight, scales, zeros_or_lut, N, K, mode, bits=4, group=128, y=None,
     _check(load().qmm_with_path(_ptr(x), DTYPES[x.dtype], _ptr(qweight), _ptr(scales),
                                 _ptr(zeros_or_lut), M, N, K, bits, group, MODES[mode], _ptr(y),
                                 _ptr(ws), nbytes, _stream(), PATHS[path]), "qmm")
+    return y
+
+
+def qmm_noalloc(x, qweight, scales, zeros_or_lut, N, K, mode, bits=4, group=128, y=None):
+    """y = x . dequant(qweight)^T with the library's static scratch buffer
+    (no workspace, no allocation by the library); M <= 16."""
+    _dev(x, "x")
+    if x.dtype not in DTYPES:
+        raise ValueError("x must be fp16 or bf16")
+    M = x.shape[0]
+    if y is None:
+        y = torch.empty(M, N, dtype=x.dtype, device=x.device)
+    _check(load().qmm_noalloc(_ptr(x), DTYPES[x.dtype], _ptr(qweight), _ptr(scales),
+                              _ptr(zeros_or_lut), M, N, K, bits, group, MODES[mode], _ptr(y),
+                              _stream()), "qmm_noalloc")
     return y
 
 

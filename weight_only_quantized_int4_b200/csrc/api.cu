@@ -166,6 +166,34 @@ int qmm(const void* x, int xdtype, const void* qweight, const uint16_t* scales,
                        workspace, workspace_bytes, stream, QMM_PATH_AUTO);
 }
 
+int qmm_noalloc(const void* x, int xdtype, const void* qweight, const uint16_t* scales,
+                const uint16_t* zeros_or_lut, int M, int N, int K, int bits, int group, int mode,
+                void* y, void* stream) {
+  if (M < 0) return QMM_ERR_ARG;
+  int st = check_shape(N, K, bits, group, mode);
+  if (st != QMM_OK) return st;
+  if (xdtype != QMM_F16 && xdtype != QMM_BF16) return QMM_ERR_ARG;
+  if (M > 16) return QMM_ERR_TOO_LARGE;
+  if (M == 0) return QMM_OK;
+  if (!x || !qweight || !scales || !y) return QMM_ERR_ARG;
+  if (mode != QMM_SYM && !zeros_or_lut) return QMM_ERR_ARG;
+  if (!aligned(x, 16) || !aligned(qweight, 16) || !aligned(scales, 4) || !aligned(y, 2) ||
+      (mode == QMM_ASYM && !aligned(zeros_or_lut, 4)))
+    return QMM_ERR_ALIGN;
+  {
+    const char* xb = static_cast<const char*>(x);
+    const char* yb = static_cast<const char*>(y);
+    const size_t xs = (size_t)M * K * 2, ys = (size_t)M * N * 2;
+    if (xb < yb + ys && yb < xb + xs) return QMM_ERR_ARG;   // y overlaps x
+  }
+  Problem p{x, xdtype == QMM_BF16, qweight, scales, zeros_or_lut, M, N, K, bits, group, mode, y};
+  bool too_large = false;
+  const cudaError_t e =
+      launch_skinny_static(p, device_sms(), static_cast<cudaStream_t>(stream), &too_large);
+  if (too_large) return QMM_ERR_TOO_LARGE;
+  return status_of(e);
+}
+
 int qmm_dequant(const void* qweight, const uint16_t* scales, const uint16_t* zeros_or_lut, int N,
                 int K, int bits, int group, int mode, int out_dtype, void* W_out, void* stream) {
   int st = check_shape(N, K, bits, group, mode);
@@ -194,6 +222,8 @@ const char* qmm_strerror(int status) {
     case QMM_ERR_CUDA: return "CUDA runtime error";
     case QMM_ERR_TIMEOUT: return "a kernel abandoned a bounded wait";
     case QMM_ERR_WORKSPACE: return "workspace smaller than qmm_workspace_size";
+    case QMM_ERR_TOO_LARGE:
+      return "problem does not fit the library's static scratch buffer (qmm_noalloc: M <= 16)";
     default: return "unknown status";
   }
 }

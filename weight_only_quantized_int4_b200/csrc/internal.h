@@ -32,6 +32,10 @@ struct SkinnyPlan {
 SkinnyPlan plan_skinny(int M, int N, int K, int bits, int group, int mode, bool bf16, int sms);
 cudaError_t launch_skinny(const Problem& p, const SkinnyPlan& plan, void* workspace,
                           cudaStream_t stream);
+// Decode path on the library's static scratch buffer (no allocation); sets
+// *too_large instead of launching when the problem does not fit it.
+cudaError_t launch_skinny_static(const Problem& p, int sms, cudaStream_t stream, bool* too_large);
+size_t static_scratch_bytes();
 
 // Stream-K plan of the tensor-core path (tcgen05, 4-bit codes).
 struct TcPlan {

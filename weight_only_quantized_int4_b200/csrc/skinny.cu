@@ -672,3 +672,70 @@ cudaError_t launch_skinny(const Problem& pr, const SkinnyPlan& plan, void* works
 }
 
 }  // namespace qk
+
+// ---------------------------------------------------------------------------
+// Decode path with a library-owned scratch buffer, for callers that cannot
+// allocate device memory (see qmm_noalloc in qmm.h).
+namespace qk {
+namespace {
+
+constexpr size_t kStaticScratchBytes = size_t(8) << 20;   // 8 MiB per device
+__device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
+
+// Device address of g_static_scratch on the current device.  The symbol's
+// name is only a host-side stand-in, so the address is looked up once per
+// device (with that device current) and cached.
+cudaError_t static_scratch(void** out) {
+  static void* addr[kMaxDevices] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  if (!addr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_static_scratch);
+    if (e != cudaSuccess) {
+      cudaGetLastError();
+      return e;
+    }
+    addr[dev] = p;
+  }
+  *out = addr[dev];
+  return cudaSuccess;
+}
+
+}  // namespace
+
+size_t static_scratch_bytes() { return kStaticScratchBytes; }
+
+cudaError_t launch_skinny_static(const Problem& pr, int sms, cudaStream_t stream, bool* too_large) {
+  *too_large = false;
+  SkinnyPlan plan = plan_skinny(pr.M, pr.N, pr.K, pr.bits, pr.group, pr.mode, pr.bf16, sms);
+  const size_t counters = ((size_t)plan.slabs * plan.tiles_n * sizeof(unsigned) + 255) / 256 * 256;
+  const size_t slot2 = (size_t)plan.slabs * 2 * plan.rows * 8 * plan.nt * sizeof(float);  // per worker
+  if (plan.ws_bytes > kStaticScratchBytes) {
+    // fewer stream-K workers so that their partial-sum slots fit
+    if (counters + slot2 > kStaticScratchBytes) {
+      *too_large = true;
+      return cudaSuccess;
+    }
+    const long long w = (long long)((kStaticScratchBytes - counters) / slot2);
+    plan.warps = (int)std::min<long long>(plan.warps, w);
+    plan.splits = (plan.warps + kWarps - 1) / kWarps;
+    plan.ws_bytes = counters + slot2 * plan.warps;
+  }
+  void* ws = nullptr;
+  if (plan.ws_bytes) {
+    cudaError_t e = static_scratch(&ws);
+    if (e != cudaSuccess) return e;
+    // the arrival counters must start at zero; every call shares the buffer
+    e = cudaMemsetAsync(ws, 0, counters, stream);
+    if (e != cudaSuccess) {
+      cudaGetLastError();
+      return e;
+    }
+  }
+  return launch_skinny(pr, plan, ws, stream);
+}
+
+}  // namespace qk
