@@ -34,7 +34,7 @@
  *    (a bounded wait that ran out) are reported by qmm_check_error.
  *  - Shapes the GPU kernels accept: N % 16 == 0; K % 64 == 0 (4-bit) or
  *    K % 128 == 0 (2-bit); group == -1 or a power of two >= 16 that divides K;
- *    M >= 0.  Other shapes return QMM_ERR_UNSUPPORTED.
+ *    N, K <= 2^20; M >= 0.  Other shapes return QMM_ERR_UNSUPPORTED.
  *
  * Packed layout (written by qmm_pack, read by qmm and qmm_dequant):
  *  - qweight: N*K*bits/8 bytes.  Rows are taken in blocks of 16; each block is

@@ -32,6 +32,7 @@ int check_shape(int N, int K, int bits, int group, int mode) {
   if (bits != 4 && bits != 2) return QMM_ERR_ARG;
   if (bits == 2 && mode != QMM_LUT) return QMM_ERR_UNSUPPORTED;
   if (N % 16 != 0 || K % chunk_cols(bits) != 0) return QMM_ERR_UNSUPPORTED;
+  if (N > (1 << 20) || K > (1 << 20)) return QMM_ERR_UNSUPPORTED;   // 32-bit work indexing
   // groups: one per row (-1) or a power of two >= 16 dividing K
   if (group != -1 && (group < 16 || (group & (group - 1)) != 0 || K % group != 0))
     return QMM_ERR_UNSUPPORTED;
@@ -209,8 +210,9 @@ int qmm_dequant(const void* qweight, const uint16_t* scales, const uint16_t* zer
 int qmm_check_error(void* stream) {
   if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return QMM_ERR_CUDA;
   const unsigned v = tc_read_and_clear_error();
-  if (v == 0xFFFFFFFFu) return QMM_ERR_CUDA;
-  return v ? QMM_ERR_TIMEOUT : QMM_OK;
+  const unsigned w = skinny_read_and_clear_error();
+  if (v == 0xFFFFFFFFu || w == 0xFFFFFFFFu) return QMM_ERR_CUDA;
+  return (v | w) ? QMM_ERR_TIMEOUT : QMM_OK;
 }
 
 const char* qmm_strerror(int status) {

@@ -1,6 +1,8 @@
 // Internal launch interface between the C-ABI layer (api.cu) and the kernels.
 #pragma once
 
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -36,6 +38,7 @@ cudaError_t launch_skinny(const Problem& p, const SkinnyPlan& plan, void* worksp
 // *too_large instead of launching when the problem does not fit it.
 cudaError_t launch_skinny_static(const Problem& p, int sms, cudaStream_t stream, bool* too_large);
 size_t static_scratch_bytes();
+unsigned skinny_read_and_clear_error();
 
 // Stream-K plan of the tensor-core path (tcgen05, 4-bit codes).
 struct TcPlan {
@@ -57,5 +60,8 @@ cudaError_t launch_dequant(const void* qweight, const uint16_t* scales,
                            int mode, int out_dtype, void* W_out, cudaStream_t stream);
 
 int device_sms();
+
+// cuTensorMapEncodeTiled from the driver (looked up once), or nullptr.
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder();
 
 }  // namespace qk

@@ -476,27 +476,38 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1) skinny_kernel(const
 #pragma unroll
       for (int i = 0; i < NACC / 4; ++i)
         mine[i] = make_float4(outv[4 * i], outv[4 * i + 1], outv[4 * i + 2], outv[4 * i + 3]);
-      __threadfence();
       __syncwarp();
       unsigned* counter = a.counters + (size_t)slab * a.tiles + tile;
       unsigned prev = 0;
-      if (lane == 0) prev = atomicAdd(counter, 1u);
+      if (lane == 0)
+        asm volatile("atom.add.acq_rel.gpu.u32 %0, [%1], 1;" : "=r"(prev) : "l"(counter) : "memory");
       prev = __shfl_sync(0xffffffffu, prev, 0);
-      if (prev != (unsigned)(nb - 1)) continue;     // not the last: the tile is someone's
-      __threadfence();
-      // last warp: add the contributions in order (deterministic)
+      if (prev != (unsigned)(nb - 1)) continue;
 #pragma unroll
       for (int i = 0; i < NACC; ++i) outv[i] = 0.0f;
-      for (int k = 0; k < nb; ++k) {
-        const float4* src = reinterpret_cast<const float4*>(
-            slots + (size_t)(2 * (first + k) + (k == 0 ? first_e : 0)) * (NACC * 32) + lane * NACC);
+      for (int k0 = 0; k0 < nb; k0 += 4) {
+        float4 v[4][NACC / 4];
 #pragma unroll
-        for (int i = 0; i < NACC / 4; ++i) {
-          const float4 v = __ldcg(src + i);
-          outv[4 * i] += v.x;
-          outv[4 * i + 1] += v.y;
-          outv[4 * i + 2] += v.z;
-          outv[4 * i + 3] += v.w;
+        for (int kk = 0; kk < 4; ++kk) {
+          const int k = k0 + kk;
+          if (k < nb) {
+            const float4* src = reinterpret_cast<const float4*>(
+                slots + (size_t)(2 * (first + k) + (k == 0 ? first_e : 0)) * (NACC * 32) + lane * NACC);
+#pragma unroll
+            for (int i = 0; i < NACC / 4; ++i) v[kk][i] = __ldcg(src + i);
+          }
+        }
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          if (k0 + kk < nb) {
+#pragma unroll
+            for (int i = 0; i < NACC / 4; ++i) {
+              outv[4 * i] += v[kk][i].x;
+              outv[4 * i + 1] += v[kk][i].y;
+              outv[4 * i + 2] += v[kk][i].z;
+              outv[4 * i + 3] += v[kk][i].w;
+            }
+          }
         }
       }
       if (lane == 0) *counter = 0u;   // ready for the next call
@@ -623,6 +634,8 @@ SkinnyPlan plan_skinny(int M, int N, int K, int bits, int group, int mode, bool 
   });
   // one resident wave of CTAs; every warp is a stream-K worker with >= 1 unit
   long long warps = (long long)sms * (occ > 0 ? occ : 1) * kWarps;
+  const long long cap = std::max<long long>(1, units * 8 / nsc);
+  if (warps > cap) warps = cap;
   if (warps > units) warps = units;
   const long long ctas = (warps + kWarps - 1) / kWarps;
   p.splits = (int)ctas;
@@ -738,4 +751,10 @@ cudaError_t launch_skinny_static(const Problem& pr, int sms, cudaStream_t stream
   return launch_skinny(pr, plan, ws, stream);
 }
 
+}  // namespace qk
+
+namespace qk {
+// The decode path waits on nothing but its own cp.async groups (hardware
+// waits that always end): it has no bounded wait that could give up.
+unsigned skinny_read_and_clear_error() { return 0; }
 }  // namespace qk

@@ -50,36 +50,6 @@ struct TcCfg {
 
 // ------------------------------------------------------------------ PTX helpers
 
-__device__ __forceinline__ uint32_t smem_u32(const void* p) {
-  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-
-__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
-}
-
-__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
-}
-
-__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
-               "r"(bytes)
-               : "memory");
-}
-
-__device__ __forceinline__ bool mbar_try(uint64_t* bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-
 // Bounded wait for phase `parity` of `bar`.  Returns false (and raises the
 // CTA's abort flag and the device error word) if it runs out, or if another
 // thread of the CTA has already aborted.
@@ -97,18 +67,6 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   }
 }
 
-__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar,
-                                            int x, int y) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes "
-      "[%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y)
-      : "memory");
-}
-
-__device__ __forceinline__ void fence_proxy_async() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
 __device__ __forceinline__ void tc_fence_before() {
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
 }
@@ -174,7 +132,7 @@ struct TcArgs {
   int tiles_n, tiles_m, tiles;
   long long units;          // tiles * nkb
   int ctas;
-  float* slots;             // [2 * ctas][BN][128]: a CTA's first / last partial tile
+  float* slots;             // [2 * ctas][128][BN]: a CTA's first / last partial tile
   unsigned* counters;       // [tiles]
 };
 
@@ -234,6 +192,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int* last_flag = const_cast<int*>(abort_flag) + 1;
+  int* meta = last_flag + 1;   // [3]: first contributor, contributors, first's slot parity
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int b = blockIdx.x;
@@ -456,60 +415,103 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       }
       const long long t_first = (long long)tile * a.nkb;
       const bool whole = (u == t_first) && (kb1 == a.nkb);
-      int first = 0, nb = 1;
+      // partial tiles: slot 2 b + e holds this CTA's [128 rows][BN] fp32 sums
+      // (e = 1 when the tile is not the CTA's first); contributors are CTAs
+      // first .. first + nb - 1, of which only `first` can have e = 1
       float* slot = nullptr;
       if (!whole) {
-        first = owner_of_tc(t_first, a.units, a.ctas);
-        nb = owner_of_tc(t_first + a.nkb - 1, a.units, a.ctas) - first + 1;
         const int e = (tile == (int)(u_begin / a.nkb)) ? 0 : 1;
-        slot = a.slots + (size_t)(2 * b + e) * (size_t)(BN * kRowsTile);
+        slot = a.slots + (size_t)(2 * b + e) * (size_t)(BN * kRowsTile) + (size_t)row_l * BN;
+        if (threadIdx.x == 192) {     // 64-bit stream-K bookkeeping, once
+          const int first = owner_of_tc(t_first, a.units, a.ctas);
+          meta[0] = first;
+          meta[1] = owner_of_tc(t_first + a.nkb - 1, a.units, a.ctas) - first + 1;
+          meta[2] = ((long long)first * a.units / a.ctas < t_first) ? 1 : 0;
+        }
       }
 #pragma unroll 1
       for (int c0 = 0; c0 < BN; c0 += 32) {
         float v[32];
         tmem_ld32(tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * BN + c0), v);
+        if (whole) {
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const int m = tm * BN + c0 + i;
-          if (whole) {
+          for (int i = 0; i < 32; ++i) {
+            const int m = tm * BN + c0 + i;
             if (row < a.N && m < a.M) {
               const float o = v[i] * s_row;
               a.y[(size_t)m * a.N + row] = BF16 ? __bfloat16_as_ushort(__float2bfloat16_rn(o))
                                                 : __half_as_ushort(__float2half_rn(o));
             }
-          } else {
-            slot[(size_t)(c0 + i) * kRowsTile + row_l] = v[i];
           }
+        } else {
+          float4* dst = reinterpret_cast<float4*>(slot + c0);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
         }
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&acc_empty[buf]);
+      if (lane == 0) mbar_arrive(&acc_empty[buf]);     // the accumulator may be reused
       if (!whole) {
-        __threadfence();
+        // every epilogue thread's slot stores, then one release increment
         named_bar(1, 128);
-        if (threadIdx.x == 192) *last_flag = (atomicAdd(&a.counters[tile], 1u) == (unsigned)(nb - 1));
-        named_bar(1, 128);
-        if (*last_flag) {
-          __threadfence();
-          for (int cc = 0; cc < BN; ++cc) {
-            const int m = tm * BN + cc;
-            float acc = 0.0f;
-            for (int k = 0; k < nb; ++k) {
-              const int bb = first + k;
-              const int ee = ((long long)bb * a.units / a.ctas < t_first) ? 1 : 0;
-              acc += __ldcg(a.slots + (size_t)(2 * bb + ee) * (BN * kRowsTile) +
-                            (size_t)cc * kRowsTile + row_l);
-            }
-            if (row < a.N && m < a.M) {
-              const float o = acc * s_row;
-              a.y[(size_t)m * a.N + row] = BF16 ? __bfloat16_as_ushort(__float2bfloat16_rn(o))
-                                                : __half_as_ushort(__float2half_rn(o));
-            }
-          }
-          if (threadIdx.x == 192) a.counters[tile] = 0u;
+        if (threadIdx.x == 192) {
+          unsigned prev;
+          asm volatile("atom.add.acq_rel.gpu.u32 %0, [%1], 1;"
+                       : "=r"(prev)
+                       : "l"(&a.counters[tile])
+                       : "memory");
+          *last_flag = prev == (unsigned)(meta[1] - 1);
         }
         named_bar(1, 128);
+        if (*last_flag) {
+          const int first = meta[0], nb = meta[1], first_e = meta[2];
+#pragma unroll 1
+          for (int c0 = 0; c0 < BN; c0 += 32) {
+            float accv[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) accv[i] = 0.0f;
+            for (int k0 = 0; k0 < nb; k0 += 2) {      // two contributors' loads in flight
+              float4 va[8], vb[8];
+              const float4* pa = reinterpret_cast<const float4*>(
+                  a.slots + (size_t)(2 * (first + k0) + (k0 == 0 ? first_e : 0)) * (BN * kRowsTile) +
+                  (size_t)row_l * BN + c0);
+#pragma unroll
+              for (int i = 0; i < 8; ++i) va[i] = __ldcg(pa + i);
+              const bool two = k0 + 1 < nb;
+              if (two) {
+                const float4* pb = reinterpret_cast<const float4*>(
+                    a.slots + (size_t)(2 * (first + k0 + 1)) * (BN * kRowsTile) +
+                    (size_t)row_l * BN + c0);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) vb[i] = __ldcg(pb + i);
+              }
+#pragma unroll
+              for (int i = 0; i < 8; ++i) {
+                accv[4 * i] += va[i].x; accv[4 * i + 1] += va[i].y;
+                accv[4 * i + 2] += va[i].z; accv[4 * i + 3] += va[i].w;
+              }
+              if (two) {
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                  accv[4 * i] += vb[i].x; accv[4 * i + 1] += vb[i].y;
+                  accv[4 * i + 2] += vb[i].z; accv[4 * i + 3] += vb[i].w;
+                }
+              }
+            }
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              const int m = tm * BN + c0 + i;
+              if (row < a.N && m < a.M) {
+                const float o = accv[i] * s_row;
+                a.y[(size_t)m * a.N + row] = BF16 ? __bfloat16_as_ushort(__float2bfloat16_rn(o))
+                                                  : __half_as_ushort(__float2half_rn(o));
+              }
+            }
+          }
+          if (threadIdx.x == 192) a.counters[tile] = 0u;   // ready for the next call
+        }
+        named_bar(1, 128);   // last_flag / meta are reused by the next segment
       }
       u += kb1 - kb0;
     }
@@ -531,25 +533,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 namespace qk {
 namespace {
 
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  if (!fn) {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  }
-  return fn;
-}
-
 template <int MODE, int BN>
 constexpr size_t tc_smem_bytes() {
   using Cfg = TcCfg<BN>;
   return 1024 + (size_t)Cfg::STAGES * (kATileBytes + Cfg::B_BYTES) +
          (size_t)kCodeStages * kCodeBytes + (MODE == kLUT ? 256 * 32 * 4 : 0) +
-         (2 * kCodeStages + 3 * Cfg::STAGES + 4) * 8 + 16;
+         (2 * kCodeStages + 3 * Cfg::STAGES + 4) * 8 + 32;
 }
 
 template <int MODE, bool BF16, int BN, bool GM1>
@@ -602,6 +591,21 @@ cudaError_t launch_mode(bool bf16, bool gm1, int bn, const CUtensorMap& mx, cons
 
 }  // namespace
 
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    else
+      cudaGetLastError();
+  }
+  return fn;
+}
+
 // Combinations the tensor path computes within tolerance: 4-bit codes with
 // fp16 activations (the operand is fp16((q - z) s) or fp16(T s), one rounding
 // of 2^-11), or with bf16 activations when the scale is per row (the operand
@@ -634,7 +638,7 @@ TcPlan plan_tc(int M, int N, int K, int sms) {
 
 cudaError_t launch_tc(const Problem& pr, const TcPlan& plan, void* workspace,
                       cudaStream_t stream) {
-  auto encode = encode_fn();
+  auto encode = tensor_map_encoder();
   if (!encode) return cudaErrorNotSupported;
   CUtensorMap mx, mw;
   {
