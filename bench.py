@@ -159,6 +159,22 @@ class ClockSampler:
 
 # --------------------------------------------------------------------------- ours
 
+def max_over_ranks(value, dist=None, device="cpu"):
+    """The largest `value` over all ranks; every rank gets it (one all-reduce)."""
+    if dist is None:
+        return value
+    import torch
+    t = torch.tensor([float(value)], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_gbs(world, bytes_per_step, steps, ms):
+    """Algorithmic GB/s of all ranks together: every rank streams `bytes_per_step`
+    per step (replicas, weak scaling) and the job takes `ms` (the slowest rank)."""
+    return world * bytes_per_step * steps / (ms / 1e3) / 1e9
+
+
 def run_ours(args, rank, world, local_rank):
     import torch
     import weight_only_quantized_int4_b200 as q
@@ -237,13 +253,9 @@ def run_ours(args, rank, world, local_rank):
         barrier()
         torch.cuda.synchronize()
     clocks = clock.stop()
-    ms = e0.elapsed_time(e1)
-    if dist is not None:
-        t = torch.tensor([ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(e0.elapsed_time(e1), dist, dev)
     ms_per_step = ms / args.steps
-    value = world * step_bytes * args.steps / (ms / 1e3) / 1e9
+    value = whole_job_gbs(world, step_bytes, args.steps, ms)
 
     # ---- end to end through the public API: pinned host x in, y out, per step
     hx = [c["x"].cpu().pin_memory() for c in calls]
@@ -271,12 +283,8 @@ def run_ours(args, rank, world, local_rank):
         a1.record(stream)
         torch.cuda.synchronize()
         barrier()
-    e2e_ms = a0.elapsed_time(a1)
-    if dist is not None:
-        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    e2e_value = world * step_bytes * e2e_steps / (e2e_ms / 1e3) / 1e9
+    e2e_ms = max_over_ranks(a0.elapsed_time(a1), dist, dev)
+    e2e_value = whole_job_gbs(world, step_bytes, e2e_steps, e2e_ms)
 
     peak, peak_kind = peaks()
     achieved = step_bytes / (ms_per_step / 1e3) / 1e9      # one GPU, the skinny kernel only

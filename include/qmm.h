@@ -98,8 +98,8 @@ size_t qmm_packed_size(int N, int K, int bits, int group, int mode,
  *   W        device, fp32 [N, K] row-major, finite values.
  *   lut      device, 2^bits fp16 entries (QMM_LUT), else NULL.
  *   qweight  device, qmm_packed_size bytes, 16-byte aligned (written).
- *   scales   device, fp16, scales_bytes (written).
- *   zeros    device, fp16, zeros_bytes (QMM_ASYM, written), else NULL.
+ *   scales   device, fp16, scales_bytes, 16-byte aligned (written).
+ *   zeros    device, fp16, zeros_bytes, 16-byte aligned (QMM_ASYM, written), else NULL.
  * bits: 4 for SYM/ASYM; 4 or 2 for LUT. */
 int qmm_pack(const float* W, int N, int K, int mode, int bits, int group,
              const uint16_t* lut, void* qweight, uint16_t* scales, uint16_t* zeros,
@@ -121,7 +121,8 @@ size_t qmm_workspace_size_for(int M, int N, int K, int bits, int group, int mode
  *   x             device, [M, K] row-major, xdtype (fp16 or bf16), 16-byte aligned.
  *   qweight, scales, zeros_or_lut
  *                 device, as written by qmm_pack (zeros for ASYM, the table
- *                 for LUT, NULL for SYM).  ASYM zeros are exact for integer
+ *                 for LUT, NULL for SYM); scales and ASYM zeros 16-byte
+ *                 aligned (they are copied in 16-byte pieces).  ASYM zeros are exact for integer
  *                 zero-points; a fractional zero is applied with one fp16 rounding.
  *   y             device, [M, N] row-major, same dtype as x, must not overlap x.
  *   workspace     device, workspace_bytes >= qmm_workspace_size(...), zero

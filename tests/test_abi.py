@@ -78,6 +78,14 @@ def test_bad_arguments_return_status_without_launching(lib):
     # misaligned x
     assert lib.qmm(P(0x1002), 0, fake, fake, None, 1, 64, 64, 4, 64, 0, P(0x90000), None, 0,
                    None) == -3
+    # scales / ASYM zeros must be 16-byte aligned (copied in 16-byte pieces)
+    assert lib.qmm(fake, 0, fake, P(0x1004), None, 1, 64, 64, 4, 64, 0, P(0x90000), None, 0,
+                   None) == -3
+    assert lib.qmm(fake, 0, fake, fake, P(0x1008), 1, 64, 64, 4, 64, 1, P(0x90000), None, 0,
+                   None) == -3
+    assert lib.qmm_noalloc(fake, 0, fake, P(0x1004), None, 1, 64, 64, 4, 64, 0, P(0x90000),
+                           None) == -3
+    assert lib.qmm_pack(fake, 64, 64, 0, 4, 64, None, fake, P(0x1002), None, None) == -3
     # y overlapping x
     assert lib.qmm(fake, 0, P(0x200000), fake, None, 2, 64, 64, 4, 64, 0, P(0x1040), None, 0,
                    None) == -1

@@ -1,0 +1,73 @@
+"""bench.py with several ranks, on the CPU: world size 2 over gloo.
+
+The decode path has no data exchange between GPUs (each rank is an
+independent replica), so the only multi-rank logic is the timing: every rank
+times its own K steps, the job time is the slowest rank's, and the reported
+throughput is all ranks' bytes over that time.  These tests run that logic in
+two real processes, and check that the reference arm under torchrun does its
+work on rank 0 only.
+"""
+import json
+import os
+import socket
+import subprocess
+import sys
+
+import pytest
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+import bench  # noqa: E402
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank, world, port, out_dir):
+    import datetime
+
+    import torch.distributed as dist
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank,
+                            world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        # the bench's collective sequence: barrier, max of the device time,
+        # barrier, max of the end-to-end time -- same steps on every rank
+        dist.barrier()
+        ms = bench.max_over_ranks(10.0 + 5.0 * rank, dist)
+        dist.barrier()
+        e2e = bench.max_over_ranks(30.0 - 7.0 * rank, dist)
+        value = bench.whole_job_gbs(world, 2.0e9, 100, ms)
+        with open(os.path.join(out_dir, f"rank{rank}.json"), "w") as f:
+            json.dump({"ms": ms, "e2e": e2e, "value": value}, f)
+    finally:
+        dist.destroy_process_group()
+
+
+def test_max_over_ranks_and_whole_job_value_two_ranks(tmp_path):
+    world = 2
+    mp.start_processes(_rank_main, args=(world, _free_port(), str(tmp_path)), nprocs=world,
+                       join=True, start_method="spawn")
+    res = [json.load(open(tmp_path / f"rank{r}.json")) for r in range(world)]
+    for r in res:
+        assert r["ms"] == 15.0            # the slowest rank's device time
+        assert r["e2e"] == 30.0
+        # 2 ranks x 2 GB per step x 100 steps in 15 ms
+        assert r["value"] == pytest.approx(2 * 2.0e9 * 100 / 0.015 / 1e9)
+
+
+def test_single_rank_needs_no_process_group():
+    assert bench.max_over_ranks(3.5) == 3.5
+    assert bench.whole_job_gbs(1, 1.0e9, 10, 1000.0) == pytest.approx(10.0)
+
+
+def test_reference_arm_runs_on_rank_zero_only():
+    env = dict(os.environ, RANK="1", WORLD_SIZE="2", LOCAL_RANK="1")
+    p = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                        "--steps", "3", "--warmup", "3"], env=env, capture_output=True,
+                       text=True, timeout=120)
+    assert p.returncode == 0, p.stderr
+    assert p.stdout.strip() == ""

@@ -90,8 +90,8 @@ int qmm_pack(const float* W, int N, int K, int mode, int bits, int group, const 
   if (!W || !qweight || !scales) return QMM_ERR_ARG;
   if (mode == QMM_ASYM && !zeros) return QMM_ERR_ARG;
   if (mode == QMM_LUT && !lut) return QMM_ERR_ARG;
-  if (!aligned(W, 16) || !aligned(qweight, 16) || !aligned(scales, 4) ||
-      (zeros && !aligned(zeros, 4)))
+  if (!aligned(W, 16) || !aligned(qweight, 16) || !aligned(scales, 16) ||
+      (zeros && !aligned(zeros, 16)))
     return QMM_ERR_ALIGN;
   return status_of(launch_pack(W, N, K, mode, bits, group, lut, qweight, scales, zeros,
                                static_cast<cudaStream_t>(stream)));
@@ -129,8 +129,8 @@ int qmm_with_path(const void* x, int xdtype, const void* qweight, const uint16_t
   if (M == 0) return QMM_OK;
   if (!x || !qweight || !scales || !y) return QMM_ERR_ARG;
   if (mode != QMM_SYM && !zeros_or_lut) return QMM_ERR_ARG;
-  if (!aligned(x, 16) || !aligned(qweight, 16) || !aligned(scales, 4) || !aligned(y, 2) ||
-      (mode == QMM_ASYM && !aligned(zeros_or_lut, 4)) || (workspace && !aligned(workspace, 256)))
+  if (!aligned(x, 16) || !aligned(qweight, 16) || !aligned(scales, 16) || !aligned(y, 2) ||
+      (mode == QMM_ASYM && !aligned(zeros_or_lut, 16)) || (workspace && !aligned(workspace, 256)))
     return QMM_ERR_ALIGN;
   {
     const char* xb = static_cast<const char*>(x);
@@ -178,8 +178,8 @@ int qmm_noalloc(const void* x, int xdtype, const void* qweight, const uint16_t* 
   if (M == 0) return QMM_OK;
   if (!x || !qweight || !scales || !y) return QMM_ERR_ARG;
   if (mode != QMM_SYM && !zeros_or_lut) return QMM_ERR_ARG;
-  if (!aligned(x, 16) || !aligned(qweight, 16) || !aligned(scales, 4) || !aligned(y, 2) ||
-      (mode == QMM_ASYM && !aligned(zeros_or_lut, 4)))
+  if (!aligned(x, 16) || !aligned(qweight, 16) || !aligned(scales, 16) || !aligned(y, 2) ||
+      (mode == QMM_ASYM && !aligned(zeros_or_lut, 16)))
     return QMM_ERR_ALIGN;
   {
     const char* xb = static_cast<const char*>(x);
