@@ -8,8 +8,10 @@ shapes of one decoder layer -- fused QKV (K 4096, N 12288), O (4096, 4096),
 fused gate/up (4096, 22016), down (11008, 4096) -- at M = 1, 2, 4, 8 and 16
 tokens: 20 qmm calls per step, symmetric int4, group 128, fp16 activations.
 Each call has its own weights (522 MB in all, over 4x the 126 MB L2), so every
-call streams its codes from HBM.  The 20 launches are captured once in a CUDA
-graph and a step is one replay.
+call streams its codes from HBM; smaller workloads get as many weight copies
+as it takes to pass twice the L2 size, rotated step by step.  The launches of
+a step are captured in a CUDA graph (one per weight copy) and a step is one
+replay.
 
 Prints one JSON line (rank 0).  `value` is HBM throughput in GB/s: algorithmic
 bytes (codes + scales + x + y) of all calls on all ranks / max-over-ranks
@@ -51,6 +53,7 @@ WORKLOADS = {
     "lut2": ("lut", 2, 64, "f16", [(4096, 14336)], [1, 8]),
 }
 SIGMA = {"sym": 0.02, "asym": 0.015, "lut": 0.02}
+L2_BYTES = 126 * 1000 * 1000     # B200 L2
 SKINNY_SOURCES = ("weight_only_quantized_int4_b200/csrc/skinny.cu",
                   "weight_only_quantized_int4_b200/csrc/common.cuh")
 
@@ -184,41 +187,54 @@ def run_ours(args, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     probs = problems(args.workload)
     gen = torch.Generator(device=dev).manual_seed(1234 + rank)
-    calls = []
-    for i, (mode, bits, group, xdt, M, K, N) in enumerate(probs):
-        W = torch.randn(N, K, generator=gen, device=dev) * SIGMA[mode]
-        lut = None
-        if mode == "lut":
-            from weight_only_quantized_int4_b200 import synth
-            t = synth.nf4_table() if bits == 4 else synth.lut2_table(0)
-            lut = torch.from_numpy(t.view(np.int16)).to(dev)
-        qw, sc, ze = q.pack(W, mode, bits, group, lut=lut)
-        del W
-        tdt = torch.float16 if xdt == "f16" else torch.bfloat16
-        x = torch.randn(M, K, generator=gen, device=dev).to(tdt)
-        y = torch.empty(M, N, dtype=tdt, device=dev)
-        ws = q.workspace(M, N, K, mode, bits, group, device=dev)
-        zl = ze if mode == "asym" else lut
-        calls.append(dict(x=x, qw=qw, sc=sc, zl=zl, y=y, ws=ws, M=M, N=N, K=K, mode=mode,
-                          bits=bits, group=group, bytes=alg_bytes(mode, bits, group, M, K, N)))
+    # enough weight copies that the codes of consecutive steps never fit in L2
+    codes_per_copy = sum(N * K * bits // 8 for (_, bits, _, _, _, K, N) in probs)
+    copies = max(1, -(-2 * L2_BYTES // codes_per_copy))
+    sets = []
+    for _ in range(copies):
+        calls = []
+        for (mode, bits, group, xdt, M, K, N) in probs:
+            W = torch.randn(N, K, generator=gen, device=dev) * SIGMA[mode]
+            lut = None
+            if mode == "lut":
+                from weight_only_quantized_int4_b200 import synth
+                t = synth.nf4_table() if bits == 4 else synth.lut2_table(0)
+                lut = torch.from_numpy(t.view(np.int16)).to(dev)
+            qw, sc, ze = q.pack(W, mode, bits, group, lut=lut)
+            del W
+            tdt = torch.float16 if xdt == "f16" else torch.bfloat16
+            x = torch.randn(M, K, generator=gen, device=dev).to(tdt)
+            y = torch.empty(M, N, dtype=tdt, device=dev)
+            ws = q.workspace(M, N, K, mode, bits, group, device=dev)
+            zl = ze if mode == "asym" else lut
+            calls.append(dict(x=x, qw=qw, sc=sc, zl=zl, y=y, ws=ws, M=M, N=N, K=K, mode=mode,
+                              bits=bits, group=group,
+                              bytes=alg_bytes(mode, bits, group, M, K, N)))
+        sets.append(calls)
     torch.cuda.synchronize()
+    calls = sets[0]
     step_bytes = sum(c["bytes"] for c in calls)
 
-    def step():
-        for c in calls:
+    def step(i=0):
+        for c in sets[i % copies]:
             q.qmm(c["x"], c["qw"], c["sc"], c["zl"], c["N"], c["K"], c["mode"], c["bits"],
                   c["group"], y=c["y"], ws=c["ws"])
 
-    # warm-up outside the graph (first calls set kernel attributes), then capture
-    step()
+    # warm-up outside the graphs (first calls set kernel attributes), then one
+    # graph per weight copy; step i replays graph i % copies
+    for i in range(copies):
+        step(i)
     torch.cuda.synchronize()
     stream = torch.cuda.Stream(device=dev)
-    graph = torch.cuda.CUDAGraph()
+    graphs = []
     with torch.cuda.stream(stream):
         step()
         torch.cuda.synchronize()
-        with torch.cuda.graph(graph, stream=stream):
-            step()
+        for i in range(copies):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                step(i)
+            graphs.append(g)
     torch.cuda.synchronize()
 
     dist = None
@@ -232,13 +248,13 @@ def run_ours(args, rank, world, local_rank):
     clock = ClockSampler(local_rank)
     clock.start()
     with torch.cuda.stream(stream):
-        for _ in range(args.warmup):
-            graph.replay()
+        for i in range(args.warmup):
+            graphs[i % copies].replay()
         # keep the GPU busy ~0.3 s so the clock samples see it under load
         t_end = time.time() + 0.3
         while time.time() < t_end:
-            for _ in range(50):
-                graph.replay()
+            for i in range(50):
+                graphs[i % copies].replay()
             torch.cuda.synchronize()
         torch.cuda.synchronize()
         barrier()
@@ -246,8 +262,8 @@ def run_ours(args, rank, world, local_rank):
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
         e0.record(stream)
-        for _ in range(args.steps):
-            graph.replay()
+        for i in range(args.steps):
+            graphs[i % copies].replay()
         e1.record(stream)
         torch.cuda.synchronize()
         barrier()
@@ -260,25 +276,26 @@ def run_ours(args, rank, world, local_rank):
     # ---- end to end through the public API: pinned host x in, y out, per step
     hx = [c["x"].cpu().pin_memory() for c in calls]
     hy = [torch.empty_like(c["y"], device="cpu").pin_memory() for c in calls]
+    e2e_calls = lambda i: sets[i % copies]
     h2d = sum(t.numel() * t.element_size() for t in hx)
     d2h = sum(t.numel() * t.element_size() for t in hy)
     e2e_steps = max(3, min(args.steps, 50))
     with torch.cuda.stream(stream):
-        for _ in range(2):
-            for c, h in zip(calls, hx):
+        for i in range(2):
+            for c, h in zip(e2e_calls(i), hx):
                 c["x"].copy_(h, non_blocking=True)
-            step()
+            step(i)
         torch.cuda.synchronize()
         barrier()
         torch.cuda.synchronize()
         a0 = torch.cuda.Event(enable_timing=True)
         a1 = torch.cuda.Event(enable_timing=True)
         a0.record(stream)
-        for _ in range(e2e_steps):
-            for c, h in zip(calls, hx):
+        for i in range(e2e_steps):
+            for c, h in zip(e2e_calls(i), hx):
                 c["x"].copy_(h, non_blocking=True)
-            step()
-            for c, h in zip(calls, hy):
+            step(i)
+            for c, h in zip(e2e_calls(i), hy):
                 h.copy_(c["y"], non_blocking=True)
         a1.record(stream)
         torch.cuda.synchronize()
@@ -301,8 +318,10 @@ def run_ours(args, rank, world, local_rank):
            "config": {"workload": args.workload, "calls_per_step": len(calls),
                       "shapes_KN": WORKLOADS[args.workload][4], "M": WORKLOADS[args.workload][5],
                       "mode": WORKLOADS[args.workload][0], "group": WORKLOADS[args.workload][2],
-                      "l2": "inputs larger than L2: every call has its own weights "
-                            f"({sum(c['qw'].numel() for c in calls) / 1e6:.0f} MB of codes)",
+                      "l2": f"inputs larger than L2: {copies} weight cop"
+                            f"{'y' if copies == 1 else 'ies'} of the step rotated, "
+                            f"{copies * codes_per_copy / 1e6:.0f} MB of codes in all "
+                            f"(L2 {L2_BYTES / 1e6:.0f} MB)",
                       "launch": "CUDA graph of the step, programmatic dependent launch",
                       "parallelism": f"replicas x{world}"},
            "roofline": roofline,
@@ -314,7 +333,7 @@ def run_ours(args, rank, world, local_rank):
            "clocks": clocks}
     if rank == 0 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(args.workload, args.cpu_seconds)
-    del graph
+    del graphs
     return out
 
 
