@@ -129,6 +129,7 @@ struct TcArgs {
   const uint16_t* zl;
   uint16_t* y;
   int M, N, K, L, G, nrb, nkb;
+  int lg;                   // log2 of the group length; 30 for one group per row
   int tiles_n, tiles_m, tiles;
   long long units;          // tiles * nkb
   int ctas;
@@ -138,6 +139,12 @@ struct TcArgs {
 
 __device__ __forceinline__ int owner_of_tc(long long u, long long U, int C) {
   return (int)(((u + 1) * (long long)C - 1) / U);
+}
+
+__device__ __forceinline__ uint32_t hmul2_u(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
 }
 
 // Scaled decoded pair (row of the pair, two k) -> packed fp16 / bf16.
@@ -311,89 +318,117 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const int dw = warp - 2;                 // row blocks 2dw, 2dw + 1 of the tile
     const int g = lane >> 2, t = lane & 3;
     const unsigned char* tabp = sT;
-    int kc = 0, ks = 0;
-    for (long long u = u_begin; u < u_end && !*abort_flag;) {
-      int tile, kb0, kb1;
-      seg_of(u, tile, kb0, kb1);
-      const int tn = tile % a.tiles_n;
-      bool ok = true;
-      for (int kb = kb0; kb < kb1; ++kb, ++kc, ++ks) {
-        const int c = kc % kCodeStages, s = ks % S;
-        if (!mbar_wait(&code_full[c], (kc / kCodeStages) & 1, abort_flag) ||
-            !mbar_wait(&ab_empty[s], ((ks / S) & 1) ^ 1, abort_flag)) {
-          ok = false;
-          break;
-        }
-        unsigned char* At = sA + s * kATileBytes;
+    // Group scales (and ASYM zero-points) of the lane's rows g and g + 8 in its
+    // two row blocks, one word per 16-column slice of the k block, read from
+    // global memory one k block ahead so that the loads overlap a decode.
+    constexpr bool kScales = !GM1;
+    constexpr bool kZeros = MODE == kASYM;
+    uint32_t sw_n[2][4] = {}, zw_n[2][4] = {};
+    auto load_meta = [&](int tl, int k) {
+      if constexpr (kScales || kZeros) {
+        const int tn = tl % a.tiles_n;
 #pragma unroll
         for (int rr = 0; rr < 2; ++rr) {
-          const int rbl = 2 * dw + rr;                       // row block in the tile
-          const int rb = tn * 8 + rbl;
-          const uint4 wv = *reinterpret_cast<const uint4*>(sC + c * kCodeBytes + rbl * 512 + lane * 16);
-          const int R0 = rbl * 16 + g, R1 = R0 + 8;
+          const int rb = tn * 8 + 2 * dw + rr;
+          const bool in = rb < a.nrb;
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
-            const uint32_t w = (&wv.x)[j];
-            uint32_t af[4];
-            if constexpr (MODE == kSYM) {
-              decode_int4<BF16, 8>(w, af);
-            } else if constexpr (MODE == kASYM) {
-              decode_int4<BF16, 0>(w, af);
-              const int gi = (kb * kKB + 16 * j) / a.L;
-              uint32_t zw = 0;
-              if (rb < a.nrb)
-                zw = *reinterpret_cast<const uint32_t*>(a.zl + ((size_t)rb * a.G + gi) * 16 + 2 * g);
-              if constexpr (BF16) {
-                const float2 zf = __half22float2(*reinterpret_cast<const __half2*>(&zw));
-                zw = pack2<true>(zf.x, zf.y);
-              }
-              sub_zero<BF16>(__byte_perm(zw, 0, 0x1010), __byte_perm(zw, 0, 0x3232), af);
-            } else {
-              const uint32_t l4 = (uint32_t)lane << 2;
-              af[0] = *reinterpret_cast<const uint32_t*>(tabp + lop3_and_or(w << 7, 0x7F80u, l4));
-              af[1] = *reinterpret_cast<const uint32_t*>(tabp + lop3_and_or(w >> 1, 0x7F80u, l4));
-              af[2] = *reinterpret_cast<const uint32_t*>(tabp + lop3_and_or(w >> 9, 0x7F80u, l4));
-              af[3] = *reinterpret_cast<const uint32_t*>(tabp + lop3_and_or(w >> 17, 0x7F80u, l4));
+            const int gi = (k * kKB + 16 * j) >> a.lg;
+            const size_t off = ((size_t)rb * a.G + gi) * 16 + 2 * g;
+            if constexpr (kScales)
+              sw_n[rr][j] = in ? __ldg(reinterpret_cast<const unsigned int*>(a.scales + off)) : 0u;
+            if constexpr (kZeros)
+              zw_n[rr][j] = in ? __ldg(reinterpret_cast<const unsigned int*>(a.zl + off)) : 0u;
+          }
+        }
+      }
+    };
+    int ct = (int)(u_begin / a.nkb), ck = (int)(u_begin % a.nkb);   // unit u = ct nkb + ck
+    if (u_begin < u_end) load_meta(ct, ck);
+    int kc = 0, ks = 0;
+    for (long long u = u_begin; u < u_end && !*abort_flag; ++u, ++kc, ++ks) {
+      uint32_t sw[2][4], zw[2][4];
+#pragma unroll
+      for (int rr = 0; rr < 2; ++rr)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          sw[rr][j] = sw_n[rr][j];
+          zw[rr][j] = zw_n[rr][j];
+        }
+      if (++ck == a.nkb) {
+        ck = 0;
+        ++ct;
+      }
+      if (u + 1 < u_end) load_meta(ct, ck);
+      const int c = kc % kCodeStages, s = ks % S;
+      if (!mbar_wait(&code_full[c], (kc / kCodeStages) & 1, abort_flag) ||
+          !mbar_wait(&ab_empty[s], ((ks / S) & 1) ^ 1, abort_flag))
+        break;
+      unsigned char* At = sA + s * kATileBytes;
+#pragma unroll
+      for (int rr = 0; rr < 2; ++rr) {
+        const int rbl = 2 * dw + rr;                       // row block in the tile
+        const uint4 wv = *reinterpret_cast<const uint4*>(sC + c * kCodeBytes + rbl * 512 + lane * 16);
+        const int R0 = rbl * 16 + g, R1 = R0 + 8;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const uint32_t w = (&wv.x)[j];
+          uint32_t af[4];
+          if constexpr (MODE == kSYM) {
+            decode_int4<BF16, 8>(w, af);
+          } else if constexpr (MODE == kASYM) {
+            decode_int4<BF16, 0>(w, af);
+            uint32_t z = zw[rr][j];
+            if constexpr (BF16) {
+              const float2 zf = __half22float2(*reinterpret_cast<const __half2*>(&z));
+              z = pack2<true>(zf.x, zf.y);
             }
+            sub_zero<BF16>(__byte_perm(z, 0, 0x1010), __byte_perm(z, 0, 0x3232), af);
+          } else {
+            const uint32_t l4 = (uint32_t)lane << 2;
+            af[0] = *reinterpret_cast<const uint32_t*>(tabp + lop3_and_or(w << 7, 0x7F80u, l4));
+            af[1] = *reinterpret_cast<const uint32_t*>(tabp + lop3_and_or(w >> 1, 0x7F80u, l4));
+            af[2] = *reinterpret_cast<const uint32_t*>(tabp + lop3_and_or(w >> 9, 0x7F80u, l4));
+            af[3] = *reinterpret_cast<const uint32_t*>(tabp + lop3_and_or(w >> 17, 0x7F80u, l4));
+          }
+          if constexpr (kScales && !BF16 && MODE != kLUT) {
+            // (s_g, s_g) and (s_g8, s_g8) as fp16 pairs: one HMUL2 per register
+            const uint32_t sg = __byte_perm(sw[rr][j], 0, 0x1010);
+            const uint32_t sg8 = __byte_perm(sw[rr][j], 0, 0x3232);
+            af[0] = hmul2_u(af[0], sg);
+            af[2] = hmul2_u(af[2], sg);
+            af[1] = hmul2_u(af[1], sg8);
+            af[3] = hmul2_u(af[3], sg8);
+          } else if constexpr (kScales || MODE == kLUT) {
             float2 sc = make_float2(1.f, 1.f);
-            if constexpr (!GM1) {
-              const int gi = (kb * kKB + 16 * j) / a.L;
-              sc = make_float2(0.f, 0.f);
-              if (rb < a.nrb) {
-                const uint32_t sw = *reinterpret_cast<const uint32_t*>(
-                    a.scales + ((size_t)rb * a.G + gi) * 16 + 2 * g);
-                sc = __half22float2(*reinterpret_cast<const __half2*>(&sw));
-              }
-            }
+            if constexpr (kScales) sc = __half22float2(*reinterpret_cast<const __half2*>(&sw[rr][j]));
             if constexpr (MODE == kLUT) {
               af[0] = lut_pair<BF16, GM1>(af[0], sc.x);
               af[2] = lut_pair<BF16, GM1>(af[2], sc.x);
               af[1] = lut_pair<BF16, GM1>(af[1], sc.y);
               af[3] = lut_pair<BF16, GM1>(af[3], sc.y);
-            } else if constexpr (!GM1) {
+            } else {
               af[0] = scale_pair<BF16>(af[0], sc.x);
               af[2] = scale_pair<BF16>(af[2], sc.x);
               af[1] = scale_pair<BF16>(af[1], sc.y);
               af[3] = scale_pair<BF16>(af[3], sc.y);
             }
-            // k_local = 16 j + 4 t: 16-byte chunk 2j + t/2, offset 8 (t & 1)
-            const int ch = 2 * j + (t >> 1);
-            const int off = 8 * (t & 1);
-            *reinterpret_cast<uint2*>(At + R0 * 128 + ((ch ^ (R0 & 7)) << 4) + off) =
-                make_uint2(af[0], af[2]);
-            *reinterpret_cast<uint2*>(At + R1 * 128 + ((ch ^ (R1 & 7)) << 4) + off) =
-                make_uint2(af[1], af[3]);
           }
-        }
-        fence_proxy_async();
-        __syncwarp();
-        if (lane == 0) {
-          mbar_arrive(&code_empty[c]);
-          mbar_arrive(&a_full[s]);
+          // k_local = 16 j + 4 t: 16-byte chunk 2j + t/2, offset 8 (t & 1)
+          const int ch = 2 * j + (t >> 1);
+          const int off = 8 * (t & 1);
+          *reinterpret_cast<uint2*>(At + R0 * 128 + ((ch ^ (R0 & 7)) << 4) + off) =
+              make_uint2(af[0], af[2]);
+          *reinterpret_cast<uint2*>(At + R1 * 128 + ((ch ^ (R1 & 7)) << 4) + off) =
+              make_uint2(af[1], af[3]);
         }
       }
-      if (!ok) break;
-      u += kb1 - kb0;
+      fence_proxy_async();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&code_empty[c]);
+        mbar_arrive(&a_full[s]);
+      }
     }
   } else {
     // ------------------------------------------------------------ epilogue warps
@@ -673,6 +708,7 @@ cudaError_t launch_tc(const Problem& pr, const TcPlan& plan, void* workspace,
   a.K = pr.K;
   a.L = pr.group == -1 ? pr.K : pr.group;
   a.G = pr.K / a.L;
+  a.lg = pr.group == -1 ? 30 : __builtin_ctz((unsigned)pr.group);
   a.nrb = pr.N / 16;
   a.nkb = plan.nkb;
   a.tiles_n = plan.tiles_n;
