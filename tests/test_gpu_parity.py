@@ -125,6 +125,26 @@ def test_qmm_small(mode, bits, group, xdtype):
             cases.compare(to_f64(y, xdtype), y_ref, bound, f"{mode}{bits} g{group} M{M} {path}")
 
 
+@pytest.mark.parametrize("mode,bits,group,xdtype", [
+    ("sym", 4, 64, "f16"), ("sym", 4, -1, "f16"), ("asym", 4, 64, "bf16"), ("lut", 4, 64, "f16"),
+    ("sym", 4, 32, "bf16"), ("lut", 4, 64, "bf16")])
+@pytest.mark.parametrize("K", [320, 704])
+def test_qmm_k_ends_mid_stage(mode, bits, group, xdtype, K):
+    """K % 128 == 64: the decode path's last 128-column stage holds one valid
+    64-column chunk (the second must contribute nothing); the tensor path's
+    64-column k blocks end exactly at K."""
+    N = 48
+    for M in (1, 5, 16, 17, 64):
+        p = cases.make(mode, bits, group, M, N, K, xdtype, seed=300 + M + K)
+        y_ref, bound = cases.expected(p)
+        x, qw, sp, zl = upload(p)
+        for path in ("auto", "skinny"):
+            ws = q.workspace(M, N, K, mode, bits, group, path=path)
+            y = q.qmm(x, qw, sp, zl, N, K, mode, bits, group, ws=ws, path=path)
+            torch.cuda.synchronize()
+            cases.compare(to_f64(y, xdtype), y_ref, bound, f"{mode} g{group} K{K} M{M} {path}")
+
+
 TC_CASES = [("sym", 4, 128, "f16"), ("sym", 4, -1, "f16"), ("asym", 4, 128, "f16"),
             ("lut", 4, 64, "f16"), ("lut", 4, -1, "f16"), ("sym", 4, 32, "f16"),
             ("sym", 4, -1, "bf16"), ("asym", 4, -1, "bf16")]
