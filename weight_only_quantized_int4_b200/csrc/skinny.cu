@@ -10,23 +10,33 @@
 // scales multiply the fp32 partial sums after each group, so the MMA operands
 // are exact.
 //
-// Memory pipeline: every warp owns a ring of kStages shared-memory stages and
-// keeps kStages - 1 chunks in flight with cp.async (codes of R row blocks, the
-// x slice of the chunk, the chunk's scales and zeros), so an SM has tens of KB
-// of HBM reads outstanding without spending registers on them.
+// Memory pipeline: every warp owns a ring of shared-memory stages (one row
+// tile x 128 columns of K each) and keeps all but one in flight with 16-byte
+// cp.async copies (L2 only): a warp-wide copy instruction moves 512
+// contiguous bytes of codes, so a stage costs the warp R x 2 code copies, one
+// x copy per two token rows and one scale (and zero) copy.  (On this part the
+// TMA bulk-copy engine was measured slower than cp.async for these small
+// per-warp stages.)  x rows sit at a 272-byte pitch, so that a warp's 8-byte
+// B-fragment loads take the minimum two wavefronts; token rows past M are
+// zeroed once and never copied.
 //
-// Work split (stream-K): the (row tile, K chunk) units are divided evenly over
-// a grid of exactly the resident CTAs.  A CTA's warps take interleaved chunks
-// of each tile segment, reduce through shared memory, and either store y
-// (whole tile) or leave an fp32 partial in the workspace; the last CTA to
-// finish a tile adds the partials in CTA order (deterministic) and stores y.
-// No CTA waits for another.
+// Work split (stream-K): the (row tile, K stage) units are divided evenly over
+// every warp of a grid of exactly the resident CTAs.  A warp whose range
+// covers a whole tile stores y; otherwise it leaves an fp32 partial in the
+// workspace and the last warp to finish the tile adds the partials in warp
+// order (deterministic) and stores y.  No warp waits for another.
 #include <algorithm>
 
 #include "common.cuh"
 #include "internal.h"
 
 namespace qk {
+
+// Device error word of the decode path.  Its waits are cp.async group waits,
+// which always end, so nothing sets it today; qmm_check_error reads it with
+// the tensor path's.
+__device__ unsigned g_skinny_error = 0;
+
 namespace {
 
 constexpr int kWarps = 8;
@@ -34,14 +44,14 @@ constexpr int kThreads = kWarps * 32;
 constexpr int kMaxDevices = 64;
 constexpr int kSC = 128;                 // K columns per stage (a "super-chunk"): 8 tiles of 16
 constexpr int kTiles = kSC / 16;
+constexpr int kXPitch = kSC * 2 + 16;    // bytes per x row in a stage (272: no bank conflicts)
 
-// Row blocks (16 rows) per tile: 2 for one token tile, 4 for two (keeps the
-// x bytes read per code byte at or below one).
+// Row blocks (16 rows) per tile.
 template <int NT>
-constexpr int rb_per_tile() { return NT == 1 ? 2 : 4; }
+constexpr int rb_per_tile() { return 2; }
 
 // Ring depth per warp (stages in flight = depth - 1), sized so that one token
-// tile fits two CTAs per SM and two token tiles one CTA per SM.
+// tile fits two CTAs per SM.
 template <int MODE, int NT>
 constexpr int ring_stages() { return (NT == 1 && MODE != kLUT) ? 3 : 2; }
 
@@ -57,15 +67,17 @@ struct SkinnyArgs {
   long long units;     // tiles * nsc
   int ctas;            // CTAs per slab
   int warps;           // stream-K workers per slab (<= 8 ctas)
-  float* slots;        // [slabs][2 * ctas][rows * tokens]: a CTA's first / last partial tile
+  double inv_units;     // 1 / units
+  double inv_warps;     // 1 / warps
+  float* slots;        // [slabs][2 * warps][rows * tokens]: a warp's first / last partial tile
   unsigned* counters;  // [slabs][tiles]
 };
 
 template <int MODE>
 constexpr size_t kTabBytes = MODE == kLUT ? 256 * 32 * 4 : 0;
 
-// Stage layout of one warp's ring slot: codes [R][CPS][512] | x [TOK][256 B]
-// (16-byte pieces swizzled by row) | scales [R][GPS][32 B] | zeros (ASYM).
+// Stage layout of one warp's ring slot: codes [R][CPS][512] | x [TOK][272]
+// | scales [R][GPS][32 B] | zeros (ASYM) [R][GPS][32 B].
 template <int BITS, int MODE, int NT, int TPG>
 struct Stage {
   static constexpr int R = rb_per_tile<NT>();
@@ -73,23 +85,41 @@ struct Stage {
   static constexpr int CPS = kSC / chunk_cols(BITS);   // chunks per stage
   static constexpr int GPS = kTiles / TPG;             // groups per stage
   static constexpr int X_OFF = R * CPS * 512;
-  static constexpr int S_OFF = X_OFF + TOK * kSC * 2;
+  static constexpr int S_OFF = X_OFF + TOK * kXPitch;
   static constexpr int Z_OFF = S_OFF + R * GPS * 32;
   static constexpr int BYTES = Z_OFF + (MODE == kASYM ? R * GPS * 32 : 0);
-  static constexpr int XPL = TOK * 16 / 32;           // x pieces per lane
-  static constexpr int SPL = (R * GPS * 2 + 31) / 32; // scale pieces per lane (upper bound)
+  static_assert(BYTES % 16 == 0, "stages must stay 16-byte aligned");
 };
 
-// CTA index of the stream-K range that holds unit u (ranges start at
-// floor(b * U / C)).
-__device__ __forceinline__ int owner_of(long long u, long long U, int C) {
-  return (int)(((u + 1) * (long long)C - 1) / U);
+// floor(a / d) for 0 <= a < 2^53, d > 0, from a double estimate (inv_d =
+// 1 / d) and exact integer corrections: 64-bit integer division is a long
+// software sequence on the GPU.
+__device__ __forceinline__ long long floor_div(long long a, long long d, double inv_d) {
+  long long q = (long long)((double)a * inv_d);
+  if (q * d > a) --q;
+  else if ((q + 1) * d <= a) ++q;
+  return q;
 }
 
+// Worker of the stream-K range that holds unit u (worker b's range starts at
+// floor(b U / W)): the largest b with b U < (u + 1) W.
+__device__ __forceinline__ int owner_of(long long u, long long U, long long W, double inv_U) {
+  return (int)floor_div((u + 1) * W - 1, U, inv_U);
+}
+
+// ---------------------------------------------------------------- PTX helpers
+
+__device__ __forceinline__ void sts128_zero(uint32_t a) {
+  asm volatile("st.shared.v4.u32 [%0], {%1,%1,%1,%1};" ::"r"(a), "r"(0u) : "memory");
+}
+// 16-byte asynchronous copy global -> shared, L2 only; `valid` false writes zeros.
 __device__ __forceinline__ void cp_async16(uint32_t saddr, const void* src, bool valid) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(saddr), "l"(src),
                "r"(valid ? 16 : 0)
                : "memory");
+}
+__device__ __forceinline__ void cp_async16_all(uint32_t saddr, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(saddr), "l"(src) : "memory");
 }
 __device__ __forceinline__ void cp_async_commit() {
   asm volatile("cp.async.commit_group;" ::: "memory");
@@ -119,153 +149,48 @@ __device__ __forceinline__ void mma_16816_first(float (&d)[4], const uint32_t (&
   }
 }
 
-// The CTA's unit range as tiles and super-chunks (computed once, 64-bit).
-struct Range {
-  int tb, sb;   // first tile, its first super-chunk
-  int te, se;   // tile holding the end, super-chunk where it ends (exclusive)
-  __device__ __forceinline__ int s0(int t) const { return t == tb ? sb : 0; }
-  __device__ __forceinline__ int s1(int t, int n) const { return t == te ? se : n; }
-  __device__ __forceinline__ bool has(int t) const { return t < te || (t == te && se > 0); }
-};
-
-// The super-chunks a warp processes, in order: in every tile segment
-// [s0, s1) of the CTA, s0 + w, s0 + w + 8, ...
-struct Seq {
-  int t, s;
-  __device__ __forceinline__ void norm(const Range& r, int n, int w) {
-    while (r.has(t) && s >= r.s1(t, n)) {
-      ++t;
-      s = r.s0(t) + w;
-    }
-  }
-  __device__ __forceinline__ void start(const Range& r, int n, int w) {
-    t = r.tb;
-    s = r.s0(t) + w;
-    norm(r, n, w);
-  }
-  __device__ __forceinline__ void next(const Range& r, int n, int w) {
-    s += kWarps;
-    norm(r, n, w);
-  }
-};
-
 template <int BITS, int MODE, bool BF16, int NT, int TPG>
 __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1) skinny_kernel(const SkinnyArgs a) {
   using St = Stage<BITS, MODE, NT, TPG>;
-  constexpr int kStages = ring_stages<MODE, NT>();
+  constexpr int S = ring_stages<MODE, NT>();
   constexpr int R = St::R;
   constexpr int TOK = St::TOK;
-  constexpr int NACC = R * NT * 4;        // fp32 values per lane per tile
   constexpr int CPS = St::CPS;
+  constexpr int GPS = St::GPS;
+  constexpr int NACC = R * NT * 4;        // fp32 values per lane per tile
 
-  extern __shared__ __align__(16) unsigned char smem[];
+  extern __shared__ __align__(128) unsigned char smem[];
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, t = lane & 3;
   const int slab = blockIdx.y;
   const int m_base = slab * TOK;
+  const int mrows = min(TOK, a.M - m_base);   // token rows of this slab (>= 1)
   const int n = a.nsc;
-  // this warp's stream-K range of (tile, super-chunk) units (64-bit, once)
+  // this warp's stream-K range of (tile, super-chunk) units
   const int gw = blockIdx.x * kWarps + warp;
   const long long W = a.warps;
-  Range rg;
-  {
-    const long long ub = (long long)gw * a.units / W;
-    const long long ue = (long long)(gw + 1) * a.units / W;
-    rg.tb = (int)(ub / n);
-    rg.sb = (int)(ub - (long long)rg.tb * n);
-    rg.te = (int)(ue / n);
-    rg.se = (int)(ue - (long long)rg.te * n);
+  long long ub = 0, ue = 0;
+  if (gw < W) {
+    ub = floor_div((long long)gw * a.units, W, a.inv_warps);
+    ue = floor_div((long long)(gw + 1) * a.units, W, a.inv_warps);
   }
   const int lg = a.lg;
 
   unsigned char* tabp = smem;
-  unsigned char* ring = smem + kTabBytes<MODE> + (size_t)warp * kStages * St::BYTES;
-  const uint32_t ring_s = static_cast<uint32_t>(__cvta_generic_to_shared(ring));
+  unsigned char* ring = smem + kTabBytes<MODE> + (size_t)warp * S * St::BYTES;
+  const uint32_t ring_s = smem_u32(ring);
 
-  // ---- lane-constant parts of the copies
-  const uint16_t* xsrc[St::XPL];
-  uint32_t xdst[St::XPL];
-  int xcol[St::XPL];
-  bool xrow_ok[St::XPL];
-#pragma unroll
-  for (int i = 0; i < St::XPL; ++i) {
-    const int q = lane + 32 * i, row = q >> 4, p = q & 15;
-    const int m = m_base + row;
-    xrow_ok[i] = m < a.M;
-    xcol[i] = p * 8;
-    xsrc[i] = a.x + (size_t)(xrow_ok[i] ? m : 0) * a.K + p * 8;
-    xdst[i] = St::X_OFF + row * (kSC * 2) + (((p & 8) | ((p ^ row) & 7)) << 4);
+  // ---- per-warp setup: stage barriers; token rows past M zeroed in every
+  // stage (they are never copied, and the fragment loads read all TOK rows)
+  for (int s = 0; s < S; ++s) {
+    const uint32_t xb = ring_s + s * St::BYTES + St::X_OFF + mrows * kXPitch;
+    for (int i = lane; i < (TOK - mrows) * (kXPitch / 16); i += 32) sts128_zero(xb + 16 * i);
   }
-  // scale / zero pieces: piece q = (r * GPS + k) * 2 + h
-  int sc_r[St::SPL], sc_k[St::SPL];
-  bool sc_on[St::SPL];
-  size_t sc_h8[St::SPL];
-#pragma unroll
-  for (int i = 0; i < St::SPL; ++i) {
-    const int q = lane + 32 * i;
-    sc_on[i] = q < R * St::GPS * 2;
-    sc_h8[i] = (size_t)(q & 1) * 8;
-    sc_k[i] = (q >> 1) % St::GPS;
-    sc_r[i] = (q >> 1) / St::GPS;
-  }
-  const int nsc_full = a.K / kSC;         // super-chunks with no column past K
+  __syncwarp();
 
   pdl_wait();                 // inputs of this call may come from the previous grid
   pdl_launch_dependents();    // let the next grid get resident while this one runs
-
-  // ---- prefetch state: per-tile base pointers, refreshed when the tile changes
-  const uint8_t* cbase[R];
-  bool rok[R];
-  const uint16_t* sbase[St::SPL];
-  bool srok[St::SPL];
-  int pf_tile = -1;
-  auto set_tile = [&](int tile) {
-    pf_tile = tile;
-#pragma unroll
-    for (int r = 0; r < R; ++r) {
-      const int rb = tile * R + r;
-      rok[r] = rb < a.nrb;
-      cbase[r] = a.qw + (rok[r] ? (size_t)rb * a.nchunks * 512 : 0) + lane * 16;
-    }
-#pragma unroll
-    for (int i = 0; i < St::SPL; ++i) {
-      const int rb = tile * R + sc_r[i];
-      srok[i] = sc_on[i] && rb < a.nrb;
-      sbase[i] = a.scales + (srok[i] ? (size_t)rb * a.G * 16 : 0) + sc_h8[i];
-    }
-  };
-  // ---- issue the loads of super-chunk (tile, sc) into ring stage `st`
-  auto issue = [&](int tile, int sc, int st) {
-    if (tile != pf_tile) set_tile(tile);
-    const uint32_t base = ring_s + st * St::BYTES;
-    const bool full = sc < nsc_full;
-#pragma unroll
-    for (int r = 0; r < R; ++r)
-#pragma unroll
-      for (int cc = 0; cc < CPS; ++cc) {
-        const int c = sc * CPS + cc;
-        cp_async16(base + (r * CPS + cc) * 512 + lane * 16, cbase[r] + (size_t)c * 512,
-                   rok[r] && (full || c < a.nchunks));
-      }
-    const int k0 = sc * kSC;
-#pragma unroll
-    for (int i = 0; i < St::XPL; ++i)
-      cp_async16(base + xdst[i], xsrc[i] + k0, xrow_ok[i] && (full || k0 + xcol[i] < a.K));
-    const int gi0 = lg < 0 ? 0 : (k0 >> lg);
-#pragma unroll
-    for (int i = 0; i < St::SPL; ++i) {
-      if (sc_on[i]) {
-        const int gi = gi0 + sc_k[i];
-        const bool ok = srok[i] && gi < a.G;
-        const size_t off = ok ? (size_t)gi * 16 : 0;
-        const int q = lane + 32 * i;
-        cp_async16(base + St::S_OFF + q * 16, sbase[i] + off, ok);
-        if constexpr (MODE == kASYM)
-          cp_async16(base + St::Z_OFF + q * 16, (sbase[i] - a.scales) + a.zl + off, ok);
-      }
-    }
-  };
 
   if constexpr (MODE == kLUT) {
     // Pair table, replicated so that every lane reads its own bank.
@@ -306,32 +231,116 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1) skinny_kernel(const
     __syncthreads();
   }
 
-  if (gw >= W) return;   // spare warps of the last CTA (plans with fewer workers)
-  if (rg.tb == rg.te && rg.sb == rg.se) return;   // no units (never planned)
+  if (ub >= ue) return;   // no units (spare warps of the last CTA)
 
-  // ---- prologue: kStages - 1 super-chunks in flight (the warp's own units,
-  // in order: consecutive super-chunks, then the next tile)
-  int pf_t = rg.tb, pf_s = rg.sb;
-  auto pf_valid = [&]() { return pf_t < rg.te || (pf_t == rg.te && pf_s < rg.se); };
+  const int nsc_full = a.K / kSC;         // super-chunks with no column past K
+
+  // ---- copies of super-chunk (tile, sc) into ring stage st with 16-byte
+  // cp.async pieces: per lane, R x CPS code pieces, one x piece per two token
+  // rows, one scale (and zero) piece
+  const int xrow0 = lane >> 4, xp = lane & 15;
+  const int xi_n = (mrows + 1) >> 1;                       // warp-uniform
+  const uint32_t xdst0 = St::X_OFF + xrow0 * kXPitch + xp * 16;
+  const uint16_t* xsrc[(TOK + 1) / 2];
+#pragma unroll
+  for (int i = 0; i < (TOK + 1) / 2; ++i) {
+    const int m = min(m_base + xrow0 + 2 * i, a.M - 1);
+    xsrc[i] = a.x + (size_t)m * a.K + xp * 8;
+  }
+  const bool sq_on = lane < R * GPS * 2;
+  const int sq_r = lane / (2 * GPS), sq_k = (lane >> 1) % GPS, sq_h = lane & 1;
+  const uint8_t* cbase[R];
+  bool rok[R];
+  bool tile_ok = true;
+  const uint16_t* sbase = a.scales;
+  bool srok = false;
+  int pf_tile = -1;
+  auto set_tile = [&](int tile) {
+    pf_tile = tile;
+    tile_ok = true;
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      const int rb = tile * R + r;
+      rok[r] = rb < a.nrb;
+      tile_ok = tile_ok && rok[r];
+      cbase[r] = a.qw + (size_t)(rok[r] ? rb : 0) * a.nchunks * 512 + lane * 16;
+    }
+    const int rbs = tile * R + sq_r;
+    srok = sq_on && rbs < a.nrb;
+    sbase = a.scales + (size_t)(srok ? rbs : 0) * a.G * 16 + sq_h * 8;
+  };
+  auto issue = [&](int tile, int sc, int st) {
+    if (tile != pf_tile) set_tile(tile);
+    const uint32_t base = ring_s + st * St::BYTES;
+    const bool full = sc < nsc_full;
+    if (tile_ok && full) {
+#pragma unroll
+      for (int r = 0; r < R; ++r) {
+        const uint8_t* src = cbase[r] + (size_t)sc * (CPS * 512);
+#pragma unroll
+        for (int cc = 0; cc < CPS; ++cc)
+          cp_async16_all(base + (r * CPS + cc) * 512 + lane * 16, src + cc * 512);
+      }
+    } else {
+#pragma unroll
+      for (int r = 0; r < R; ++r)
+#pragma unroll
+        for (int cc = 0; cc < CPS; ++cc) {
+          const int c = sc * CPS + cc;
+          const bool ok = rok[r] && c < a.nchunks;
+          cp_async16(base + (r * CPS + cc) * 512 + lane * 16, cbase[r] + (size_t)(ok ? c : 0) * 512, ok);
+        }
+    }
+    const int k0 = sc * kSC;
+    const bool xk = full || k0 + xp * 8 < a.K;
+#pragma unroll
+    for (int i = 0; i < (TOK + 1) / 2; ++i) {
+      if (i < xi_n) {   // warp-uniform
+        const bool ok = xrow0 + 2 * i < mrows && xk;
+        cp_async16(base + xdst0 + 2 * i * kXPitch, xsrc[i] + (ok ? k0 : 0), ok);
+      }
+    }
+    if (sq_on) {
+      const int gi = (lg < 0 ? 0 : (k0 >> lg)) + sq_k;
+      const bool ok = srok && gi < a.G;
+      const size_t off = ok ? (size_t)gi * 16 : 0;
+      cp_async16(base + St::S_OFF + lane * 16, sbase + off, ok);
+      if constexpr (MODE == kASYM)
+        cp_async16(base + St::Z_OFF + lane * 16, a.zl + (sbase - a.scales) + off, ok);
+    }
+  };
+
+  // ---- prologue: S - 1 super-chunks in flight (the warp's own units, in
+  // order: consecutive super-chunks, then the next tile)
+  long long pf_u = ub;
+  const int tb = (int)((unsigned)ub / (unsigned)n);   // the warp's first tile (ub < 2^31)
+  int pf_t = tb, pf_s = (int)(ub - (long long)tb * n);
   auto pf_next = [&]() {
+    ++pf_u;
     if (++pf_s == n) {
       pf_s = 0;
       ++pf_t;
     }
   };
 #pragma unroll
-  for (int s = 0; s < kStages - 1; ++s) {
-    if (pf_valid()) {
+  for (int s = 0; s < S - 1; ++s) {
+    if (pf_u < ue) {
       issue(pf_t, pf_s, s);
       pf_next();
     }
     cp_async_commit();
   }
 
+  int tile = tb, sc = (int)(ub - (long long)tb * n);
+  long long u = ub;
   int st_c = 0;                          // ring stage being computed
-  int st_f = kStages - 1;                // ring stage being filled
-  for (int tile = rg.tb; rg.has(tile); ++tile) {
-    const int s0 = rg.s0(tile), s1 = rg.s1(tile, n);
+  int st_f = S - 1;                      // ring stage being filled
+
+  while (u < ue) {
+    // this warp's segment of the tile: super-chunks [s0, s1)
+    const int s0 = sc;
+    const long long tile_end = (long long)(tile + 1) * n;
+    const int s1 = (int)((ue < tile_end ? ue : tile_end) - (long long)tile * n);
 
     float acc[R][NT][4];
 #pragma unroll
@@ -341,31 +350,40 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1) skinny_kernel(const
 #pragma unroll
         for (int i = 0; i < 4; ++i) acc[r][nt][i] = 0.0f;
 
-    for (int sc = s0; sc < s1; ++sc) {
+    for (; sc < s1; ++sc, ++u) {
       // keep the ring full: the stage refilled here was drained last iteration
-      if (pf_valid()) {
+      if (pf_u < ue) {
         issue(pf_t, pf_s, st_f);
         pf_next();
       }
       cp_async_commit();
-      cp_async_wait<kStages - 1>();
+      cp_async_wait<S - 1>();
       __syncwarp();
 
       const unsigned char* st = ring + st_c * St::BYTES;
+      const bool full = sc < nsc_full;   // else the stage holds only its first 64 columns
+
+      // B fragments (tokens) of the eight tiles.  The packed layout gives lane
+      // (g, t) the columns 4t .. 4t + 3 of each 16-column tile (the MMA's k
+      // order permuted the same way for both operands), so its b0, b1 are the
+      // 8 contiguous bytes at column 16 j + 4 t of token row g.
+      uint32_t xf[kTiles][NT][2];
+      {
+        const unsigned char* xa = st + St::X_OFF + g * kXPitch + 8 * t;
+#pragma unroll
+        for (int j = 0; j < kTiles; ++j)
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt) {
+            const uint2 v = *reinterpret_cast<const uint2*>(xa + nt * 8 * kXPitch + 32 * j);
+            xf[j][nt][0] = v.x;
+            xf[j][nt][1] = v.y;
+          }
+      }
       float gacc[R][NT][4];
       uint4 cw[R];
 
 #pragma unroll
       for (int j = 0; j < kTiles; ++j) {
-        uint2 xf[NT];
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-          const int row = g + 8 * nt;
-          const int p = 2 * j + (t >> 1);
-          const int phys = (p & 8) | ((p ^ g) & 7);
-          xf[nt] = *reinterpret_cast<const uint2*>(st + St::X_OFF + row * (kSC * 2) + phys * 16 +
-                                                   8 * (t & 1));
-        }
         const int grp = j / TPG;            // group within the stage (compile-time)
         // the lane's 16 code bytes of chunk j / 4 (4-bit) or of the stage (2-bit)
         if ((BITS == 4 && (j & 3) == 0) || j == 0) {
@@ -374,75 +392,78 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1) skinny_kernel(const
             cw[r] = *reinterpret_cast<const uint4*>(st + (r * CPS + (BITS == 4 ? (j >> 2) : 0)) * 512 +
                                                     lane * 16);
         }
+        if (full || j < 4) {
 #pragma unroll
-        for (int r = 0; r < R; ++r) {
-          uint32_t af[4], aflo[4];
-          if constexpr (BITS == 4) {
-            // tile j: chunk j / 4 of the stage, word j % 4 of the lane
-            const uint32_t w = (&cw[r].x)[j & 3];
-            if constexpr (MODE == kSYM) {
-              decode_int4<BF16, 8>(w, af);
-            } else if constexpr (MODE == kASYM) {
-              decode_int4<BF16, 0>(w, af);
-              uint32_t zw = *reinterpret_cast<const uint32_t*>(st + St::Z_OFF +
-                                                               (r * St::GPS + grp) * 32 + 4 * g);
-              if constexpr (BF16) {
-                const float2 zf = __half22float2(*reinterpret_cast<const __half2*>(&zw));
-                zw = pack2<true>(zf.x, zf.y);
+          for (int r = 0; r < R; ++r) {
+            uint32_t af[4], aflo[4];
+            if constexpr (BITS == 4) {
+              // tile j: chunk j / 4 of the stage, word j % 4 of the lane
+              const uint32_t w = (&cw[r].x)[j & 3];
+              if constexpr (MODE == kSYM) {
+                decode_int4<BF16, 8>(w, af);
+              } else if constexpr (MODE == kASYM) {
+                decode_int4<BF16, 0>(w, af);
+                uint32_t zw = *reinterpret_cast<const uint32_t*>(st + St::Z_OFF +
+                                                                 (r * GPS + grp) * 32 + 4 * g);
+                if constexpr (BF16) {
+                  const float2 zf = __half22float2(*reinterpret_cast<const __half2*>(&zw));
+                  zw = pack2<true>(zf.x, zf.y);
+                }
+                sub_zero<BF16>(__byte_perm(zw, 0, 0x1010), __byte_perm(zw, 0, 0x3232), af);
+              } else if constexpr (!BF16) {
+                const uint32_t l4 = (uint32_t)lane << 2;
+                af[0] = *reinterpret_cast<const uint32_t*>(tabp + lop3_and_or(w << 7, 0x7F80u, l4));
+                af[1] = *reinterpret_cast<const uint32_t*>(tabp + lop3_and_or(w >> 1, 0x7F80u, l4));
+                af[2] = *reinterpret_cast<const uint32_t*>(tabp + lop3_and_or(w >> 9, 0x7F80u, l4));
+                af[3] = *reinterpret_cast<const uint32_t*>(tabp + lop3_and_or(w >> 17, 0x7F80u, l4));
+              } else {
+                // (hi, lo) per pair: 8-byte entries, 16 copies
+                const uint32_t l8 = (uint32_t)(lane & 15) << 3;
+                const uint2 e0 = *reinterpret_cast<const uint2*>(tabp + lop3_and_or(w << 7, 0x7F80u, l8));
+                const uint2 e1 = *reinterpret_cast<const uint2*>(tabp + lop3_and_or(w >> 1, 0x7F80u, l8));
+                const uint2 e2 = *reinterpret_cast<const uint2*>(tabp + lop3_and_or(w >> 9, 0x7F80u, l8));
+                const uint2 e3 = *reinterpret_cast<const uint2*>(tabp + lop3_and_or(w >> 17, 0x7F80u, l8));
+                af[0] = e0.x; af[1] = e1.x; af[2] = e2.x; af[3] = e3.x;
+                aflo[0] = e0.y; aflo[1] = e1.y; aflo[2] = e2.y; aflo[3] = e3.y;
               }
-              sub_zero<BF16>(__byte_perm(zw, 0, 0x1010), __byte_perm(zw, 0, 0x3232), af);
-            } else if constexpr (!BF16) {
-              const uint32_t l4 = (uint32_t)lane << 2;
-              af[0] = *reinterpret_cast<const uint32_t*>(tabp + lop3_and_or(w << 7, 0x7F80u, l4));
-              af[1] = *reinterpret_cast<const uint32_t*>(tabp + lop3_and_or(w >> 1, 0x7F80u, l4));
-              af[2] = *reinterpret_cast<const uint32_t*>(tabp + lop3_and_or(w >> 9, 0x7F80u, l4));
-              af[3] = *reinterpret_cast<const uint32_t*>(tabp + lop3_and_or(w >> 17, 0x7F80u, l4));
             } else {
-              // (hi, lo) per pair: 8-byte entries, 16 copies
-              const uint32_t l8 = (uint32_t)(lane & 15) << 3;
-              const uint2 e0 = *reinterpret_cast<const uint2*>(tabp + lop3_and_or(w << 7, 0x7F80u, l8));
-              const uint2 e1 = *reinterpret_cast<const uint2*>(tabp + lop3_and_or(w >> 1, 0x7F80u, l8));
-              const uint2 e2 = *reinterpret_cast<const uint2*>(tabp + lop3_and_or(w >> 9, 0x7F80u, l8));
-              const uint2 e3 = *reinterpret_cast<const uint2*>(tabp + lop3_and_or(w >> 17, 0x7F80u, l8));
-              af[0] = e0.x; af[1] = e1.x; af[2] = e2.x; af[3] = e3.x;
-              aflo[0] = e0.y; aflo[1] = e1.y; aflo[2] = e2.y; aflo[3] = e3.y;
+              // 2-bit LUT: word j/2 of the lane, bytes 2 (j % 2) and 2 (j % 2) + 1
+              const uint32_t w = (&cw[r].x)[j >> 1];
+              const int sh = 16 * (j & 1);
+              const uint32_t s0w = sh >= 7 ? (w >> (sh - 7)) : (w << 7);
+              const uint32_t s1w = w >> (sh + 1);
+              if constexpr (!BF16) {
+                const uint32_t l8 = (uint32_t)(lane & 15) << 3;
+                const uint2 e0 = *reinterpret_cast<const uint2*>(tabp + lop3_and_or(s0w, 0x7F80u, l8));
+                const uint2 e1 = *reinterpret_cast<const uint2*>(tabp + lop3_and_or(s1w, 0x7F80u, l8));
+                af[0] = e0.x; af[1] = e0.y; af[2] = e1.x; af[3] = e1.y;
+              } else {
+                // (hi hi, lo lo) per byte: 16-byte entries, 8 copies
+                const uint32_t l16 = (uint32_t)(lane & 7) << 4;
+                const uint4 e0 = *reinterpret_cast<const uint4*>(tabp + lop3_and_or(s0w, 0x7F80u, l16));
+                const uint4 e1 = *reinterpret_cast<const uint4*>(tabp + lop3_and_or(s1w, 0x7F80u, l16));
+                af[0] = e0.x; af[1] = e0.y; af[2] = e1.x; af[3] = e1.y;
+                aflo[0] = e0.z; aflo[1] = e0.w; aflo[2] = e1.z; aflo[3] = e1.w;
+              }
             }
-          } else {
-            // 2-bit LUT: word j/2 of the lane, bytes 2 (j % 2) and 2 (j % 2) + 1
-            const uint32_t w = (&cw[r].x)[j >> 1];
-            const int sh = 16 * (j & 1);
-            const uint32_t s0w = sh >= 7 ? (w >> (sh - 7)) : (w << 7);
-            const uint32_t s1w = w >> (sh + 1);
-            if constexpr (!BF16) {
-              const uint32_t l8 = (uint32_t)(lane & 15) << 3;
-              const uint2 e0 = *reinterpret_cast<const uint2*>(tabp + lop3_and_or(s0w, 0x7F80u, l8));
-              const uint2 e1 = *reinterpret_cast<const uint2*>(tabp + lop3_and_or(s1w, 0x7F80u, l8));
-              af[0] = e0.x; af[1] = e0.y; af[2] = e1.x; af[3] = e1.y;
-            } else {
-              // (hi hi, lo lo) per byte: 16-byte entries, 8 copies
-              const uint32_t l16 = (uint32_t)(lane & 7) << 4;
-              const uint4 e0 = *reinterpret_cast<const uint4*>(tabp + lop3_and_or(s0w, 0x7F80u, l16));
-              const uint4 e1 = *reinterpret_cast<const uint4*>(tabp + lop3_and_or(s1w, 0x7F80u, l16));
-              af[0] = e0.x; af[1] = e0.y; af[2] = e1.x; af[3] = e1.y;
-              aflo[0] = e0.z; aflo[1] = e0.w; aflo[2] = e1.z; aflo[3] = e1.w;
-            }
-          }
 #pragma unroll
-          for (int nt = 0; nt < NT; ++nt) {
-            if (j % TPG == 0)
-              mma_16816_first<BF16>(gacc[r][nt], af, xf[nt].x, xf[nt].y);
-            else
-              mma_16816<BF16>(gacc[r][nt], af, xf[nt].x, xf[nt].y);
-            if constexpr (MODE == kLUT && BF16) mma_16816<BF16>(gacc[r][nt], aflo, xf[nt].x, xf[nt].y);
+            for (int nt = 0; nt < NT; ++nt) {
+              if (j % TPG == 0)
+                mma_16816_first<BF16>(gacc[r][nt], af, xf[j][nt][0], xf[j][nt][1]);
+              else
+                mma_16816<BF16>(gacc[r][nt], af, xf[j][nt][0], xf[j][nt][1]);
+              if constexpr (MODE == kLUT && BF16)
+                mma_16816<BF16>(gacc[r][nt], aflo, xf[j][nt][0], xf[j][nt][1]);
+            }
           }
         }
-        // the group ends after this tile (position fixed at compile time):
-        // fold the group's sums into acc with its scales
-        if ((j + 1) % TPG == 0) {
+        // the group ends after this tile (position fixed at compile time): fold
+        // its sums into acc with its scales (a group wholly past K is skipped)
+        if ((j + 1) % TPG == 0 && (full || j + 1 - TPG < 4)) {
 #pragma unroll
           for (int r = 0; r < R; ++r) {
             const uint32_t sw = *reinterpret_cast<const uint32_t*>(st + St::S_OFF +
-                                                                   (r * St::GPS + grp) * 32 + 4 * g);
+                                                                   (r * GPS + grp) * 32 + 4 * g);
             const float2 s = __half22float2(*reinterpret_cast<const __half2*>(&sw));
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) {
@@ -455,22 +476,25 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1) skinny_kernel(const
         }
       }
       __syncwarp();   // every lane is done with this stage before it is refilled
-      st_c = st_c + 1 == kStages ? 0 : st_c + 1;
-      st_f = st_f + 1 == kStages ? 0 : st_f + 1;
+      st_c = st_c + 1 == S ? 0 : st_c + 1;
+      st_f = st_f + 1 == S ? 0 : st_f + 1;
     }
 
     // ---- this warp's result for the tile segment: store y (whole tile) or
     // hand a partial to the last warp that finishes the tile
     const bool whole = s0 == 0 && s1 == n;
     float* outv = &acc[0][0][0];
+    bool store = true;
     if (!whole) {
       const long long t_first = (long long)tile * n;
-      const int first = owner_of(t_first, a.units, (int)W);
-      const int nb = owner_of(t_first + n - 1, a.units, (int)W) - first + 1;
-      const int first_e = ((long long)first * a.units / W < t_first) ? 1 : 0;
+      const int first = owner_of(t_first, a.units, W, a.inv_units);
+      const int nb = owner_of(t_first + n - 1, a.units, W, a.inv_units) - first + 1;
+      // `first` started before this tile (its range start floor(first U / W)
+      // is below t_first) exactly when first U < t_first W
+      const int first_e = ((long long)first * a.units < t_first * W) ? 1 : 0;
       // slot 2 gw + e, e = 1 when the tile is not the warp's first; of the
       // contributors only `first` can have e = 1
-      const int e = (tile == rg.tb) ? 0 : 1;
+      const int e = (tile == tb) ? 0 : 1;
       float* slots = a.slots + (size_t)slab * 2 * W * (NACC * 32);
       float4* mine = reinterpret_cast<float4*>(slots + (size_t)(2 * gw + e) * (NACC * 32) + lane * NACC);
 #pragma unroll
@@ -482,54 +506,61 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1) skinny_kernel(const
       if (lane == 0)
         asm volatile("atom.add.acq_rel.gpu.u32 %0, [%1], 1;" : "=r"(prev) : "l"(counter) : "memory");
       prev = __shfl_sync(0xffffffffu, prev, 0);
-      if (prev != (unsigned)(nb - 1)) continue;
+      if (prev != (unsigned)(nb - 1)) {
+        store = false;
+      } else {
 #pragma unroll
-      for (int i = 0; i < NACC; ++i) outv[i] = 0.0f;
-      for (int k0 = 0; k0 < nb; k0 += 4) {
-        float4 v[4][NACC / 4];
+        for (int i = 0; i < NACC; ++i) outv[i] = 0.0f;
+        for (int k0 = 0; k0 < nb; k0 += 4) {
+          float4 v[4][NACC / 4];
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-          const int k = k0 + kk;
-          if (k < nb) {
-            const float4* src = reinterpret_cast<const float4*>(
-                slots + (size_t)(2 * (first + k) + (k == 0 ? first_e : 0)) * (NACC * 32) + lane * NACC);
+          for (int kk = 0; kk < 4; ++kk) {
+            const int k = k0 + kk;
+            if (k < nb) {
+              const float4* src = reinterpret_cast<const float4*>(
+                  slots + (size_t)(2 * (first + k) + (k == 0 ? first_e : 0)) * (NACC * 32) + lane * NACC);
 #pragma unroll
-            for (int i = 0; i < NACC / 4; ++i) v[kk][i] = __ldcg(src + i);
+              for (int i = 0; i < NACC / 4; ++i) v[kk][i] = __ldcg(src + i);
+            }
           }
-        }
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-          if (k0 + kk < nb) {
+          for (int kk = 0; kk < 4; ++kk) {
+            if (k0 + kk < nb) {
 #pragma unroll
-            for (int i = 0; i < NACC / 4; ++i) {
-              outv[4 * i] += v[kk][i].x;
-              outv[4 * i + 1] += v[kk][i].y;
-              outv[4 * i + 2] += v[kk][i].z;
-              outv[4 * i + 3] += v[kk][i].w;
+              for (int i = 0; i < NACC / 4; ++i) {
+                outv[4 * i] += v[kk][i].x;
+                outv[4 * i + 1] += v[kk][i].y;
+                outv[4 * i + 2] += v[kk][i].z;
+                outv[4 * i + 3] += v[kk][i].w;
+              }
             }
           }
         }
+        if (lane == 0) *counter = 0u;   // ready for the next call
       }
-      if (lane == 0) *counter = 0u;   // ready for the next call
     }
-    // fragment (r, nt, i) of this lane: row (tile R + r) 16 + g + 8 (i / 2),
-    // token m_base + 8 nt + 2 t + (i % 2)
+    if (store) {
+      // fragment (r, nt, i) of this lane: row (tile R + r) 16 + g + 8 (i / 2),
+      // token m_base + 8 nt + 2 t + (i % 2)
 #pragma unroll
-    for (int r = 0; r < R; ++r)
+      for (int r = 0; r < R; ++r)
 #pragma unroll
-      for (int nt = 0; nt < NT; ++nt)
+        for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int row = (tile * R + r) * 16 + g + 8 * (i >> 1);
-          const int m = m_base + 8 * nt + 2 * t + (i & 1);
-          if (row < a.N && m < a.M) {
-            const float v = acc[r][nt][i];
-            if constexpr (BF16)
-              a.y[(size_t)m * a.N + row] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
-            else
-              a.y[(size_t)m * a.N + row] = __half_as_ushort(__float2half_rn(v));
+          for (int i = 0; i < 4; ++i) {
+            const int row = (tile * R + r) * 16 + g + 8 * (i >> 1);
+            const int m = m_base + 8 * nt + 2 * t + (i & 1);
+            if (row < a.N && m < a.M) {
+              const float v = acc[r][nt][i];
+              if constexpr (BF16)
+                a.y[(size_t)m * a.N + row] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
+              else
+                a.y[(size_t)m * a.N + row] = __half_as_ushort(__float2half_rn(v));
+            }
           }
-        }
+    }
+    ++tile;
+    sc = 0;
   }
   cp_async_wait<0>();   // nothing may still land in shared memory after exit
 }
@@ -537,7 +568,8 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1) skinny_kernel(const
 template <int BITS, int MODE, int NT, int TPG>
 constexpr size_t smem_bytes() {
   using St = Stage<BITS, MODE, NT, TPG>;
-  return kTabBytes<MODE> + (size_t)kWarps * ring_stages<MODE, NT>() * St::BYTES;
+  constexpr int S = ring_stages<MODE, NT>();
+  return kTabBytes<MODE> + (size_t)kWarps * S * St::BYTES;
 }
 
 // Opts the kernel into `smem` bytes of dynamic shared memory (once per device)
@@ -583,7 +615,6 @@ cudaError_t launch(const SkinnyArgs& args, int slabs, cudaStream_t stream) {
   if (e != cudaSuccess) cudaGetLastError();   // report it once, here
   return e;
 }
-
 // Calls f.template operator()<BITS, MODE, BF16, NT, TPG>() for the runtime values.
 template <int B, int MO, bool BF, int T, class F>
 auto dispatch_tpg(int tpg, F&& f) {
@@ -618,7 +649,7 @@ int tiles_per_group(int group) { return (group == -1 || group >= kSC) ? 8 : grou
 SkinnyPlan plan_skinny(int M, int N, int K, int bits, int group, int mode, bool bf16, int sms) {
   SkinnyPlan p{};
   p.nt = M <= 8 ? 1 : 2;
-  const int R = p.nt == 1 ? 2 : 4;
+  const int R = p.nt == 1 ? rb_per_tile<1>() : rb_per_tile<2>();
   p.rows = 16 * R;
   const int nrb = N / 16;
   p.tiles_n = (nrb + R - 1) / R;
@@ -672,6 +703,8 @@ cudaError_t launch_skinny(const Problem& pr, const SkinnyPlan& plan, void* works
   a.units = (long long)plan.tiles_n * a.nsc;
   a.ctas = plan.splits;
   a.warps = plan.warps;
+  a.inv_units = 1.0 / (double)a.units;
+  a.inv_warps = 1.0 / (double)a.warps;
   if (plan.ws_bytes) {
     const size_t counters = ((size_t)plan.slabs * plan.tiles_n * sizeof(unsigned) + 255) / 256 * 256;
     a.counters = reinterpret_cast<unsigned*>(workspace);
@@ -754,7 +787,10 @@ cudaError_t launch_skinny_static(const Problem& pr, int sms, cudaStream_t stream
 }  // namespace qk
 
 namespace qk {
-// The decode path waits on nothing but its own cp.async groups (hardware
-// waits that always end): it has no bounded wait that could give up.
-unsigned skinny_read_and_clear_error() { return 0; }
+unsigned skinny_read_and_clear_error() {
+  unsigned v = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&v, g_skinny_error, sizeof(v)) != cudaSuccess) return 0xFFFFFFFFu;
+  if (v) cudaMemcpyToSymbol(g_skinny_error, &zero, sizeof(zero));
+  return v;
+}
 }  // namespace qk
