@@ -46,7 +46,10 @@ WORKLOADS = {
     "gateup_m1": ("sym", 4, 128, "f16", [(4096, 22016)], [1]),
     "gateup_m16": ("sym", 4, 128, "f16", [(4096, 22016)], [16]),
     "prefill_m64": ("sym", 4, 128, "f16", [(4096, 11008)], [64]),
+    "prefill_m256": ("sym", 4, 128, "f16", [(4096, 11008)], [256]),
+    "prefill_m1024": ("sym", 4, 128, "f16", [(4096, 11008)], [1024]),
     "prefill_m4096": ("sym", 4, 128, "f16", [(4096, 11008)], [4096]),
+    "prefill_m4096_rowscale": ("sym", 4, -1, "f16", [(4096, 11008)], [4096]),
     "llama70b_asym_bf16": ("asym", 4, 128, "bf16",
                            [(8192, 10240), (8192, 57344), (28672, 8192)], [1, 16]),
     "lut4_nf4": ("lut", 4, 64, "f16", [(4096, 14336)], [1, 8]),
