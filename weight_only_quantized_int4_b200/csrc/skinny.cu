@@ -16,9 +16,10 @@
 // contiguous bytes of codes, so a stage costs the warp R x 2 code copies, one
 // x copy per two token rows and one scale (and zero) copy.  (On this part the
 // TMA bulk-copy engine was measured slower than cp.async for these small
-// per-warp stages.)  x rows sit at a 272-byte pitch, so that a warp's 8-byte
-// B-fragment loads take the minimum two wavefronts; token rows past M are
-// zeroed once and never copied.
+// per-warp stages.)  x rows sit at a 288-byte pitch (72 words: rows g and
+// g + 1 start 8 banks apart), so that the 8-byte B-fragment loads of each
+// half-warp (rows g .. g + 3, 32 bytes per row) hit 32 distinct banks; token
+// rows past M are zeroed once and never copied.
 //
 // Work split (stream-K): the (row tile, K stage) units are divided evenly over
 // every warp of a grid of exactly the resident CTAs.  A warp whose range
@@ -44,7 +45,7 @@ constexpr int kThreads = kWarps * 32;
 constexpr int kMaxDevices = 64;
 constexpr int kSC = 128;                 // K columns per stage (a "super-chunk"): 8 tiles of 16
 constexpr int kTiles = kSC / 16;
-constexpr int kXPitch = kSC * 2 + 16;    // bytes per x row in a stage (272: no bank conflicts)
+constexpr int kXPitch = kSC * 2 + 32;    // bytes per x row in a stage (288: rows 8 banks apart)
 
 // Row blocks (16 rows) per tile.
 template <int NT>

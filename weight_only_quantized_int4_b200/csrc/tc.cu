@@ -320,11 +320,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const unsigned char* tabp = sT;
     // Group scales (and ASYM zero-points) of the lane's rows g and g + 8 in its
     // two row blocks, one word per 16-column slice of the k block, read from
-    // global memory one k block ahead so that the loads overlap a decode.
+    // global memory two k blocks ahead so that the loads overlap decodes.
     constexpr bool kScales = !GM1;
     constexpr bool kZeros = MODE == kASYM;
-    uint32_t sw_n[2][4] = {}, zw_n[2][4] = {};
-    auto load_meta = [&](int tl, int k) {
+    uint32_t sw_n[2][4] = {}, zw_n[2][4] = {};     // unit u + 1
+    uint32_t sw_nn[2][4] = {}, zw_nn[2][4] = {};   // unit u + 2
+    auto load_meta = [&](int tl, int k, uint32_t (&sw_o)[2][4], uint32_t (&zw_o)[2][4]) {
       if constexpr (kScales || kZeros) {
         const int tn = tl % a.tiles_n;
 #pragma unroll
@@ -336,15 +337,25 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             const int gi = (k * kKB + 16 * j) >> a.lg;
             const size_t off = ((size_t)rb * a.G + gi) * 16 + 2 * g;
             if constexpr (kScales)
-              sw_n[rr][j] = in ? __ldg(reinterpret_cast<const unsigned int*>(a.scales + off)) : 0u;
+              sw_o[rr][j] = in ? __ldg(reinterpret_cast<const unsigned int*>(a.scales + off)) : 0u;
             if constexpr (kZeros)
-              zw_n[rr][j] = in ? __ldg(reinterpret_cast<const unsigned int*>(a.zl + off)) : 0u;
+              zw_o[rr][j] = in ? __ldg(reinterpret_cast<const unsigned int*>(a.zl + off)) : 0u;
           }
         }
       }
     };
-    int ct = (int)(u_begin / a.nkb), ck = (int)(u_begin % a.nkb);   // unit u = ct nkb + ck
-    if (u_begin < u_end) load_meta(ct, ck);
+    // (ct, ck): the unit two ahead of the one being decoded, u = ct nkb + ck
+    int ct = (int)(u_begin / a.nkb), ck = (int)(u_begin % a.nkb);
+    auto advance = [&]() {
+      if (++ck == a.nkb) {
+        ck = 0;
+        ++ct;
+      }
+    };
+    if (u_begin < u_end) load_meta(ct, ck, sw_n, zw_n);
+    advance();
+    if (u_begin + 1 < u_end) load_meta(ct, ck, sw_nn, zw_nn);
+    advance();
     int kc = 0, ks = 0;
     for (long long u = u_begin; u < u_end && !*abort_flag; ++u, ++kc, ++ks) {
       uint32_t sw[2][4], zw[2][4];
@@ -354,12 +365,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         for (int j = 0; j < 4; ++j) {
           sw[rr][j] = sw_n[rr][j];
           zw[rr][j] = zw_n[rr][j];
+          sw_n[rr][j] = sw_nn[rr][j];
+          zw_n[rr][j] = zw_nn[rr][j];
         }
-      if (++ck == a.nkb) {
-        ck = 0;
-        ++ct;
-      }
-      if (u + 1 < u_end) load_meta(ct, ck);
+      if (u + 2 < u_end) load_meta(ct, ck, sw_nn, zw_nn);
+      advance();
       const int c = kc % kCodeStages, s = ks % S;
       if (!mbar_wait(&code_full[c], (kc / kCodeStages) & 1, abort_flag) ||
           !mbar_wait(&ab_empty[s], ((ks / S) & 1) ^ 1, abort_flag))
