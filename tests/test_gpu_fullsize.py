@@ -26,6 +26,9 @@ CONFIGS = {
     "lut2": ("lut", 2, 64, "f16", [(4096, 14336)], [1, 8, 32]),
     "prefill_gm1": ("sym", 4, -1, "f16", [(4096, 11008)], [64, 256, 1024, 4096]),
     "prefill_g128": ("sym", 4, 128, "f16", [(4096, 11008)], [64, 256, 1024, 4096]),
+    # the largest K and N the packed layout accepts (2^20), each with the
+    # smallest other dimension: 8192 K stages in one row tile, 65536 row blocks
+    "max_sizes": ("sym", 4, 128, "f16", [(1 << 20, 16), (128, 1 << 20)], [1, 16, 64]),
 }
 
 
