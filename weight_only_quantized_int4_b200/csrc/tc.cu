@@ -9,11 +9,11 @@
 //
 // per 64-column K block, with A = decoded weights (fp16/bf16, written into
 // shared memory in the 128-byte-swizzled K-major layout by decode warps) and
-// B = a TMA-loaded tile of x.  Warp roles (10 warps):
+// B = a TMA-loaded tile of x.  Warp roles:
 //   warp 0      TMA producer: code tiles (4 KB, 8 row blocks) and x tiles
 //   warp 1      TMEM owner and MMA issuer (one elected thread)
-//   warps 2-5   decode: codes (smem) -> (q - z) s, T[q] s -> A tile (smem)
-//   warps 6-9   epilogue: TMEM -> registers -> y (or split-K partials)
+//   next kDecWarps warps   decode: codes (smem) -> (q - z) s, T[q] s -> A tile
+//   last 4 warps           epilogue: TMEM -> registers -> y (or split-K partials)
 // Work is split stream-K over (tile, K block) units across a grid of one CTA
 // per SM, like the decode path; partial tiles are reduced deterministically by
 // the last CTA that finishes them.  Every mbarrier wait is bounded: a wait
@@ -33,7 +33,10 @@ __device__ unsigned g_tc_error = 0;
 
 namespace {
 
-constexpr int kTcThreads = 320;
+constexpr int kDecWarps = 4;                        // decode warps (8 row blocks between them)
+constexpr int kRbPerDec = 8 / kDecWarps;            // row blocks per decode warp
+constexpr int kTcThreads = 32 * (2 + kDecWarps + 4);
+constexpr int kEpi0 = 32 * (2 + kDecWarps);          // first epilogue thread
 constexpr int kKB = 64;             // K columns per stage (one 128-byte swizzle row of fp16)
 constexpr int kRowsTile = 128;      // weight rows per tile (UMMA M)
 constexpr int kCodeStages = 8;
@@ -209,11 +212,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   if (threadIdx.x == 0) {
     for (int i = 0; i < kCodeStages; ++i) {
       mbar_init(&code_full[i], 1);
-      mbar_init(&code_empty[i], 4);
+      mbar_init(&code_empty[i], kDecWarps);
     }
     for (int i = 0; i < S; ++i) {
       mbar_init(&b_full[i], 1);
-      mbar_init(&a_full[i], 4);
+      mbar_init(&a_full[i], kDecWarps);
       mbar_init(&ab_empty[i], 1);
     }
     for (int i = 0; i < 2; ++i) {
@@ -313,9 +316,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         u += kb1 - kb0;
       }
     }
-  } else if (warp < 6) {
+  } else if (warp < 2 + kDecWarps) {
     // ------------------------------------------------------------ decode warps
-    const int dw = warp - 2;                 // row blocks 2dw, 2dw + 1 of the tile
+    const int dw = warp - 2;                 // row blocks kRbPerDec dw + rr of the tile
     const int g = lane >> 2, t = lane & 3;
     const unsigned char* tabp = sT;
     // Group scales (and ASYM zero-points) of the lane's rows g and g + 8 in its
@@ -323,14 +326,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     // global memory two k blocks ahead so that the loads overlap decodes.
     constexpr bool kScales = !GM1;
     constexpr bool kZeros = MODE == kASYM;
-    uint32_t sw_n[2][4] = {}, zw_n[2][4] = {};     // unit u + 1
-    uint32_t sw_nn[2][4] = {}, zw_nn[2][4] = {};   // unit u + 2
-    auto load_meta = [&](int tl, int k, uint32_t (&sw_o)[2][4], uint32_t (&zw_o)[2][4]) {
+    uint32_t sw_n[kRbPerDec][4] = {}, zw_n[kRbPerDec][4] = {};     // unit u + 1
+    uint32_t sw_nn[kRbPerDec][4] = {}, zw_nn[kRbPerDec][4] = {};   // unit u + 2
+    auto load_meta = [&](int tl, int k, uint32_t (&sw_o)[kRbPerDec][4], uint32_t (&zw_o)[kRbPerDec][4]) {
       if constexpr (kScales || kZeros) {
         const int tn = tl % a.tiles_n;
 #pragma unroll
-        for (int rr = 0; rr < 2; ++rr) {
-          const int rb = tn * 8 + 2 * dw + rr;
+        for (int rr = 0; rr < kRbPerDec; ++rr) {
+          const int rb = tn * 8 + kRbPerDec * dw + rr;
           const bool in = rb < a.nrb;
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
@@ -358,9 +361,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     advance();
     int kc = 0, ks = 0;
     for (long long u = u_begin; u < u_end && !*abort_flag; ++u, ++kc, ++ks) {
-      uint32_t sw[2][4], zw[2][4];
+      uint32_t sw[kRbPerDec][4], zw[kRbPerDec][4];
 #pragma unroll
-      for (int rr = 0; rr < 2; ++rr)
+      for (int rr = 0; rr < kRbPerDec; ++rr)
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           sw[rr][j] = sw_n[rr][j];
@@ -376,8 +379,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         break;
       unsigned char* At = sA + s * kATileBytes;
 #pragma unroll
-      for (int rr = 0; rr < 2; ++rr) {
-        const int rbl = 2 * dw + rr;                       // row block in the tile
+      for (int rr = 0; rr < kRbPerDec; ++rr) {
+        const int rbl = kRbPerDec * dw + rr;               // row block in the tile
         const uint4 wv = *reinterpret_cast<const uint4*>(sC + c * kCodeBytes + rbl * 512 + lane * 16);
         const int R0 = rbl * 16 + g, R1 = R0 + 8;
 #pragma unroll
@@ -467,7 +470,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       if (!whole) {
         const int e = (tile == (int)(u_begin / a.nkb)) ? 0 : 1;
         slot = a.slots + (size_t)(2 * b + e) * (size_t)(BN * kRowsTile) + (size_t)row_l * BN;
-        if (threadIdx.x == 192) {     // 64-bit stream-K bookkeeping, once
+        if (threadIdx.x == kEpi0) {     // 64-bit stream-K bookkeeping, once
           const int first = owner_of_tc(t_first, a.units, a.ctas);
           meta[0] = first;
           meta[1] = owner_of_tc(t_first + a.nkb - 1, a.units, a.ctas) - first + 1;
@@ -500,7 +503,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       if (!whole) {
         // every epilogue thread's slot stores, then one release increment
         named_bar(1, 128);
-        if (threadIdx.x == 192) {
+        if (threadIdx.x == kEpi0) {
           unsigned prev;
           asm volatile("atom.add.acq_rel.gpu.u32 %0, [%1], 1;"
                        : "=r"(prev)
@@ -554,7 +557,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
               }
             }
           }
-          if (threadIdx.x == 192) a.counters[tile] = 0u;   // ready for the next call
+          if (threadIdx.x == kEpi0) a.counters[tile] = 0u;   // ready for the next call
         }
         named_bar(1, 128);   // last_flag / meta are reused by the next segment
       }
