@@ -177,6 +177,35 @@ int qmm_noalloc(const void* x, int xdtype, const void* qweight, const uint16_t* 
                 const uint16_t* zeros_or_lut, int M, int N, int K, int bits, int group, int mode,
                 void* y, void* stream);
 
+/* Fused feed-forward gate: the GPTQ-Triton summary ("How It Works") fuses
+ * the FFN layers into the quantized matmul.  For a LLaMA-style FFN with gate
+ * and up projections Wg, Wu [I, K]:
+ *
+ *     y[M, I] = silu(x . dequant(Wg)^T) * (x . dequant(Wu)^T),  silu(v) = v / (1 + e^-v)
+ *
+ * in one pass over the codes of both matrices.
+ *
+ * qmm_pack_gated packs Wg and Wu (device, fp32 [I, K] row-major each, 16-byte
+ * aligned) as one [2I, K] matrix in the layout of qmm_pack whose 16-row blocks
+ * alternate: packed block 2b is rows 16b .. 16b + 15 of Wg, block 2b + 1 the
+ * same rows of Wu.  Quantization is per row as in qmm_pack, so the codes,
+ * scales and zeros equal those qmm_pack writes for that interleaved matrix.
+ * Buffer sizes: qmm_packed_size(2 I, K, ...).  I must be a multiple of 16.
+ *
+ * qmm_gated runs the product on such a buffer (qweight, scales, zeros_or_lut
+ * as written by qmm_pack_gated; I as given to it) and writes y [M, I] (same
+ * dtype as x, must not overlap x); the sums are fp32 and the gate, the SiLU
+ * and the product are taken in fp32 before the single rounding to y's type.
+ * Workspace: qmm_workspace_size(M, 2 I, K, bits, group, mode) bytes, same
+ * rules as qmm (NULL / 0 allowed).  Paths and statuses are those of qmm on
+ * the [2I, K] problem. */
+int qmm_pack_gated(const float* Wg, const float* Wu, int I, int K, int mode, int bits, int group,
+                   const uint16_t* lut, void* qweight, uint16_t* scales, uint16_t* zeros,
+                   void* stream);
+int qmm_gated(const void* x, int xdtype, const void* qweight, const uint16_t* scales,
+              const uint16_t* zeros_or_lut, int M, int I, int K, int bits, int group, int mode,
+              void* y, void* workspace, size_t workspace_bytes, void* stream);
+
 /* Decode the packed weights into W_out[N, K] row-major (fp16 or bf16 by
  * out_dtype): W_out = round_to_nearest_even((q - z) * s) (SYM z = 8) or
  * round(T[q] * s), the product taken exactly in fp32 (exact for integer

@@ -54,6 +54,7 @@ def _load():
             lib.oracle_round.argtypes = [P, S, I, P]
             lib.oracle_widen.argtypes = [P, S, I, P]
             lib.oracle_qmm.argtypes = [P, I, P, P, P, I, I, I, I, I, I, I, I, P]
+            lib.oracle_qmm_gated.argtypes = [P, I, P, P, P, I, I, I, I, I, I, I, I, P]
             lib.oracle_packed_bytes.argtypes = [I, I, I]
             lib.oracle_packed_bytes.restype = S
             _lib = lib
@@ -156,6 +157,21 @@ def qmm(x, xdtype, qweight, scales_p, zeros_or_lut, M, N, K, mode, bits, group,
     y = np.empty((M, n1 - n0), np.float64)
     _check(_load().oracle_qmm(_p(x), DTYPES[xdtype], _p(qweight), _p(sp), _p(zl), M, N, K,
                               MODES[mode], bits, group, n0, n1, _p(y)), "oracle_qmm")
+    return y
+
+
+def qmm_gated(x, xdtype, qweight, scales_p, zeros_or_lut, M, I, K, mode, bits, group,
+              i0=0, i1=None):
+    """silu(gate) * up [M, i1 - i0] (float64) from a gated packed buffer (2I rows
+    whose 16-row blocks alternate gate, up), for outputs [i0, i1)."""
+    i1 = I if i1 is None else i1
+    x = np.ascontiguousarray(x, dtype=np.uint16)
+    qweight = np.ascontiguousarray(qweight, dtype=np.uint8)
+    sp = np.ascontiguousarray(scales_p, dtype=np.uint16)
+    zl = None if zeros_or_lut is None else np.ascontiguousarray(zeros_or_lut, dtype=np.uint16)
+    y = np.empty((M, i1 - i0), np.float64)
+    _check(_load().oracle_qmm_gated(_p(x), DTYPES[xdtype], _p(qweight), _p(sp), _p(zl), M, I, K,
+                                    MODES[mode], bits, group, i0, i1, _p(y)), "oracle_qmm_gated")
     return y
 
 

@@ -363,6 +363,22 @@ int oracle_widen(const uint16_t* in, size_t n, int dtype, double* out) {
   return OK;
 }
 
+// W~[n, k] for k = 0 .. K-1 of packed row n, into w.
+static void dequant_row(int n, const uint8_t* qweight, const uint16_t* scales_p,
+                        const uint16_t* zeros_or_lut, int K, int mode, int bits, int G, int L,
+                        double* w) {
+  for (int k = 0; k < K; ++k) {
+    size_t byte;
+    int shift;
+    code_place(n, k, K, mode, bits, &byte, &shift);
+    int q = (qweight[byte] >> shift) & ((1 << bits) - 1);
+    int gi = k / L;
+    double s = half_value(scales_p[scale_index(n, gi, G)]);
+    double z = (mode == MODE_ASYM) ? half_value(zeros_or_lut[scale_index(n, gi, G)]) : 0.0;
+    w[k] = decode(q, s, z, zeros_or_lut, mode);
+  }
+}
+
 // y[m, n] = sum_k x[m, k] * W~[n, k] for output columns n in [n0, n1), read
 // straight from the packed buffers ([GT] decode-then-multiply, [EX] the
 // activations stay in their fp16/bf16 input precision).  The sum runs over k in
@@ -379,16 +395,7 @@ int oracle_qmm(const uint16_t* x, int xdtype, const uint8_t* qweight, const uint
   for (size_t i = 0; i < (size_t)M * K; ++i)
     xv[i] = xdtype == DT_BF16 ? bf16_value(x[i]) : half_value(x[i]);
   for (int n = n0; n < n1; ++n) {
-    for (int k = 0; k < K; ++k) {
-      size_t byte;
-      int shift;
-      code_place(n, k, K, mode, bits, &byte, &shift);
-      int q = (qweight[byte] >> shift) & ((1 << bits) - 1);
-      int gi = k / L;
-      double s = half_value(scales_p[scale_index(n, gi, G)]);
-      double z = (mode == MODE_ASYM) ? half_value(zeros_or_lut[scale_index(n, gi, G)]) : 0.0;
-      w[k] = decode(q, s, z, zeros_or_lut, mode);
-    }
+    dequant_row(n, qweight, scales_p, zeros_or_lut, K, mode, bits, G, L, w);
     for (int m = 0; m < M; ++m) {
       double acc = 0.0;
       for (int k = 0; k < K; ++k) acc += xv[(size_t)m * K + k] * w[k];
@@ -397,6 +404,46 @@ int oracle_qmm(const uint16_t* x, int xdtype, const uint8_t* qweight, const uint
   }
   delete[] xv;
   delete[] w;
+  return OK;
+}
+
+// Fused feed-forward gate ([GT] "How It Works": the FFN layers are fused into
+// the quantized matmul).  The packed matrix has 2I rows whose 16-row blocks
+// alternate gate and up: output i reads gate row 32 (i / 16) + i % 16 and the
+// up row 16 below it.  y[m, i] = silu(g) * u with g, u the two rows' sums as in
+// oracle_qmm and silu(v) = v / (1 + exp(-v)), all in double; outputs
+// i in [i0, i1), y is [M, i1 - i0] row-major.
+int oracle_qmm_gated(const uint16_t* x, int xdtype, const uint8_t* qweight,
+                     const uint16_t* scales_p, const uint16_t* zeros_or_lut, int M, int I, int K,
+                     int mode, int bits, int group, int i0, int i1, double* y) {
+  if (!x || !qweight || !scales_p || !y || M < 0 || I <= 0 || I % 16 || i0 < 0 || i1 > I ||
+      i0 > i1)
+    return ERR_ARG;
+  const int N = 2 * I;
+  if (!shape_ok(N, K, mode, bits, group)) return ERR_ARG;
+  if (mode != MODE_SYM && !zeros_or_lut) return ERR_ARG;
+  const int G = n_groups(K, group), L = group_len(K, group);
+  double* xv = new double[(size_t)M * K];
+  double* wg = new double[(size_t)K];
+  double* wu = new double[(size_t)K];
+  for (size_t i = 0; i < (size_t)M * K; ++i)
+    xv[i] = xdtype == DT_BF16 ? bf16_value(x[i]) : half_value(x[i]);
+  for (int i = i0; i < i1; ++i) {
+    const int ng = 32 * (i / 16) + i % 16, nu = ng + 16;
+    dequant_row(ng, qweight, scales_p, zeros_or_lut, K, mode, bits, G, L, wg);
+    dequant_row(nu, qweight, scales_p, zeros_or_lut, K, mode, bits, G, L, wu);
+    for (int m = 0; m < M; ++m) {
+      double g = 0.0, u = 0.0;
+      for (int k = 0; k < K; ++k) {
+        g += xv[(size_t)m * K + k] * wg[k];
+        u += xv[(size_t)m * K + k] * wu[k];
+      }
+      y[(size_t)m * (i1 - i0) + (i - i0)] = g / (1.0 + std::exp(-g)) * u;
+    }
+  }
+  delete[] xv;
+  delete[] wg;
+  delete[] wu;
   return OK;
 }
 

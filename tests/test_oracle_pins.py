@@ -395,3 +395,52 @@ def test_tables():
     assert np.array_equal(t, -t[::-1])
     t2 = h2f(synth.lut2_table(0))
     assert np.all(np.diff(t2) > 0) and np.max(np.abs(t2)) == 1.0
+
+
+# ------------------------------------------------- fused feed-forward gate
+
+def _negate_f16(x):
+    """-x for fp16 bit patterns (flip the sign bit: exact)."""
+    return (np.asarray(x, np.uint16) ^ np.uint16(0x8000)).astype(np.uint16)
+
+
+@pytest.mark.parametrize("mode,bits,group", [("sym", 4, 128), ("asym", 4, 64), ("lut", 4, 64)])
+def test_gated_odd_even_identity(mode, bits, group):
+    """silu(g) u + silu(-g) (-u) = g u for any g, u (silu(v) - silu(-v) = v), so
+    gated(x) + gated(-x) equals the product of the plain sums of the gate and
+    up rows.  The interleave (which packed rows are the gate and the up rows of
+    output i) and the composition are checked against the pinned plain oracle;
+    the exponential cancels out."""
+    M, I, K = 3, 32, 256
+    p = _problem(mode, bits, group, M, 2 * I, K, 21)
+    x = p["x"]
+    g_plus = oracle.qmm_gated(x, "f16", p["qw"], p["sp"], p["zl"], M, I, K, mode, bits, group)
+    g_minus = oracle.qmm_gated(_negate_f16(x), "f16", p["qw"], p["sp"], p["zl"], M, I, K, mode,
+                               bits, group)
+    y = oracle.qmm(x, "f16", p["qw"], p["sp"], p["zl"], M, 2 * I, K, mode, bits, group)
+    gate = np.concatenate([y[:, 32 * b: 32 * b + 16] for b in range(I // 16)], axis=1)
+    up = np.concatenate([y[:, 32 * b + 16: 32 * b + 32] for b in range(I // 16)], axis=1)
+    assert np.allclose(g_plus + g_minus, gate * up, rtol=1e-9, atol=1e-12)
+
+
+def test_gated_gate_and_up_roles():
+    """Gate rows with a large negative sum switch the output off (silu -> 0);
+    a large positive one passes the up sum through (silu(v) -> v); a zero gate
+    gives exactly 0.  Swapping gate and up would break each of these."""
+    I, K, g = 48, 128, 128
+    x = oracle.round_to(np.ones((1, K)), "f16")
+    codes = np.full((2 * I, K), 8, np.uint8)
+    blocks = [slice(32 * b, 32 * b + 16) for b in range(I // 16)]
+    ups = [slice(32 * b + 16, 32 * b + 32) for b in range(I // 16)]
+    codes[blocks[0]] = 0          # outputs 0..15: gate sum -8 K s = -1024 s
+    codes[blocks[1]] = 15         # outputs 16..31: gate sum +7 K s
+    codes[blocks[2]] = 8          # outputs 32..47: gate sum 0
+    for u in ups:
+        codes[u] = 11             # up sum +3 K s
+    scales = np.full((2 * I, 1), 0x3C00, np.uint16)     # s = 1
+    qw, sp, _ = oracle.pack(codes, scales, None, "sym", 4, g)
+    y = oracle.qmm_gated(x, "f16", qw, sp, None, 1, I, K, "sym", 4, g)[0]
+    up = 3.0 * K
+    assert np.all(np.abs(y[0:16]) < 1e-300 * up + 1e-200)          # silu(-1024) ~ -1024 e^-1024
+    assert np.allclose(y[16:32], 7.0 * K * up, rtol=1e-12)         # silu(896) = 896 (to 1e-300)
+    assert np.all(y[32:48] == 0.0)

@@ -28,7 +28,8 @@ PATH_NAMES = {1: "skinny", 2: "tensor"}
 
 SYMBOLS = ("qmm_packed_size", "qmm_pack", "qmm_workspace_size", "qmm_workspace_size_for", "qmm",
            "qmm_with_path",
-           "qmm_path", "qmm_dequant", "qmm_check_error", "qmm_strerror", "qmm_noalloc")
+           "qmm_path", "qmm_dequant", "qmm_check_error", "qmm_strerror", "qmm_noalloc",
+           "qmm_pack_gated", "qmm_gated")
 
 _lib = None
 _lock = threading.Lock()
@@ -61,6 +62,8 @@ def load(path: str = LIB_PATH):
             lib.qmm_with_path.argtypes = [P, I, P, P, P, I, I, I, I, I, I, P, P, S, P, I]
             lib.qmm_path.argtypes = [I, I, I, I, I, I]
             lib.qmm_noalloc.argtypes = [P, I, P, P, P, I, I, I, I, I, I, P, P]
+            lib.qmm_pack_gated.argtypes = [P, P, I, I, I, I, I, P, P, P, P, P]
+            lib.qmm_gated.argtypes = [P, I, P, P, P, I, I, I, I, I, I, P, P, S, P]
             lib.qmm_dequant.argtypes = [P, P, P, I, I, I, I, I, I, P, P]
             lib.qmm_check_error.argtypes = [P]
             lib.qmm_strerror.argtypes = [I]
@@ -116,6 +119,40 @@ def pack(W, mode, bits=4, group=128, lut=None, out=None):
     _check(load().qmm_pack(_ptr(W), N, K, MODES[mode], bits, group, _ptr(lut), _ptr(qw),
                            _ptr(sc), _ptr(ze), _stream()), "qmm_pack")
     return qw, sc, ze
+
+
+def pack_gated(Wg, Wu, mode, bits=4, group=128, lut=None):
+    """Quantize the FFN gate and up projections (fp32 [I, K] each, CUDA) into
+    one packed [2I, K] buffer with alternating 16-row gate / up blocks."""
+    _dev(Wg, "Wg")
+    _dev(Wu, "Wu")
+    I, K = Wg.shape
+    if tuple(Wu.shape) != (I, K):
+        raise ValueError("Wg and Wu must have the same shape")
+    qb, sb, zb = packed_size(2 * I, K, mode, bits, group)
+    qw = torch.empty(qb, dtype=torch.uint8, device=Wg.device)
+    sc = torch.empty(sb // 2, dtype=torch.int16, device=Wg.device)
+    ze = torch.empty(zb // 2, dtype=torch.int16, device=Wg.device) if zb else None
+    _check(load().qmm_pack_gated(_ptr(Wg), _ptr(Wu), I, K, MODES[mode], bits, group, _ptr(lut),
+                                 _ptr(qw), _ptr(sc), _ptr(ze), _stream()), "qmm_pack_gated")
+    return qw, sc, ze
+
+
+def qmm_gated(x, qweight, scales, zeros_or_lut, I, K, mode, bits=4, group=128, y=None, ws=None):
+    """y[M, I] = silu(x . dequant(Wg)^T) * (x . dequant(Wu)^T) on a pack_gated buffer."""
+    _dev(x, "x")
+    if x.dtype not in DTYPES:
+        raise ValueError("x must be fp16 or bf16")
+    M = x.shape[0]
+    if x.shape[1] != K:
+        raise ValueError("x.shape[1] != K")
+    if y is None:
+        y = torch.empty(M, I, dtype=x.dtype, device=x.device)
+    nbytes = 0 if ws is None else ws.numel() * ws.element_size()
+    _check(load().qmm_gated(_ptr(x), DTYPES[x.dtype], _ptr(qweight), _ptr(scales),
+                            _ptr(zeros_or_lut), M, I, K, bits, group, MODES[mode], _ptr(y),
+                            _ptr(ws), nbytes, _stream()), "qmm_gated")
+    return y
 
 
 def workspace_size(M, N, K, mode, bits=4, group=128, path="auto"):

@@ -72,6 +72,52 @@ Plan make_plan(int M, int N, int K, int bits, int group, int mode, bool bf16, in
 
 using namespace qk;
 
+static int run_qmm(const void* x, int xdtype, const void* qweight, const uint16_t* scales,
+                   const uint16_t* zeros_or_lut, int M, int N, int K, int bits, int group,
+                   int mode, void* y, void* workspace, size_t workspace_bytes, void* stream,
+                   int path, bool gated) {
+  if (M < 0) return QMM_ERR_ARG;
+  int st = check_shape(N, K, bits, group, mode);
+  if (st != QMM_OK) return st;
+  if (xdtype != QMM_F16 && xdtype != QMM_BF16) return QMM_ERR_ARG;
+  if (path != QMM_PATH_AUTO && path != QMM_PATH_SKINNY && path != QMM_PATH_TENSOR)
+    return QMM_ERR_ARG;
+  if (M == 0) return QMM_OK;
+  if (!x || !qweight || !scales || !y) return QMM_ERR_ARG;
+  if (mode != QMM_SYM && !zeros_or_lut) return QMM_ERR_ARG;
+  if (!aligned(x, 16) || !aligned(qweight, 16) || !aligned(scales, 16) || !aligned(y, 2) ||
+      (mode == QMM_ASYM && !aligned(zeros_or_lut, 16)) || (workspace && !aligned(workspace, 256)))
+    return QMM_ERR_ALIGN;
+  {
+    const char* xb = static_cast<const char*>(x);
+    const char* yb = static_cast<const char*>(y);
+    const size_t xs = (size_t)M * K * 2, ys = (size_t)M * (gated ? N / 2 : N) * 2;
+    if (xb < yb + ys && yb < xb + xs) return QMM_ERR_ARG;   // y overlaps x
+  }
+  Problem p{x, xdtype == QMM_BF16, qweight, scales, zeros_or_lut, M, N, K, bits, group, mode, y};
+  p.gated = gated;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  Plan plan = make_plan(M, N, K, bits, group, mode, xdtype == QMM_BF16, path);
+  if (plan.ws_bytes()) {
+    if (!workspace) {
+      // no workspace: every CTA owns whole tiles over all of K, no partial sums
+      if (plan.path == QMM_PATH_TENSOR) {
+        plan.tc.ctas = plan.tc.tiles_n * plan.tc.tiles_m;
+        plan.tc.ws_bytes = 0;
+      } else {
+        plan.sk.warps = plan.sk.tiles_n;
+        plan.sk.splits = (plan.sk.tiles_n + 7) / 8;
+        plan.sk.ws_bytes = 0;
+      }
+    } else if (workspace_bytes < plan.ws_bytes()) {
+      return QMM_ERR_WORKSPACE;
+    }
+  }
+  if (plan.path == QMM_PATH_TENSOR) return status_of(launch_tc(p, plan.tc, workspace, s));
+  return status_of(launch_skinny(p, plan.sk, workspace, s));
+}
+
+
 extern "C" {
 
 size_t qmm_packed_size(int N, int K, int bits, int group, int mode, size_t* scales_bytes,
@@ -93,7 +139,24 @@ int qmm_pack(const float* W, int N, int K, int mode, int bits, int group, const 
   if (!aligned(W, 16) || !aligned(qweight, 16) || !aligned(scales, 16) ||
       (zeros && !aligned(zeros, 16)))
     return QMM_ERR_ALIGN;
-  return status_of(launch_pack(W, N, K, mode, bits, group, lut, qweight, scales, zeros,
+  return status_of(launch_pack(W, nullptr, N, K, mode, bits, group, lut, qweight, scales, zeros,
+                               static_cast<cudaStream_t>(stream)));
+}
+
+int qmm_pack_gated(const float* Wg, const float* Wu, int I, int K, int mode, int bits, int group,
+                   const uint16_t* lut, void* qweight, uint16_t* scales, uint16_t* zeros,
+                   void* stream) {
+  if (I <= 0 || I > (1 << 19)) return I <= 0 ? QMM_ERR_ARG : QMM_ERR_UNSUPPORTED;
+  int st = check_shape(2 * I, K, bits, group, mode);
+  if (st != QMM_OK) return st;
+  if (I % 16 != 0) return QMM_ERR_UNSUPPORTED;
+  if (!Wg || !Wu || !qweight || !scales) return QMM_ERR_ARG;
+  if (mode == QMM_ASYM && !zeros) return QMM_ERR_ARG;
+  if (mode == QMM_LUT && !lut) return QMM_ERR_ARG;
+  if (!aligned(Wg, 16) || !aligned(Wu, 16) || !aligned(qweight, 16) || !aligned(scales, 16) ||
+      (zeros && !aligned(zeros, 16)))
+    return QMM_ERR_ALIGN;
+  return status_of(launch_pack(Wg, Wu, 2 * I, K, mode, bits, group, lut, qweight, scales, zeros,
                                static_cast<cudaStream_t>(stream)));
 }
 
@@ -120,44 +183,17 @@ int qmm_with_path(const void* x, int xdtype, const void* qweight, const uint16_t
                   const uint16_t* zeros_or_lut, int M, int N, int K, int bits, int group,
                   int mode, void* y, void* workspace, size_t workspace_bytes, void* stream,
                   int path) {
-  if (M < 0) return QMM_ERR_ARG;
-  int st = check_shape(N, K, bits, group, mode);
-  if (st != QMM_OK) return st;
-  if (xdtype != QMM_F16 && xdtype != QMM_BF16) return QMM_ERR_ARG;
-  if (path != QMM_PATH_AUTO && path != QMM_PATH_SKINNY && path != QMM_PATH_TENSOR)
-    return QMM_ERR_ARG;
-  if (M == 0) return QMM_OK;
-  if (!x || !qweight || !scales || !y) return QMM_ERR_ARG;
-  if (mode != QMM_SYM && !zeros_or_lut) return QMM_ERR_ARG;
-  if (!aligned(x, 16) || !aligned(qweight, 16) || !aligned(scales, 16) || !aligned(y, 2) ||
-      (mode == QMM_ASYM && !aligned(zeros_or_lut, 16)) || (workspace && !aligned(workspace, 256)))
-    return QMM_ERR_ALIGN;
-  {
-    const char* xb = static_cast<const char*>(x);
-    const char* yb = static_cast<const char*>(y);
-    const size_t xs = (size_t)M * K * 2, ys = (size_t)M * N * 2;
-    if (xb < yb + ys && yb < xb + xs) return QMM_ERR_ARG;   // y overlaps x
-  }
-  Problem p{x, xdtype == QMM_BF16, qweight, scales, zeros_or_lut, M, N, K, bits, group, mode, y};
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  Plan plan = make_plan(M, N, K, bits, group, mode, xdtype == QMM_BF16, path);
-  if (plan.ws_bytes()) {
-    if (!workspace) {
-      // no workspace: every CTA owns whole tiles over all of K, no partial sums
-      if (plan.path == QMM_PATH_TENSOR) {
-        plan.tc.ctas = plan.tc.tiles_n * plan.tc.tiles_m;
-        plan.tc.ws_bytes = 0;
-      } else {
-        plan.sk.warps = plan.sk.tiles_n;
-        plan.sk.splits = (plan.sk.tiles_n + 7) / 8;
-        plan.sk.ws_bytes = 0;
-      }
-    } else if (workspace_bytes < plan.ws_bytes()) {
-      return QMM_ERR_WORKSPACE;
-    }
-  }
-  if (plan.path == QMM_PATH_TENSOR) return status_of(launch_tc(p, plan.tc, workspace, s));
-  return status_of(launch_skinny(p, plan.sk, workspace, s));
+  return run_qmm(x, xdtype, qweight, scales, zeros_or_lut, M, N, K, bits, group, mode, y,
+                 workspace, workspace_bytes, stream, path, false);
+}
+
+int qmm_gated(const void* x, int xdtype, const void* qweight, const uint16_t* scales,
+              const uint16_t* zeros_or_lut, int M, int I, int K, int bits, int group, int mode,
+              void* y, void* workspace, size_t workspace_bytes, void* stream) {
+  if (I <= 0) return QMM_ERR_ARG;
+  if (I % 16 != 0 || I > (1 << 19)) return QMM_ERR_UNSUPPORTED;
+  return run_qmm(x, xdtype, qweight, scales, zeros_or_lut, M, 2 * I, K, bits, group, mode, y,
+                 workspace, workspace_bytes, stream, QMM_PATH_AUTO, true);
 }
 
 int qmm(const void* x, int xdtype, const void* qweight, const uint16_t* scales,

@@ -151,6 +151,9 @@ __device__ __forceinline__ void fence_proxy_async() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// SiLU (x times the logistic sigmoid of x) of the fused FFN gate.
+__device__ __forceinline__ float silu(float v) { return v / (1.0f + __expf(-v)); }
+
 // ------------------------------------------------------------- code decoding
 //
 // One 32-bit word of a 4-bit SYM/ASYM chunk holds a lane's 8 codes of one

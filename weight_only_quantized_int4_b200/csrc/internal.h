@@ -17,6 +17,7 @@ struct Problem {
   const uint16_t* zl;     // zeros (ASYM) or table (LUT)
   int M, N, K, bits, group, mode;
   void* y;
+  bool gated = false;     // fused gate/up rows: y[M, N/2] = silu(gate) * up
 };
 
 // Split-K plan of the skinny (M <= 16 per slab) decode path.
@@ -52,9 +53,9 @@ TcPlan plan_tc(int M, int N, int K, int sms);
 cudaError_t launch_tc(const Problem& p, const TcPlan& plan, void* workspace, cudaStream_t stream);
 unsigned tc_read_and_clear_error();
 
-cudaError_t launch_pack(const float* W, int N, int K, int mode, int bits, int group,
-                        const uint16_t* lut, void* qweight, uint16_t* scales, uint16_t* zeros,
-                        cudaStream_t stream);
+cudaError_t launch_pack(const float* W, const float* W2, int N, int K, int mode, int bits,
+                        int group, const uint16_t* lut, void* qweight, uint16_t* scales,
+                        uint16_t* zeros, cudaStream_t stream);
 cudaError_t launch_dequant(const void* qweight, const uint16_t* scales,
                            const uint16_t* zeros_or_lut, int N, int K, int bits, int group,
                            int mode, int out_dtype, void* W_out, cudaStream_t stream);

@@ -32,17 +32,27 @@ __device__ __forceinline__ uint16_t scale_to_half(float s32) {
   return b;
 }
 
+// Source row of packed row n.  With a second matrix W2 (the gated layout),
+// 16-row blocks alternate: packed block 2b is block b of W, block 2b + 1 is
+// block b of W2.
+__device__ __forceinline__ const float* src_row(const float* W, const float* W2, int n, int K) {
+  if (!W2) return W + (size_t)n * K;
+  const int b = n >> 4;
+  return ((b & 1) ? W2 : W) + (size_t)((b >> 1) * 16 + (n & 15)) * K;
+}
+
 // One warp per (row n, group gi): reduce |w| or (min, max) over the group,
 // write the fp16 scale (and zero) at the packed position.
-__global__ void __launch_bounds__(256) pack_scales_kernel(const float* __restrict__ W, int N, int K,
+__global__ void __launch_bounds__(256) pack_scales_kernel(const float* __restrict__ W,
+                                                          const float* __restrict__ W2, int N, int K,
                                                           int mode, int L, int G,
                                                           uint16_t* __restrict__ scales,
                                                           uint16_t* __restrict__ zeros) {
-  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const long long warp = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
-  if (warp >= N * G) return;
-  const int n = warp / G, gi = warp % G;
-  const float* w = W + (size_t)n * K + (size_t)gi * L;
+  if (warp >= (long long)N * G) return;
+  const int n = (int)(warp / G), gi = (int)(warp % G);
+  const float* w = src_row(W, W2, n, K) + (size_t)gi * L;
   float amax = 0.0f, mn = INFINITY, mx = -INFINITY;
   for (int i = lane; i < L; i += 32) {
     float v = w[i];
@@ -72,6 +82,7 @@ __global__ void __launch_bounds__(256) pack_scales_kernel(const float* __restric
 
 struct CodeCtx {
   const float* W;
+  const float* W2;   // gated layout: the second matrix (else null)
   int K, mode, bits, L, G, nchunks;
   const uint16_t* scales;
   const uint16_t* zeros;
@@ -121,7 +132,7 @@ __global__ void __launch_bounds__(256) pack_codes_kernel(CodeCtx c, uint32_t* __
       const size_t sidx = ((size_t)rb * c.G + gi) * 16 + scale_slot(g + 8 * h);
       const float s = __half2float(__ushort_as_half(c.scales[sidx]));
       const float z = c.mode == kASYM ? __half2float(__ushort_as_half(c.zeros[sidx])) : 0.0f;
-      const float4 wv = *reinterpret_cast<const float4*>(c.W + (size_t)n * c.K + k0);
+      const float4 wv = *reinterpret_cast<const float4*>(src_row(c.W, c.W2, n, c.K) + k0);
       const float wc[4] = {wv.x, wv.y, wv.z, wv.w};
       for (int cc = 0; cc < 4; ++cc) {
         const uint32_t q = (uint32_t)encode(wc[cc], s, z, c, lut);
@@ -199,18 +210,19 @@ __global__ void __launch_bounds__(256) dequant_kernel(const uint32_t* __restrict
 
 }  // namespace
 
-cudaError_t launch_pack(const float* W, int N, int K, int mode, int bits, int group,
-                        const uint16_t* lut, void* qweight, uint16_t* scales, uint16_t* zeros,
-                        cudaStream_t stream) {
+cudaError_t launch_pack(const float* W, const float* W2, int N, int K, int mode, int bits,
+                        int group, const uint16_t* lut, void* qweight, uint16_t* scales,
+                        uint16_t* zeros, cudaStream_t stream) {
   const int L = group == -1 ? K : group;
   const int G = K / L;
-  const int warps = N * G;
-  pack_scales_kernel<<<(warps * 32 + 255) / 256, 256, 0, stream>>>(W, N, K, mode, L, G, scales,
-                                                                   zeros);
+  const long long warps = (long long)N * G;
+  pack_scales_kernel<<<(unsigned)((warps * 32 + 255) / 256), 256, 0, stream>>>(
+      W, W2, N, K, mode, L, G, scales, zeros);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   CodeCtx c;
   c.W = W;
+  c.W2 = W2;
   c.K = K;
   c.mode = mode;
   c.bits = bits;

@@ -49,7 +49,7 @@ constexpr int kXPitch = kSC * 2 + 32;    // bytes per x row in a stage (288: row
 
 // Row blocks (16 rows) per tile.
 template <int NT>
-constexpr int rb_per_tile() { return 2; }
+constexpr int rb_per_tile() { return 2; }   // the fused gate / up epilogue relies on 2
 
 // Ring depth per warp (stages in flight = depth - 1), sized so that one token
 // tile fits two CTAs per SM.
@@ -64,6 +64,7 @@ struct SkinnyArgs {
   uint16_t* y;
   int M, N, K, G, nchunks, nrb, tiles, nsc;
   int lg;              // log2 of the group length; -1 for one group per row
+  int gated;           // 1: rows are alternating 16-row gate / up blocks, y[M, N/2] = silu(gate) up
   int stage_bytes;     // bytes of one ring stage
   long long units;     // tiles * nsc
   int ctas;            // CTAs per slab
@@ -541,24 +542,44 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1) skinny_kernel(const
       }
     }
     if (store) {
-      // fragment (r, nt, i) of this lane: row (tile R + r) 16 + g + 8 (i / 2),
-      // token m_base + 8 nt + 2 t + (i % 2)
-#pragma unroll
-      for (int r = 0; r < R; ++r)
+      if (a.gated) {
+        // the tile's two row blocks are gate block `tile` (r = 0) and up block
+        // `tile` (r = 1): each lane holds both values of its outputs
+        const int ny = a.N >> 1;
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
-            const int row = (tile * R + r) * 16 + g + 8 * (i >> 1);
+            const int col = tile * 16 + g + 8 * (i >> 1);
             const int m = m_base + 8 * nt + 2 * t + (i & 1);
-            if (row < a.N && m < a.M) {
-              const float v = acc[r][nt][i];
+            if (col < ny && m < a.M) {
+              const float v = silu(acc[0][nt][i]) * acc[1][nt][i];
               if constexpr (BF16)
-                a.y[(size_t)m * a.N + row] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
+                a.y[(size_t)m * ny + col] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
               else
-                a.y[(size_t)m * a.N + row] = __half_as_ushort(__float2half_rn(v));
+                a.y[(size_t)m * ny + col] = __half_as_ushort(__float2half_rn(v));
             }
           }
+      } else {
+        // fragment (r, nt, i) of this lane: row (tile R + r) 16 + g + 8 (i / 2),
+        // token m_base + 8 nt + 2 t + (i % 2)
+#pragma unroll
+        for (int r = 0; r < R; ++r)
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const int row = (tile * R + r) * 16 + g + 8 * (i >> 1);
+              const int m = m_base + 8 * nt + 2 * t + (i & 1);
+              if (row < a.N && m < a.M) {
+                const float v = acc[r][nt][i];
+                if constexpr (BF16)
+                  a.y[(size_t)m * a.N + row] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
+                else
+                  a.y[(size_t)m * a.N + row] = __half_as_ushort(__float2half_rn(v));
+              }
+            }
+      }
     }
     ++tile;
     sc = 0;
@@ -694,6 +715,7 @@ cudaError_t launch_skinny(const Problem& pr, const SkinnyPlan& plan, void* works
   a.M = pr.M;
   a.N = pr.N;
   a.K = pr.K;
+  a.gated = pr.gated ? 1 : 0;
   const int L = pr.group == -1 ? pr.K : pr.group;
   a.G = pr.K / L;
   a.lg = pr.group == -1 ? -1 : __builtin_ctz((unsigned)pr.group);

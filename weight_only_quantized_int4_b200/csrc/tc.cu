@@ -133,6 +133,7 @@ struct TcArgs {
   uint16_t* y;
   int M, N, K, L, G, nrb, nkb;
   int lg;                   // log2 of the group length; 30 for one group per row
+  int gated;                // 1: alternating 16-row gate / up blocks, y[M, N/2] = silu(gate) up
   int tiles_n, tiles_m, tiles;
   long long units;          // tiles * nkb
   int ctas;
@@ -477,20 +478,41 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           meta[2] = ((long long)first * a.units / a.ctas < t_first) ? 1 : 0;
         }
       }
+      // y for 32 tokens of this thread's row.  Gated layout: the quadrant's 32
+      // rows are one gate block (lanes 0-15) and its up block (lanes 16-31).
+      auto store32 = [&](const float (&vals)[32], int c0) {
+        if (!a.gated) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const int m = tm * BN + c0 + i;
+            if (row < a.N && m < a.M) {
+              const float o = vals[i] * s_row;
+              a.y[(size_t)m * a.N + row] = BF16 ? __bfloat16_as_ushort(__float2bfloat16_rn(o))
+                                                : __half_as_ushort(__float2half_rn(o));
+            }
+          }
+        } else {
+          const int ny = a.N >> 1;
+          const int col = (row >> 5) * 16 + (row & 15);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const float o = vals[i] * s_row;
+            const float up = __shfl_down_sync(0xffffffffu, o, 16);
+            const int m = tm * BN + c0 + i;
+            if (lane < 16 && row < a.N && m < a.M) {
+              const float gv = silu(o) * up;
+              a.y[(size_t)m * ny + col] = BF16 ? __bfloat16_as_ushort(__float2bfloat16_rn(gv))
+                                               : __half_as_ushort(__float2half_rn(gv));
+            }
+          }
+        }
+      };
 #pragma unroll 1
       for (int c0 = 0; c0 < BN; c0 += 32) {
         float v[32];
         tmem_ld32(tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * BN + c0), v);
         if (whole) {
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const int m = tm * BN + c0 + i;
-            if (row < a.N && m < a.M) {
-              const float o = v[i] * s_row;
-              a.y[(size_t)m * a.N + row] = BF16 ? __bfloat16_as_ushort(__float2bfloat16_rn(o))
-                                                : __half_as_ushort(__float2half_rn(o));
-            }
-          }
+          store32(v, c0);
         } else {
           float4* dst = reinterpret_cast<float4*>(slot + c0);
 #pragma unroll
@@ -547,15 +569,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 }
               }
             }
-#pragma unroll
-            for (int i = 0; i < 32; ++i) {
-              const int m = tm * BN + c0 + i;
-              if (row < a.N && m < a.M) {
-                const float o = accv[i] * s_row;
-                a.y[(size_t)m * a.N + row] = BF16 ? __bfloat16_as_ushort(__float2bfloat16_rn(o))
-                                                  : __half_as_ushort(__float2half_rn(o));
-              }
-            }
+            store32(accv, c0);
           }
           if (threadIdx.x == kEpi0) a.counters[tile] = 0u;   // ready for the next call
         }
@@ -719,6 +733,7 @@ cudaError_t launch_tc(const Problem& pr, const TcPlan& plan, void* workspace,
   a.M = pr.M;
   a.N = pr.N;
   a.K = pr.K;
+  a.gated = pr.gated ? 1 : 0;
   a.L = pr.group == -1 ? pr.K : pr.group;
   a.G = pr.K / a.L;
   a.lg = pr.group == -1 ? 30 : __builtin_ctz((unsigned)pr.group);
