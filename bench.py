@@ -54,18 +54,23 @@ WORKLOADS = {
                            [(8192, 10240), (8192, 57344), (28672, 8192)], [1, 16]),
     "lut4_nf4": ("lut", 4, 64, "f16", [(4096, 14336)], [1, 8]),
     "lut2": ("lut", 2, 64, "f16", [(4096, 14336)], [1, 8]),
+    # LLaMA-7B feed-forward gate fused into the matmul: gate and up (I = 11008
+    # each, N = 2 I rows packed together), y[M, I] = silu(gate) * up
+    "ffn_gated": ("sym", 4, 128, "f16", [(4096, 22016)], [1, 2, 4, 8, 16]),
 }
+GATED = {"ffn_gated"}
 SIGMA = {"sym": 0.02, "asym": 0.015, "lut": 0.02}
 L2_BYTES = 126 * 1000 * 1000     # B200 L2
 SKINNY_SOURCES = ("weight_only_quantized_int4_b200/csrc/skinny.cu",
                   "weight_only_quantized_int4_b200/csrc/common.cuh")
 
 
-def alg_bytes(mode, bits, group, M, K, N):
-    """Bytes a call must move at least once: codes, scales (+ zeros), x, y."""
+def alg_bytes(mode, bits, group, M, K, N, gated=False):
+    """Bytes a call must move at least once: codes, scales (+ zeros), x, y
+    (y has N / 2 columns for the fused gate)."""
     G = 1 if group == -1 else K // group
     meta = N * G * 2 * (2 if mode == "asym" else 1)
-    return N * K * bits // 8 + meta + M * K * 2 + M * N * 2
+    return N * K * bits // 8 + meta + M * K * 2 + M * (N // 2 if gated else N) * 2
 
 
 def problems(name):
@@ -189,6 +194,7 @@ def run_ours(args, rank, world, local_rank):
     q.load()
     dev = torch.device("cuda", local_rank)
     probs = problems(args.workload)
+    gated = args.workload in GATED
     gen = torch.Generator(device=dev).manual_seed(1234 + rank)
     # enough weight copies that the codes of consecutive steps never fit in L2
     codes_per_copy = sum(N * K * bits // 8 for (_, bits, _, _, _, K, N) in probs)
@@ -203,16 +209,19 @@ def run_ours(args, rank, world, local_rank):
                 from weight_only_quantized_int4_b200 import synth
                 t = synth.nf4_table() if bits == 4 else synth.lut2_table(0)
                 lut = torch.from_numpy(t.view(np.int16)).to(dev)
-            qw, sc, ze = q.pack(W, mode, bits, group, lut=lut)
+            if gated:
+                qw, sc, ze = q.pack_gated(W[: N // 2], W[N // 2:], mode, bits, group, lut=lut)
+            else:
+                qw, sc, ze = q.pack(W, mode, bits, group, lut=lut)
             del W
             tdt = torch.float16 if xdt == "f16" else torch.bfloat16
             x = torch.randn(M, K, generator=gen, device=dev).to(tdt)
-            y = torch.empty(M, N, dtype=tdt, device=dev)
+            y = torch.empty(M, N // 2 if gated else N, dtype=tdt, device=dev)
             ws = q.workspace(M, N, K, mode, bits, group, device=dev)
             zl = ze if mode == "asym" else lut
             calls.append(dict(x=x, qw=qw, sc=sc, zl=zl, y=y, ws=ws, M=M, N=N, K=K, mode=mode,
                               bits=bits, group=group,
-                              bytes=alg_bytes(mode, bits, group, M, K, N)))
+                              bytes=alg_bytes(mode, bits, group, M, K, N, gated)))
         sets.append(calls)
     torch.cuda.synchronize()
     calls = sets[0]
@@ -220,8 +229,12 @@ def run_ours(args, rank, world, local_rank):
 
     def step(i=0):
         for c in sets[i % copies]:
-            q.qmm(c["x"], c["qw"], c["sc"], c["zl"], c["N"], c["K"], c["mode"], c["bits"],
-                  c["group"], y=c["y"], ws=c["ws"])
+            if gated:
+                q.qmm_gated(c["x"], c["qw"], c["sc"], c["zl"], c["N"] // 2, c["K"], c["mode"],
+                            c["bits"], c["group"], y=c["y"], ws=c["ws"])
+            else:
+                q.qmm(c["x"], c["qw"], c["sc"], c["zl"], c["N"], c["K"], c["mode"], c["bits"],
+                      c["group"], y=c["y"], ws=c["ws"])
 
     # warm-up outside the graphs (first calls set kernel attributes), then one
     # graph per weight copy; step i replays graph i % copies
@@ -347,7 +360,10 @@ def _oracle_sample(workload, rows_per_problem, seed=0):
     import oracle
     from weight_only_quantized_int4_b200 import synth
     items = []
+    gated = workload in GATED
     for i, (mode, bits, group, xdt, M, K, N) in enumerate(problems(workload)):
+        if gated:   # whole (gate, up) block pairs
+            rows_per_problem = max(32, rows_per_problem // 32 * 32)
         rows = np.arange(rows_per_problem)
         W = synth.weights(seed + i, "W", N, K, SIGMA[mode], rows=rows)
         lut = None
@@ -359,7 +375,7 @@ def _oracle_sample(workload, rows_per_problem, seed=0):
         zl = zp if mode == "asym" else lut
         frac = rows_per_problem / N
         items.append((x, xdt, qw, sp, zl, M, rows_per_problem, K, mode, bits, group,
-                      frac * alg_bytes(mode, bits, group, M, K, N)))
+                      frac * alg_bytes(mode, bits, group, M, K, N, gated), gated))
     return items
 
 
@@ -367,8 +383,11 @@ def _run_oracle(items, threads):
     import oracle
     t0 = time.perf_counter()
     total = 0.0
-    for (x, xdt, qw, sp, zl, M, n, K, mode, bits, group, b) in items:
-        oracle.qmm_threaded(x, xdt, qw, sp, zl, M, n, K, mode, bits, group, 0, n, threads)
+    for (x, xdt, qw, sp, zl, M, n, K, mode, bits, group, b, gated) in items:
+        if gated:
+            oracle.qmm_gated(x, xdt, qw, sp, zl, M, n // 2, K, mode, bits, group)
+        else:
+            oracle.qmm_threaded(x, xdt, qw, sp, zl, M, n, K, mode, bits, group, 0, n, threads)
         total += b
     return time.perf_counter() - t0, total
 
