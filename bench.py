@@ -343,8 +343,8 @@ def run_ours(args, rank, world, local_rank):
            "roofline": roofline,
            "e2e": {"value": round(e2e_value, 1), "unit": "GB/s", "h2d_bytes_per_step": h2d,
                    "d2h_bytes_per_step": d2h, "steps": e2e_steps,
-                   "how": "per step: pinned x -> device, the 20 qmm calls through the Python "
-                          "API, y -> pinned host; CUDA events on the stream"},
+                   "how": f"per step: pinned x -> device, the {len(calls)} calls through the "
+                          "Python API, y -> pinned host; CUDA events on the stream"},
            "gpu_launches": len(calls) * args.steps,
            "clocks": clocks}
     if rank == 0 and not args.no_cpu_baseline:
