@@ -77,7 +77,12 @@ typedef enum {
 } qmm_status;
 
 /* Paths for qmm_with_path. */
-enum { QMM_PATH_AUTO = 0, QMM_PATH_SKINNY = 1, QMM_PATH_TENSOR = 2 };
+/* Paths.  QMM_PATH_SKINNY_STREAMK is the decode path with its split-K plan
+ * forced: for problems with few row tiles the decode path normally gives each
+ * tile one CTA (its warps split K and add their sums in shared memory); this
+ * value keeps the warp-level stream-K split with workspace partials instead
+ * (for tests and tuning; same results within rounding). */
+enum { QMM_PATH_AUTO = 0, QMM_PATH_SKINNY = 1, QMM_PATH_TENSOR = 2, QMM_PATH_SKINNY_STREAMK = 3 };
 
 /* Byte sizes of the packed buffers for an [N, K] weight.  Returns the size of
  * qweight (N*K*bits/8) and writes the scale and zero buffer sizes (zeros: 0

@@ -118,7 +118,7 @@ def test_qmm_small(mode, bits, group, xdtype):
         p = cases.make(mode, bits, group, M, N, K, xdtype, seed=M)
         y_ref, bound = cases.expected(p)
         x, qw, sp, zl = upload(p)
-        for path in ("auto", "skinny", "tensor"):
+        for path in ("auto", "skinny", "skinny_streamk", "tensor"):
             ws = q.workspace(M, N, K, mode, bits, group, path=path)
             y = q.qmm(x, qw, sp, zl, N, K, mode, bits, group, ws=ws, path=path)
             torch.cuda.synchronize()
@@ -138,7 +138,7 @@ def test_qmm_k_ends_mid_stage(mode, bits, group, xdtype, K):
         p = cases.make(mode, bits, group, M, N, K, xdtype, seed=300 + M + K)
         y_ref, bound = cases.expected(p)
         x, qw, sp, zl = upload(p)
-        for path in ("auto", "skinny"):
+        for path in ("auto", "skinny", "skinny_streamk"):
             ws = q.workspace(M, N, K, mode, bits, group, path=path)
             y = q.qmm(x, qw, sp, zl, N, K, mode, bits, group, ws=ws, path=path)
             torch.cuda.synchronize()
@@ -177,9 +177,10 @@ def test_qmm_workspace_modes(ws_kind):
     p = cases.make("sym", 4, 128, M, N, K, seed=21)
     y_ref, bound = cases.expected(p)
     x, qw, sp, _ = upload(p)
-    ws = q.workspace(M, N, K, "sym") if ws_kind == "sized" else None
-    y1 = q.qmm(x, qw, sp, None, N, K, "sym", 4, 128, ws=ws)
-    y2 = q.qmm(x, qw, sp, None, N, K, "sym", 4, 128, ws=ws)
+    # the decode path's stream-K plan (the one that needs a workspace)
+    ws = q.workspace(M, N, K, "sym", path="skinny_streamk") if ws_kind == "sized" else None
+    y1 = q.qmm(x, qw, sp, None, N, K, "sym", 4, 128, ws=ws, path="skinny_streamk")
+    y2 = q.qmm(x, qw, sp, None, N, K, "sym", 4, 128, ws=ws, path="skinny_streamk")
     torch.cuda.synchronize()
     cases.compare(to_f64(y1, "f16"), y_ref, bound, ws_kind)
     assert torch.equal(y1, y2), "repeated calls must be bit-identical (deterministic split-K)"
@@ -190,14 +191,13 @@ def test_qmm_workspace_modes(ws_kind):
 
 def test_qmm_rejects_small_workspace():
     M, N, K = 5, 2048, 4096
-    need = q.workspace_size(M, N, K, "sym")
-    if need == 0:
-        pytest.skip("this device plan needs no workspace")
+    need = q.workspace_size(M, N, K, "sym", path="skinny_streamk")
+    assert need > 0
     p = cases.make("sym", 4, 128, M, N, K, seed=22)
     x, qw, sp, _ = upload(p)
     small = torch.zeros(need - 256, dtype=torch.uint8, device="cuda")
     with pytest.raises(q.QmmError) as e:
-        q.qmm(x, qw, sp, None, N, K, "sym", 4, 128, ws=small)
+        q.qmm(x, qw, sp, None, N, K, "sym", 4, 128, ws=small, path="skinny_streamk")
     assert e.value.status == -6
 
 

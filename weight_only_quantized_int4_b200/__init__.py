@@ -23,7 +23,7 @@ LIB_PATH = os.path.join(_HERE, "libqmm.so")
 
 MODES = {"sym": 0, "asym": 1, "lut": 2}
 DTYPES = {torch.float16: 0, torch.bfloat16: 1}
-PATHS = {"auto": 0, "skinny": 1, "tensor": 2}
+PATHS = {"auto": 0, "skinny": 1, "tensor": 2, "skinny_streamk": 3}
 PATH_NAMES = {1: "skinny", 2: "tensor"}
 
 SYMBOLS = ("qmm_packed_size", "qmm_pack", "qmm_workspace_size", "qmm_workspace_size_for", "qmm",

@@ -60,10 +60,13 @@ struct Plan {
 
 Plan make_plan(int M, int N, int K, int bits, int group, int mode, bool bf16, int path) {
   Plan p{};
-  p.path = path == QMM_PATH_AUTO ? choose_path(M, bits, mode, bf16, group) : path;
+  const bool streamk = path == QMM_PATH_SKINNY_STREAMK;
+  p.path = path == QMM_PATH_AUTO ? choose_path(M, bits, mode, bf16, group)
+           : streamk            ? QMM_PATH_SKINNY
+                                : path;
   if (p.path == QMM_PATH_TENSOR && !tc_supported(bits, mode, bf16, group)) p.path = QMM_PATH_SKINNY;
   if (p.path == QMM_PATH_TENSOR) p.tc = plan_tc(M, N, K, device_sms());
-  else p.sk = plan_skinny(M, N, K, bits, group, mode, bf16, device_sms());
+  else p.sk = plan_skinny(M, N, K, bits, group, mode, bf16, device_sms(), streamk);
   return p;
 }
 
@@ -80,8 +83,7 @@ static int run_qmm(const void* x, int xdtype, const void* qweight, const uint16_
   int st = check_shape(N, K, bits, group, mode);
   if (st != QMM_OK) return st;
   if (xdtype != QMM_F16 && xdtype != QMM_BF16) return QMM_ERR_ARG;
-  if (path != QMM_PATH_AUTO && path != QMM_PATH_SKINNY && path != QMM_PATH_TENSOR)
-    return QMM_ERR_ARG;
+  if (path < QMM_PATH_AUTO || path > QMM_PATH_SKINNY_STREAMK) return QMM_ERR_ARG;
   if (M == 0) return QMM_OK;
   if (!x || !qweight || !scales || !y) return QMM_ERR_ARG;
   if (mode != QMM_SYM && !zeros_or_lut) return QMM_ERR_ARG;
@@ -169,7 +171,7 @@ int qmm_path(int M, int N, int K, int bits, int group, int mode) {
 
 size_t qmm_workspace_size_for(int M, int N, int K, int bits, int group, int mode, int path) {
   if (M <= 0 || check_shape(N, K, bits, group, mode) != QMM_OK) return 0;
-  if (path != QMM_PATH_AUTO && path != QMM_PATH_SKINNY && path != QMM_PATH_TENSOR) return 0;
+  if (path < QMM_PATH_AUTO || path > QMM_PATH_SKINNY_STREAMK) return 0;
   // the activation dtype is not an argument here: size for the larger of the two
   return std::max(make_plan(M, N, K, bits, group, mode, false, path).ws_bytes(),
                   make_plan(M, N, K, bits, group, mode, true, path).ws_bytes());

@@ -23,6 +23,7 @@ struct Problem {
 // Split-K plan of the skinny (M <= 16 per slab) decode path.
 struct SkinnyPlan {
   int nt;          // token tiles of 8 per slab (1 or 2)
+  int cta_tiles;   // 1: one CTA per row tile, warps split K, no workspace
   int rows;        // rows per CTA tile (16 * row blocks)
   int tiles_n;     // CTA tiles along N
   int slabs;       // token slabs (ceil(M / (8 nt)))
@@ -32,7 +33,8 @@ struct SkinnyPlan {
   size_t ws_bytes; // workspace needed (0 when every CTA owns whole tiles)
 };
 
-SkinnyPlan plan_skinny(int M, int N, int K, int bits, int group, int mode, bool bf16, int sms);
+SkinnyPlan plan_skinny(int M, int N, int K, int bits, int group, int mode, bool bf16, int sms,
+                       bool force_streamk = false);
 cudaError_t launch_skinny(const Problem& p, const SkinnyPlan& plan, void* workspace,
                           cudaStream_t stream);
 // Decode path on the library's static scratch buffer (no allocation); sets

@@ -65,6 +65,7 @@ struct SkinnyArgs {
   int M, N, K, G, nchunks, nrb, tiles, nsc;
   int lg;              // log2 of the group length; -1 for one group per row
   int gated;           // 1: rows are alternating 16-row gate / up blocks, y[M, N/2] = silu(gate) up
+  int cta_tiles;       // 1: CTA b owns tile b, its warps take the super-chunks round-robin
   int stage_bytes;     // bytes of one ring stage
   long long units;     // tiles * nsc
   int ctas;            // CTAs per slab
@@ -173,7 +174,14 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1) skinny_kernel(const
   const int gw = blockIdx.x * kWarps + warp;
   const long long W = a.warps;
   long long ub = 0, ue = 0;
-  if (gw < W) {
+  // CTA-per-tile mode (problems with few row tiles): CTA b owns tile b, warp w
+  // takes its super-chunks w, w + 8, ... and the warps' sums are added in
+  // shared memory; otherwise warp-level stream-K over contiguous unit ranges
+  const bool ctile = a.cta_tiles != 0;
+  const int sc_step = ctile ? kWarps : 1;
+  if (ctile) {
+    ue = warp < n ? (n - warp + kWarps - 1) / kWarps : 0;
+  } else if (gw < W) {
     ub = floor_div((long long)gw * a.units, W, a.inv_warps);
     ue = floor_div((long long)(gw + 1) * a.units, W, a.inv_warps);
   }
@@ -233,7 +241,7 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1) skinny_kernel(const
     __syncthreads();
   }
 
-  if (ub >= ue) return;   // no units (spare warps of the last CTA)
+  if (ub >= ue && !ctile) return;   // no units (spare warps of the last CTA)
 
   const int nsc_full = a.K / kSC;         // super-chunks with no column past K
 
@@ -315,12 +323,15 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1) skinny_kernel(const
   // ---- prologue: S - 1 super-chunks in flight (the warp's own units, in
   // order: consecutive super-chunks, then the next tile)
   long long pf_u = ub;
-  const int tb = (int)((unsigned)ub / (unsigned)n);   // the warp's first tile (ub < 2^31)
-  int pf_t = tb, pf_s = (int)(ub - (long long)tb * n);
+  // the warp's first tile and super-chunk (ub < 2^31)
+  const int tb = ctile ? (int)blockIdx.x : (int)((unsigned)ub / (unsigned)n);
+  const int sb = ctile ? warp : (int)(ub - (long long)tb * n);
+  int pf_t = tb, pf_s = sb;
   auto pf_next = [&]() {
     ++pf_u;
-    if (++pf_s == n) {
-      pf_s = 0;
+    pf_s += sc_step;
+    if (pf_s >= n) {
+      pf_s -= n;
       ++pf_t;
     }
   };
@@ -333,16 +344,61 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1) skinny_kernel(const
     cp_async_commit();
   }
 
-  int tile = tb, sc = (int)(ub - (long long)tb * n);
+  int tile = tb, sc = sb;
   long long u = ub;
+  float part[NACC];                      // CTA-per-tile mode: this warp's sums
+#pragma unroll
+  for (int i = 0; i < NACC; ++i) part[i] = 0.0f;
   int st_c = 0;                          // ring stage being computed
   int st_f = S - 1;                      // ring stage being filled
+
+  // y for the lane's fragments of `tile` (fused gate: silu(gate) * up)
+  auto store_y = [&](const float (&acc)[R][NT][4], int tile) {
+    if (a.gated) {
+      // the tile's two row blocks are gate block `tile` (r = 0) and up block
+      // `tile` (r = 1): each lane holds both values of its outputs
+      const int ny = a.N >> 1;
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int col = tile * 16 + g + 8 * (i >> 1);
+          const int m = m_base + 8 * nt + 2 * t + (i & 1);
+          if (col < ny && m < a.M) {
+            const float v = silu(acc[0][nt][i]) * acc[1][nt][i];
+            if constexpr (BF16)
+              a.y[(size_t)m * ny + col] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
+            else
+              a.y[(size_t)m * ny + col] = __half_as_ushort(__float2half_rn(v));
+          }
+        }
+    } else {
+      // fragment (r, nt, i) of this lane: row (tile R + r) 16 + g + 8 (i / 2),
+      // token m_base + 8 nt + 2 t + (i % 2)
+#pragma unroll
+      for (int r = 0; r < R; ++r)
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int row = (tile * R + r) * 16 + g + 8 * (i >> 1);
+            const int m = m_base + 8 * nt + 2 * t + (i & 1);
+            if (row < a.N && m < a.M) {
+              const float v = acc[r][nt][i];
+              if constexpr (BF16)
+                a.y[(size_t)m * a.N + row] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
+              else
+                a.y[(size_t)m * a.N + row] = __half_as_ushort(__float2half_rn(v));
+            }
+          }
+    }
+  };
 
   while (u < ue) {
     // this warp's segment of the tile: super-chunks [s0, s1)
     const int s0 = sc;
     const long long tile_end = (long long)(tile + 1) * n;
-    const int s1 = (int)((ue < tile_end ? ue : tile_end) - (long long)tile * n);
+    const int s1 = ctile ? n : (int)((ue < tile_end ? ue : tile_end) - (long long)tile * n);
 
     float acc[R][NT][4];
 #pragma unroll
@@ -352,7 +408,7 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1) skinny_kernel(const
 #pragma unroll
         for (int i = 0; i < 4; ++i) acc[r][nt][i] = 0.0f;
 
-    for (; sc < s1; ++sc, ++u) {
+    for (; sc < s1; sc += sc_step, ++u) {
       // keep the ring full: the stage refilled here was drained last iteration
       if (pf_u < ue) {
         issue(pf_t, pf_s, st_f);
@@ -482,10 +538,15 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1) skinny_kernel(const
       st_f = st_f + 1 == S ? 0 : st_f + 1;
     }
 
+    float* outv = &acc[0][0][0];
+    if (ctile) {
+#pragma unroll
+      for (int i = 0; i < NACC; ++i) part[i] = outv[i];
+      break;
+    }
     // ---- this warp's result for the tile segment: store y (whole tile) or
     // hand a partial to the last warp that finishes the tile
     const bool whole = s0 == 0 && s1 == n;
-    float* outv = &acc[0][0][0];
     bool store = true;
     if (!whole) {
       const long long t_first = (long long)tile * n;
@@ -541,50 +602,40 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1) skinny_kernel(const
         if (lane == 0) *counter = 0u;   // ready for the next call
       }
     }
-    if (store) {
-      if (a.gated) {
-        // the tile's two row blocks are gate block `tile` (r = 0) and up block
-        // `tile` (r = 1): each lane holds both values of its outputs
-        const int ny = a.N >> 1;
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const int col = tile * 16 + g + 8 * (i >> 1);
-            const int m = m_base + 8 * nt + 2 * t + (i & 1);
-            if (col < ny && m < a.M) {
-              const float v = silu(acc[0][nt][i]) * acc[1][nt][i];
-              if constexpr (BF16)
-                a.y[(size_t)m * ny + col] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
-              else
-                a.y[(size_t)m * ny + col] = __half_as_ushort(__float2half_rn(v));
-            }
-          }
-      } else {
-        // fragment (r, nt, i) of this lane: row (tile R + r) 16 + g + 8 (i / 2),
-        // token m_base + 8 nt + 2 t + (i % 2)
-#pragma unroll
-        for (int r = 0; r < R; ++r)
-#pragma unroll
-          for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              const int row = (tile * R + r) * 16 + g + 8 * (i >> 1);
-              const int m = m_base + 8 * nt + 2 * t + (i & 1);
-              if (row < a.N && m < a.M) {
-                const float v = acc[r][nt][i];
-                if constexpr (BF16)
-                  a.y[(size_t)m * a.N + row] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
-                else
-                  a.y[(size_t)m * a.N + row] = __half_as_ushort(__float2half_rn(v));
-              }
-            }
-      }
-    }
+    if (store) store_y(acc, tile);
     ++tile;
     sc = 0;
   }
   cp_async_wait<0>();   // nothing may still land in shared memory after exit
+  if (ctile) {
+    // the CTA's warps add their sums in warp order (deterministic) through
+    // shared memory (the rings are free once every warp is past this barrier)
+    __syncthreads();
+    float* red = reinterpret_cast<float*>(smem + kTabBytes<MODE>);   // [kWarps][32][NACC]
+    float4* mine = reinterpret_cast<float4*>(red + ((size_t)warp * 32 + lane) * NACC);
+#pragma unroll
+    for (int i = 0; i < NACC / 4; ++i)
+      mine[i] = make_float4(part[4 * i], part[4 * i + 1], part[4 * i + 2], part[4 * i + 3]);
+    __syncthreads();
+    if (warp == 0) {
+      float acc[R][NT][4];
+      float* outv = &acc[0][0][0];
+#pragma unroll
+      for (int i = 0; i < NACC; ++i) outv[i] = 0.0f;
+      for (int w = 0; w < kWarps; ++w) {
+        const float4* src = reinterpret_cast<const float4*>(red + ((size_t)w * 32 + lane) * NACC);
+#pragma unroll
+        for (int i = 0; i < NACC / 4; ++i) {
+          const float4 v = src[i];
+          outv[4 * i] += v.x;
+          outv[4 * i + 1] += v.y;
+          outv[4 * i + 2] += v.z;
+          outv[4 * i + 3] += v.w;
+        }
+      }
+      store_y(acc, (int)blockIdx.x);
+    }
+  }
 }
 
 template <int BITS, int MODE, int NT, int TPG>
@@ -668,7 +719,8 @@ int tiles_per_group(int group) { return (group == -1 || group >= kSC) ? 8 : grou
 
 }  // namespace
 
-SkinnyPlan plan_skinny(int M, int N, int K, int bits, int group, int mode, bool bf16, int sms) {
+SkinnyPlan plan_skinny(int M, int N, int K, int bits, int group, int mode, bool bf16, int sms,
+                       bool force_streamk) {
   SkinnyPlan p{};
   p.nt = M <= 8 ? 1 : 2;
   const int R = p.nt == 1 ? rb_per_tile<1>() : rb_per_tile<2>();
@@ -688,6 +740,15 @@ SkinnyPlan plan_skinny(int M, int N, int K, int bits, int group, int mode, bool 
   // one resident wave of CTAs; every warp is a stream-K worker with >= 1 unit
   long long warps = (long long)sms * (occ > 0 ? occ : 1) * kWarps;
   const long long cap = std::max<long long>(1, units * 8 / nsc);
+  if (!force_streamk && warps >= (long long)p.tiles_n * kWarps) {
+    // few row tiles: one CTA per tile, its warps split K, sums added in
+    // shared memory (no split-K workspace)
+    p.cta_tiles = 1;
+    p.splits = p.tiles_n;
+    p.warps = p.tiles_n * kWarps;
+    p.ws_bytes = 0;
+    return p;
+  }
   if (warps > cap) warps = cap;
   if (warps > units) warps = units;
   const long long ctas = (warps + kWarps - 1) / kWarps;
@@ -716,6 +777,7 @@ cudaError_t launch_skinny(const Problem& pr, const SkinnyPlan& plan, void* works
   a.N = pr.N;
   a.K = pr.K;
   a.gated = pr.gated ? 1 : 0;
+  a.cta_tiles = plan.cta_tiles;
   const int L = pr.group == -1 ? pr.K : pr.group;
   a.G = pr.K / L;
   a.lg = pr.group == -1 ? -1 : __builtin_ctz((unsigned)pr.group);
