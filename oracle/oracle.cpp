@@ -51,6 +51,11 @@
 //                      nibble 2p + 1.
 //      2-bit LUT:      word j/2 of the lane, byte 2 (j % 2) + p / 2; inside the
 //                      byte the 2-bit field 2 (p % 2) + (c % 2).
+//      3-bit LUT:      chunks of 128 columns and 768 bytes, lane l owning bytes
+//                      [24 l, 24 l + 24): words 0..3 hold the codes' two low bits
+//                      exactly as the 2-bit layout places 2-bit codes; words
+//                      4 and 5 hold the high bits, tile j's eight in byte j % 4 of
+//                      word 4 + j / 4, pair p member c % 2 at bit 2 p + (c % 2).
 //    Words are little-endian uint32; nibble/field f occupies bits [b f, b f + b).
 //  * scales (and ASYM zeros): fp16, [N/16][G][16]; inside the 16 the row r of
 //    the block sits at 2 (r % 8) + r / 8.
@@ -155,13 +160,14 @@ uint16_t scale_bits(float s32) {
 int n_groups(int K, int group) { return group == -1 ? 1 : K / group; }
 int group_len(int K, int group) { return group == -1 ? K : group; }
 int chunk_cols(int bits) { return bits == 4 ? 64 : 128; }
+int chunk_bytes(int bits) { return bits == 3 ? 768 : 512; }
 
 // Shapes the quantizer and the logical decode accept: any N, K > 0 with the
 // group dividing K.
 bool logical_ok(int N, int K, int mode, int bits, int group) {
   if (N <= 0 || K <= 0) return false;
   if (mode != MODE_SYM && mode != MODE_ASYM && mode != MODE_LUT) return false;
-  if (bits != 4 && !(bits == 2 && mode == MODE_LUT)) return false;
+  if (bits != 4 && !((bits == 2 || bits == 3) && mode == MODE_LUT)) return false;
   if (group != -1 && (group <= 0 || K % group != 0)) return false;
   return true;
 }
@@ -175,7 +181,8 @@ bool shape_ok(int N, int K, int mode, int bits, int group) {
   return true;
 }
 
-// Byte offset and bit shift of code (n, k) in the packed code buffer.
+// Byte offset and bit shift of code (n, k) in the packed code buffer (2- and
+// 4-bit codes; for 3-bit codes, of their two low bits).
 void code_place(int n, int k, int K, int mode, int bits, size_t* byte, int* shift) {
   int kc_cols = chunk_cols(bits);
   int rb = n / 16, r = n % 16;
@@ -185,7 +192,8 @@ void code_place(int n, int k, int K, int mode, int bits, size_t* byte, int* shif
   int lane = 4 * g + t;
   int p = h + 2 * (c / 2);
   int hi = c % 2;
-  size_t chunk_base = ((size_t)rb * (K / kc_cols) + chunk) * 512 + (size_t)lane * 16;
+  size_t chunk_base = ((size_t)rb * (K / kc_cols) + chunk) * chunk_bytes(bits) +
+                      (size_t)lane * (chunk_bytes(bits) / 32);
   if (bits == 4) {
     int nib = (mode == MODE_LUT) ? (2 * p + hi) : (p + 4 * hi);
     *byte = chunk_base + (size_t)j * 4 + nib / 2;
@@ -196,6 +204,42 @@ void code_place(int n, int k, int K, int mode, int bits, size_t* byte, int* shif
     *byte = chunk_base + (size_t)(j / 2) * 4 + byte_in_word;
     *shift = 2 * field;
   }
+}
+
+// 3-bit codes: byte offset and bit of the code's high bit.
+void code_place_high(int n, int k, int K, size_t* byte, int* shift) {
+  int rb = n / 16, r = n % 16;
+  int g = r % 8, h = r / 8;
+  int chunk = k / 128, kk = k % 128;
+  int j = kk / 16, t = (kk % 16) / 4, c = kk % 4;
+  int lane = 4 * g + t;
+  int p = h + 2 * (c / 2);
+  size_t lane_base = ((size_t)rb * (K / 128) + chunk) * 768 + (size_t)lane * 24;
+  *byte = lane_base + 16 + (size_t)(j / 4) * 4 + (j % 4);
+  *shift = 2 * p + c % 2;
+}
+
+int get_code(const uint8_t* qw, int n, int k, int K, int mode, int bits) {
+  size_t byte;
+  int shift;
+  code_place(n, k, K, mode, bits, &byte, &shift);
+  if (bits != 3) return (qw[byte] >> shift) & ((1 << bits) - 1);
+  int q = (qw[byte] >> shift) & 3;
+  code_place_high(n, k, K, &byte, &shift);
+  return q | (((qw[byte] >> shift) & 1) << 2);
+}
+
+void put_code(uint8_t* qw, int n, int k, int K, int mode, int bits, int q) {
+  size_t byte;
+  int shift;
+  code_place(n, k, K, mode, bits, &byte, &shift);
+  if (bits != 3) {
+    qw[byte] |= (uint8_t)((q & ((1 << bits) - 1)) << shift);
+    return;
+  }
+  qw[byte] |= (uint8_t)((q & 3) << shift);
+  code_place_high(n, k, K, &byte, &shift);
+  qw[byte] |= (uint8_t)(((q >> 2) & 1) << shift);
 }
 
 // Index of (row n, group gi) in the packed scale / zero buffers.
@@ -289,12 +333,7 @@ int oracle_pack(const uint8_t* codes, const uint16_t* scales, const uint16_t* ze
   const int G = n_groups(K, group);
   std::memset(qweight, 0, oracle_packed_bytes(N, K, bits));
   for (int n = 0; n < N; ++n)
-    for (int k = 0; k < K; ++k) {
-      size_t byte;
-      int shift;
-      code_place(n, k, K, mode, bits, &byte, &shift);
-      qweight[byte] |= (uint8_t)((codes[(size_t)n * K + k] & ((1 << bits) - 1)) << shift);
-    }
+    for (int k = 0; k < K; ++k) put_code(qweight, n, k, K, mode, bits, codes[(size_t)n * K + k]);
   for (int n = 0; n < N; ++n)
     for (int gi = 0; gi < G; ++gi) {
       scales_p[scale_index(n, gi, G)] = scales[(size_t)n * G + gi];
@@ -310,12 +349,7 @@ int oracle_unpack(const uint8_t* qweight, const uint16_t* scales_p, const uint16
   if (!qweight || !codes || !shape_ok(N, K, mode, bits, group)) return ERR_ARG;
   const int G = n_groups(K, group);
   for (int n = 0; n < N; ++n)
-    for (int k = 0; k < K; ++k) {
-      size_t byte;
-      int shift;
-      code_place(n, k, K, mode, bits, &byte, &shift);
-      codes[(size_t)n * K + k] = (uint8_t)((qweight[byte] >> shift) & ((1 << bits) - 1));
-    }
+    for (int k = 0; k < K; ++k) codes[(size_t)n * K + k] = (uint8_t)get_code(qweight, n, k, K, mode, bits);
   for (int n = 0; n < N; ++n)
     for (int gi = 0; gi < G; ++gi) {
       if (scales && scales_p) scales[(size_t)n * G + gi] = scales_p[scale_index(n, gi, G)];
@@ -368,10 +402,7 @@ static void dequant_row(int n, const uint8_t* qweight, const uint16_t* scales_p,
                         const uint16_t* zeros_or_lut, int K, int mode, int bits, int G, int L,
                         double* w) {
   for (int k = 0; k < K; ++k) {
-    size_t byte;
-    int shift;
-    code_place(n, k, K, mode, bits, &byte, &shift);
-    int q = (qweight[byte] >> shift) & ((1 << bits) - 1);
+    int q = get_code(qweight, n, k, K, mode, bits);
     int gi = k / L;
     double s = half_value(scales_p[scale_index(n, gi, G)]);
     double z = (mode == MODE_ASYM) ? half_value(zeros_or_lut[scale_index(n, gi, G)]) : 0.0;

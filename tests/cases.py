@@ -23,7 +23,7 @@ SIGMA = {"sym": 0.02, "asym": 0.015, "lut": 0.02}
 def table(mode, bits):
     if mode != "lut":
         return None
-    return synth.nf4_table() if bits == 4 else synth.lut2_table(0)
+    return {4: synth.nf4_table, 3: synth.nf3_table, 2: lambda: synth.lut2_table(0)}[bits]()
 
 
 @dataclass

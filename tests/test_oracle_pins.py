@@ -221,9 +221,9 @@ def test_asym_codes_are_nearest_grid_points():
     assert np.all(Wg.max(axis=2) <= hi + h2f(scales) * 0.51)
 
 
-@pytest.mark.parametrize("bits", [4, 2])
+@pytest.mark.parametrize("bits", [4, 3, 2])
 def test_lut_codes_are_nearest_entries(bits):
-    T = synth.nf4_table() if bits == 4 else synth.lut2_table(0)
+    T = {4: synth.nf4_table(), 3: synth.nf3_table(), 2: synth.lut2_table(0)}[bits]
     W = _rand_w(32, 128, 0.02, 5)
     codes, scales, _ = oracle.quantize(W, "lut", bits, 64, lut=T)
     s = np.repeat(h2f(scales).astype(np.float32), 64, axis=1)
@@ -263,7 +263,47 @@ def test_layout_is_a_bijection(bits, mode):
     assert np.all(qw == 0xFF)
 
 
-@pytest.mark.parametrize("bits,mode", [(4, "sym"), (4, "asym"), (4, "lut"), (2, "lut")])
+def test_layout3_planes_and_bijection():
+    """3-bit codes: every code owns three bits, two adjacent ones in the low
+    plane (bytes 0..15 of its lane's 24) and one in the high plane (bytes
+    16..23); no bit is shared and all bits are used."""
+    N, K = 32, 256
+    seen = np.zeros(N * K * 3, np.int32)
+    for n in range(0, N, 3):
+        for k in range(0, K, 5):
+            codes = np.zeros((N, K), np.uint8)
+            codes[n, k] = 7
+            qw, _, _ = oracle.pack(codes, np.zeros((N, K // 64), np.uint16), None, "lut", 3, 64)
+            on = np.nonzero(np.unpackbits(qw, bitorder="little"))[0]
+            assert len(on) == 3
+            lo, hi = on[:2], on[2]
+            assert lo[1] - lo[0] == 1 and lo[0] % 2 == 0
+            assert (lo[0] // 8) % 24 < 16 and (hi // 8) % 24 >= 16
+            seen[on] += 1
+    assert seen.max() == 1
+    qw, _, _ = oracle.pack(np.full((N, K), 7, np.uint8), np.zeros((N, 4), np.uint16), None,
+                           "lut", 3, 64)
+    assert np.all(qw == 0xFF)
+
+
+def test_layout3_hand_position():
+    """Code 5 (binary 101) at row 9, column 21, worked out from the layout's
+    definition: g = 1, h = 1, tile j = 1, t = 1, c = 1 -> lane 5 (bytes
+    120..143 of chunk 0), pair p = 1, member 1.  Low bits: word 0, byte
+    2 (j % 2) + p / 2 = 2, field 2 (p % 2) + 1 = 3 -> byte 122 bits 6-7 = 01.
+    High bit: byte 16 + j % 4 = 17 of the lane -> byte 137, bit 2 p + 1 = 3."""
+    N, K = 16, 128
+    codes = np.zeros((N, K), np.uint8)
+    codes[9, 21] = 5
+    qw, _, _ = oracle.pack(codes, np.zeros((N, 2), np.uint16), None, "lut", 3, 64)
+    expect = np.zeros(N * K * 3 // 8, np.uint8)
+    expect[122] = 0x40
+    expect[137] = 0x08
+    assert np.array_equal(qw, expect)
+
+
+@pytest.mark.parametrize("bits,mode", [(4, "sym"), (4, "asym"), (4, "lut"), (3, "lut"),
+                                       (2, "lut")])
 def test_pack_unpack_round_trip(bits, mode):
     rng = np.random.default_rng(7)
     N, K, g = 48, 384, 128
@@ -272,6 +312,7 @@ def test_pack_unpack_round_trip(bits, mode):
     scales = rng.integers(0, 0x7BFF, (N, G)).astype(np.uint16)
     zeros = rng.integers(0, 16, (N, G)).astype(np.uint16) if mode == "asym" else None
     qw, sp, zp = oracle.pack(codes, scales, zeros, mode, bits, g)
+    assert qw.size == N * K * bits // 8
     c2, s2, z2 = oracle.unpack(qw, sp, zp, N, K, mode, bits, g)
     assert np.array_equal(c2, codes) and np.array_equal(s2, scales)
     if mode == "asym":
@@ -288,7 +329,7 @@ def _problem(mode, bits, group, M, N, K, seed, xdtype="f16"):
     W = _rand_w(N, K, 0.02, seed)
     lut = None
     if mode == "lut":
-        lut = synth.nf4_table() if bits == 4 else synth.lut2_table(0)
+        lut = {4: synth.nf4_table(), 3: synth.nf3_table(), 2: synth.lut2_table(0)}[bits]
     codes, scales, zeros = oracle.quantize(W, mode, bits, group, lut=lut)
     qw, sp, zp = oracle.pack(codes, scales, zeros, mode, bits, group)
     x = synth.activations(seed, "x", M, K, xdtype)
@@ -298,7 +339,7 @@ def _problem(mode, bits, group, M, N, K, seed, xdtype="f16"):
 
 @pytest.mark.parametrize("mode,bits,group,xdt", [("sym", 4, 128, "f16"), ("sym", 4, -1, "f16"),
                                                  ("asym", 4, 64, "bf16"), ("lut", 4, 64, "f16"),
-                                                 ("lut", 2, 64, "f16")])
+                                                 ("lut", 3, 64, "f16"), ("lut", 2, 64, "f16")])
 def test_qmm_matches_numpy_matmul(mode, bits, group, xdt):
     """x . W~^T through numpy's matmul (a library routine) on the decoded weights."""
     M, N, K = 5, 48, 256
@@ -395,6 +436,11 @@ def test_tables():
     assert np.array_equal(t, -t[::-1])
     t2 = h2f(synth.lut2_table(0))
     assert np.all(np.diff(t2) > 0) and np.max(np.abs(t2)) == 1.0
+    t3 = h2f(synth.nf3_table())
+    assert len(t3) == 8 and t3[0] == -1.0 and t3[-1] == 1.0 and np.all(np.diff(t3) > 0)
+    assert np.array_equal(t3, -t3[::-1])
+    # T[5] = q(5.5 / 8) / q(7.5 / 8) with q the normal quantile (values from scipy)
+    assert abs(t3[5] - 0.48877641 / 1.53412054) < 1e-3
 
 
 # ------------------------------------------------- fused feed-forward gate

@@ -113,15 +113,26 @@ def _norm_ppf(p: float) -> float:
     return 0.5 * (lo + hi)
 
 
-def nf4_table() -> np.ndarray:
-    """16-entry normal-quantile table over [-1, 1] as fp16 bits.
+def nf_table(bits: int) -> np.ndarray:
+    """2^bits-entry normal-quantile table over [-1, 1] as fp16 bits.
 
-    T[i] = q((i + 0.5) / 16) / q(15.5 / 16) with q the standard normal quantile:
-    symmetric, ascending, endpoints exactly -1 and 1.
+    T[i] = q((i + 0.5) / 2^bits) / q((2^bits - 0.5) / 2^bits) with q the standard
+    normal quantile: symmetric, ascending, endpoints exactly -1 and 1.
     """
-    top = _norm_ppf(15.5 / 16)
-    t = np.array([_norm_ppf((i + 0.5) / 16) / top for i in range(16)])
+    n = 1 << bits
+    top = _norm_ppf((n - 0.5) / n)
+    t = np.array([_norm_ppf((i + 0.5) / n) / top for i in range(n)])
     return t.astype(np.float16).view(np.uint16)
+
+
+def nf4_table() -> np.ndarray:
+    """The 16-entry NF4-style table (nf_table(4))."""
+    return nf_table(4)
+
+
+def nf3_table() -> np.ndarray:
+    """The 8-entry NF3-style table (nf_table(3))."""
+    return nf_table(3)
 
 
 def lut2_table(seed: int = 0) -> np.ndarray:
