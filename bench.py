@@ -54,6 +54,7 @@ WORKLOADS = {
                            [(8192, 10240), (8192, 57344), (28672, 8192)], [1, 16]),
     "lut4_nf4": ("lut", 4, 64, "f16", [(4096, 14336)], [1, 8]),
     "lut2": ("lut", 2, 64, "f16", [(4096, 14336)], [1, 8]),
+    "lut3_nf3": ("lut", 3, 64, "f16", [(4096, 14336)], [1, 8]),
     # LLaMA-7B feed-forward gate fused into the matmul: gate and up (I = 11008
     # each, N = 2 I rows packed together), y[M, I] = silu(gate) * up
     "ffn_gated": ("sym", 4, 128, "f16", [(4096, 22016)], [1, 2, 4, 8, 16]),
@@ -207,7 +208,7 @@ def run_ours(args, rank, world, local_rank):
             lut = None
             if mode == "lut":
                 from weight_only_quantized_int4_b200 import synth
-                t = synth.nf4_table() if bits == 4 else synth.lut2_table(0)
+                t = {4: synth.nf4_table, 3: synth.nf3_table, 2: lambda: synth.lut2_table(0)}[bits]()
                 lut = torch.from_numpy(t.view(np.int16)).to(dev)
             if gated:
                 qw, sc, ze = q.pack_gated(W[: N // 2], W[N // 2:], mode, bits, group, lut=lut)
@@ -368,7 +369,7 @@ def _oracle_sample(workload, rows_per_problem, seed=0):
         W = synth.weights(seed + i, "W", N, K, SIGMA[mode], rows=rows)
         lut = None
         if mode == "lut":
-            lut = synth.nf4_table() if bits == 4 else synth.lut2_table(0)
+            lut = {4: synth.nf4_table, 3: synth.nf3_table, 2: lambda: synth.lut2_table(0)}[bits]()
         codes, scales, zeros = oracle.quantize(W, mode, bits, group, lut=lut)
         qw, sp, zp = oracle.pack(codes, scales, zeros, mode, bits, group)
         x = synth.activations(seed + i, "x", M, K, xdt)

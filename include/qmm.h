@@ -33,7 +33,7 @@
  *    cudaGetLastError right after the launch.  Errors raised later by a kernel
  *    (a bounded wait that ran out) are reported by qmm_check_error.
  *  - Shapes the GPU kernels accept: N % 16 == 0; K % 64 == 0 (4-bit) or
- *    K % 128 == 0 (2-bit); group == -1 or a power of two >= 16 that divides K;
+ *    K % 128 == 0 (2- and 3-bit); group == -1 or a power of two >= 16 that divides K;
  *    N, K <= 2^20; M >= 0.  Other shapes return QMM_ERR_UNSUPPORTED.
  *
  * Packed layout (written by qmm_pack, read by qmm and qmm_dequant):
@@ -48,6 +48,11 @@
  *    2p and 2p + 1.  2-bit LUT: word j / 2, byte 2 (j % 2) + p / 2, 2-bit field
  *    2 (p % 2) + (c % 2).  Words are little-endian; field f holds bits
  *    [bits*f, bits*f + bits).
+ *    3-bit LUT (the FLUTE summary's 2/3/4-bit tables): chunks of 128 columns
+ *    and 768 bytes, lane l owning bytes [24 l, 24 l + 24); words 0..3 of the
+ *    lane hold the codes' two low bits placed as the 2-bit layout places 2-bit
+ *    codes, words 4 and 5 the high bits: tile j's eight in byte j % 4 of word
+ *    4 + j / 4, pair p member c % 2 at bit 2 p + (c % 2).
  *  - scales (and zeros): fp16, G = K/group groups (1 for group -1), stored as
  *    [N/16][G][16] with row r of a block at position 2 (r % 8) + r / 8, i.e.
  *    rows g and g + 8 side by side.
@@ -105,7 +110,7 @@ size_t qmm_packed_size(int N, int K, int bits, int group, int mode,
  *   qweight  device, qmm_packed_size bytes, 16-byte aligned (written).
  *   scales   device, fp16, scales_bytes, 16-byte aligned (written).
  *   zeros    device, fp16, zeros_bytes, 16-byte aligned (QMM_ASYM, written), else NULL.
- * bits: 4 for SYM/ASYM; 4 or 2 for LUT. */
+ * bits: 4 for SYM/ASYM; 4, 3 or 2 for LUT. */
 int qmm_pack(const float* W, int N, int K, int mode, int bits, int group,
              const uint16_t* lut, void* qweight, uint16_t* scales, uint16_t* zeros,
              void* stream);

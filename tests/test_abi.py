@@ -55,7 +55,9 @@ def test_sizes_and_paths(lib):
     (4608, 4608, 4, 48, "sym", -2),     # group not a power of two
     (4096, 4096, 4, 384, "sym", -2),    # group does not divide K
     (0, 4096, 4, 128, "sym", -1),
-    (4096, 4096, 3, 128, "lut", -1),
+    (4096, 4096, 5, 128, "lut", -1),   # no 5-bit codes
+    (4096, 4096, 3, 128, "sym", -2),   # 3-bit needs LUT
+    (4096, 4160, 3, 64, "lut", -2),    # 3-bit needs K % 128
 ])
 def test_bad_shapes_are_rejected(lib, N, K, bits, group, mode, status):
     assert lib.qmm_path(1, N, K, bits, group, q.MODES[mode]) == status

@@ -24,6 +24,7 @@ CONFIGS = {
                            [(8192, 10240), (8192, 57344), (28672, 8192)], [1, 16, 64]),
     "lut4_nf4": ("lut", 4, 64, "f16", [(4096, 14336)], [1, 8, 32]),
     "lut2": ("lut", 2, 64, "f16", [(4096, 14336)], [1, 8, 32]),
+    "lut3_nf3": ("lut", 3, 64, "f16", [(4096, 14336)], [1, 8, 32]),
     "prefill_gm1": ("sym", 4, -1, "f16", [(4096, 11008)], [64, 256, 1024, 4096]),
     "prefill_g128": ("sym", 4, 128, "f16", [(4096, 11008)], [64, 256, 1024, 4096]),
     # the largest K and N the packed layout accepts (2^20), each with the

@@ -47,7 +47,8 @@ def upload(p):
 
 MODES = [("sym", 4, 128), ("sym", 4, -1), ("sym", 4, 64), ("sym", 4, 32), ("asym", 4, 128),
          ("asym", 4, 64), ("lut", 4, 64), ("lut", 4, 128), ("lut", 2, 64), ("lut", 2, 128),
-         ("lut", 2, 32), ("sym", 4, 16), ("sym", 4, 256), ("asym", 4, 256)]
+         ("lut", 2, 32), ("sym", 4, 16), ("sym", 4, 256), ("asym", 4, 256), ("lut", 3, 64),
+         ("lut", 3, 128)]
 
 
 # ------------------------------------------------------------------ packing

@@ -29,8 +29,8 @@ bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) %
 int check_shape(int N, int K, int bits, int group, int mode) {
   if (N <= 0 || K <= 0) return QMM_ERR_ARG;
   if (mode != QMM_SYM && mode != QMM_ASYM && mode != QMM_LUT) return QMM_ERR_ARG;
-  if (bits != 4 && bits != 2) return QMM_ERR_ARG;
-  if (bits == 2 && mode != QMM_LUT) return QMM_ERR_UNSUPPORTED;
+  if (bits < 2 || bits > 4) return QMM_ERR_ARG;
+  if (bits != 4 && mode != QMM_LUT) return QMM_ERR_UNSUPPORTED;   // 2- and 3-bit: LUT only
   if (N % 16 != 0 || K % chunk_cols(bits) != 0) return QMM_ERR_UNSUPPORTED;
   if (N > (1 << 20) || K > (1 << 20)) return QMM_ERR_UNSUPPORTED;   // 32-bit work indexing
   // groups: one per row (-1) or a power of two >= 16 dividing K

@@ -12,8 +12,10 @@ namespace qk {
 
 constexpr int kSYM = QMM_SYM, kASYM = QMM_ASYM, kLUT = QMM_LUT;
 
-// Chunk of K covered by one 512-byte block of codes (16 rows x KC columns).
+// Chunk of K covered by one block of codes (16 rows x KC columns): 512 bytes
+// for 4- and 2-bit codes, 768 bytes for 3-bit codes.
 __host__ __device__ constexpr int chunk_cols(int bits) { return bits == 4 ? 64 : 128; }
+__host__ __device__ constexpr int chunk_bytes(int bits) { return bits == 3 ? 768 : 512; }
 
 // Position of row r (0..15) of a row block inside its 16 scales.
 __host__ __device__ constexpr int scale_slot(int r) { return 2 * (r & 7) + (r >> 3); }

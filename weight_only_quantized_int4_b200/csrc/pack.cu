@@ -156,6 +156,91 @@ __global__ void __launch_bounds__(256) pack_codes_kernel(CodeCtx c, uint32_t* __
 
 // One thread per packed word: decode its codes to (q - z) * s (or T[q] * s),
 // exact in fp32 for integer zero-points, then round once to fp16 / bf16.
+// 3-bit codes: one thread per 32-bit word, six words per lane of a 768-byte
+// chunk (128 columns).  Words 0..3 take the codes' two low bits in the 2-bit
+// layout (word w: tiles 2w, 2w + 1); words 4, 5 take the high bits (word 4 + u:
+// tiles 4u .. 4u + 3, tile j in byte j % 4, pair p member c % 2 at bit 2p + c % 2).
+__global__ void __launch_bounds__(256) pack_codes3_kernel(CodeCtx c, uint32_t* __restrict__ out,
+                                                          size_t nwords) {
+  const size_t wid = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (wid >= nwords) return;
+  const int w6 = (int)(wid % 6);
+  const int lane = (int)((wid / 6) % 32);
+  const size_t blk = wid / 192;                      // 192 words per 768-byte chunk
+  const int chunk = (int)(blk % c.nchunks);
+  const int rb = (int)(blk / c.nchunks);
+  const int g = lane >> 2, t = lane & 3;
+  float lut[16];
+  for (int e = 0; e < 16; ++e)
+    lut[e] = e < c.nlut ? __half2float(__ushort_as_half(c.lut[e])) : 0.0f;
+  const bool low = w6 < 4;
+  const int ntiles = low ? 2 : 4;
+  uint32_t v = 0;
+  for (int sub = 0; sub < ntiles; ++sub) {
+    const int j = low ? 2 * w6 + sub : 4 * (w6 - 4) + sub;   // 16-column tile
+    const int k0 = chunk * 128 + 16 * j + 4 * t;
+    const int gi = k0 / c.L;
+    for (int h = 0; h < 2; ++h) {
+      const int n = rb * 16 + g + 8 * h;
+      const size_t sidx = ((size_t)rb * c.G + gi) * 16 + scale_slot(g + 8 * h);
+      const float s = __half2float(__ushort_as_half(c.scales[sidx]));
+      const float4 wv = *reinterpret_cast<const float4*>(src_row(c.W, c.W2, n, c.K) + k0);
+      const float wc[4] = {wv.x, wv.y, wv.z, wv.w};
+      for (int cc = 0; cc < 4; ++cc) {
+        const uint32_t q = (uint32_t)encode(wc[cc], s, 0.0f, c, lut);
+        const int p = h + 2 * (cc >> 1), hi = cc & 1;
+        if (low)
+          v |= (q & 3u) << (8 * (2 * sub + (p >> 1)) + 2 * (2 * (p & 1) + hi));
+        else
+          v |= ((q >> 2) & 1u) << (8 * sub + 2 * p + hi);
+      }
+    }
+  }
+  out[wid] = v;
+  __threadfence();   // visible to any kernel that starts after this grid
+}
+
+// 3-bit codes: one thread per (row block, chunk, lane) decodes its 64 codes.
+__global__ void __launch_bounds__(256) dequant3_kernel(const uint32_t* __restrict__ qw,
+                                                       const uint16_t* __restrict__ scales,
+                                                       const uint16_t* __restrict__ lut, int K,
+                                                       int L, int G, int nchunks, bool bf16,
+                                                       void* out, size_t nthreads) {
+  const size_t tid = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (tid >= nthreads) return;
+  const int lane = (int)(tid % 32);
+  const size_t blk = tid / 32;
+  const int chunk = (int)(blk % nchunks);
+  const int rb = (int)(blk / nchunks);
+  const int g = lane >> 2, t = lane & 3;
+  const uint32_t* w = qw + blk * 192 + (size_t)lane * 6;
+  for (int j = 0; j < 8; ++j) {
+    const uint32_t lo = w[j >> 1], hw = w[4 + (j >> 2)];
+    const int k0 = chunk * 128 + 16 * j + 4 * t;
+    const int gi = k0 / L;
+    for (int h = 0; h < 2; ++h) {
+      const int n = rb * 16 + g + 8 * h;
+      const size_t sidx = ((size_t)rb * G + gi) * 16 + scale_slot(g + 8 * h);
+      const float s = __half2float(__ushort_as_half(scales[sidx]));
+      float r[4];
+      for (int cc = 0; cc < 4; ++cc) {
+        const int p = h + 2 * (cc >> 1), hi = cc & 1;
+        const uint32_t q = ((lo >> (8 * (2 * (j & 1) + (p >> 1)) + 2 * (2 * (p & 1) + hi))) & 3u) |
+                           (((hw >> (8 * (j & 3) + 2 * p + hi)) & 1u) << 2);
+        r[cc] = __fmul_rn(__half2float(__ushort_as_half(lut[q])), s);
+      }
+      const size_t o = (size_t)n * K + k0;
+      if (bf16) {
+        __nv_bfloat16* p = reinterpret_cast<__nv_bfloat16*>(out) + o;
+        for (int cc = 0; cc < 4; ++cc) p[cc] = __float2bfloat16_rn(r[cc]);
+      } else {
+        __half* p = reinterpret_cast<__half*>(out) + o;
+        for (int cc = 0; cc < 4; ++cc) p[cc] = __float2half_rn(r[cc]);
+      }
+    }
+  }
+}
+
 __global__ void __launch_bounds__(256) dequant_kernel(const uint32_t* __restrict__ qw,
                                                       const uint16_t* __restrict__ scales,
                                                       const uint16_t* __restrict__ zl, int K,
@@ -235,7 +320,10 @@ cudaError_t launch_pack(const float* W, const float* W2, int N, int K, int mode,
   c.nlut = 1 << bits;
   const size_t nwords = (size_t)N * K * bits / 32;
   const unsigned blocks = (unsigned)((nwords + 255) / 256);
-  pack_codes_kernel<<<blocks, 256, 0, stream>>>(c, reinterpret_cast<uint32_t*>(qweight), nwords);
+  if (bits == 3)
+    pack_codes3_kernel<<<blocks, 256, 0, stream>>>(c, reinterpret_cast<uint32_t*>(qweight), nwords);
+  else
+    pack_codes_kernel<<<blocks, 256, 0, stream>>>(c, reinterpret_cast<uint32_t*>(qweight), nwords);
   return cudaGetLastError();
 }
 
@@ -244,6 +332,13 @@ cudaError_t launch_dequant(const void* qweight, const uint16_t* scales,
                            int mode, int out_dtype, void* W_out, cudaStream_t stream) {
   const int L = group == -1 ? K : group;
   const int G = K / L;
+  if (bits == 3) {
+    const size_t nthreads = (size_t)(N / 16) * (K / 128) * 32;
+    dequant3_kernel<<<(unsigned)((nthreads + 255) / 256), 256, 0, stream>>>(
+        reinterpret_cast<const uint32_t*>(qweight), scales, zeros_or_lut, K, L, G, K / 128,
+        out_dtype == QMM_BF16, W_out, nthreads);
+    return cudaGetLastError();
+  }
   const size_t nwords = (size_t)N * K * bits / 32;
   const unsigned blocks = (unsigned)((nwords + 255) / 256);
   dequant_kernel<<<blocks, 256, 0, stream>>>(reinterpret_cast<const uint32_t*>(qweight), scales,

@@ -79,7 +79,7 @@ struct SkinnyArgs {
 template <int MODE>
 constexpr size_t kTabBytes = MODE == kLUT ? 256 * 32 * 4 : 0;
 
-// Stage layout of one warp's ring slot: codes [R][CPS][512] | x [TOK][272]
+// Stage layout of one warp's ring slot: codes [R][CPS][CB] | x [TOK][288]
 // | scales [R][GPS][32 B] | zeros (ASYM) [R][GPS][32 B].
 template <int BITS, int MODE, int NT, int TPG>
 struct Stage {
@@ -87,7 +87,8 @@ struct Stage {
   static constexpr int TOK = 8 * NT;
   static constexpr int CPS = kSC / chunk_cols(BITS);   // chunks per stage
   static constexpr int GPS = kTiles / TPG;             // groups per stage
-  static constexpr int X_OFF = R * CPS * 512;
+  static constexpr int CB = chunk_bytes(BITS);         // bytes per chunk
+  static constexpr int X_OFF = R * CPS * CB;
   static constexpr int S_OFF = X_OFF + TOK * kXPitch;
   static constexpr int Z_OFF = S_OFF + R * GPS * 32;
   static constexpr int BYTES = Z_OFF + (MODE == kASYM ? R * GPS * 32 : 0);
@@ -224,14 +225,22 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1) skinny_kernel(const
         lv[i] = 0;
       }
     }
-    constexpr int VALS = BITS == 4 ? 2 : 4;              // values per entry
+    //  3-bit: entry[6-bit index] = the pair (low bits of both members, then
+    //  their high bits), 64 entries.
+    constexpr int VALS = BITS == 2 ? 4 : 2;              // values per entry
     constexpr int WORDS = (BF16 ? 2 : 1) * VALS / 2;     // 32-bit words per entry copy
     constexpr int COPIES = 32 / WORDS;
-    for (int i = threadIdx.x; i < 256 * COPIES; i += kThreads) {
+    constexpr int NENT = BITS == 3 ? 64 : 256;
+    for (int i = threadIdx.x; i < NENT * COPIES; i += kThreads) {
       const int e = i / COPIES;
       uint32_t v[4];
+      if constexpr (BITS == 3) {
+        v[0] = (e & 3) | (((e >> 4) & 1) << 2);
+        v[1] = ((e >> 2) & 3) | (((e >> 5) & 1) << 2);
+      } else {
 #pragma unroll
-      for (int k = 0; k < VALS; ++k) v[k] = BITS == 4 ? ((e >> (4 * k)) & 15) : ((e >> (2 * k)) & 3);
+        for (int k = 0; k < VALS; ++k) v[k] = BITS == 4 ? ((e >> (4 * k)) & 15) : ((e >> (2 * k)) & 3);
+      }
 #pragma unroll
       for (int w = 0; w < VALS / 2; ++w) {
         tab[i * WORDS + w] = hv[v[2 * w]] | (hv[v[2 * w + 1]] << 16);
@@ -273,7 +282,7 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1) skinny_kernel(const
       const int rb = tile * R + r;
       rok[r] = rb < a.nrb;
       tile_ok = tile_ok && rok[r];
-      cbase[r] = a.qw + (size_t)(rok[r] ? rb : 0) * a.nchunks * 512 + lane * 16;
+      cbase[r] = a.qw + (size_t)(rok[r] ? rb : 0) * a.nchunks * St::CB + lane * 16;
     }
     const int rbs = tile * R + sq_r;
     srok = sq_on && rbs < a.nrb;
@@ -283,22 +292,29 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1) skinny_kernel(const
     if (tile != pf_tile) set_tile(tile);
     const uint32_t base = ring_s + st * St::BYTES;
     const bool full = sc < nsc_full;
+    // a row block's codes of the stage: CPS chunks, contiguous, copied as
+    // 512-byte warp-wide pieces (the last one partial for 3-bit chunks)
+    constexpr int RB_BYTES = CPS * St::CB;
+    constexpr int PIECES = (RB_BYTES + 511) / 512;
     if (tile_ok && full) {
 #pragma unroll
       for (int r = 0; r < R; ++r) {
-        const uint8_t* src = cbase[r] + (size_t)sc * (CPS * 512);
+        const uint8_t* src = cbase[r] + (size_t)sc * RB_BYTES;
 #pragma unroll
-        for (int cc = 0; cc < CPS; ++cc)
-          cp_async16_all(base + (r * CPS + cc) * 512 + lane * 16, src + cc * 512);
+        for (int i = 0; i < PIECES; ++i)
+          if (RB_BYTES % 512 == 0 || i * 512 + lane * 16 < RB_BYTES)
+            cp_async16_all(base + r * RB_BYTES + i * 512 + lane * 16, src + i * 512);
       }
     } else {
 #pragma unroll
       for (int r = 0; r < R; ++r)
 #pragma unroll
-        for (int cc = 0; cc < CPS; ++cc) {
-          const int c = sc * CPS + cc;
+        for (int i = 0; i < PIECES; ++i) {
+          if (RB_BYTES % 512 != 0 && i * 512 + lane * 16 >= RB_BYTES) continue;
+          const int c = sc * CPS + (i * 512) / St::CB;      // chunk of the piece
           const bool ok = rok[r] && c < a.nchunks;
-          cp_async16(base + (r * CPS + cc) * 512 + lane * 16, cbase[r] + (size_t)(ok ? c : 0) * 512, ok);
+          cp_async16(base + r * RB_BYTES + i * 512 + lane * 16,
+                     cbase[r] + (ok ? (size_t)sc * RB_BYTES + i * 512 : 0), ok);
         }
     }
     const int k0 = sc * kSC;
@@ -439,12 +455,24 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1) skinny_kernel(const
       }
       float gacc[R][NT][4];
       uint4 cw[R];
+      uint32_t cw3[BITS == 3 ? R : 1][6];   // 3-bit: the lane's 24 bytes of the stage
 
 #pragma unroll
       for (int j = 0; j < kTiles; ++j) {
         const int grp = j / TPG;            // group within the stage (compile-time)
         // the lane's 16 code bytes of chunk j / 4 (4-bit) or of the stage (2-bit)
-        if ((BITS == 4 && (j & 3) == 0) || j == 0) {
+        if constexpr (BITS == 3) {
+          if (j == 0) {
+#pragma unroll
+            for (int r = 0; r < R; ++r)
+#pragma unroll
+              for (int q = 0; q < 3; ++q) {
+                const uint2 v = *reinterpret_cast<const uint2*>(st + r * St::CB + lane * 24 + 8 * q);
+                cw3[r][2 * q] = v.x;
+                cw3[r][2 * q + 1] = v.y;
+              }
+          }
+        } else if ((BITS == 4 && (j & 3) == 0) || j == 0) {
 #pragma unroll
           for (int r = 0; r < R; ++r)
             cw[r] = *reinterpret_cast<const uint4*>(st + (r * CPS + (BITS == 4 ? (j >> 2) : 0)) * 512 +
@@ -483,6 +511,28 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1) skinny_kernel(const
                 const uint2 e3 = *reinterpret_cast<const uint2*>(tabp + lop3_and_or(w >> 17, 0x7F80u, l8));
                 af[0] = e0.x; af[1] = e1.x; af[2] = e2.x; af[3] = e3.x;
                 aflo[0] = e0.y; aflo[1] = e1.y; aflo[2] = e2.y; aflo[3] = e3.y;
+              }
+            } else if constexpr (BITS == 3) {
+              // 3-bit LUT: pair p's two low bits at 16 (j % 2) + 4 p of word j / 2,
+              // its two high bits at 8 (j % 4) + 2 p of word 4 + j / 4; together
+              // a 6-bit index into the 64-entry pair table (entries 128 bytes apart)
+              const uint32_t lo = cw3[r][j >> 1], hw = cw3[r][4 + (j >> 2)];
+#pragma unroll
+              for (int p = 0; p < 4; ++p) {
+                const int sl = 16 * (j & 1) + 4 * p, sh = 8 * (j & 3) + 2 * p;
+                const uint32_t al = sl >= 7 ? lo >> (sl - 7) : lo << (7 - sl);     // bits 7..10
+                const uint32_t ah = sh >= 11 ? hw >> (sh - 11) : hw << (11 - sh);  // bits 11..12
+                if constexpr (!BF16) {
+                  const uint32_t l4 = (uint32_t)lane << 2;
+                  af[p] = *reinterpret_cast<const uint32_t*>(
+                      tabp + lop3_and_or(al, 0x780u, lop3_and_or(ah, 0x1800u, l4)));
+                } else {
+                  const uint32_t l8 = (uint32_t)(lane & 15) << 3;
+                  const uint2 e = *reinterpret_cast<const uint2*>(
+                      tabp + lop3_and_or(al, 0x780u, lop3_and_or(ah, 0x1800u, l8)));
+                  af[p] = e.x;
+                  aflo[p] = e.y;
+                }
               }
             } else {
               // 2-bit LUT: word j/2 of the lane, bytes 2 (j % 2) and 2 (j % 2) + 1
@@ -708,7 +758,8 @@ auto dispatch(int bits, int mode, bool bf16, int nt, int tpg, F&& f) {
   QMM_CASE(4, kASYM, true, 1) QMM_CASE(4, kASYM, true, 2) QMM_CASE(4, kLUT, false, 1)
   QMM_CASE(4, kLUT, false, 2) QMM_CASE(4, kLUT, true, 1) QMM_CASE(4, kLUT, true, 2)
   QMM_CASE(2, kLUT, false, 1) QMM_CASE(2, kLUT, false, 2) QMM_CASE(2, kLUT, true, 1)
-  QMM_CASE(2, kLUT, true, 2)
+  QMM_CASE(2, kLUT, true, 2) QMM_CASE(3, kLUT, false, 1) QMM_CASE(3, kLUT, false, 2)
+  QMM_CASE(3, kLUT, true, 1) QMM_CASE(3, kLUT, true, 2)
 #undef QMM_CASE
   return dispatch_tpg<4, kSYM, false, 1>(tpg, f);
 }
