@@ -478,4 +478,313 @@ int oracle_qmm_gated(const uint16_t* x, int xdtype, const uint8_t* qweight,
   return OK;
 }
 
+// ------------------------------------------------ zero-point options ([MZ])
+//
+// [MZ] (mobicham's and efrantar's replies) raises two variants of the fp16
+// zero-point: zero-points quantized to low-bit integers, and a zero-point group
+// size different from the scale group size (scale per row with a zero-point per
+// 8 weights).  Readings taken here:
+//  R18 the zero-point group zg nests inside the scale group (zg divides the
+//      scale group, group -1 counting as K); the reverse nesting is the one
+//      the page reports as useless and is not defined.
+//  R19 quantizer: s = (max - min) / 15 over the scale group (as R4), rounded to
+//      fp16; per zero-point group z = clamp(rint(-min_zg / s), 0, 15) from that
+//      group's own minimum; q = clamp(rint(w / s) + z, 0, 15).  With zg equal
+//      to the scale group this is the plain asymmetric quantizer.
+//  R20 zero storage: zbits 16 = fp16 value (as R4); zbits 4 = the same integer
+//      in 4 bits, packed [N/16][Gz][8 bytes]: the block's rows in the order of
+//      the scales (row r at slot 2 (r % 8) + r / 8), slot i at byte i / 2, the
+//      low nibble for even i.
+// Logical zeros are fp16 bit patterns [N, Gz] in every case.
+
+static int zgroup_len(int K, int zgroup) { return zgroup == -1 ? K : zgroup; }
+
+static bool zopts_ok(int K, int group, int zgroup, int zbits) {
+  if (zbits != 16 && zbits != 4) return false;
+  const int L = group_len(K, group);
+  if (zgroup != -1 && (zgroup <= 0 || K % zgroup != 0)) return false;
+  const int LZ = zgroup_len(K, zgroup);
+  return LZ <= L && L % LZ == 0;
+}
+
+// Per row: scale per group of `group`, zero-point per group of `zgroup` (R18,
+// R19).  codes[N*K], scales[N*G], zeros[N*Gz] (fp16 bits of integers).
+int oracle_quantize_asym(const float* W, int N, int K, int group, int zgroup, uint8_t* codes,
+                         uint16_t* scales, uint16_t* zeros) {
+  if (!W || !codes || !scales || !zeros || !logical_ok(N, K, MODE_ASYM, 4, group)) return ERR_ARG;
+  if (!zopts_ok(K, group, zgroup, 16)) return ERR_ARG;
+  const int G = n_groups(K, group), L = group_len(K, group);
+  const int LZ = zgroup_len(K, zgroup), GZ = K / LZ;
+  for (int n = 0; n < N; ++n) {
+    const float* row = W + (size_t)n * K;
+    for (int gi = 0; gi < G; ++gi) {
+      // the scale from the scale group's range
+      float mn = row[gi * L], mx = row[gi * L];
+      for (int i = gi * L; i < (gi + 1) * L; ++i) {
+        if (row[i] < mn) mn = row[i];
+        if (row[i] > mx) mx = row[i];
+      }
+      const uint16_t s16 = scale_bits((mx - mn) / 15.0f);
+      const float s = (float)half_value(s16);
+      scales[(size_t)n * G + gi] = s16;
+      // a zero-point per zero group inside it, from that group's minimum
+      for (int zi = gi * L / LZ; zi < (gi + 1) * L / LZ; ++zi) {
+        float zmn = row[zi * LZ];
+        for (int i = zi * LZ; i < (zi + 1) * LZ; ++i)
+          if (row[i] < zmn) zmn = row[i];
+        const int z = (s == 0.0f) ? 0 : clamp_code(std::rint(-zmn / s), 15);
+        zeros[(size_t)n * GZ + zi] = half_bits((double)z);
+        for (int i = zi * LZ; i < (zi + 1) * LZ; ++i)
+          codes[(size_t)n * K + i] =
+              (uint8_t)(s == 0.0f ? 0 : clamp_code(std::rint(row[i] / s) + (float)z, 15));
+      }
+    }
+  }
+  return OK;
+}
+
+// Packed zero buffer bytes (R20).
+size_t oracle_zeros_bytes(int N, int K, int zgroup, int zbits) {
+  const size_t GZ = (size_t)K / zgroup_len(K, zgroup);
+  return zbits == 4 ? (size_t)N * GZ / 2 : (size_t)N * GZ * 2;
+}
+
+// The integer zero-point of row n, zero group zi, as a double, from the packed
+// zero buffer (fp16 value, or the 4-bit integer of R20).
+static double packed_zero(const uint8_t* zeros_p, int n, int zi, int GZ, int zbits) {
+  const size_t idx = scale_index(n, zi, GZ);
+  if (zbits == 16) {
+    uint16_t h;
+    std::memcpy(&h, zeros_p + 2 * idx, 2);
+    return half_value(h);
+  }
+  return (double)((zeros_p[idx / 2] >> (4 * (idx % 2))) & 15);
+}
+
+// Logical (codes, scales, zeros) -> packed buffers; zeros written per R20.
+// A zero that is not an integer in [0, 15] cannot be stored in 4 bits (ERR_ARG).
+int oracle_pack_asym(const uint8_t* codes, const uint16_t* scales, const uint16_t* zeros, int N,
+                     int K, int group, int zgroup, int zbits, uint8_t* qweight,
+                     uint16_t* scales_p, uint8_t* zeros_p) {
+  if (!codes || !scales || !zeros || !qweight || !scales_p || !zeros_p) return ERR_ARG;
+  if (!shape_ok(N, K, MODE_ASYM, 4, group) || !zopts_ok(K, group, zgroup, zbits)) return ERR_ARG;
+  const int LZ = zgroup_len(K, zgroup), GZ = K / LZ;
+  if (LZ % 8 != 0) return ERR_ARG;
+  int st = oracle_pack(codes, scales, scales, N, K, MODE_SYM, 4, group, qweight, scales_p, nullptr);
+  if (st != OK) return st;
+  // SYM and ASYM place 4-bit codes identically; the zeros go separately
+  std::memset(zeros_p, 0, oracle_zeros_bytes(N, K, zgroup, zbits));
+  for (int n = 0; n < N; ++n)
+    for (int zi = 0; zi < GZ; ++zi) {
+      const uint16_t zb = zeros[(size_t)n * GZ + zi];
+      const size_t idx = scale_index(n, zi, GZ);
+      if (zbits == 16) {
+        std::memcpy(zeros_p + 2 * idx, &zb, 2);
+      } else {
+        const double z = half_value(zb);
+        if (!(z >= 0.0 && z <= 15.0 && z == std::floor(z))) return ERR_ARG;
+        zeros_p[idx / 2] |= (uint8_t)((int)z << (4 * (idx % 2)));
+      }
+    }
+  return OK;
+}
+
+// Logical codes -> exact W~[N*K] = (q - z[n, k / zg]) s[n, k / group].
+int oracle_dequant_asym(const uint8_t* codes, const uint16_t* scales, const uint16_t* zeros, int N,
+                        int K, int group, int zgroup, double* out) {
+  if (!codes || !scales || !zeros || !out || !logical_ok(N, K, MODE_ASYM, 4, group)) return ERR_ARG;
+  if (!zopts_ok(K, group, zgroup, 16)) return ERR_ARG;
+  const int G = n_groups(K, group), L = group_len(K, group);
+  const int LZ = zgroup_len(K, zgroup), GZ = K / LZ;
+  for (int n = 0; n < N; ++n)
+    for (int k = 0; k < K; ++k) {
+      const double s = half_value(scales[(size_t)n * G + k / L]);
+      const double z = half_value(zeros[(size_t)n * GZ + k / LZ]);
+      out[(size_t)n * K + k] = decode(codes[(size_t)n * K + k], s, z, nullptr, MODE_ASYM);
+    }
+  return OK;
+}
+
+// y[m, n] = sum_k x[m, k] (q - z) s read from the packed buffers, columns
+// [n0, n1), double sums in ascending k (as oracle_qmm).
+int oracle_qmm_asym(const uint16_t* x, int xdtype, const uint8_t* qweight,
+                    const uint16_t* scales_p, const uint8_t* zeros_p, int M, int N, int K,
+                    int group, int zgroup, int zbits, int n0, int n1, double* y) {
+  if (!x || !qweight || !scales_p || !zeros_p || !y || M < 0 || n0 < 0 || n1 > N || n0 > n1)
+    return ERR_ARG;
+  if (!shape_ok(N, K, MODE_ASYM, 4, group) || !zopts_ok(K, group, zgroup, zbits)) return ERR_ARG;
+  const int G = n_groups(K, group), L = group_len(K, group);
+  const int LZ = zgroup_len(K, zgroup), GZ = K / LZ;
+  double* xv = new double[(size_t)M * K];
+  double* w = new double[(size_t)K];
+  for (size_t i = 0; i < (size_t)M * K; ++i)
+    xv[i] = xdtype == DT_BF16 ? bf16_value(x[i]) : half_value(x[i]);
+  for (int n = n0; n < n1; ++n) {
+    for (int k = 0; k < K; ++k) {
+      const double s = half_value(scales_p[scale_index(n, k / L, G)]);
+      const double z = packed_zero(zeros_p, n, k / LZ, GZ, zbits);
+      w[k] = decode(get_code(qweight, n, k, K, MODE_ASYM, 4), s, z, nullptr, MODE_ASYM);
+    }
+    for (int m = 0; m < M; ++m) {
+      double acc = 0.0;
+      for (int k = 0; k < K; ++k) acc += xv[(size_t)m * K + k] * w[k];
+      y[(size_t)m * (n1 - n0) + (n - n0)] = acc;
+    }
+  }
+  delete[] xv;
+  delete[] w;
+  return OK;
+}
+
+// ------------------------------------------------------------- act-order
+//
+// [GT] "Limitations & Caveats" names GPTQ's act-order option without
+// describing it.  Reading R21 (GPTQ's convention): the quantizer visits the
+// columns in a chosen order and forms its groups along that order, so the
+// group of column k is g_idx[k] and a group is any set of columns; the weight
+// keeps its column order.  W~[n, k] = decode(q[n, k], s[n, g_idx[k]],
+// z[n, g_idx[k]]).  Packed layout: the codes of group i occupy packed columns
+// [i L, (i + 1) L), members in ascending original column (so every group must
+// hold exactly L columns); scales and zeros stay per group.
+
+static bool gidx_ok(const int* g_idx, int K, int G) {
+  for (int k = 0; k < K; ++k)
+    if (g_idx[k] < 0 || g_idx[k] >= G) return false;
+  return true;
+}
+
+// Packed column of every original column: pos[k] = g_idx[k] L + (number of
+// earlier columns in the same group).  False if a group does not hold exactly
+// L columns.
+static bool packed_columns(const int* g_idx, int K, int G, int L, int* pos) {
+  int* cnt = new int[G]();
+  bool ok = true;
+  for (int k = 0; k < K; ++k) pos[k] = g_idx[k] * L + cnt[g_idx[k]]++;
+  for (int i = 0; i < G; ++i) ok = ok && cnt[i] == L;
+  delete[] cnt;
+  return ok;
+}
+
+// Quantize with groups given by g_idx (R21); otherwise oracle_quantize's
+// arithmetic.  Reductions run over the group's members in ascending column.
+int oracle_quantize_gidx(const float* W, int N, int K, int mode, int bits, int group,
+                         const int* g_idx, const uint16_t* lut, uint8_t* codes, uint16_t* scales,
+                         uint16_t* zeros) {
+  if (!W || !g_idx || !codes || !scales || !logical_ok(N, K, mode, bits, group)) return ERR_ARG;
+  if (mode == MODE_ASYM && !zeros) return ERR_ARG;
+  if (mode == MODE_LUT && !lut) return ERR_ARG;
+  const int G = n_groups(K, group);
+  if (!gidx_ok(g_idx, K, G)) return ERR_ARG;
+  // gather each group's members into a contiguous row, quantize that row with
+  // the plain quantizer (one group per row), scatter the codes back
+  float* gw = new float[K];
+  uint8_t* gq = new uint8_t[K];
+  int* members = new int[K];
+  int st = OK;
+  for (int n = 0; n < N && st == OK; ++n)
+    for (int gi = 0; gi < G && st == OK; ++gi) {
+      int cnt = 0;
+      for (int k = 0; k < K; ++k)
+        if (g_idx[k] == gi) {
+          members[cnt] = k;
+          gw[cnt++] = W[(size_t)n * K + k];
+        }
+      if (cnt == 0) {   // an empty group: no weights, scale 0
+        scales[(size_t)n * G + gi] = 0;
+        if (mode == MODE_ASYM) zeros[(size_t)n * G + gi] = 0;
+        continue;
+      }
+      uint16_t s16, z16 = 0;
+      st = oracle_quantize(gw, 1, cnt, mode, bits, -1, lut, gq, &s16,
+                           mode == MODE_ASYM ? &z16 : nullptr);
+      scales[(size_t)n * G + gi] = s16;
+      if (mode == MODE_ASYM) zeros[(size_t)n * G + gi] = z16;
+      for (int i = 0; i < cnt; ++i) codes[(size_t)n * K + members[i]] = gq[i];
+    }
+  delete[] gw;
+  delete[] gq;
+  delete[] members;
+  return st;
+}
+
+// Logical codes -> exact W~ with per-column groups g_idx.
+int oracle_dequant_gidx(const uint8_t* codes, const uint16_t* scales, const uint16_t* zeros_or_lut,
+                        int N, int K, int mode, int bits, int group, const int* g_idx,
+                        double* out) {
+  if (!codes || !scales || !g_idx || !out || !logical_ok(N, K, mode, bits, group)) return ERR_ARG;
+  if (mode != MODE_SYM && !zeros_or_lut) return ERR_ARG;
+  const int G = n_groups(K, group);
+  if (!gidx_ok(g_idx, K, G)) return ERR_ARG;
+  for (int n = 0; n < N; ++n)
+    for (int k = 0; k < K; ++k) {
+      const int gi = g_idx[k];
+      const double s = half_value(scales[(size_t)n * G + gi]);
+      const double z = (mode == MODE_ASYM) ? half_value(zeros_or_lut[(size_t)n * G + gi]) : 0.0;
+      out[(size_t)n * K + k] = decode(codes[(size_t)n * K + k], s, z, zeros_or_lut, mode);
+    }
+  return OK;
+}
+
+// Logical codes (original column order) -> packed buffers with the act-order
+// column placement of R21.
+int oracle_pack_gidx(const uint8_t* codes, const uint16_t* scales, const uint16_t* zeros,
+                     const int* g_idx, int N, int K, int mode, int bits, int group,
+                     uint8_t* qweight, uint16_t* scales_p, uint16_t* zeros_p) {
+  if (!codes || !g_idx || !shape_ok(N, K, mode, bits, group)) return ERR_ARG;
+  const int G = n_groups(K, group), L = group_len(K, group);
+  if (!gidx_ok(g_idx, K, G)) return ERR_ARG;
+  int* pos = new int[K];
+  uint8_t* moved = new uint8_t[(size_t)N * K];
+  const bool ok = packed_columns(g_idx, K, G, L, pos);
+  int st = ERR_ARG;
+  if (ok) {
+    for (int n = 0; n < N; ++n)
+      for (int k = 0; k < K; ++k) moved[(size_t)n * K + pos[k]] = codes[(size_t)n * K + k];
+    st = oracle_pack(moved, scales, zeros, N, K, mode, bits, group, qweight, scales_p, zeros_p);
+  }
+  delete[] pos;
+  delete[] moved;
+  return st;
+}
+
+// y[m, n] = sum_k x[m, k] W~[n, k] in original column order, the code of column
+// k read at its packed column and its scale (zero) at group g_idx[k].
+int oracle_qmm_gidx(const uint16_t* x, int xdtype, const uint8_t* qweight,
+                    const uint16_t* scales_p, const uint16_t* zeros_or_lut, const int* g_idx,
+                    int M, int N, int K, int mode, int bits, int group, int n0, int n1,
+                    double* y) {
+  if (!x || !qweight || !scales_p || !g_idx || !y || M < 0 || n0 < 0 || n1 > N || n0 > n1)
+    return ERR_ARG;
+  if (!shape_ok(N, K, mode, bits, group)) return ERR_ARG;
+  if (mode != MODE_SYM && !zeros_or_lut) return ERR_ARG;
+  const int G = n_groups(K, group), L = group_len(K, group);
+  if (!gidx_ok(g_idx, K, G)) return ERR_ARG;
+  int* pos = new int[K];
+  if (!packed_columns(g_idx, K, G, L, pos)) {
+    delete[] pos;
+    return ERR_ARG;
+  }
+  double* xv = new double[(size_t)M * K];
+  double* w = new double[(size_t)K];
+  for (size_t i = 0; i < (size_t)M * K; ++i)
+    xv[i] = xdtype == DT_BF16 ? bf16_value(x[i]) : half_value(x[i]);
+  for (int n = n0; n < n1; ++n) {
+    for (int k = 0; k < K; ++k) {
+      const int gi = g_idx[k];
+      const double s = half_value(scales_p[scale_index(n, gi, G)]);
+      const double z = (mode == MODE_ASYM) ? half_value(zeros_or_lut[scale_index(n, gi, G)]) : 0.0;
+      w[k] = decode(get_code(qweight, n, pos[k], K, mode, bits), s, z, zeros_or_lut, mode);
+    }
+    for (int m = 0; m < M; ++m) {
+      double acc = 0.0;
+      for (int k = 0; k < K; ++k) acc += xv[(size_t)m * K + k] * w[k];
+      y[(size_t)m * (n1 - n0) + (n - n0)] = acc;
+    }
+  }
+  delete[] pos;
+  delete[] xv;
+  delete[] w;
+  return OK;
+}
+
 }  // extern "C"
