@@ -58,20 +58,42 @@ WORKLOADS = {
     # LLaMA-7B feed-forward gate fused into the matmul: gate and up (I = 11008
     # each, N = 2 I rows packed together), y[M, I] = silu(gate) * up
     "ffn_gated": ("sym", 4, 128, "f16", [(4096, 22016)], [1, 2, 4, 8, 16]),
+    # zero-point options (Marlin zero-point issue): scale per row with a 4-bit
+    # zero-point per 8 columns (mobicham's HQQ+ layout); and the 70B asymmetric
+    # layers with their zero-points stored in 4 bits
+    "asym_rowscale_zg8_u4": ("asym", 4, -1, "f16", [(4096, 14336)], [1, 8]),
+    "llama70b_asym_zq4_bf16": ("asym", 4, 128, "bf16",
+                               [(8192, 10240), (8192, 57344), (28672, 8192)], [1, 16]),
+    # act-order groups (GPTQ-Triton summary, Limitations): the LLaMA-7B decode
+    # layers with a random column order per matrix; x gathered per call
+    "actorder_llama7b": ("sym", 4, 128, "f16",
+                         [(4096, 12288), (4096, 4096), (4096, 22016), (11008, 4096)],
+                         [1, 2, 4, 8, 16]),
 }
 GATED = {"ffn_gated"}
+# workload -> zero-point options (zero group, zero bits)
+ZOPTS = {"asym_rowscale_zg8_u4": (8, 4), "llama70b_asym_zq4_bf16": (128, 4)}
+ACTORDER = {"actorder_llama7b"}
 SIGMA = {"sym": 0.02, "asym": 0.015, "lut": 0.02}
 L2_BYTES = 126 * 1000 * 1000     # B200 L2
 SKINNY_SOURCES = ("weight_only_quantized_int4_b200/csrc/skinny.cu",
                   "weight_only_quantized_int4_b200/csrc/common.cuh")
 
 
-def alg_bytes(mode, bits, group, M, K, N, gated=False):
+def alg_bytes(mode, bits, group, M, K, N, gated=False, zopts=None, actorder=False):
     """Bytes a call must move at least once: codes, scales (+ zeros), x, y
-    (y has N / 2 columns for the fused gate)."""
+    (y has N / 2 columns for the fused gate); with zero-point options the zero
+    records of their own group and width; with act-order the int32 column
+    permutation."""
     G = 1 if group == -1 else K // group
-    meta = N * G * 2 * (2 if mode == "asym" else 1)
-    return N * K * bits // 8 + meta + M * K * 2 + M * (N // 2 if gated else N) * 2
+    if zopts is not None:
+        zg, zbits = zopts
+        GZ = K // (K if zg == -1 else zg)
+        meta = N * G * 2 + N * GZ * zbits // 8
+    else:
+        meta = N * G * 2 * (2 if mode == "asym" else 1)
+    perm = 4 * K if actorder else 0
+    return N * K * bits // 8 + meta + perm + M * K * 2 + M * (N // 2 if gated else N) * 2
 
 
 def problems(name):
@@ -196,6 +218,8 @@ def run_ours(args, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     probs = problems(args.workload)
     gated = args.workload in GATED
+    zopts = ZOPTS.get(args.workload)
+    actorder = args.workload in ACTORDER
     gen = torch.Generator(device=dev).manual_seed(1234 + rank)
     # enough weight copies that the codes of consecutive steps never fit in L2
     codes_per_copy = sum(N * K * bits // 8 for (_, bits, _, _, _, K, N) in probs)
@@ -210,19 +234,31 @@ def run_ours(args, rank, world, local_rank):
                 from weight_only_quantized_int4_b200 import synth
                 t = {4: synth.nf4_table, 3: synth.nf3_table, 2: lambda: synth.lut2_table(0)}[bits]()
                 lut = torch.from_numpy(t.view(np.int16)).to(dev)
+            perm = None
             if gated:
                 qw, sc, ze = q.pack_gated(W[: N // 2], W[N // 2:], mode, bits, group, lut=lut)
+            elif zopts is not None:
+                qw, sc, ze = q.pack_asym(W, group, zopts[0], zopts[1])
+            elif actorder:
+                perm = torch.randperm(K, generator=gen, device=dev).to(torch.int32)
+                qw, sc, ze = q.pack_actorder(W, perm, mode, bits, group, lut=lut)
             else:
                 qw, sc, ze = q.pack(W, mode, bits, group, lut=lut)
             del W
             tdt = torch.float16 if xdt == "f16" else torch.bfloat16
             x = torch.randn(M, K, generator=gen, device=dev).to(tdt)
             y = torch.empty(M, N // 2 if gated else N, dtype=tdt, device=dev)
-            ws = q.workspace(M, N, K, mode, bits, group, device=dev)
+            if zopts is not None:
+                ws = q.workspace_asym(M, N, K, group, zopts[0], zopts[1], device=dev)
+            elif actorder:
+                ws = q.workspace_actorder(M, N, K, mode, bits, group, device=dev)
+            else:
+                ws = q.workspace(M, N, K, mode, bits, group, device=dev)
             zl = ze if mode == "asym" else lut
             calls.append(dict(x=x, qw=qw, sc=sc, zl=zl, y=y, ws=ws, M=M, N=N, K=K, mode=mode,
-                              bits=bits, group=group,
-                              bytes=alg_bytes(mode, bits, group, M, K, N, gated)))
+                              bits=bits, group=group, perm=perm,
+                              bytes=alg_bytes(mode, bits, group, M, K, N, gated, zopts,
+                                              actorder)))
         sets.append(calls)
     torch.cuda.synchronize()
     calls = sets[0]
@@ -233,6 +269,12 @@ def run_ours(args, rank, world, local_rank):
             if gated:
                 q.qmm_gated(c["x"], c["qw"], c["sc"], c["zl"], c["N"] // 2, c["K"], c["mode"],
                             c["bits"], c["group"], y=c["y"], ws=c["ws"])
+            elif zopts is not None:
+                q.qmm_asym(c["x"], c["qw"], c["sc"], c["zl"], c["N"], c["K"], c["group"],
+                           zopts[0], zopts[1], y=c["y"], ws=c["ws"])
+            elif actorder:
+                q.qmm_actorder(c["x"], c["perm"], c["qw"], c["sc"], c["zl"], c["N"], c["K"],
+                               c["mode"], c["bits"], c["group"], y=c["y"], ws=c["ws"])
             else:
                 q.qmm(c["x"], c["qw"], c["sc"], c["zl"], c["N"], c["K"], c["mode"], c["bits"],
                       c["group"], y=c["y"], ws=c["ws"])
@@ -326,7 +368,8 @@ def run_ours(args, rank, world, local_rank):
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                 "frac": round(achieved / peak, 4), "peak_source": peak_kind,
                 "traffic": None if tpb is None else round(tpb * step_bytes / len(calls)),
-                "kernel": "skinny_kernel (all launches of the step)",
+                "kernel": "skinny_kernel (all launches of the step)" if not actorder else
+                          "permute_x_kernel + skinny_kernel (all launches of the step)",
                 "algorithmic_bytes_per_launch": round(step_bytes / len(calls))}
     out = {"metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world,
            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5),
@@ -335,6 +378,8 @@ def run_ours(args, rank, world, local_rank):
            "config": {"workload": args.workload, "calls_per_step": len(calls),
                       "shapes_KN": WORKLOADS[args.workload][4], "M": WORKLOADS[args.workload][5],
                       "mode": WORKLOADS[args.workload][0], "group": WORKLOADS[args.workload][2],
+                      **({"zero_group": zopts[0], "zero_bits": zopts[1]} if zopts else {}),
+                      **({"act_order": "random column order per matrix"} if actorder else {}),
                       "l2": f"inputs larger than L2: {copies} weight cop"
                             f"{'y' if copies == 1 else 'ies'} of the step rotated, "
                             f"{copies * codes_per_copy / 1e6:.0f} MB of codes in all "
@@ -346,7 +391,7 @@ def run_ours(args, rank, world, local_rank):
                    "d2h_bytes_per_step": d2h, "steps": e2e_steps,
                    "how": f"per step: pinned x -> device, the {len(calls)} calls through the "
                           "Python API, y -> pinned host; CUDA events on the stream"},
-           "gpu_launches": len(calls) * args.steps,
+           "gpu_launches": len(calls) * args.steps * (2 if actorder else 1),
            "clocks": clocks}
     if rank == 0 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(args.workload, args.cpu_seconds)
@@ -362,6 +407,8 @@ def _oracle_sample(workload, rows_per_problem, seed=0):
     from weight_only_quantized_int4_b200 import synth
     items = []
     gated = workload in GATED
+    zopts = ZOPTS.get(workload)
+    actorder = workload in ACTORDER
     for i, (mode, bits, group, xdt, M, K, N) in enumerate(problems(workload)):
         if gated:   # whole (gate, up) block pairs
             rows_per_problem = max(32, rows_per_problem // 32 * 32)
@@ -370,25 +417,62 @@ def _oracle_sample(workload, rows_per_problem, seed=0):
         lut = None
         if mode == "lut":
             lut = {4: synth.nf4_table, 3: synth.nf3_table, 2: lambda: synth.lut2_table(0)}[bits]()
-        codes, scales, zeros = oracle.quantize(W, mode, bits, group, lut=lut)
-        qw, sp, zp = oracle.pack(codes, scales, zeros, mode, bits, group)
         x = synth.activations(seed + i, "x", M, K, xdt)
-        zl = zp if mode == "asym" else lut
-        frac = rows_per_problem / N
-        items.append((x, xdt, qw, sp, zl, M, rows_per_problem, K, mode, bits, group,
-                      frac * alg_bytes(mode, bits, group, M, K, N, gated), gated))
+        n = rows_per_problem
+        b = n / N * alg_bytes(mode, bits, group, M, K, N, gated, zopts, actorder)
+        if zopts is not None:
+            codes, scales, zeros = oracle.quantize_asym(W, group, zopts[0])
+            qw, sp, zp = oracle.pack_asym(codes, scales, zeros, group, zopts[0], zopts[1])
+            fn = (lambda a, b, x=x, xdt=xdt, qw=qw, sp=sp, zp=zp, M=M, n=n, K=K, group=group:
+                  oracle.qmm_asym(x, xdt, qw, sp, zp, M, n, K, group, zopts[0], zopts[1], a, b))
+            parts = n
+        elif actorder:
+            gidx = np.empty(K, np.int32)
+            gidx[np.random.default_rng(seed + i).permutation(K)] = np.arange(K) // group
+            codes, scales, zeros = oracle.quantize_gidx(W, mode, bits, group, gidx, lut=lut)
+            qw, sp, zp = oracle.pack_gidx(codes, scales, zeros, gidx, mode, bits, group)
+            zl = zp if mode == "asym" else lut
+            fn = (lambda a, b, x=x, xdt=xdt, qw=qw, sp=sp, zl=zl, gidx=gidx, M=M, n=n, K=K,
+                  mode=mode, bits=bits, group=group:
+                  oracle.qmm_gidx(x, xdt, qw, sp, zl, gidx, M, n, K, mode, bits, group, a, b))
+            parts = n
+        else:
+            codes, scales, zeros = oracle.quantize(W, mode, bits, group, lut=lut)
+            qw, sp, zp = oracle.pack(codes, scales, zeros, mode, bits, group)
+            zl = zp if mode == "asym" else lut
+            if gated:   # outputs i = 0 .. n/2 - 1
+                fn = (lambda a, b, x=x, xdt=xdt, qw=qw, sp=sp, zl=zl, M=M, n=n, K=K, mode=mode,
+                      bits=bits, group=group:
+                      oracle.qmm_gated(x, xdt, qw, sp, zl, M, n // 2, K, mode, bits, group, a, b))
+                parts = n // 2
+            else:
+                fn = (lambda a, b, x=x, xdt=xdt, qw=qw, sp=sp, zl=zl, M=M, n=n, K=K, mode=mode,
+                      bits=bits, group=group:
+                      oracle.qmm(x, xdt, qw, sp, zl, M, n, K, mode, bits, group, a, b))
+                parts = n
+        items.append((fn, parts, b))
     return items
 
 
+def _split_run(fn, parts, threads):
+    """fn(a, b) over [0, parts) in `threads` contiguous ranges on host threads
+    (ctypes releases the GIL during each oracle call)."""
+    bounds = np.linspace(0, parts, threads + 1).astype(int)
+    ts = [threading.Thread(target=fn, args=(int(bounds[i]), int(bounds[i + 1])))
+          for i in range(threads) if bounds[i + 1] > bounds[i]]
+    for t in ts:
+        t.start()
+    for t in ts:
+        t.join()
+
+
 def _run_oracle(items, threads):
-    import oracle
+    """Runs every sampled call, its output columns split over `threads` host
+    threads; returns (seconds, algorithmic bytes)."""
     t0 = time.perf_counter()
     total = 0.0
-    for (x, xdt, qw, sp, zl, M, n, K, mode, bits, group, b, gated) in items:
-        if gated:
-            oracle.qmm_gated(x, xdt, qw, sp, zl, M, n // 2, K, mode, bits, group)
-        else:
-            oracle.qmm_threaded(x, xdt, qw, sp, zl, M, n, K, mode, bits, group, 0, n, threads)
+    for fn, parts, b in items:
+        _split_run(fn, parts, threads)
         total += b
     return time.perf_counter() - t0, total
 

@@ -216,6 +216,73 @@ int qmm_gated(const void* x, int xdtype, const void* qweight, const uint16_t* sc
               const uint16_t* zeros_or_lut, int M, int I, int K, int bits, int group, int mode,
               void* y, void* workspace, size_t workspace_bytes, void* stream);
 
+/* ---- Zero-point options (asymmetric 4-bit codes).
+ *
+ * "Does Marlin support zero-point quantization?" (IST-DASLab/marlin issue 5):
+ * efrantar's reply names zero-points quantized to low-bit integers, and
+ * mobicham's reports HQQ+ runs with a zero-point group smaller than the
+ * scale group (scale per row, zero-point per 8 weights).  Both are supported
+ * for QMM_ASYM codes:
+ *   zgroup  the zero-point group along K: -1 (the whole row) or a power of two
+ *           >= 8 that divides K and the scale group (a zero group never
+ *           straddles two scale groups; group -1 counts as K).  Equal to
+ *           `group` gives the plain ASYM format.
+ *   zbits   16: fp16 zero-points, [N/16][K/zgroup][16] in the slot order of
+ *           the scales;  4: the integer zero-points 0..15 in 4 bits,
+ *           [N/16][K/zgroup][8 bytes], slot i at byte i / 2, low nibble for
+ *           even i.  Buffer size: qmm_zeros_size.
+ * Codes, code layout and scales are those of QMM_ASYM.  Decode:
+ *   w = (q - z[n, k / zgroup]) * s[n, k / group].
+ * qmm_pack_asym quantizes: s = (max - min) / 15 over the scale group (rounded
+ * to fp16 as in qmm_pack), then per zero group z = clamp(rint(-min_zg / s),
+ * 0, 15) from the zero group's own minimum, q = clamp(rint(w / s) + z, 0, 15).
+ * With zgroup == group and zbits == 16 every function below equals its plain
+ * QMM_ASYM counterpart byte for byte.
+ * qmm_asym runs the decode path for every M (the tensor-core path does not
+ * take these formats; M > 16 runs in slabs of 16 tokens); zeros must be
+ * 16-byte aligned; other arguments and statuses as for qmm. */
+size_t qmm_zeros_size(int N, int K, int group, int zgroup, int zbits);
+int qmm_pack_asym(const float* W, int N, int K, int group, int zgroup, int zbits, void* qweight,
+                  uint16_t* scales, void* zeros, void* stream);
+size_t qmm_workspace_size_asym(int M, int N, int K, int group, int zgroup, int zbits);
+int qmm_asym(const void* x, int xdtype, const void* qweight, const uint16_t* scales,
+             const void* zeros, int M, int N, int K, int group, int zgroup, int zbits, void* y,
+             void* workspace, size_t workspace_bytes, void* stream);
+int qmm_dequant_asym(const void* qweight, const uint16_t* scales, const void* zeros, int N, int K,
+                     int group, int zgroup, int zbits, int out_dtype, void* W_out, void* stream);
+
+/* ---- Act-order (GPTQ-Triton summary, "Limitations & Caveats": the act-order
+ * option).  A GPTQ quantizer run with act-order forms its groups along its own
+ * column order, so column k of W belongs to group g_idx[k] (int32, 0 .. K/group
+ * - 1) and every group holds `group` columns.  The packed layout keeps each
+ * group's columns together:
+ *   perm    int32 [K], device, 16-byte aligned: packed column j holds original
+ *           column perm[j]; group i occupies packed columns [i group,
+ *           (i + 1) group), its members in ascending original column.
+ * qmm_actorder_perm computes perm from g_idx on the device and writes to the
+ * device int *bad_groups the number of groups that do not hold exactly
+ * `group` columns (perm is incomplete unless it reads 0).  O(K^2 / group) work.
+ * qmm_pack_actorder is qmm_pack for the weight whose packed column j is
+ * W[:, perm[j]]: scales (zeros) are per act-order group, codes in packed
+ * order (qmm_dequant of the result gives W~ in packed column order).
+ * qmm_actorder computes y = x . W~^T over the original columns: it writes
+ * x'[m, j] = x[m, perm[j]] into the workspace and runs qmm on x'.  Workspace:
+ * qmm_workspace_size_actorder bytes (required; the first
+ * qmm_workspace_size(...) bytes, rounded up to 256, follow qmm's rules, the rest
+ * holds x'); y must overlap neither x nor the workspace.  perm entries
+ * outside [0, K) read column 0 (no access outside W or x).  Other arguments
+ * and statuses as for qmm_pack / qmm. */
+int qmm_actorder_perm(const int32_t* g_idx, int K, int group, int32_t* perm, int32_t* bad_groups,
+                      void* stream);
+int qmm_pack_actorder(const float* W, const int32_t* perm, int N, int K, int mode, int bits,
+                      int group, const uint16_t* lut, void* qweight, uint16_t* scales,
+                      uint16_t* zeros, void* stream);
+size_t qmm_workspace_size_actorder(int M, int N, int K, int bits, int group, int mode);
+int qmm_actorder(const void* x, int xdtype, const int32_t* perm, const void* qweight,
+                 const uint16_t* scales, const uint16_t* zeros_or_lut, int M, int N, int K,
+                 int bits, int group, int mode, void* y, void* workspace, size_t workspace_bytes,
+                 void* stream);
+
 /* Decode the packed weights into W_out[N, K] row-major (fp16 or bf16 by
  * out_dtype): W_out = round_to_nearest_even((q - z) * s) (SYM z = 8) or
  * round(T[q] * s), the product taken exactly in fp32 (exact for integer

@@ -675,20 +675,28 @@ int oracle_quantize_gidx(const float* W, int N, int K, int mode, int bits, int g
   if (mode == MODE_LUT && !lut) return ERR_ARG;
   const int G = n_groups(K, group);
   if (!gidx_ok(g_idx, K, G)) return ERR_ARG;
+  // the members of every group, in ascending column: group gi's are
+  // members[first[gi] .. first[gi + 1])
+  int* first = new int[G + 1]();
+  int* members = new int[K];
+  for (int k = 0; k < K; ++k) ++first[g_idx[k] + 1];
+  for (int gi = 0; gi < G; ++gi) first[gi + 1] += first[gi];
+  {
+    int* fill = new int[G];
+    for (int gi = 0; gi < G; ++gi) fill[gi] = first[gi];
+    for (int k = 0; k < K; ++k) members[fill[g_idx[k]]++] = k;
+    delete[] fill;
+  }
   // gather each group's members into a contiguous row, quantize that row with
   // the plain quantizer (one group per row), scatter the codes back
   float* gw = new float[K];
   uint8_t* gq = new uint8_t[K];
-  int* members = new int[K];
   int st = OK;
   for (int n = 0; n < N && st == OK; ++n)
     for (int gi = 0; gi < G && st == OK; ++gi) {
-      int cnt = 0;
-      for (int k = 0; k < K; ++k)
-        if (g_idx[k] == gi) {
-          members[cnt] = k;
-          gw[cnt++] = W[(size_t)n * K + k];
-        }
+      const int* mem = members + first[gi];
+      const int cnt = first[gi + 1] - first[gi];
+      for (int i = 0; i < cnt; ++i) gw[i] = W[(size_t)n * K + mem[i]];
       if (cnt == 0) {   // an empty group: no weights, scale 0
         scales[(size_t)n * G + gi] = 0;
         if (mode == MODE_ASYM) zeros[(size_t)n * G + gi] = 0;
@@ -699,11 +707,12 @@ int oracle_quantize_gidx(const float* W, int N, int K, int mode, int bits, int g
                            mode == MODE_ASYM ? &z16 : nullptr);
       scales[(size_t)n * G + gi] = s16;
       if (mode == MODE_ASYM) zeros[(size_t)n * G + gi] = z16;
-      for (int i = 0; i < cnt; ++i) codes[(size_t)n * K + members[i]] = gq[i];
+      for (int i = 0; i < cnt; ++i) codes[(size_t)n * K + mem[i]] = gq[i];
     }
   delete[] gw;
   delete[] gq;
   delete[] members;
+  delete[] first;
   return st;
 }
 

@@ -105,3 +105,59 @@ def test_strerror_covers_every_status(lib):
     for s in (0, -1, -2, -3, -4, -5, -6):
         assert q.strerror(s) != "unknown status"
     assert q.strerror(-99) == "unknown status"
+
+
+def test_zero_point_options_sizes_and_rejections(lib):
+    # 4-bit zero records: N * (K / zgroup) / 2 bytes; fp16: N * (K / zgroup) * 2
+    assert lib.qmm_zeros_size(4096, 14336, -1, 8, 4) == 4096 * 1792 // 2
+    assert lib.qmm_zeros_size(4096, 14336, -1, 8, 16) == 4096 * 1792 * 2
+    assert lib.qmm_zeros_size(64, 1024, 128, 128, 4) == 64 * 8 // 2
+    assert lib.qmm_zeros_size(64, 1024, -1, -1, 4) == 64 // 2
+    for group, zgroup, zbits in ((64, 128, 4), (-1, 24, 4), (-1, 4, 4), (-1, 8, 8),
+                                 (128, 8, 2)):
+        assert lib.qmm_zeros_size(64, 1024, group, zgroup, zbits) == 0
+    P = ctypes.c_void_p
+    fake = P(0x1000)
+    # zero group larger than the scale group; zbits not 4 / 16; zeros missing or misaligned
+    assert lib.qmm_asym(fake, 0, fake, fake, fake, 1, 64, 1024, 64, 128, 4, P(0x900000), None, 0,
+                        None) == -2
+    assert lib.qmm_asym(fake, 0, fake, fake, fake, 1, 64, 1024, -1, 8, 8, P(0x900000), None, 0,
+                        None) == -1
+    assert lib.qmm_asym(fake, 0, fake, fake, None, 1, 64, 1024, -1, 8, 4, P(0x900000), None, 0,
+                        None) == -1
+    assert lib.qmm_asym(fake, 0, fake, fake, P(0x1008), 1, 64, 1024, -1, 8, 4, P(0x900000), None,
+                        0, None) == -3
+    assert lib.qmm_pack_asym(fake, 64, 1024, -1, 8, 4, fake, fake, None, None) == -1
+    assert lib.qmm_pack_asym(fake, 64, 1024, 64, 128, 4, fake, fake, fake, None) == -2
+    assert lib.qmm_dequant_asym(fake, fake, fake, 64, 1024, -1, 8, 4, 3, fake, None) == -1
+    # the options only take 4-bit ASYM codes: the shape rules of qmm apply
+    assert lib.qmm_asym(fake, 0, fake, fake, fake, 1, 60, 1024, -1, 8, 4, P(0x900000), None, 0,
+                        None) == -2
+
+
+def test_actorder_argument_checks(lib):
+    P = ctypes.c_void_p
+    fake = P(0x1000)
+    # perm from g_idx: bad group, bad K, null pointers
+    assert lib.qmm_actorder_perm(fake, 1024, 48, fake, fake, None) == -2
+    assert lib.qmm_actorder_perm(fake, 0, 128, fake, fake, None) == -1
+    assert lib.qmm_actorder_perm(fake, 1024, 128, None, fake, None) == -1
+    # pack: perm required and 16-byte aligned
+    assert lib.qmm_pack_actorder(fake, None, 64, 1024, 0, 4, 128, None, fake, fake, None,
+                                 None) == -1
+    assert lib.qmm_pack_actorder(fake, P(0x1004), 64, 1024, 0, 4, 128, None, fake, fake, None,
+                                 None) == -3
+    # the product needs its workspace (x is gathered into it)
+    n = lib.qmm_workspace_size_actorder(3, 64, 1024, 4, 128, 0)
+    plain = lib.qmm_workspace_size(3, 64, 1024, 4, 128, 0)
+    assert n == (plain + 255) // 256 * 256 + 3 * 1024 * 2
+    assert lib.qmm_actorder(fake, 0, fake, fake, fake, None, 3, 64, 1024, 4, 128, 0,
+                            P(0x900000), None, 0, None) == -6
+    assert lib.qmm_actorder(fake, 0, fake, fake, fake, None, 3, 64, 1024, 4, 128, 0,
+                            P(0x900000), P(0x100000), n - 256, None) == -6
+    # y overlapping the workspace
+    assert lib.qmm_actorder(fake, 0, fake, fake, fake, None, 3, 64, 1024, 4, 128, 0,
+                            P(0x100100), P(0x100000), n, None) == -1
+    # M == 0 is a no-op
+    assert lib.qmm_actorder(fake, 0, fake, fake, fake, None, 0, 64, 1024, 4, 128, 0,
+                            P(0x900000), None, 0, None) == 0

@@ -29,7 +29,9 @@ PATH_NAMES = {1: "skinny", 2: "tensor"}
 SYMBOLS = ("qmm_packed_size", "qmm_pack", "qmm_workspace_size", "qmm_workspace_size_for", "qmm",
            "qmm_with_path",
            "qmm_path", "qmm_dequant", "qmm_check_error", "qmm_strerror", "qmm_noalloc",
-           "qmm_pack_gated", "qmm_gated")
+           "qmm_pack_gated", "qmm_gated", "qmm_zeros_size", "qmm_pack_asym",
+           "qmm_workspace_size_asym", "qmm_asym", "qmm_dequant_asym", "qmm_actorder_perm",
+           "qmm_pack_actorder", "qmm_workspace_size_actorder", "qmm_actorder")
 
 _lib = None
 _lock = threading.Lock()
@@ -65,6 +67,18 @@ def load(path: str = LIB_PATH):
             lib.qmm_pack_gated.argtypes = [P, P, I, I, I, I, I, P, P, P, P, P]
             lib.qmm_gated.argtypes = [P, I, P, P, P, I, I, I, I, I, I, P, P, S, P]
             lib.qmm_dequant.argtypes = [P, P, P, I, I, I, I, I, I, P, P]
+            lib.qmm_zeros_size.argtypes = [I, I, I, I, I]
+            lib.qmm_zeros_size.restype = S
+            lib.qmm_pack_asym.argtypes = [P, I, I, I, I, I, P, P, P, P]
+            lib.qmm_workspace_size_asym.argtypes = [I, I, I, I, I, I]
+            lib.qmm_workspace_size_asym.restype = S
+            lib.qmm_asym.argtypes = [P, I, P, P, P, I, I, I, I, I, I, P, P, S, P]
+            lib.qmm_dequant_asym.argtypes = [P, P, P, I, I, I, I, I, I, P, P]
+            lib.qmm_actorder_perm.argtypes = [P, I, I, P, P, P]
+            lib.qmm_pack_actorder.argtypes = [P, P, I, I, I, I, I, P, P, P, P, P]
+            lib.qmm_workspace_size_actorder.argtypes = [I, I, I, I, I, I]
+            lib.qmm_workspace_size_actorder.restype = S
+            lib.qmm_actorder.argtypes = [P, I, P, P, P, P, I, I, I, I, I, I, P, P, S, P]
             lib.qmm_check_error.argtypes = [P]
             lib.qmm_strerror.argtypes = [I]
             lib.qmm_strerror.restype = ctypes.c_char_p
@@ -214,6 +228,110 @@ def dequant(qweight, scales, zeros_or_lut, N, K, mode, bits=4, group=128, dtype=
                               MODES[mode], DTYPES[out.dtype], _ptr(out), _stream()),
            "qmm_dequant")
     return out
+
+
+# ---- zero-point options: zero group inside the scale group, fp16 or 4-bit zeros
+
+def pack_asym(W, group=-1, zgroup=8, zbits=4):
+    """Quantize fp32 W[N, K] (CUDA) into ASYM codes with zero-points per group
+    of `zgroup` (fp16 or 4-bit) -> (qweight uint8, scales int16 bits, zeros uint8 bytes)."""
+    _dev(W, "W")
+    N, K = W.shape
+    qb, sb, _ = packed_size(N, K, "asym", 4, group)
+    zb = load().qmm_zeros_size(N, K, group, zgroup, zbits)
+    if zb == 0:
+        raise QmmError(-2, "qmm_zeros_size")
+    qw = torch.empty(qb, dtype=torch.uint8, device=W.device)
+    sc = torch.empty(sb // 2, dtype=torch.int16, device=W.device)
+    ze = torch.empty(zb, dtype=torch.uint8, device=W.device)
+    _check(load().qmm_pack_asym(_ptr(W), N, K, group, zgroup, zbits, _ptr(qw), _ptr(sc), _ptr(ze),
+                                _stream()), "qmm_pack_asym")
+    return qw, sc, ze
+
+
+def workspace_asym(M, N, K, group, zgroup, zbits, device="cuda"):
+    n = load().qmm_workspace_size_asym(M, N, K, group, zgroup, zbits)
+    return torch.zeros(n, dtype=torch.uint8, device=device) if n else None
+
+
+def qmm_asym(x, qweight, scales, zeros, N, K, group=-1, zgroup=8, zbits=4, y=None, ws=None):
+    """y = x . dequant(qweight)^T for a pack_asym buffer."""
+    _dev(x, "x")
+    if x.dtype not in DTYPES:
+        raise ValueError("x must be fp16 or bf16")
+    M = x.shape[0]
+    if x.shape[1] != K:
+        raise ValueError("x.shape[1] != K")
+    if y is None:
+        y = torch.empty(M, N, dtype=x.dtype, device=x.device)
+    nbytes = 0 if ws is None else ws.numel() * ws.element_size()
+    _check(load().qmm_asym(_ptr(x), DTYPES[x.dtype], _ptr(qweight), _ptr(scales), _ptr(zeros), M,
+                           N, K, group, zgroup, zbits, _ptr(y), _ptr(ws), nbytes, _stream()),
+           "qmm_asym")
+    return y
+
+
+def dequant_asym(qweight, scales, zeros, N, K, group=-1, zgroup=8, zbits=4, dtype=torch.float16):
+    out = torch.empty(N, K, dtype=dtype, device=qweight.device)
+    _check(load().qmm_dequant_asym(_ptr(qweight), _ptr(scales), _ptr(zeros), N, K, group, zgroup,
+                                   zbits, DTYPES[out.dtype], _ptr(out), _stream()),
+           "qmm_dequant_asym")
+    return out
+
+
+# ---- act-order: per-column groups
+
+def actorder_perm(g_idx, group):
+    """perm (int32 [K], CUDA) from g_idx (int32 [K], CUDA); raises if a group
+    does not hold exactly `group` columns (synchronizes the stream)."""
+    _dev(g_idx, "g_idx")
+    K = g_idx.shape[0]
+    perm = torch.empty(K, dtype=torch.int32, device=g_idx.device)
+    bad = torch.zeros(1, dtype=torch.int32, device=g_idx.device)
+    _check(load().qmm_actorder_perm(_ptr(g_idx), K, group, _ptr(perm), _ptr(bad), _stream()),
+           "qmm_actorder_perm")
+    if int(bad.item()) != 0:
+        raise ValueError(f"g_idx: {int(bad.item())} groups do not hold exactly {group} columns")
+    return perm
+
+
+def pack_actorder(W, perm, mode, bits=4, group=128, lut=None):
+    """Quantize fp32 W[N, K] with act-order groups: packed column j = W[:, perm[j]]."""
+    _dev(W, "W")
+    _dev(perm, "perm")
+    N, K = W.shape
+    qb, sb, zb = packed_size(N, K, mode, bits, group)
+    qw = torch.empty(qb, dtype=torch.uint8, device=W.device)
+    sc = torch.empty(sb // 2, dtype=torch.int16, device=W.device)
+    ze = torch.empty(zb // 2, dtype=torch.int16, device=W.device) if zb else None
+    _check(load().qmm_pack_actorder(_ptr(W), _ptr(perm), N, K, MODES[mode], bits, group, _ptr(lut),
+                                    _ptr(qw), _ptr(sc), _ptr(ze), _stream()), "qmm_pack_actorder")
+    return qw, sc, ze
+
+
+def workspace_actorder(M, N, K, mode, bits=4, group=128, device="cuda"):
+    n = load().qmm_workspace_size_actorder(M, N, K, bits, group, MODES[mode])
+    return torch.zeros(n, dtype=torch.uint8, device=device)
+
+
+def qmm_actorder(x, perm, qweight, scales, zeros_or_lut, N, K, mode, bits=4, group=128, y=None,
+                 ws=None):
+    """y = x . W~^T over the original columns for a pack_actorder buffer."""
+    _dev(x, "x")
+    if x.dtype not in DTYPES:
+        raise ValueError("x must be fp16 or bf16")
+    M = x.shape[0]
+    if x.shape[1] != K:
+        raise ValueError("x.shape[1] != K")
+    if y is None:
+        y = torch.empty(M, N, dtype=x.dtype, device=x.device)
+    if ws is None:
+        ws = workspace_actorder(M, N, K, mode, bits, group, device=x.device)
+    nbytes = ws.numel() * ws.element_size()
+    _check(load().qmm_actorder(_ptr(x), DTYPES[x.dtype], _ptr(perm), _ptr(qweight), _ptr(scales),
+                               _ptr(zeros_or_lut), M, N, K, bits, group, MODES[mode], _ptr(y),
+                               _ptr(ws), nbytes, _stream()), "qmm_actorder")
+    return y
 
 
 def check_error():

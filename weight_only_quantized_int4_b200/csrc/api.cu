@@ -41,6 +41,27 @@ int check_shape(int N, int K, int bits, int group, int mode) {
 
 int status_of(cudaError_t e) { return e == cudaSuccess ? QMM_OK : QMM_ERR_CUDA; }
 
+// Zero-point options: zbits 16 (fp16) or 4; the zero group is -1 (the row) or
+// a power of two >= 8 that divides K and nests inside the scale group.
+int check_zopts(int K, int group, int zgroup, int zbits) {
+  if (zbits != 16 && zbits != 4) return QMM_ERR_ARG;
+  if (zgroup != -1 && (zgroup < 8 || (zgroup & (zgroup - 1)) != 0 || K % zgroup != 0))
+    return QMM_ERR_UNSUPPORTED;
+  const int L = group == -1 ? K : group, LZ = zgroup == -1 ? K : zgroup;
+  if (LZ > L || L % LZ != 0) return QMM_ERR_UNSUPPORTED;
+  return QMM_OK;
+}
+
+// Internal (mode, zgroup) of an ASYM format with zero-point options: the plain
+// ASYM format when the zero group is the scale group and zeros are fp16.
+void zero_mode(int K, int group, int zgroup, int zbits, int* mode, int* zg) {
+  const int L = group == -1 ? K : group, LZ = zgroup == -1 ? K : zgroup;
+  *zg = LZ == L ? 0 : zgroup;
+  *mode = zbits == 4 ? kASYMQ : (*zg == 0 ? QMM_ASYM : kASYMX);
+}
+
+size_t round256(size_t b) { return (b + 255) / 256 * 256; }
+
 // Decode path while the product is bandwidth-bound (few tokens), tensor-core
 // path once it becomes a dense contraction.  Combinations the tensor path does
 // not cover (2-bit codes; bf16 with group scales or a table) take the decode
@@ -58,6 +79,7 @@ struct Plan {
   size_t ws_bytes() const { return path == QMM_PATH_TENSOR ? tc.ws_bytes : sk.ws_bytes; }
 };
 
+// `mode` may be an internal zero-point-options mode (kASYMX, kASYMQ).
 Plan make_plan(int M, int N, int K, int bits, int group, int mode, bool bf16, int path) {
   Plan p{};
   const bool streamk = path == QMM_PATH_SKINNY_STREAMK;
@@ -78,9 +100,9 @@ using namespace qk;
 static int run_qmm(const void* x, int xdtype, const void* qweight, const uint16_t* scales,
                    const uint16_t* zeros_or_lut, int M, int N, int K, int bits, int group,
                    int mode, void* y, void* workspace, size_t workspace_bytes, void* stream,
-                   int path, bool gated) {
+                   int path, bool gated, int zgroup = 0, int zbits = 16) {
   if (M < 0) return QMM_ERR_ARG;
-  int st = check_shape(N, K, bits, group, mode);
+  int st = check_shape(N, K, bits, group, zero_opts(mode) ? QMM_ASYM : mode);
   if (st != QMM_OK) return st;
   if (xdtype != QMM_F16 && xdtype != QMM_BF16) return QMM_ERR_ARG;
   if (path < QMM_PATH_AUTO || path > QMM_PATH_SKINNY_STREAMK) return QMM_ERR_ARG;
@@ -88,7 +110,8 @@ static int run_qmm(const void* x, int xdtype, const void* qweight, const uint16_
   if (!x || !qweight || !scales || !y) return QMM_ERR_ARG;
   if (mode != QMM_SYM && !zeros_or_lut) return QMM_ERR_ARG;
   if (!aligned(x, 16) || !aligned(qweight, 16) || !aligned(scales, 16) || !aligned(y, 2) ||
-      (mode == QMM_ASYM && !aligned(zeros_or_lut, 16)) || (workspace && !aligned(workspace, 256)))
+      ((mode == QMM_ASYM || zero_opts(mode)) && !aligned(zeros_or_lut, 16)) ||
+      (workspace && !aligned(workspace, 256)))
     return QMM_ERR_ALIGN;
   {
     const char* xb = static_cast<const char*>(x);
@@ -98,6 +121,8 @@ static int run_qmm(const void* x, int xdtype, const void* qweight, const uint16_
   }
   Problem p{x, xdtype == QMM_BF16, qweight, scales, zeros_or_lut, M, N, K, bits, group, mode, y};
   p.gated = gated;
+  p.zgroup = zgroup;
+  p.zbits = zbits;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   Plan plan = make_plan(M, N, K, bits, group, mode, xdtype == QMM_BF16, path);
   if (plan.ws_bytes()) {
@@ -141,8 +166,8 @@ int qmm_pack(const float* W, int N, int K, int mode, int bits, int group, const 
   if (!aligned(W, 16) || !aligned(qweight, 16) || !aligned(scales, 16) ||
       (zeros && !aligned(zeros, 16)))
     return QMM_ERR_ALIGN;
-  return status_of(launch_pack(W, nullptr, N, K, mode, bits, group, lut, qweight, scales, zeros,
-                               static_cast<cudaStream_t>(stream)));
+  return status_of(launch_pack(W, nullptr, nullptr, N, K, mode, bits, group, 0, 16, lut, qweight,
+                               scales, zeros, static_cast<cudaStream_t>(stream)));
 }
 
 int qmm_pack_gated(const float* Wg, const float* Wu, int I, int K, int mode, int bits, int group,
@@ -158,8 +183,8 @@ int qmm_pack_gated(const float* Wg, const float* Wu, int I, int K, int mode, int
   if (!aligned(Wg, 16) || !aligned(Wu, 16) || !aligned(qweight, 16) || !aligned(scales, 16) ||
       (zeros && !aligned(zeros, 16)))
     return QMM_ERR_ALIGN;
-  return status_of(launch_pack(Wg, Wu, 2 * I, K, mode, bits, group, lut, qweight, scales, zeros,
-                               static_cast<cudaStream_t>(stream)));
+  return status_of(launch_pack(Wg, Wu, nullptr, 2 * I, K, mode, bits, group, 0, 16, lut, qweight,
+                               scales, zeros, static_cast<cudaStream_t>(stream)));
 }
 
 int qmm_path(int M, int N, int K, int bits, int group, int mode) {
@@ -241,8 +266,137 @@ int qmm_dequant(const void* qweight, const uint16_t* scales, const uint16_t* zer
   if (!qweight || !scales || !W_out) return QMM_ERR_ARG;
   if (mode != QMM_SYM && !zeros_or_lut) return QMM_ERR_ARG;
   if (!aligned(qweight, 16) || !aligned(W_out, 8)) return QMM_ERR_ALIGN;
-  return status_of(launch_dequant(qweight, scales, zeros_or_lut, N, K, bits, group, mode,
+  return status_of(launch_dequant(qweight, scales, zeros_or_lut, N, K, bits, group, 0, 16, mode,
                                   out_dtype, W_out, static_cast<cudaStream_t>(stream)));
+}
+
+// ------------------------------------------------------ zero-point options
+
+size_t qmm_zeros_size(int N, int K, int group, int zgroup, int zbits) {
+  if (check_shape(N, K, 4, group, QMM_ASYM) != QMM_OK) return 0;
+  if (check_zopts(K, group, zgroup, zbits) != QMM_OK) return 0;
+  const size_t GZ = (size_t)K / (zgroup == -1 ? K : zgroup);
+  return zbits == 4 ? (size_t)N * GZ / 2 : (size_t)N * GZ * 2;
+}
+
+int qmm_pack_asym(const float* W, int N, int K, int group, int zgroup, int zbits, void* qweight,
+                  uint16_t* scales, void* zeros, void* stream) {
+  int st = check_shape(N, K, 4, group, QMM_ASYM);
+  if (st != QMM_OK) return st;
+  st = check_zopts(K, group, zgroup, zbits);
+  if (st != QMM_OK) return st;
+  if (!W || !qweight || !scales || !zeros) return QMM_ERR_ARG;
+  if (!aligned(W, 16) || !aligned(qweight, 16) || !aligned(scales, 16) || !aligned(zeros, 16))
+    return QMM_ERR_ALIGN;
+  int mode, zg;
+  zero_mode(K, group, zgroup, zbits, &mode, &zg);
+  return status_of(launch_pack(W, nullptr, nullptr, N, K, QMM_ASYM, 4, group, zg, zbits, nullptr,
+                               qweight, scales, zeros, static_cast<cudaStream_t>(stream)));
+}
+
+size_t qmm_workspace_size_asym(int M, int N, int K, int group, int zgroup, int zbits) {
+  if (M <= 0 || check_shape(N, K, 4, group, QMM_ASYM) != QMM_OK) return 0;
+  if (check_zopts(K, group, zgroup, zbits) != QMM_OK) return 0;
+  int mode, zg;
+  zero_mode(K, group, zgroup, zbits, &mode, &zg);
+  return std::max(make_plan(M, N, K, 4, group, mode, false, QMM_PATH_AUTO).ws_bytes(),
+                  make_plan(M, N, K, 4, group, mode, true, QMM_PATH_AUTO).ws_bytes());
+}
+
+int qmm_asym(const void* x, int xdtype, const void* qweight, const uint16_t* scales,
+             const void* zeros, int M, int N, int K, int group, int zgroup, int zbits, void* y,
+             void* workspace, size_t workspace_bytes, void* stream) {
+  int st = check_shape(N, K, 4, group, QMM_ASYM);
+  if (st != QMM_OK) return st;
+  st = check_zopts(K, group, zgroup, zbits);
+  if (st != QMM_OK) return st;
+  int mode, zg;
+  zero_mode(K, group, zgroup, zbits, &mode, &zg);
+  return run_qmm(x, xdtype, qweight, scales, static_cast<const uint16_t*>(zeros), M, N, K, 4,
+                 group, mode, y, workspace, workspace_bytes, stream, QMM_PATH_AUTO, false, zg,
+                 zbits);
+}
+
+int qmm_dequant_asym(const void* qweight, const uint16_t* scales, const void* zeros, int N, int K,
+                     int group, int zgroup, int zbits, int out_dtype, void* W_out, void* stream) {
+  int st = check_shape(N, K, 4, group, QMM_ASYM);
+  if (st != QMM_OK) return st;
+  st = check_zopts(K, group, zgroup, zbits);
+  if (st != QMM_OK) return st;
+  if (out_dtype != QMM_F16 && out_dtype != QMM_BF16) return QMM_ERR_ARG;
+  if (!qweight || !scales || !zeros || !W_out) return QMM_ERR_ARG;
+  if (!aligned(qweight, 16) || !aligned(W_out, 8)) return QMM_ERR_ALIGN;
+  int mode, zg;
+  zero_mode(K, group, zgroup, zbits, &mode, &zg);
+  return status_of(launch_dequant(qweight, scales, zeros, N, K, 4, group, zg, zbits, QMM_ASYM,
+                                  out_dtype, W_out, static_cast<cudaStream_t>(stream)));
+}
+
+// ---------------------------------------------------------------- act-order
+
+int qmm_actorder_perm(const int32_t* g_idx, int K, int group, int32_t* perm, int32_t* bad_groups,
+                      void* stream) {
+  if (K <= 0 || K > (1 << 20)) return K <= 0 ? QMM_ERR_ARG : QMM_ERR_UNSUPPORTED;
+  if (group != -1 && (group < 16 || (group & (group - 1)) != 0 || K % group != 0))
+    return QMM_ERR_UNSUPPORTED;
+  if (!g_idx || !perm || !bad_groups) return QMM_ERR_ARG;
+  if (!aligned(g_idx, 4) || !aligned(perm, 4) || !aligned(bad_groups, 4)) return QMM_ERR_ALIGN;
+  return status_of(launch_gidx_perm(g_idx, K, group, perm, bad_groups,
+                                    static_cast<cudaStream_t>(stream)));
+}
+
+int qmm_pack_actorder(const float* W, const int32_t* perm, int N, int K, int mode, int bits,
+                      int group, const uint16_t* lut, void* qweight, uint16_t* scales,
+                      uint16_t* zeros, void* stream) {
+  int st = check_shape(N, K, bits, group, mode);
+  if (st != QMM_OK) return st;
+  if (!W || !perm || !qweight || !scales) return QMM_ERR_ARG;
+  if (mode == QMM_ASYM && !zeros) return QMM_ERR_ARG;
+  if (mode == QMM_LUT && !lut) return QMM_ERR_ARG;
+  if (!aligned(W, 16) || !aligned(perm, 16) || !aligned(qweight, 16) || !aligned(scales, 16) ||
+      (zeros && !aligned(zeros, 16)))
+    return QMM_ERR_ALIGN;
+  return status_of(launch_pack(W, nullptr, perm, N, K, mode, bits, group, 0, 16, lut, qweight,
+                               scales, zeros, static_cast<cudaStream_t>(stream)));
+}
+
+size_t qmm_workspace_size_actorder(int M, int N, int K, int bits, int group, int mode) {
+  if (M <= 0 || check_shape(N, K, bits, group, mode) != QMM_OK) return 0;
+  return round256(qmm_workspace_size(M, N, K, bits, group, mode)) + round256((size_t)M * K * 2);
+}
+
+int qmm_actorder(const void* x, int xdtype, const int32_t* perm, const void* qweight,
+                 const uint16_t* scales, const uint16_t* zeros_or_lut, int M, int N, int K,
+                 int bits, int group, int mode, void* y, void* workspace, size_t workspace_bytes,
+                 void* stream) {
+  if (M < 0) return QMM_ERR_ARG;
+  int st = check_shape(N, K, bits, group, mode);
+  if (st != QMM_OK) return st;
+  if (xdtype != QMM_F16 && xdtype != QMM_BF16) return QMM_ERR_ARG;
+  if (M == 0) return QMM_OK;
+  if (!x || !perm || !y || !qweight || !scales) return QMM_ERR_ARG;
+  if (mode != QMM_SYM && !zeros_or_lut) return QMM_ERR_ARG;
+  if (!aligned(x, 16) || !aligned(perm, 16) || !aligned(qweight, 16) || !aligned(scales, 16) ||
+      !aligned(y, 2) || (mode == QMM_ASYM && !aligned(zeros_or_lut, 16)) ||
+      (workspace && !aligned(workspace, 256)))
+    return QMM_ERR_ALIGN;
+  // the workspace holds the product's own workspace, then x in packed column order
+  const size_t plain = round256(qmm_workspace_size(M, N, K, bits, group, mode));
+  if (!workspace || workspace_bytes < plain + (size_t)M * K * 2) return QMM_ERR_WORKSPACE;
+  {
+    const char* xb = static_cast<const char*>(x);
+    const char* yb = static_cast<const char*>(y);
+    const char* wb = static_cast<const char*>(workspace);
+    const size_t xs = (size_t)M * K * 2, ys = (size_t)M * N * 2, ws = plain + xs;
+    if (xb < yb + ys && yb < xb + xs) return QMM_ERR_ARG;   // y overlaps x
+    if (wb < yb + ys && yb < wb + ws) return QMM_ERR_ARG;   // y overlaps the workspace
+  }
+  void* xp = static_cast<char*>(workspace) + plain;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  st = status_of(launch_permute_x(x, perm, M, K, xp, s));
+  if (st != QMM_OK) return st;
+  return run_qmm(xp, xdtype, qweight, scales, zeros_or_lut, M, N, K, bits, group, mode, y,
+                 workspace, plain, stream, QMM_PATH_AUTO, false);
 }
 
 int qmm_check_error(void* stream) {

@@ -18,6 +18,9 @@ struct Problem {
   int M, N, K, bits, group, mode;
   void* y;
   bool gated = false;     // fused gate/up rows: y[M, N/2] = silu(gate) * up
+  // ASYM zero-point options (modes kASYMX / kASYMQ): zero group (columns; 0 =
+  // the scale group, -1 = the row) and storage (16 = fp16, 4 = 4-bit integers)
+  int zgroup = 0, zbits = 16;
 };
 
 // Split-K plan of the skinny (M <= 16 per slab) decode path.
@@ -55,12 +58,23 @@ TcPlan plan_tc(int M, int N, int K, int sms);
 cudaError_t launch_tc(const Problem& p, const TcPlan& plan, void* workspace, cudaStream_t stream);
 unsigned tc_read_and_clear_error();
 
-cudaError_t launch_pack(const float* W, const float* W2, int N, int K, int mode, int bits,
-                        int group, const uint16_t* lut, void* qweight, uint16_t* scales,
-                        uint16_t* zeros, cudaStream_t stream);
+// Quantize + pack.  W2: second matrix of the gated layout (else null); perm:
+// act-order column permutation (else null); zgroup / zbits: ASYM zero-point
+// options (0 / 16 for the plain format).
+cudaError_t launch_pack(const float* W, const float* W2, const int* perm, int N, int K, int mode,
+                        int bits, int group, int zgroup, int zbits, const uint16_t* lut,
+                        void* qweight, uint16_t* scales, void* zeros, cudaStream_t stream);
 cudaError_t launch_dequant(const void* qweight, const uint16_t* scales,
-                           const uint16_t* zeros_or_lut, int N, int K, int bits, int group,
-                           int mode, int out_dtype, void* W_out, cudaStream_t stream);
+                           const void* zeros_or_lut, int N, int K, int bits, int group,
+                           int zgroup, int zbits, int mode, int out_dtype, void* W_out,
+                           cudaStream_t stream);
+
+// Act-order: perm from per-column group indices (*bad counts groups without
+// exactly `group` members), and x'[m, j] = x[m, perm[j]].
+cudaError_t launch_gidx_perm(const int* g_idx, int K, int group, int* perm, int* bad,
+                             cudaStream_t stream);
+cudaError_t launch_permute_x(const void* x, const int* perm, int M, int K, void* xp,
+                             cudaStream_t stream);
 
 int device_sms();
 

@@ -32,6 +32,14 @@ __device__ __forceinline__ uint16_t scale_to_half(float s32) {
   return b;
 }
 
+// Column k of a source row; with an act-order permutation, packed column k
+// takes original column perm[k] (entries outside [0, K) read column 0).
+__device__ __forceinline__ float wcol(const float* row, const int* perm, int k, int K) {
+  if (!perm) return row[k];
+  const unsigned c = (unsigned)perm[k];
+  return row[c < (unsigned)K ? c : 0u];
+}
+
 // Source row of packed row n.  With a second matrix W2 (the gated layout),
 // 16-row blocks alternate: packed block 2b is block b of W, block 2b + 1 is
 // block b of W2.
@@ -42,20 +50,22 @@ __device__ __forceinline__ const float* src_row(const float* W, const float* W2,
 }
 
 // One warp per (row n, group gi): reduce |w| or (min, max) over the group,
-// write the fp16 scale (and zero) at the packed position.
+// write the fp16 scale (and, if `zeros` is given, the zero) at the packed
+// position.
 __global__ void __launch_bounds__(256) pack_scales_kernel(const float* __restrict__ W,
-                                                          const float* __restrict__ W2, int N, int K,
-                                                          int mode, int L, int G,
+                                                          const float* __restrict__ W2,
+                                                          const int* __restrict__ perm, int N,
+                                                          int K, int mode, int L, int G,
                                                           uint16_t* __restrict__ scales,
                                                           uint16_t* __restrict__ zeros) {
   const long long warp = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (warp >= (long long)N * G) return;
   const int n = (int)(warp / G), gi = (int)(warp % G);
-  const float* w = src_row(W, W2, n, K) + (size_t)gi * L;
+  const float* row = src_row(W, W2, n, K);
   float amax = 0.0f, mn = INFINITY, mx = -INFINITY;
   for (int i = lane; i < L; i += 32) {
-    float v = w[i];
+    float v = wcol(row, perm, gi * L + i, K);
     amax = fmaxf(amax, fabsf(v));
     mn = fminf(mn, v);
     mx = fmaxf(mx, v);
@@ -73,19 +83,70 @@ __global__ void __launch_bounds__(256) pack_scales_kernel(const float* __restric
   const uint16_t s16 = scale_to_half(s32);
   const size_t idx = ((size_t)(n >> 4) * G + gi) * 16 + scale_slot(n & 15);
   scales[idx] = s16;
-  if (mode == kASYM) {
+  if (mode == kASYM && zeros) {
     const float s = __half2float(__ushort_as_half(s16));
     const int z = (s == 0.0f) ? 0 : clamp_code(rintf(__fdiv_rn(-mn, s)), 15);
     zeros[idx] = __half_as_ushort(__int2half_rn(z));
   }
 }
 
+// Zero-point storage: fp16 values [N/16][GZ][16] (zbits 16), or the same
+// integers in 4 bits, [N/16][GZ][8 bytes] with slot i at byte i / 2, the low
+// nibble for even i (zbits 4).  Groups of LZ columns.
+struct ZeroFmt {
+  const void* z;
+  int LZ, GZ, zbits;
+};
+
+__device__ __forceinline__ float zero_value(const ZeroFmt& f, int rb, int zi, int slot) {
+  const size_t idx = ((size_t)rb * f.GZ + zi) * 16 + slot;
+  if (f.zbits == 16) return __half2float(__ushort_as_half(static_cast<const uint16_t*>(f.z)[idx]));
+  return (float)((static_cast<const uint8_t*>(f.z)[idx >> 1] >> (4 * (idx & 1))) & 15u);
+}
+
+// Zero-points of zero groups nested in the scale groups (efrantar's and
+// mobicham's replies in the Marlin zero-point issue: integer zero-points,
+// zero group smaller than the scale group): one thread per (row block, zero
+// group, g) takes rows g and g + 8 (adjacent slots, one byte in 4-bit form):
+// z = clamp(rint(-min / s), 0, 15) from the zero group's minimum and the fp16
+// scale of the scale group around it.
+__global__ void __launch_bounds__(256) pack_zeros_kernel(const float* __restrict__ W, int N, int K,
+                                                         int L, int G, int LZ, int GZ, int zbits,
+                                                         const uint16_t* __restrict__ scales,
+                                                         void* __restrict__ zeros) {
+  const size_t tid = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (tid >= (size_t)(N / 16) * GZ * 8) return;
+  const int g = (int)(tid & 7);
+  const size_t rz = tid >> 3;
+  const int zi = (int)(rz % GZ), rb = (int)(rz / GZ);
+  const int gi = (int)(((long long)zi * LZ) / L);
+  int zv[2];
+  for (int h = 0; h < 2; ++h) {
+    const int n = rb * 16 + g + 8 * h;
+    const float* w = W + (size_t)n * K + (size_t)zi * LZ;
+    float mn = w[0];
+    for (int i = 1; i < LZ; ++i) mn = fminf(mn, w[i]);
+    const float s = __half2float(
+        __ushort_as_half(scales[((size_t)rb * G + gi) * 16 + scale_slot(g + 8 * h)]));
+    zv[h] = (s == 0.0f) ? 0 : clamp_code(rintf(__fdiv_rn(-mn, s)), 15);
+  }
+  const size_t idx = ((size_t)rb * GZ + zi) * 16 + 2 * g;   // slots 2g (row g), 2g + 1 (row g + 8)
+  if (zbits == 16) {
+    uint16_t* z = static_cast<uint16_t*>(zeros);
+    z[idx] = __half_as_ushort(__int2half_rn(zv[0]));
+    z[idx + 1] = __half_as_ushort(__int2half_rn(zv[1]));
+  } else {
+    static_cast<uint8_t*>(zeros)[idx >> 1] = (uint8_t)(zv[0] | (zv[1] << 4));
+  }
+}
+
 struct CodeCtx {
   const float* W;
   const float* W2;   // gated layout: the second matrix (else null)
+  const int* perm;   // act-order: packed column k takes original column perm[k] (else null)
   int K, mode, bits, L, G, nchunks;
   const uint16_t* scales;
-  const uint16_t* zeros;
+  ZeroFmt zf;        // ASYM zero-points
   const uint16_t* lut;   // 2^bits fp16 entries (LUT mode)
   int nlut;
 };
@@ -131,9 +192,16 @@ __global__ void __launch_bounds__(256) pack_codes_kernel(CodeCtx c, uint32_t* __
       const int n = rb * 16 + g + 8 * h;
       const size_t sidx = ((size_t)rb * c.G + gi) * 16 + scale_slot(g + 8 * h);
       const float s = __half2float(__ushort_as_half(c.scales[sidx]));
-      const float z = c.mode == kASYM ? __half2float(__ushort_as_half(c.zeros[sidx])) : 0.0f;
-      const float4 wv = *reinterpret_cast<const float4*>(src_row(c.W, c.W2, n, c.K) + k0);
-      const float wc[4] = {wv.x, wv.y, wv.z, wv.w};
+      const float z = c.mode == kASYM ? zero_value(c.zf, rb, k0 / c.zf.LZ, scale_slot(g + 8 * h))
+                                      : 0.0f;
+      float wc[4];
+      const float* row = src_row(c.W, c.W2, n, c.K);
+      if (c.perm) {
+        for (int cc = 0; cc < 4; ++cc) wc[cc] = wcol(row, c.perm, k0 + cc, c.K);
+      } else {
+        const float4 wv = *reinterpret_cast<const float4*>(row + k0);
+        wc[0] = wv.x; wc[1] = wv.y; wc[2] = wv.z; wc[3] = wv.w;
+      }
       for (int cc = 0; cc < 4; ++cc) {
         const uint32_t q = (uint32_t)encode(wc[cc], s, z, c, lut);
         const int p = h + 2 * (cc >> 1), hi = cc & 1;
@@ -184,8 +252,9 @@ __global__ void __launch_bounds__(256) pack_codes3_kernel(CodeCtx c, uint32_t* _
       const int n = rb * 16 + g + 8 * h;
       const size_t sidx = ((size_t)rb * c.G + gi) * 16 + scale_slot(g + 8 * h);
       const float s = __half2float(__ushort_as_half(c.scales[sidx]));
-      const float4 wv = *reinterpret_cast<const float4*>(src_row(c.W, c.W2, n, c.K) + k0);
-      const float wc[4] = {wv.x, wv.y, wv.z, wv.w};
+      const float* row = src_row(c.W, c.W2, n, c.K);
+      float wc[4];
+      for (int cc = 0; cc < 4; ++cc) wc[cc] = wcol(row, c.perm, k0 + cc, c.K);
       for (int cc = 0; cc < 4; ++cc) {
         const uint32_t q = (uint32_t)encode(wc[cc], s, 0.0f, c, lut);
         const int p = h + 2 * (cc >> 1), hi = cc & 1;
@@ -243,8 +312,8 @@ __global__ void __launch_bounds__(256) dequant3_kernel(const uint32_t* __restric
 
 __global__ void __launch_bounds__(256) dequant_kernel(const uint32_t* __restrict__ qw,
                                                       const uint16_t* __restrict__ scales,
-                                                      const uint16_t* __restrict__ zl, int K,
-                                                      int bits, int mode, int L, int G,
+                                                      const uint16_t* __restrict__ zl, ZeroFmt zf,
+                                                      int K, int bits, int mode, int L, int G,
                                                       int nchunks, bool bf16, void* out,
                                                       size_t nwords) {
   const size_t wid = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
@@ -266,8 +335,9 @@ __global__ void __launch_bounds__(256) dequant_kernel(const uint32_t* __restrict
       const int n = rb * 16 + g + 8 * h;
       const size_t sidx = ((size_t)rb * G + gi) * 16 + scale_slot(g + 8 * h);
       const float s = __half2float(__ushort_as_half(scales[sidx]));
-      const float z = mode == kSYM ? 8.0f
-                      : mode == kASYM ? __half2float(__ushort_as_half(zl[sidx])) : 0.0f;
+      const float z = mode == kSYM    ? 8.0f
+                      : mode == kASYM ? zero_value(zf, rb, k0 / zf.LZ, scale_slot(g + 8 * h))
+                                      : 0.0f;
       float r[4];
       for (int cc = 0; cc < 4; ++cc) {
         const int p = h + 2 * (cc >> 1), hi = cc & 1;
@@ -295,19 +365,29 @@ __global__ void __launch_bounds__(256) dequant_kernel(const uint32_t* __restrict
 
 }  // namespace
 
-cudaError_t launch_pack(const float* W, const float* W2, int N, int K, int mode, int bits,
-                        int group, const uint16_t* lut, void* qweight, uint16_t* scales,
-                        uint16_t* zeros, cudaStream_t stream) {
+cudaError_t launch_pack(const float* W, const float* W2, const int* perm, int N, int K, int mode,
+                        int bits, int group, int zgroup, int zbits, const uint16_t* lut,
+                        void* qweight, uint16_t* scales, void* zeros, cudaStream_t stream) {
   const int L = group == -1 ? K : group;
   const int G = K / L;
+  const int LZ = zgroup == 0 ? L : (zgroup == -1 ? K : zgroup);
+  const bool own_zeros = mode == kASYM && (LZ != L || zbits != 16);   // zero-point options
   const long long warps = (long long)N * G;
   pack_scales_kernel<<<(unsigned)((warps * 32 + 255) / 256), 256, 0, stream>>>(
-      W, W2, N, K, mode, L, G, scales, zeros);
+      W, W2, perm, N, K, mode, L, G, scales, own_zeros ? nullptr : static_cast<uint16_t*>(zeros));
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
+  if (own_zeros) {
+    const size_t threads = (size_t)(N / 16) * (K / LZ) * 8;
+    pack_zeros_kernel<<<(unsigned)((threads + 255) / 256), 256, 0, stream>>>(
+        W, N, K, L, G, LZ, K / LZ, zbits, scales, zeros);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
   CodeCtx c;
   c.W = W;
   c.W2 = W2;
+  c.perm = perm;
   c.K = K;
   c.mode = mode;
   c.bits = bits;
@@ -315,7 +395,7 @@ cudaError_t launch_pack(const float* W, const float* W2, int N, int K, int mode,
   c.G = G;
   c.nchunks = K / chunk_cols(bits);
   c.scales = scales;
-  c.zeros = zeros;
+  c.zf = ZeroFmt{zeros, LZ, K / LZ, mode == kASYM ? zbits : 16};
   c.lut = lut;
   c.nlut = 1 << bits;
   const size_t nwords = (size_t)N * K * bits / 32;
@@ -328,21 +408,25 @@ cudaError_t launch_pack(const float* W, const float* W2, int N, int K, int mode,
 }
 
 cudaError_t launch_dequant(const void* qweight, const uint16_t* scales,
-                           const uint16_t* zeros_or_lut, int N, int K, int bits, int group,
-                           int mode, int out_dtype, void* W_out, cudaStream_t stream) {
+                           const void* zeros_or_lut, int N, int K, int bits, int group,
+                           int zgroup, int zbits, int mode, int out_dtype, void* W_out,
+                           cudaStream_t stream) {
   const int L = group == -1 ? K : group;
   const int G = K / L;
+  const int LZ = zgroup == 0 ? L : (zgroup == -1 ? K : zgroup);
+  const ZeroFmt zf{zeros_or_lut, LZ, K / LZ, zbits};
+  const uint16_t* zl = static_cast<const uint16_t*>(zeros_or_lut);
   if (bits == 3) {
     const size_t nthreads = (size_t)(N / 16) * (K / 128) * 32;
     dequant3_kernel<<<(unsigned)((nthreads + 255) / 256), 256, 0, stream>>>(
-        reinterpret_cast<const uint32_t*>(qweight), scales, zeros_or_lut, K, L, G, K / 128,
+        reinterpret_cast<const uint32_t*>(qweight), scales, zl, K, L, G, K / 128,
         out_dtype == QMM_BF16, W_out, nthreads);
     return cudaGetLastError();
   }
   const size_t nwords = (size_t)N * K * bits / 32;
   const unsigned blocks = (unsigned)((nwords + 255) / 256);
   dequant_kernel<<<blocks, 256, 0, stream>>>(reinterpret_cast<const uint32_t*>(qweight), scales,
-                                             zeros_or_lut, K, bits, mode, L, G,
+                                             zl, zf, K, bits, mode, L, G,
                                              K / chunk_cols(bits), out_dtype == QMM_BF16, W_out,
                                              nwords);
   return cudaGetLastError();

@@ -51,10 +51,10 @@ constexpr int kXPitch = kSC * 2 + 32;    // bytes per x row in a stage (288: row
 template <int NT>
 constexpr int rb_per_tile() { return 2; }   // the fused gate / up epilogue relies on 2
 
-// Ring depth per warp (stages in flight = depth - 1), sized so that one token
-// tile fits two CTAs per SM.
-template <int MODE, int NT>
-constexpr int ring_stages() { return (NT == 1 && MODE != kLUT) ? 3 : 2; }
+// Zero-point bytes per row block and stage with zero-point options: up to 16
+// zero groups (groups of 8 columns) of 16 fp16 values, or of 16 nibbles.
+template <int MODE>
+constexpr int kZxRb = MODE == kASYMX ? 512 : 128;
 
 struct SkinnyArgs {
   const uint16_t* x;
@@ -64,6 +64,7 @@ struct SkinnyArgs {
   uint16_t* y;
   int M, N, K, G, nchunks, nrb, tiles, nsc;
   int lg;              // log2 of the group length; -1 for one group per row
+  int lgz, GZ;         // zero-point options: log2 of the zero group, zero groups per row
   int gated;           // 1: rows are alternating 16-row gate / up blocks, y[M, N/2] = silu(gate) up
   int cta_tiles;       // 1: CTA b owns tile b, its warps take the super-chunks round-robin
   int stage_bytes;     // bytes of one ring stage
@@ -80,7 +81,8 @@ template <int MODE>
 constexpr size_t kTabBytes = MODE == kLUT ? 256 * 32 * 4 : 0;
 
 // Stage layout of one warp's ring slot: codes [R][CPS][CB] | x [TOK][288]
-// | scales [R][GPS][32 B] | zeros (ASYM) [R][GPS][32 B].
+// | scales [R][GPS][32 B] | zeros: ASYM [R][GPS][32 B]; zero-point options
+// [R][512 B] (the stage's zero groups, fp16 or 4-bit records).
 template <int BITS, int MODE, int NT, int TPG>
 struct Stage {
   static constexpr int R = rb_per_tile<NT>();
@@ -91,9 +93,22 @@ struct Stage {
   static constexpr int X_OFF = R * CPS * CB;
   static constexpr int S_OFF = X_OFF + TOK * kXPitch;
   static constexpr int Z_OFF = S_OFF + R * GPS * 32;
-  static constexpr int BYTES = Z_OFF + (MODE == kASYM ? R * GPS * 32 : 0);
+  static constexpr int BYTES =
+      Z_OFF + (MODE == kASYM ? R * GPS * 32 : (zero_opts(MODE) ? R * kZxRb<MODE> : 0));
   static_assert(BYTES % 16 == 0, "stages must stay 16-byte aligned");
 };
+
+// Ring depth per warp (stages in flight = depth - 1): 3 for one token tile
+// where the 8 warps' rings still fit two CTAs per SM (228 KB, 1 KB reserved
+// per CTA), else 2.
+template <int BITS, int MODE, int NT, int TPG>
+constexpr int ring_stages() {
+  if (NT != 1) return 2;
+  if (MODE == kSYM || MODE == kASYM) return 3;
+  if (MODE == kASYMQ && 2 * (3 * kWarps * Stage<BITS, MODE, NT, TPG>::BYTES + 1024) <= 228 * 1024)
+    return 3;
+  return 2;
+}
 
 // floor(a / d) for 0 <= a < 2^53, d > 0, from a double estimate (inv_d =
 // 1 / d) and exact integer corrections: 64-bit integer division is a long
@@ -115,6 +130,12 @@ __device__ __forceinline__ int owner_of(long long u, long long U, long long W, d
 
 __device__ __forceinline__ void sts128_zero(uint32_t a) {
   asm volatile("st.shared.v4.u32 [%0], {%1,%1,%1,%1};" ::"r"(a), "r"(0u) : "memory");
+}
+// 8-byte asynchronous copy global -> shared; `valid` false writes zeros.
+__device__ __forceinline__ void cp_async8(uint32_t saddr, const void* src, bool valid) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 8, %2;" ::"r"(saddr), "l"(src),
+               "r"(valid ? 8 : 0)
+               : "memory");
 }
 // 16-byte asynchronous copy global -> shared, L2 only; `valid` false writes zeros.
 __device__ __forceinline__ void cp_async16(uint32_t saddr, const void* src, bool valid) {
@@ -156,7 +177,7 @@ __device__ __forceinline__ void mma_16816_first(float (&d)[4], const uint32_t (&
 template <int BITS, int MODE, bool BF16, int NT, int TPG>
 __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1) skinny_kernel(const SkinnyArgs a) {
   using St = Stage<BITS, MODE, NT, TPG>;
-  constexpr int S = ring_stages<MODE, NT>();
+  constexpr int S = ring_stages<BITS, MODE, NT, TPG>();
   constexpr int R = St::R;
   constexpr int TOK = St::TOK;
   constexpr int CPS = St::CPS;
@@ -266,6 +287,25 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1) skinny_kernel(const
     const int m = min(m_base + xrow0 + 2 * i, a.M - 1);
     xsrc[i] = a.x + (size_t)m * a.K + xp * 8;
   }
+  // zero-point options: bytes per zero group record (16 fp16 or 16 nibbles),
+  // zero groups per stage, bytes of a row block's zeros per stage
+  constexpr int zrec = MODE == kASYMX ? 32 : 8;
+  const int zps = a.lgz >= 7 ? 1 : (kSC >> a.lgz);
+  const uint8_t* zbytes = reinterpret_cast<const uint8_t*>(a.zl);
+  // this lane's zero group inside a tile: columns 4t .. 4t + 3 lie in the
+  // tile's half t / 2 (groups of 8 or more columns never split a half)
+  const int zhalf = 8 * (t >> 1);
+  const int lgzc = a.lgz < 7 ? a.lgz : 7;
+  // this lane's zero-record pieces of a stage (at most two: pieces lane and
+  // lane + 32 of R * zppr), row block and piece index fixed for the whole call
+  constexpr int zppz = zrec == 32 ? 2 : 1;               // pieces per record
+  const int zppr = zps * zppz;                           // pieces per row block (<= 32)
+  int zr[2], zpc[2];
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    zr[h] = (lane + 32 * h) / zppr;
+    zpc[h] = lane + 32 * h - zr[h] * zppr;
+  }
   const bool sq_on = lane < R * GPS * 2;
   const int sq_r = lane / (2 * GPS), sq_k = (lane >> 1) % GPS, sq_h = lane & 1;
   const uint8_t* cbase[R];
@@ -333,6 +373,27 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1) skinny_kernel(const
       cp_async16(base + St::S_OFF + lane * 16, sbase + off, ok);
       if constexpr (MODE == kASYM)
         cp_async16(base + St::Z_OFF + lane * 16, a.zl + (sbase - a.scales) + off, ok);
+    }
+    if constexpr (zero_opts(MODE)) {
+      // the zps zero groups that meet the stage's 128 columns, per row block:
+      // fp16 records (32 bytes) in two 16-byte pieces each, 4-bit records
+      // (8 bytes) in one 8-byte piece each; a piece never spans two records,
+      // so its validity is its record's and its source stays aligned
+      const int zf = k0 >> a.lgz;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        if (lane + 32 * h < R * zppr) {   // warp-uniform for h = 0 once zppr >= 16
+          const int r = zr[h], pc = zpc[h];
+          const int rb = tile * R + r;
+          const int zi = zf + pc / zppz;
+          const bool ok = rb < a.nrb && zi < a.GZ;
+          const uint8_t* src = zbytes + ((size_t)rb * a.GZ + zi) * zrec + (pc % zppz) * 16;
+          if constexpr (zrec == 32)
+            cp_async16(base + St::Z_OFF + r * kZxRb<MODE> + pc * 16, ok ? src : zbytes, ok);
+          else
+            cp_async8(base + St::Z_OFF + r * kZxRb<MODE> + pc * 8, ok ? src : zbytes, ok);
+        }
+      }
     }
   };
 
@@ -494,6 +555,27 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1) skinny_kernel(const
                 if constexpr (BF16) {
                   const float2 zf = __half22float2(*reinterpret_cast<const __half2*>(&zw));
                   zw = pack2<true>(zf.x, zf.y);
+                }
+                sub_zero<BF16>(__byte_perm(zw, 0, 0x1010), __byte_perm(zw, 0, 0x3232), af);
+              } else if constexpr (zero_opts(MODE)) {
+                decode_int4<BF16, 0>(w, af);
+                // zero group of (tile j, this lane's half) inside the stage
+                const int zl = (16 * j + zhalf) >> lgzc;
+                const unsigned char* zp = st + St::Z_OFF + r * kZxRb<MODE>;
+                uint32_t zw;
+                if constexpr (MODE == kASYMX) {
+                  zw = *reinterpret_cast<const uint32_t*>(zp + zl * 32 + 4 * g);
+                  if constexpr (BF16) {
+                    const float2 zf2 = __half22float2(*reinterpret_cast<const __half2*>(&zw));
+                    zw = pack2<true>(zf2.x, zf2.y);
+                  }
+                } else {
+                  // rows g, g + 8 = the low and high nibble of byte g of the record
+                  const uint32_t b = zp[zl * 8 + g];
+                  if constexpr (BF16)   // (128 + z) - 128 in bf16, exact
+                    zw = bsub2_u(lop3_and_or(b | (b << 12), 0x000F000Fu, 0x43004300u), 0x43004300u);
+                  else                  // (1024 + z) - 1024 in fp16, exact
+                    zw = hsub2_u(lop3_and_or(b | (b << 12), 0x000F000Fu, 0x64006400u), 0x64006400u);
                 }
                 sub_zero<BF16>(__byte_perm(zw, 0, 0x1010), __byte_perm(zw, 0, 0x3232), af);
               } else if constexpr (!BF16) {
@@ -691,7 +773,7 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1) skinny_kernel(const
 template <int BITS, int MODE, int NT, int TPG>
 constexpr size_t smem_bytes() {
   using St = Stage<BITS, MODE, NT, TPG>;
-  constexpr int S = ring_stages<MODE, NT>();
+  constexpr int S = ring_stages<BITS, MODE, NT, TPG>();
   return kTabBytes<MODE> + (size_t)kWarps * S * St::BYTES;
 }
 
@@ -760,6 +842,9 @@ auto dispatch(int bits, int mode, bool bf16, int nt, int tpg, F&& f) {
   QMM_CASE(2, kLUT, false, 1) QMM_CASE(2, kLUT, false, 2) QMM_CASE(2, kLUT, true, 1)
   QMM_CASE(2, kLUT, true, 2) QMM_CASE(3, kLUT, false, 1) QMM_CASE(3, kLUT, false, 2)
   QMM_CASE(3, kLUT, true, 1) QMM_CASE(3, kLUT, true, 2)
+  QMM_CASE(4, kASYMX, false, 1) QMM_CASE(4, kASYMX, false, 2) QMM_CASE(4, kASYMX, true, 1)
+  QMM_CASE(4, kASYMX, true, 2) QMM_CASE(4, kASYMQ, false, 1) QMM_CASE(4, kASYMQ, false, 2)
+  QMM_CASE(4, kASYMQ, true, 1) QMM_CASE(4, kASYMQ, true, 2)
 #undef QMM_CASE
   return dispatch_tpg<4, kSYM, false, 1>(tpg, f);
 }
@@ -832,6 +917,13 @@ cudaError_t launch_skinny(const Problem& pr, const SkinnyPlan& plan, void* works
   const int L = pr.group == -1 ? pr.K : pr.group;
   a.G = pr.K / L;
   a.lg = pr.group == -1 ? -1 : __builtin_ctz((unsigned)pr.group);
+  {
+    const int LZ = pr.zgroup == 0 ? L : (pr.zgroup == -1 ? pr.K : pr.zgroup);
+    a.GZ = pr.K / LZ;
+    // zero groups of 128 columns or more: one per stage (lgz only decides the
+    // group's index, K >> lgz; a row-long group gets a shift past every k)
+    a.lgz = pr.zgroup == -1 || (pr.zgroup == 0 && pr.group == -1) ? 30 : __builtin_ctz((unsigned)LZ);
+  }
   a.nchunks = pr.K / chunk_cols(pr.bits);
   a.nsc = (pr.K + kSC - 1) / kSC;
   a.nrb = pr.N / 16;

@@ -675,7 +675,7 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
 // scales with bf16 would round every weight to 8 bits, which together with the
 // bf16 output exceeds the error budget; those run on the decode path.
 bool tc_supported(int bits, int mode, bool bf16, int group) {
-  if (bits != 4) return false;
+  if (bits != 4 || zero_opts(mode)) return false;
   if (!bf16) return true;
   return group == -1 && mode != kLUT;
 }
