@@ -100,8 +100,7 @@ using namespace qk;
 static int run_qmm(const void* x, int xdtype, const void* qweight, const uint16_t* scales,
                    const uint16_t* zeros_or_lut, int M, int N, int K, int bits, int group,
                    int mode, void* y, void* workspace, size_t workspace_bytes, void* stream,
-                   int path, bool gated, int zgroup = 0, int zbits = 16,
-                   bool early_weights = false) {
+                   int path, bool gated, int zgroup = 0, int zbits = 16) {
   if (M < 0) return QMM_ERR_ARG;
   int st = check_shape(N, K, bits, group, zero_opts(mode) ? QMM_ASYM : mode);
   if (st != QMM_OK) return st;
@@ -124,7 +123,6 @@ static int run_qmm(const void* x, int xdtype, const void* qweight, const uint16_
   p.gated = gated;
   p.zgroup = zgroup;
   p.zbits = zbits;
-  p.early_weights = early_weights;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   Plan plan = make_plan(M, N, K, bits, group, mode, xdtype == QMM_BF16, path);
   if (plan.ws_bytes()) {
@@ -397,9 +395,8 @@ int qmm_actorder(const void* x, int xdtype, const int32_t* perm, const void* qwe
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   st = status_of(launch_permute_x(x, perm, M, K, xp, s));
   if (st != QMM_OK) return st;
-  // the product's predecessor is the gather, which writes only x'
   return run_qmm(xp, xdtype, qweight, scales, zeros_or_lut, M, N, K, bits, group, mode, y,
-                 workspace, plain, stream, QMM_PATH_AUTO, false, 0, 16, true);
+                 workspace, plain, stream, QMM_PATH_AUTO, false);
 }
 
 int qmm_check_error(void* stream) {

@@ -21,10 +21,6 @@ struct Problem {
   // ASYM zero-point options (modes kASYMX / kASYMQ): zero group (columns; 0 =
   // the scale group, -1 = the row) and storage (16 = fp16, 4 = 4-bit integers)
   int zgroup = 0, zbits = 16;
-  // The previous grid in the stream writes only x (the act-order gather, which
-  // waited for its own predecessor before releasing this grid): the decode
-  // path may request its first weight stages before its dependency wait.
-  bool early_weights = false;
 };
 
 // Split-K plan of the skinny (M <= 16 per slab) decode path.

@@ -67,7 +67,6 @@ struct SkinnyArgs {
   int lgz, GZ;         // zero-point options: log2 of the zero group, zero groups per row
   int gated;           // 1: rows are alternating 16-row gate / up blocks, y[M, N/2] = silu(gate) up
   int cta_tiles;       // 1: CTA b owns tile b, its warps take the super-chunks round-robin
-  int early_weights;   // 1: the previous grid writes x only (see the prologue)
   int stage_bytes;     // bytes of one ring stage
   long long units;     // tiles * nsc
   int ctas;            // CTAs per slab
@@ -222,15 +221,8 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1) skinny_kernel(const
   }
   __syncwarp();
 
-  // Programmatic dependent launch: every input may come from the previous grid,
-  // so nothing global is read before the wait -- except with early_weights,
-  // where the previous grid is the activation gather of this call, which writes
-  // only x and itself waited for its own predecessor before it let this grid
-  // start: the weights' first stages are then requested before the wait.
-  if (!a.early_weights) {
-    pdl_wait();
-    pdl_launch_dependents();   // let the next grid get resident while this one runs
-  }
+  pdl_wait();                 // inputs of this call may come from the previous grid
+  pdl_launch_dependents();    // let the next grid get resident while this one runs
 
   if constexpr (MODE == kLUT) {
     // Pair table, replicated so that every lane reads its own bank.
@@ -336,23 +328,10 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1) skinny_kernel(const
     srok = sq_on && rbs < a.nrb;
     sbase = a.scales + (size_t)(srok ? rbs : 0) * a.G * 16 + sq_h * 8;
   };
-  // what: 1 = the stage's weights (codes, scales, zeros), 2 = its x rows
-  auto issue = [&](int tile, int sc, int st, int what = 3) {
+  auto issue = [&](int tile, int sc, int st) {
     if (tile != pf_tile) set_tile(tile);
     const uint32_t base = ring_s + st * St::BYTES;
     const bool full = sc < nsc_full;
-    const int k0 = sc * kSC;
-    if (what & 2) {
-      const bool xk = full || k0 + xp * 8 < a.K;
-#pragma unroll
-      for (int i = 0; i < (TOK + 1) / 2; ++i) {
-        if (i < xi_n) {   // warp-uniform
-          const bool ok = xrow0 + 2 * i < mrows && xk;
-          cp_async16(base + xdst0 + 2 * i * kXPitch, xsrc[i] + (ok ? k0 : 0), ok);
-        }
-      }
-    }
-    if (!(what & 1)) return;
     // a row block's codes of the stage: CPS chunks, contiguous, copied as
     // 512-byte warp-wide pieces (the last one partial for 3-bit chunks)
     constexpr int RB_BYTES = CPS * St::CB;
@@ -377,6 +356,15 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1) skinny_kernel(const
           cp_async16(base + r * RB_BYTES + i * 512 + lane * 16,
                      cbase[r] + (ok ? (size_t)sc * RB_BYTES + i * 512 : 0), ok);
         }
+    }
+    const int k0 = sc * kSC;
+    const bool xk = full || k0 + xp * 8 < a.K;
+#pragma unroll
+    for (int i = 0; i < (TOK + 1) / 2; ++i) {
+      if (i < xi_n) {   // warp-uniform
+        const bool ok = xrow0 + 2 * i < mrows && xk;
+        cp_async16(base + xdst0 + 2 * i * kXPitch, xsrc[i] + (ok ? k0 : 0), ok);
+      }
     }
     if (sq_on) {
       const int gi = (lg < 0 ? 0 : (k0 >> lg)) + sq_k;
@@ -424,28 +412,10 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1) skinny_kernel(const
       ++pf_t;
     }
   };
-  if (a.early_weights) {
-    // the weights of the first S - 1 stages, then the wait, then their x rows
-    // (the first commit group holds all of them: one stage's wait covers them)
-    const long long u0 = pf_u;
-    const int t0 = pf_t, s0 = pf_s;
-#pragma unroll
-    for (int s = 0; s < S - 1; ++s) {
-      if (pf_u < ue) {
-        issue(pf_t, pf_s, s, 1);
-        pf_next();
-      }
-    }
-    pf_u = u0;
-    pf_t = t0;
-    pf_s = s0;
-    pdl_wait();
-    pdl_launch_dependents();
-  }
 #pragma unroll
   for (int s = 0; s < S - 1; ++s) {
     if (pf_u < ue) {
-      issue(pf_t, pf_s, s, a.early_weights ? 2 : 3);
+      issue(pf_t, pf_s, s);
       pf_next();
     }
     cp_async_commit();
@@ -944,7 +914,6 @@ cudaError_t launch_skinny(const Problem& pr, const SkinnyPlan& plan, void* works
   a.K = pr.K;
   a.gated = pr.gated ? 1 : 0;
   a.cta_tiles = plan.cta_tiles;
-  a.early_weights = pr.early_weights ? 1 : 0;
   const int L = pr.group == -1 ? pr.K : pr.group;
   a.G = pr.K / L;
   a.lg = pr.group == -1 ? -1 : __builtin_ctz((unsigned)pr.group);
