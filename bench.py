@@ -102,12 +102,34 @@ def problems(name):
 
 
 def peaks():
+    """(HBM GB/s, source) of the roofline's memory bound."""
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
             d = json.load(f)
         return float(d["hbm_gbs"]), "measured"
     except Exception:
         return 6650.0, "fallback"
+
+
+def tensor_peak():
+    """(TFLOP/s, source) of the dense fp16/bf16 tensor bound.  The bench loops
+    for seconds under the power cap, so the sustained figure applies."""
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            d = json.load(f)
+        return float(d["bf16_tflops_sustained"]), "measured, sustained"
+    except Exception:
+        return 1400.0, "fallback, sustained"
+
+
+def tensor_bound(name):
+    """Workloads whose every call has M >= 256: reported in TFLOP/s against the
+    tensor roofline (the rest in GB/s against HBM)."""
+    return min(WORKLOADS[name][5]) >= 256
+
+
+def alg_flops(M, K, N):
+    return 2.0 * M * N * K
 
 
 def sources_hash():
@@ -263,6 +285,8 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.synchronize()
     calls = sets[0]
     step_bytes = sum(c["bytes"] for c in calls)
+    step_flops = sum(alg_flops(c["M"], c["K"], c["N"]) for c in calls)
+    tensor = tensor_bound(args.workload)
 
     def step(i=0):
         for c in sets[i % copies]:
@@ -362,16 +386,30 @@ def run_ours(args, rank, world, local_rank):
     e2e_ms = max_over_ranks(a0.elapsed_time(a1), dist, dev)
     e2e_value = whole_job_gbs(world, step_bytes, e2e_steps, e2e_ms)
 
-    peak, peak_kind = peaks()
-    achieved = step_bytes / (ms_per_step / 1e3) / 1e9      # one GPU, the skinny kernel only
-    tpb = traffic_per_byte()
-    roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-                "frac": round(achieved / peak, 4), "peak_source": peak_kind,
-                "traffic": None if tpb is None else round(tpb * step_bytes / len(calls)),
-                "kernel": "skinny_kernel (all launches of the step)" if not actorder else
-                          "permute_x_kernel + skinny_kernel (all launches of the step)",
-                "algorithmic_bytes_per_launch": round(step_bytes / len(calls))}
-    out = {"metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world,
+    if tensor:
+        # the tensor-core kernel: flops per step over the step time (one GPU)
+        peak, peak_kind = tensor_peak()
+        achieved = step_flops / (ms_per_step / 1e3) / 1e12
+        value = world * step_flops * args.steps / (ms / 1e3) / 1e12
+        e2e_value = world * step_flops * e2e_steps / (e2e_ms / 1e3) / 1e12
+        unit = "TFLOP/s"
+        roofline = {"bound": "tensor", "achieved": round(achieved, 1), "peak": peak,
+                    "unit": "TFLOP/s", "frac": round(achieved / peak, 4), "peak_source": peak_kind,
+                    "traffic": None, "kernel": "tc_kernel (all launches of the step)",
+                    "algorithmic_flops_per_launch": step_flops / len(calls),
+                    "algorithmic_bytes_per_launch": round(step_bytes / len(calls))}
+    else:
+        peak, peak_kind = peaks()
+        achieved = step_bytes / (ms_per_step / 1e3) / 1e9      # one GPU, the skinny kernel only
+        tpb = traffic_per_byte()
+        unit = "GB/s"
+        roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                    "frac": round(achieved / peak, 4), "peak_source": peak_kind,
+                    "traffic": None if tpb is None else round(tpb * step_bytes / len(calls)),
+                    "kernel": "skinny_kernel (all launches of the step)" if not actorder else
+                              "permute_x_kernel + skinny_kernel (all launches of the step)",
+                    "algorithmic_bytes_per_launch": round(step_bytes / len(calls))}
+    out = {"metric": METRIC, "value": round(value, 1), "unit": unit, "n_gpus": world,
            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5),
            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f16",
            "data": "synthetic (seeded torch.randn weights and activations)",
@@ -387,14 +425,14 @@ def run_ours(args, rank, world, local_rank):
                       "launch": "CUDA graph of the step, programmatic dependent launch",
                       "parallelism": f"replicas x{world}"},
            "roofline": roofline,
-           "e2e": {"value": round(e2e_value, 1), "unit": "GB/s", "h2d_bytes_per_step": h2d,
+           "e2e": {"value": round(e2e_value, 1), "unit": unit, "h2d_bytes_per_step": h2d,
                    "d2h_bytes_per_step": d2h, "steps": e2e_steps,
                    "how": f"per step: pinned x -> device, the {len(calls)} calls through the "
                           "Python API, y -> pinned host; CUDA events on the stream"},
            "gpu_launches": len(calls) * args.steps * (2 if actorder else 1),
            "clocks": clocks}
     if rank == 0 and not args.no_cpu_baseline:
-        out["cpu_baseline"] = cpu_baseline(args.workload, args.cpu_seconds)
+        out["cpu_baseline"] = cpu_baseline(args.workload, args.cpu_seconds, tensor)
     del graphs
     return out
 
@@ -420,6 +458,7 @@ def _oracle_sample(workload, rows_per_problem, seed=0):
         x = synth.activations(seed + i, "x", M, K, xdt)
         n = rows_per_problem
         b = n / N * alg_bytes(mode, bits, group, M, K, N, gated, zopts, actorder)
+        f = alg_flops(M, K, n)
         if zopts is not None:
             codes, scales, zeros = oracle.quantize_asym(W, group, zopts[0])
             qw, sp, zp = oracle.pack_asym(codes, scales, zeros, group, zopts[0], zopts[1])
@@ -450,7 +489,7 @@ def _oracle_sample(workload, rows_per_problem, seed=0):
                       bits=bits, group=group:
                       oracle.qmm(x, xdt, qw, sp, zl, M, n, K, mode, bits, group, a, b))
                 parts = n
-        items.append((fn, parts, b))
+        items.append((fn, parts, b, f))
     return items
 
 
@@ -466,14 +505,14 @@ def _split_run(fn, parts, threads):
         t.join()
 
 
-def _run_oracle(items, threads):
+def _run_oracle(items, threads, flops=False):
     """Runs every sampled call, its output columns split over `threads` host
-    threads; returns (seconds, algorithmic bytes)."""
+    threads; returns (seconds, algorithmic bytes or flops)."""
     t0 = time.perf_counter()
     total = 0.0
-    for fn, parts, b in items:
+    for fn, parts, b, f in items:
         _split_run(fn, parts, threads)
-        total += b
+        total += f if flops else b
     return time.perf_counter() - t0, total
 
 
@@ -484,29 +523,32 @@ def cpu_threads():
         return os.cpu_count() or 1
 
 
-def cpu_baseline(workload, seconds):
+def cpu_baseline(workload, seconds, tensor=False):
     """The oracle (plain C++, double sums) on a bounded sample of the workload:
-    the same 20 calls restricted to their first R rows of W (whole 16-row
-    blocks), R chosen so the timed run takes about `seconds`."""
+    the same calls restricted to their first R rows of W (whole 16-row
+    blocks), R chosen so the timed run takes about `seconds`.  Reported in the
+    bench line's unit (GB/s of algorithmic bytes, or TFLOP/s)."""
     threads = cpu_threads()
     probe = _oracle_sample(workload, 16)
     dt, _ = _run_oracle(probe, threads)
     rows = int(16 * max(1, round(seconds / max(dt, 1e-3))))
     rows = max(16, min(rows // 16 * 16, 4096))
     items = _oracle_sample(workload, rows)
-    dt, nbytes = _run_oracle(items, threads)
+    dt, work = _run_oracle(items, threads, tensor)
     # the sample's inputs are capped (they are generated on the host); repeat
     # the oracle on them until the CPU work reaches about `seconds`
     reps = max(1, int(round(seconds / max(dt, 1e-3))))
     for _ in range(reps - 1):
-        d, b = _run_oracle(items, threads)
+        d, w = _run_oracle(items, threads, tensor)
         dt += d
-        nbytes += b
-    return {"value": round(nbytes / dt / 1e9, 4), "unit": "GB/s", "cores": threads,
+        work += w
+    what = (f"{work / reps / 1e9:.2f} GFLOP" if tensor
+            else f"{work / reps / 1e6:.1f} MB of algorithmic bytes")
+    return {"value": round(work / dt / (1e12 if tensor else 1e9), 6),
+            "unit": "TFLOP/s" if tensor else "GB/s", "cores": threads,
             "kind": "oracle", "seconds": round(dt, 2),
             "sample": f"every call of the step on its first {rows} rows of W "
-                      f"({nbytes / reps / 1e6:.1f} MB of algorithmic bytes), run {reps} times, "
-                      f"columns split over {threads} threads"}
+                      f"({what}), run {reps} times, columns split over {threads} threads"}
 
 
 def run_reference(args):
@@ -517,24 +559,26 @@ def run_reference(args):
     budget = max(2.0, 120.0 / max(1, args.steps + args.warmup))   # whole run ~2 minutes
     rows = max(16, min(int(16 * round(budget / max(dt, 1e-3))) // 16 * 16, 4096))
     items = _oracle_sample(args.workload, rows)
+    tensor = tensor_bound(args.workload)
+    unit = "TFLOP/s" if tensor else "GB/s"
     for _ in range(args.warmup):
-        _run_oracle(items, threads)
+        _run_oracle(items, threads, tensor)
     tot_t, tot_b = 0.0, 0.0
     for _ in range(args.steps):
-        t, b = _run_oracle(items, threads)
+        t, b = _run_oracle(items, threads, tensor)
         tot_t += t
         tot_b += b
-    value = tot_b / tot_t / 1e9
+    value = tot_b / tot_t / (1e12 if tensor else 1e9)
     sample = (f"every call of the step on its first {rows} rows of W, columns split over "
               f"{threads} threads")
-    return {"impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s",
+    return {"impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": unit,
             "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(1e3 * tot_t / args.steps, 3), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": args.workload, "calls_per_step": len(items)},
-            "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": threads,
+            "cpu_baseline": {"value": round(value, 6), "unit": unit, "cores": threads,
                              "kind": "oracle", "sample": sample},
-            "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+            "e2e": {"value": round(value, 6), "unit": unit, "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
 
 

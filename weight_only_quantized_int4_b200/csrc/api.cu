@@ -57,7 +57,7 @@ int check_zopts(int K, int group, int zgroup, int zbits) {
 void zero_mode(int K, int group, int zgroup, int zbits, int* mode, int* zg) {
   const int L = group == -1 ? K : group, LZ = zgroup == -1 ? K : zgroup;
   *zg = LZ == L ? 0 : zgroup;
-  *mode = zbits == 4 ? kASYMQ : (*zg == 0 ? QMM_ASYM : kASYMX);
+  *mode = zbits == 4 ? (LZ >= 128 ? kASYMQ1 : kASYMQ) : (*zg == 0 ? QMM_ASYM : kASYMX);
 }
 
 size_t round256(size_t b) { return (b + 255) / 256 * 256; }
@@ -79,7 +79,7 @@ struct Plan {
   size_t ws_bytes() const { return path == QMM_PATH_TENSOR ? tc.ws_bytes : sk.ws_bytes; }
 };
 
-// `mode` may be an internal zero-point-options mode (kASYMX, kASYMQ).
+// `mode` may be an internal zero-point-options mode (kASYMX, kASYMQ, kASYMQ1).
 Plan make_plan(int M, int N, int K, int bits, int group, int mode, bool bf16, int path) {
   Plan p{};
   const bool streamk = path == QMM_PATH_SKINNY_STREAMK;

@@ -13,9 +13,12 @@ namespace qk {
 constexpr int kSYM = QMM_SYM, kASYM = QMM_ASYM, kLUT = QMM_LUT;
 // Internal modes: ASYM with zero-point options (a zero group inside the scale
 // group, or 4-bit integer zero-points); packed codes as for ASYM.  kASYMX has
-// fp16 zero-points, kASYMQ 4-bit ones.
-constexpr int kASYMX = 3, kASYMQ = 4;
-__host__ __device__ constexpr bool zero_opts(int mode) { return mode == kASYMX || mode == kASYMQ; }
+// fp16 zero-points, kASYMQ 4-bit ones, kASYMQ1 4-bit ones in groups of 128
+// columns or more (one zero record per 128-column stage of the decode path).
+constexpr int kASYMX = 3, kASYMQ = 4, kASYMQ1 = 5;
+__host__ __device__ constexpr bool zero_opts(int mode) {
+  return mode == kASYMX || mode == kASYMQ || mode == kASYMQ1;
+}
 
 // Chunk of K covered by one block of codes (16 rows x KC columns): 512 bytes
 // for 4- and 2-bit codes, 768 bytes for 3-bit codes.

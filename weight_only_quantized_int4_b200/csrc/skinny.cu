@@ -52,9 +52,10 @@ template <int NT>
 constexpr int rb_per_tile() { return 2; }   // the fused gate / up epilogue relies on 2
 
 // Zero-point bytes per row block and stage with zero-point options: up to 16
-// zero groups (groups of 8 columns) of 16 fp16 values, or of 16 nibbles.
+// zero groups (groups of 8 columns) of 16 fp16 values, or of 16 nibbles; one
+// 8-byte record (padded to 16) when the zero group spans the stage.
 template <int MODE>
-constexpr int kZxRb = MODE == kASYMX ? 512 : 128;
+constexpr int kZxRb = MODE == kASYMX ? 512 : (MODE == kASYMQ ? 128 : 16);
 
 struct SkinnyArgs {
   const uint16_t* x;
@@ -105,7 +106,8 @@ template <int BITS, int MODE, int NT, int TPG>
 constexpr int ring_stages() {
   if (NT != 1) return 2;
   if (MODE == kSYM || MODE == kASYM) return 3;
-  if (MODE == kASYMQ && 2 * (3 * kWarps * Stage<BITS, MODE, NT, TPG>::BYTES + 1024) <= 228 * 1024)
+  if ((MODE == kASYMQ || MODE == kASYMQ1) &&
+      2 * (3 * kWarps * Stage<BITS, MODE, NT, TPG>::BYTES + 1024) <= 228 * 1024)
     return 3;
   return 2;
 }
@@ -290,7 +292,7 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1) skinny_kernel(const
   // zero-point options: bytes per zero group record (16 fp16 or 16 nibbles),
   // zero groups per stage, bytes of a row block's zeros per stage
   constexpr int zrec = MODE == kASYMX ? 32 : 8;
-  const int zps = a.lgz >= 7 ? 1 : (kSC >> a.lgz);
+  const int zps = (MODE == kASYMQ1 || a.lgz >= 7) ? 1 : (kSC >> a.lgz);
   const uint8_t* zbytes = reinterpret_cast<const uint8_t*>(a.zl);
   // this lane's zero group inside a tile: columns 4t .. 4t + 3 lie in the
   // tile's half t / 2 (groups of 8 or more columns never split a half)
@@ -514,6 +516,19 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1) skinny_kernel(const
             xf[j][nt][1] = v.y;
           }
       }
+      // one 4-bit zero record per stage: each row block's (z_g, z_g8) pairs once
+      uint32_t zq1[MODE == kASYMQ1 ? R : 1][2];
+      if constexpr (MODE == kASYMQ1) {
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+          const uint32_t b = st[St::Z_OFF + r * kZxRb<MODE> + g];
+          const uint32_t zw =
+              BF16 ? bsub2_u(lop3_and_or(b | (b << 12), 0x000F000Fu, 0x43004300u), 0x43004300u)
+                   : hsub2_u(lop3_and_or(b | (b << 12), 0x000F000Fu, 0x64006400u), 0x64006400u);
+          zq1[r][0] = __byte_perm(zw, 0, 0x1010);
+          zq1[r][1] = __byte_perm(zw, 0, 0x3232);
+        }
+      }
       float gacc[R][NT][4];
       uint4 cw[R];
       uint32_t cw3[BITS == 3 ? R : 1][6];   // 3-bit: the lane's 24 bytes of the stage
@@ -557,6 +572,9 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1) skinny_kernel(const
                   zw = pack2<true>(zf.x, zf.y);
                 }
                 sub_zero<BF16>(__byte_perm(zw, 0, 0x1010), __byte_perm(zw, 0, 0x3232), af);
+              } else if constexpr (MODE == kASYMQ1) {
+                decode_int4<BF16, 0>(w, af);
+                sub_zero<BF16>(zq1[r][0], zq1[r][1], af);
               } else if constexpr (zero_opts(MODE)) {
                 decode_int4<BF16, 0>(w, af);
                 // zero group of (tile j, this lane's half) inside the stage
@@ -844,7 +862,8 @@ auto dispatch(int bits, int mode, bool bf16, int nt, int tpg, F&& f) {
   QMM_CASE(3, kLUT, true, 1) QMM_CASE(3, kLUT, true, 2)
   QMM_CASE(4, kASYMX, false, 1) QMM_CASE(4, kASYMX, false, 2) QMM_CASE(4, kASYMX, true, 1)
   QMM_CASE(4, kASYMX, true, 2) QMM_CASE(4, kASYMQ, false, 1) QMM_CASE(4, kASYMQ, false, 2)
-  QMM_CASE(4, kASYMQ, true, 1) QMM_CASE(4, kASYMQ, true, 2)
+  QMM_CASE(4, kASYMQ, true, 1) QMM_CASE(4, kASYMQ, true, 2) QMM_CASE(4, kASYMQ1, false, 1)
+  QMM_CASE(4, kASYMQ1, false, 2) QMM_CASE(4, kASYMQ1, true, 1) QMM_CASE(4, kASYMQ1, true, 2)
 #undef QMM_CASE
   return dispatch_tpg<4, kSYM, false, 1>(tpg, f);
 }
