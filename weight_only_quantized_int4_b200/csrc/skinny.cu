@@ -197,7 +197,7 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1) skinny_kernel(const
   // this warp's stream-K range of (tile, super-chunk) units
   const int gw = blockIdx.x * kWarps + warp;
   const long long W = a.warps;
-  long long ub = 0, ue = 0;
+  int ub = 0, ue = 0;   // unit indices: at most 2^15 tiles x 2^13 stages, 32 bits
   // CTA-per-tile mode (problems with few row tiles): CTA b owns tile b, warp w
   // takes its super-chunks w, w + 8, ... and the warps' sums are added in
   // shared memory; otherwise warp-level stream-K over contiguous unit ranges
@@ -206,8 +206,8 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1) skinny_kernel(const
   if (ctile) {
     ue = warp < n ? (n - warp + kWarps - 1) / kWarps : 0;
   } else if (gw < W) {
-    ub = floor_div((long long)gw * a.units, W, a.inv_warps);
-    ue = floor_div((long long)(gw + 1) * a.units, W, a.inv_warps);
+    ub = (int)floor_div((long long)gw * a.units, W, a.inv_warps);
+    ue = (int)floor_div((long long)(gw + 1) * a.units, W, a.inv_warps);
   }
   const int lg = a.lg;
 
@@ -310,6 +310,13 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1) skinny_kernel(const
   }
   const bool sq_on = lane < R * GPS * 2;
   const int sq_r = lane / (2 * GPS), sq_k = (lane >> 1) % GPS, sq_h = lane & 1;
+  // steady-state copy parameters fixed for the call: source bytes of this
+  // lane's x pieces (16, or 0 for a token row past M, which reads as zeros)
+  // and the shift from a stage's first column to its first group
+  uint32_t xsz[(TOK + 1) / 2];
+#pragma unroll
+  for (int i = 0; i < (TOK + 1) / 2; ++i) xsz[i] = xrow0 + 2 * i < mrows ? 16u : 0u;
+  const int lgs = lg < 0 ? 31 : lg;
   const uint8_t* cbase[R];
   bool rok[R];
   bool tile_ok = true;
@@ -330,24 +337,59 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1) skinny_kernel(const
     srok = sq_on && rbs < a.nrb;
     sbase = a.scales + (size_t)(srok ? rbs : 0) * a.G * 16 + sq_h * 8;
   };
+  auto issue_zeros = [&](int tile, int k0, uint32_t base) {
+    // the zps zero groups that meet the stage's 128 columns, per row block:
+    // fp16 records (32 bytes) in two 16-byte pieces each, 4-bit records
+    // (8 bytes) in one 8-byte piece each; a piece never spans two records,
+    // so its validity is its record's and its source stays aligned
+    const int zf = k0 >> a.lgz;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      if (lane + 32 * h < R * zppr) {   // warp-uniform for h = 0 once zppr >= 16
+        const int r = zr[h], pc = zpc[h];
+        const int rb = tile * R + r;
+        const int zi = zf + pc / zppz;
+        const bool ok = rb < a.nrb && zi < a.GZ;
+        const uint8_t* src = zbytes + ((size_t)rb * a.GZ + zi) * zrec + (pc % zppz) * 16;
+        if constexpr (zrec == 32)
+          cp_async16(base + St::Z_OFF + r * kZxRb<MODE> + pc * 16, ok ? src : zbytes, ok);
+        else
+          cp_async8(base + St::Z_OFF + r * kZxRb<MODE> + pc * 8, ok ? src : zbytes, ok);
+      }
+    }
+  };
   auto issue = [&](int tile, int sc, int st) {
     if (tile != pf_tile) set_tile(tile);
     const uint32_t base = ring_s + st * St::BYTES;
-    const bool full = sc < nsc_full;
+    const int k0 = sc * kSC;
     // a row block's codes of the stage: CPS chunks, contiguous, copied as
     // 512-byte warp-wide pieces (the last one partial for 3-bit chunks)
     constexpr int RB_BYTES = CPS * St::CB;
     constexpr int PIECES = (RB_BYTES + 511) / 512;
-    if (tile_ok && full) {
+    if (tile_ok && sc < nsc_full) {
+      // steady state (a whole stage of a tile inside N and K): every copy is
+      // in bounds, no per-piece checks; 32-bit offsets from the row-block bases
+      const uint32_t cofs = (uint32_t)sc * RB_BYTES;
 #pragma unroll
-      for (int r = 0; r < R; ++r) {
-        const uint8_t* src = cbase[r] + (size_t)sc * RB_BYTES;
+      for (int r = 0; r < R; ++r)
 #pragma unroll
         for (int i = 0; i < PIECES; ++i)
           if (RB_BYTES % 512 == 0 || i * 512 + lane * 16 < RB_BYTES)
-            cp_async16_all(base + r * RB_BYTES + i * 512 + lane * 16, src + i * 512);
+            cp_async16_all(base + r * RB_BYTES + i * 512 + lane * 16, cbase[r] + cofs + i * 512);
+#pragma unroll
+      for (int i = 0; i < (TOK + 1) / 2; ++i)
+        if (i < xi_n)   // warp-uniform
+          cp_async16(base + xdst0 + 2 * i * kXPitch, xsrc[i] + k0, xsz[i] != 0);
+      if (sq_on) {
+        const int off = ((k0 >> lgs) + sq_k) << 4;
+        cp_async16(base + St::S_OFF + lane * 16, sbase + off, srok);
+        if constexpr (MODE == kASYM)
+          cp_async16(base + St::Z_OFF + lane * 16, a.zl + (sbase - a.scales) + off, srok);
       }
     } else {
+      // a tile with row blocks past N, or the stage that K ends in: every
+      // piece checked, the missing ones zero-filled
+      const bool full = sc < nsc_full;
 #pragma unroll
       for (int r = 0; r < R; ++r)
 #pragma unroll
@@ -358,53 +400,32 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1) skinny_kernel(const
           cp_async16(base + r * RB_BYTES + i * 512 + lane * 16,
                      cbase[r] + (ok ? (size_t)sc * RB_BYTES + i * 512 : 0), ok);
         }
-    }
-    const int k0 = sc * kSC;
-    const bool xk = full || k0 + xp * 8 < a.K;
+      const bool xk = full || k0 + xp * 8 < a.K;
 #pragma unroll
-    for (int i = 0; i < (TOK + 1) / 2; ++i) {
-      if (i < xi_n) {   // warp-uniform
-        const bool ok = xrow0 + 2 * i < mrows && xk;
-        cp_async16(base + xdst0 + 2 * i * kXPitch, xsrc[i] + (ok ? k0 : 0), ok);
-      }
-    }
-    if (sq_on) {
-      const int gi = (lg < 0 ? 0 : (k0 >> lg)) + sq_k;
-      const bool ok = srok && gi < a.G;
-      const size_t off = ok ? (size_t)gi * 16 : 0;
-      cp_async16(base + St::S_OFF + lane * 16, sbase + off, ok);
-      if constexpr (MODE == kASYM)
-        cp_async16(base + St::Z_OFF + lane * 16, a.zl + (sbase - a.scales) + off, ok);
-    }
-    if constexpr (zero_opts(MODE)) {
-      // the zps zero groups that meet the stage's 128 columns, per row block:
-      // fp16 records (32 bytes) in two 16-byte pieces each, 4-bit records
-      // (8 bytes) in one 8-byte piece each; a piece never spans two records,
-      // so its validity is its record's and its source stays aligned
-      const int zf = k0 >> a.lgz;
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        if (lane + 32 * h < R * zppr) {   // warp-uniform for h = 0 once zppr >= 16
-          const int r = zr[h], pc = zpc[h];
-          const int rb = tile * R + r;
-          const int zi = zf + pc / zppz;
-          const bool ok = rb < a.nrb && zi < a.GZ;
-          const uint8_t* src = zbytes + ((size_t)rb * a.GZ + zi) * zrec + (pc % zppz) * 16;
-          if constexpr (zrec == 32)
-            cp_async16(base + St::Z_OFF + r * kZxRb<MODE> + pc * 16, ok ? src : zbytes, ok);
-          else
-            cp_async8(base + St::Z_OFF + r * kZxRb<MODE> + pc * 8, ok ? src : zbytes, ok);
+      for (int i = 0; i < (TOK + 1) / 2; ++i) {
+        if (i < xi_n) {   // warp-uniform
+          const bool ok = xrow0 + 2 * i < mrows && xk;
+          cp_async16(base + xdst0 + 2 * i * kXPitch, xsrc[i] + (ok ? k0 : 0), ok);
         }
       }
+      if (sq_on) {
+        const int gi = (lg < 0 ? 0 : (k0 >> lg)) + sq_k;
+        const bool ok = srok && gi < a.G;
+        const size_t off = ok ? (size_t)gi * 16 : 0;
+        cp_async16(base + St::S_OFF + lane * 16, sbase + off, ok);
+        if constexpr (MODE == kASYM)
+          cp_async16(base + St::Z_OFF + lane * 16, a.zl + (sbase - a.scales) + off, ok);
+      }
     }
+    if constexpr (zero_opts(MODE)) issue_zeros(tile, k0, base);
   };
 
   // ---- prologue: S - 1 super-chunks in flight (the warp's own units, in
   // order: consecutive super-chunks, then the next tile)
-  long long pf_u = ub;
+  int pf_u = ub;
   // the warp's first tile and super-chunk (ub < 2^31)
   const int tb = ctile ? (int)blockIdx.x : (int)((unsigned)ub / (unsigned)n);
-  const int sb = ctile ? warp : (int)(ub - (long long)tb * n);
+  const int sb = ctile ? warp : ub - tb * n;
   int pf_t = tb, pf_s = sb;
   auto pf_next = [&]() {
     ++pf_u;
@@ -424,7 +445,7 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1) skinny_kernel(const
   }
 
   int tile = tb, sc = sb;
-  long long u = ub;
+  int u = ub;
   float part[NACC];                      // CTA-per-tile mode: this warp's sums
 #pragma unroll
   for (int i = 0; i < NACC; ++i) part[i] = 0.0f;
@@ -476,8 +497,8 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1) skinny_kernel(const
   while (u < ue) {
     // this warp's segment of the tile: super-chunks [s0, s1)
     const int s0 = sc;
-    const long long tile_end = (long long)(tile + 1) * n;
-    const int s1 = ctile ? n : (int)((ue < tile_end ? ue : tile_end) - (long long)tile * n);
+    const int tile_end = (tile + 1) * n;
+    const int s1 = ctile ? n : (ue < tile_end ? ue : tile_end) - tile * n;
 
     float acc[R][NT][4];
 #pragma unroll
