@@ -446,9 +446,15 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1) skinny_kernel(const
 
   int tile = tb, sc = sb;
   int u = ub;
-  float part[NACC];                      // CTA-per-tile mode: this warp's sums
+  // the current tile segment's sums; in CTA-per-tile mode they stay this
+  // warp's contribution to the CTA's one tile after the loop
+  float acc[R][NT][4];
 #pragma unroll
-  for (int i = 0; i < NACC; ++i) part[i] = 0.0f;
+  for (int r = 0; r < R; ++r)
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) acc[r][nt][i] = 0.0f;
   int st_c = 0;                          // ring stage being computed
   int st_f = S - 1;                      // ring stage being filled
 
@@ -500,7 +506,6 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1) skinny_kernel(const
     const int tile_end = (tile + 1) * n;
     const int s1 = ctile ? n : (ue < tile_end ? ue : tile_end) - tile * n;
 
-    float acc[R][NT][4];
 #pragma unroll
     for (int r = 0; r < R; ++r)
 #pragma unroll
@@ -710,11 +715,7 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1) skinny_kernel(const
     }
 
     float* outv = &acc[0][0][0];
-    if (ctile) {
-#pragma unroll
-      for (int i = 0; i < NACC; ++i) part[i] = outv[i];
-      break;
-    }
+    if (ctile) break;
     // ---- this warp's result for the tile segment: store y (whole tile) or
     // hand a partial to the last warp that finishes the tile
     const bool whole = s0 == 0 && s1 == n;
@@ -784,13 +785,14 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1) skinny_kernel(const
     __syncthreads();
     float* red = reinterpret_cast<float*>(smem + kTabBytes<MODE>);   // [kWarps][32][NACC]
     float4* mine = reinterpret_cast<float4*>(red + ((size_t)warp * 32 + lane) * NACC);
+    const float* part = &acc[0][0][0];
 #pragma unroll
     for (int i = 0; i < NACC / 4; ++i)
       mine[i] = make_float4(part[4 * i], part[4 * i + 1], part[4 * i + 2], part[4 * i + 3]);
     __syncthreads();
     if (warp == 0) {
-      float acc[R][NT][4];
-      float* outv = &acc[0][0][0];
+      float sum[R][NT][4];
+      float* outv = &sum[0][0][0];
 #pragma unroll
       for (int i = 0; i < NACC; ++i) outv[i] = 0.0f;
       for (int w = 0; w < kWarps; ++w) {
@@ -804,7 +806,7 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1) skinny_kernel(const
           outv[4 * i + 3] += v.w;
         }
       }
-      store_y(acc, (int)blockIdx.x);
+      store_y(sum, (int)blockIdx.x);
     }
   }
 }
