@@ -263,22 +263,46 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   };
 
   if (warp == 0) {
-    // ------------------------------------------------------------ TMA producer
+    // ------------------------------------------------------------ TMA producers
+    // Two independent single-thread loops: lane 0 streams the code tiles from
+    // HBM as far ahead as the code ring allows (its latency is the long one),
+    // lane 1 the x tiles (L2-resident) as the A/B ring frees its stages.
     if (lane == 0) {
-      int kc = 0, ks = 0;     // running k-block counters for the code / A-B rings
+      int kc = 0;             // running k-block counter of the code ring
       for (long long u = u_begin; u < u_end && !*abort_flag;) {
         int tile, kb0, kb1;
         seg_of(u, tile, kb0, kb1);
-        const int tn = tile % a.tiles_n, tm = tile / a.tiles_n;
-        for (int kb = kb0; kb < kb1; ++kb, ++kc, ++ks) {
-          const int c = kc % kCodeStages, s = ks % S;
-          if (!mbar_wait(&code_empty[c], ((kc / kCodeStages) & 1) ^ 1, abort_flag)) break;
+        const int tn = tile % a.tiles_n;
+        bool ok = true;
+        for (int kb = kb0; kb < kb1; ++kb, ++kc) {
+          const int c = kc % kCodeStages;
+          if (!mbar_wait(&code_empty[c], ((kc / kCodeStages) & 1) ^ 1, abort_flag)) {
+            ok = false;
+            break;
+          }
           mbar_expect_tx(&code_full[c], kCodeBytes);
           tma_load_2d(sC + c * kCodeBytes, &map_w, &code_full[c], kb * 128, tn * 8);
-          if (!mbar_wait(&ab_empty[s], ((ks / S) & 1) ^ 1, abort_flag)) break;
+        }
+        if (!ok) break;
+        u += kb1 - kb0;
+      }
+    } else if (lane == 1) {
+      int ks = 0;             // running k-block counter of the A/B ring
+      for (long long u = u_begin; u < u_end && !*abort_flag;) {
+        int tile, kb0, kb1;
+        seg_of(u, tile, kb0, kb1);
+        const int tm = tile / a.tiles_n;
+        bool ok = true;
+        for (int kb = kb0; kb < kb1; ++kb, ++ks) {
+          const int s = ks % S;
+          if (!mbar_wait(&ab_empty[s], ((ks / S) & 1) ^ 1, abort_flag)) {
+            ok = false;
+            break;
+          }
           mbar_expect_tx(&b_full[s], Cfg::B_BYTES);
           tma_load_2d(sB + s * Cfg::B_BYTES, &map_x, &b_full[s], kb * kKB, tm * BN);
         }
+        if (!ok) break;
         u += kb1 - kb0;
       }
     }
