@@ -137,7 +137,8 @@ struct TcArgs {
   int tiles_n, tiles_m, tiles;
   long long units;          // tiles * nkb
   int ctas;
-  float* slots;             // [2 * ctas][128][BN]: a CTA's first / last partial tile
+  float* slots;             // [2 * ctas][BN][128]: a CTA's first / last partial tile,
+                            // column-major so that a warp's 32 rows are 128 contiguous bytes
   unsigned* counters;       // [tiles]
 };
 
@@ -488,13 +489,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       }
       const long long t_first = (long long)tile * a.nkb;
       const bool whole = (u == t_first) && (kb1 == a.nkb);
-      // partial tiles: slot 2 b + e holds this CTA's [128 rows][BN] fp32 sums
+      // partial tiles: slot 2 b + e holds this CTA's [BN][128 rows] fp32 sums
       // (e = 1 when the tile is not the CTA's first); contributors are CTAs
       // first .. first + nb - 1, of which only `first` can have e = 1
       float* slot = nullptr;
       if (!whole) {
         const int e = (tile == (int)(u_begin / a.nkb)) ? 0 : 1;
-        slot = a.slots + (size_t)(2 * b + e) * (size_t)(BN * kRowsTile) + (size_t)row_l * BN;
+        slot = a.slots + (size_t)(2 * b + e) * (size_t)(BN * kRowsTile) + row_l;
         if (threadIdx.x == kEpi0) {     // 64-bit stream-K bookkeeping, once
           const int first = owner_of_tc(t_first, a.units, a.ctas);
           meta[0] = first;
@@ -531,6 +532,56 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           }
         }
       };
+      // A partial tile whose other contributors have all arrived already (the
+      // usual case for a CTA's last segment: the tile's remainder was the next
+      // CTA's first work): this CTA is certainly the last one, so it adds the
+      // others' slots to its own sums straight from TMEM, without writing its
+      // own slot.  Contributors are added in order, as in the general path.
+      if (!whole) {
+        named_bar(1, 128);   // meta written
+        if (threadIdx.x == kEpi0) {
+          unsigned cur;
+          asm volatile("ld.acquire.gpu.u32 %0, [%1];" : "=r"(cur) : "l"(&a.counters[tile]) : "memory");
+          *last_flag = cur == (unsigned)(meta[1] - 1) ? 2 : 0;
+        }
+        named_bar(1, 128);
+      }
+      if (!whole && *last_flag == 2) {
+        const int first = meta[0], nb = meta[1], first_e = meta[2];
+        const int own = b - first;
+#pragma unroll 1
+        for (int c0 = 0; c0 < BN; c0 += 32) {
+          float accv[32];
+          tmem_ld32(tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * BN + c0), accv);
+          if (own != 0) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) accv[i] = 0.0f;
+          }
+          for (int k = 0; k < nb; ++k) {
+            float va[32];
+            if (k == own) {
+              if (k == 0) continue;   // own sums already in accv
+              tmem_ld32(tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * BN + c0), va);
+            } else {
+              const float* pa = a.slots +
+                                (size_t)(2 * (first + k) + (k == 0 ? first_e : 0)) * (BN * kRowsTile) +
+                                (size_t)c0 * kRowsTile + row_l;
+#pragma unroll
+              for (int i = 0; i < 32; ++i) va[i] = __ldcg(pa + (size_t)i * kRowsTile);
+            }
+#pragma unroll
+            for (int i = 0; i < 32; ++i) accv[i] += va[i];
+          }
+          store32(accv, c0);
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&acc_empty[buf]);     // the accumulator may be reused
+        if (threadIdx.x == kEpi0) a.counters[tile] = 0u;   // ready for the next call
+        named_bar(1, 128);   // last_flag / meta are reused by the next segment
+        u += kb1 - kb0;
+        continue;
+      }
 #pragma unroll 1
       for (int c0 = 0; c0 < BN; c0 += 32) {
         float v[32];
@@ -538,9 +589,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         if (whole) {
           store32(v, c0);
         } else {
-          float4* dst = reinterpret_cast<float4*>(slot + c0);
+          // column c of the slot: the warp's 32 rows are one 128-byte line
 #pragma unroll
-          for (int i = 0; i < 8; ++i) dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+          for (int i = 0; i < 32; ++i) __stcg(slot + (size_t)(c0 + i) * kRowsTile, v[i]);
         }
       }
       tc_fence_before();
@@ -565,33 +616,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             float accv[32];
 #pragma unroll
             for (int i = 0; i < 32; ++i) accv[i] = 0.0f;
-            for (int k0 = 0; k0 < nb; k0 += 2) {      // two contributors' loads in flight
-              float4 va[8], vb[8];
-              const float4* pa = reinterpret_cast<const float4*>(
-                  a.slots + (size_t)(2 * (first + k0) + (k0 == 0 ? first_e : 0)) * (BN * kRowsTile) +
-                  (size_t)row_l * BN + c0);
+            for (int k = 0; k < nb; ++k) {      // one contributor's 32 loads in flight
+              const float* pa = a.slots +
+                                (size_t)(2 * (first + k) + (k == 0 ? first_e : 0)) * (BN * kRowsTile) +
+                                (size_t)c0 * kRowsTile + row_l;
+              float va[32];
 #pragma unroll
-              for (int i = 0; i < 8; ++i) va[i] = __ldcg(pa + i);
-              const bool two = k0 + 1 < nb;
-              if (two) {
-                const float4* pb = reinterpret_cast<const float4*>(
-                    a.slots + (size_t)(2 * (first + k0 + 1)) * (BN * kRowsTile) +
-                    (size_t)row_l * BN + c0);
+              for (int i = 0; i < 32; ++i) va[i] = __ldcg(pa + (size_t)i * kRowsTile);
 #pragma unroll
-                for (int i = 0; i < 8; ++i) vb[i] = __ldcg(pb + i);
-              }
-#pragma unroll
-              for (int i = 0; i < 8; ++i) {
-                accv[4 * i] += va[i].x; accv[4 * i + 1] += va[i].y;
-                accv[4 * i + 2] += va[i].z; accv[4 * i + 3] += va[i].w;
-              }
-              if (two) {
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                  accv[4 * i] += vb[i].x; accv[4 * i + 1] += vb[i].y;
-                  accv[4 * i + 2] += vb[i].z; accv[4 * i + 3] += vb[i].w;
-                }
-              }
+              for (int i = 0; i < 32; ++i) accv[i] += va[i];
             }
             store32(accv, c0);
           }
