@@ -42,6 +42,12 @@ constexpr int kRowsTile = 128;      // weight rows per tile (UMMA M)
 constexpr int kCodeStages = 8;
 constexpr int kCodeBytes = 8 * 512; // 8 row blocks x one 512-byte chunk
 constexpr int kATileBytes = kRowsTile * kKB * 2;   // 16 KB
+// Per code stage, the k block's group scales (and ASYM zero-points) of the
+// tile's 8 row blocks, loaded by TMA with the codes: [8][sx] fp16, sx = 16
+// slots x the groups in 64 columns (at most 4), 1 KB each.
+constexpr int kMetaTile = 1024;
+template <int MODE>
+constexpr int kMetaBytes = MODE == kASYM ? 2 * kMetaTile : kMetaTile;
 constexpr long long kWaitCycles = 4000000000ll; // ~2 s at 1.9 GHz
 
 template <int BN>
@@ -132,6 +138,7 @@ struct TcArgs {
   const uint16_t* zl;
   uint16_t* y;
   int M, N, K, L, G, nrb, nkb;
+  int sx;                   // scale (zero) elements per row block in a k block's meta tile
   int lg;                   // log2 of the group length; 30 for one group per row
   int gated;                // 1: alternating 16-row gate / up blocks, y[M, N/2] = silu(gate) up
   int tiles_n, tiles_m, tiles;
@@ -181,17 +188,23 @@ __device__ __forceinline__ uint32_t lut_pair(uint32_t t16, float s) {
 template <int MODE, bool BF16, int BN, bool GM1>
 __global__ void __launch_bounds__(kTcThreads, 1)
     tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_w,
+              const __grid_constant__ CUtensorMap map_s, const __grid_constant__ CUtensorMap map_z,
               const TcArgs a) {
   using Cfg = TcCfg<BN>;
   constexpr int S = Cfg::STAGES;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
-  // carve: A stages | B stages | code stages | LUT table | barriers
+  // carve: A stages | B stages | code stages | meta stages | LUT table | barriers
   unsigned char* base = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   unsigned char* sA = base;
   unsigned char* sB = sA + S * kATileBytes;
   unsigned char* sC = sB + S * Cfg::B_BYTES;
-  unsigned char* sT = sC + kCodeStages * kCodeBytes;
+  unsigned char* sM = sC + kCodeStages * kCodeBytes;
+  unsigned char* sT = sM + kCodeStages * kMetaBytes<MODE>;
+  // group scales and zero-points come with the codes (per-row scales of
+  // group -1 are applied in the epilogue instead)
+  constexpr bool kScales = !GM1;
+  constexpr bool kZeros = MODE == kASYM;
   constexpr int TAB = MODE == kLUT ? 256 * 32 * 4 : 0;
   uint64_t* bars = reinterpret_cast<uint64_t*>(sT + TAB);
   uint64_t* code_full = bars;
@@ -231,6 +244,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   if (warp == 0 && lane == 0) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&map_x)) : "memory");
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&map_w)) : "memory");
+    if constexpr (kScales)
+      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&map_s)) : "memory");
+    if constexpr (kZeros)
+      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&map_z)) : "memory");
   }
   pdl_wait();                 // inputs may come from the previous grid; TMEM taken after this
   pdl_launch_dependents();
@@ -281,8 +298,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             ok = false;
             break;
           }
-          mbar_expect_tx(&code_full[c], kCodeBytes);
+          constexpr int kMetaCopies = (kScales ? 1 : 0) + (kZeros ? 1 : 0);
+          mbar_expect_tx(&code_full[c], kCodeBytes + kMetaCopies * 8 * a.sx * 2);
           tma_load_2d(sC + c * kCodeBytes, &map_w, &code_full[c], kb * 128, tn * 8);
+          // the k block's first group, 16 slots per group (the x coordinate is
+          // a multiple of 16 elements: 32-byte aligned)
+          const int gx = ((kb * kKB) >> a.lg) * 16;
+          if constexpr (kScales)
+            tma_load_2d(sM + c * kMetaBytes<MODE>, &map_s, &code_full[c], gx, tn * 8);
+          if constexpr (kZeros)
+            tma_load_2d(sM + c * kMetaBytes<MODE> + kMetaTile, &map_z, &code_full[c], gx, tn * 8);
         }
         if (!ok) break;
         u += kb1 - kb0;
@@ -347,63 +372,27 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const int dw = warp - 2;                 // row blocks kRbPerDec dw + rr of the tile
     const int g = lane >> 2, t = lane & 3;
     const unsigned char* tabp = sT;
-    // Group scales (and ASYM zero-points) of the lane's rows g and g + 8 in its
-    // two row blocks, one word per 16-column slice of the k block, read from
-    // global memory two k blocks ahead so that the loads overlap decodes.
-    constexpr bool kScales = !GM1;
-    constexpr bool kZeros = MODE == kASYM;
-    uint32_t sw_n[kRbPerDec][4] = {}, zw_n[kRbPerDec][4] = {};     // unit u + 1
-    uint32_t sw_nn[kRbPerDec][4] = {}, zw_nn[kRbPerDec][4] = {};   // unit u + 2
-    auto load_meta = [&](int tl, int k, uint32_t (&sw_o)[kRbPerDec][4], uint32_t (&zw_o)[kRbPerDec][4]) {
-      if constexpr (kScales || kZeros) {
-        const int tn = tl % a.tiles_n;
-#pragma unroll
-        for (int rr = 0; rr < kRbPerDec; ++rr) {
-          const int rb = tn * 8 + kRbPerDec * dw + rr;
-          const bool in = rb < a.nrb;
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const int gi = (k * kKB + 16 * j) >> a.lg;
-            const size_t off = ((size_t)rb * a.G + gi) * 16 + 2 * g;
-            if constexpr (kScales)
-              sw_o[rr][j] = in ? __ldg(reinterpret_cast<const unsigned int*>(a.scales + off)) : 0u;
-            if constexpr (kZeros)
-              zw_o[rr][j] = in ? __ldg(reinterpret_cast<const unsigned int*>(a.zl + off)) : 0u;
-          }
-        }
-      }
-    };
-    // (ct, ck): the unit two ahead of the one being decoded, u = ct nkb + ck
-    int ct = (int)(u_begin / a.nkb), ck = (int)(u_begin % a.nkb);
-    auto advance = [&]() {
-      if (++ck == a.nkb) {
-        ck = 0;
-        ++ct;
-      }
-    };
-    if (u_begin < u_end) load_meta(ct, ck, sw_n, zw_n);
-    advance();
-    if (u_begin + 1 < u_end) load_meta(ct, ck, sw_nn, zw_nn);
-    advance();
     int kc = 0, ks = 0;
     for (long long u = u_begin; u < u_end && !*abort_flag; ++u, ++kc, ++ks) {
-      uint32_t sw[kRbPerDec][4], zw[kRbPerDec][4];
-#pragma unroll
-      for (int rr = 0; rr < kRbPerDec; ++rr)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          sw[rr][j] = sw_n[rr][j];
-          zw[rr][j] = zw_n[rr][j];
-          sw_n[rr][j] = sw_nn[rr][j];
-          zw_n[rr][j] = zw_nn[rr][j];
-        }
-      if (u + 2 < u_end) load_meta(ct, ck, sw_nn, zw_nn);
-      advance();
       const int c = kc % kCodeStages, s = ks % S;
       if (!mbar_wait(&code_full[c], (kc / kCodeStages) & 1, abort_flag) ||
           !mbar_wait(&ab_empty[s], ((ks / S) & 1) ^ 1, abort_flag))
         break;
       unsigned char* At = sA + s * kATileBytes;
+      // group scales (and zero-points) of the lane's rows g and g + 8, one word
+      // per 16-column slice j, from the k block's meta tile (landed with the codes)
+      uint32_t sw[kRbPerDec][4], zw[kRbPerDec][4];
+      if constexpr (kScales || kZeros) {
+        const unsigned char* mt = sM + c * kMetaBytes<MODE>;
+#pragma unroll
+        for (int rr = 0; rr < kRbPerDec; ++rr)
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const int e = (kRbPerDec * dw + rr) * a.sx + ((16 * j) >> a.lg) * 16 + 2 * g;
+            if constexpr (kScales) sw[rr][j] = *reinterpret_cast<const uint32_t*>(mt + 2 * e);
+            if constexpr (kZeros) zw[rr][j] = *reinterpret_cast<const uint32_t*>(mt + kMetaTile + 2 * e);
+          }
+      }
 #pragma unroll
       for (int rr = 0; rr < kRbPerDec; ++rr) {
         const int rbl = kRbPerDec * dw + rr;               // row block in the tile
@@ -656,13 +645,13 @@ template <int MODE, int BN>
 constexpr size_t tc_smem_bytes() {
   using Cfg = TcCfg<BN>;
   return 1024 + (size_t)Cfg::STAGES * (kATileBytes + Cfg::B_BYTES) +
-         (size_t)kCodeStages * kCodeBytes + (MODE == kLUT ? 256 * 32 * 4 : 0) +
+         (size_t)kCodeStages * (kCodeBytes + kMetaBytes<MODE>) + (MODE == kLUT ? 256 * 32 * 4 : 0) +
          (2 * kCodeStages + 3 * Cfg::STAGES + 4) * 8 + 32;
 }
 
 template <int MODE, bool BF16, int BN, bool GM1>
-cudaError_t launch_tc_t(const CUtensorMap& mx, const CUtensorMap& mw, const TcArgs& args,
-                        cudaStream_t stream) {
+cudaError_t launch_tc_t(const CUtensorMap& mx, const CUtensorMap& mw, const CUtensorMap& ms,
+                        const CUtensorMap& mz, const TcArgs& args, cudaStream_t stream) {
   auto k = tc_kernel<MODE, BF16, BN, GM1>;
   constexpr size_t smem = tc_smem_bytes<MODE, BN>();
   static bool attr_set[64] = {};
@@ -686,26 +675,27 @@ cudaError_t launch_tc_t(const CUtensorMap& mx, const CUtensorMap& mw, const TcAr
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, k, mx, mw, args);
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, k, mx, mw, ms, mz, args);
   if (e != cudaSuccess) cudaGetLastError();   // report it once, here
   return e;
 }
 
 template <int MODE, bool BF16, bool GM1>
-cudaError_t launch_bn(int bn, const CUtensorMap& mx, const CUtensorMap& mw, const TcArgs& args,
-                      cudaStream_t s) {
-  if (bn == 64) return launch_tc_t<MODE, BF16, 64, GM1>(mx, mw, args, s);
-  if (bn == 128) return launch_tc_t<MODE, BF16, 128, GM1>(mx, mw, args, s);
-  return launch_tc_t<MODE, BF16, 256, GM1>(mx, mw, args, s);
+cudaError_t launch_bn(int bn, const CUtensorMap& mx, const CUtensorMap& mw, const CUtensorMap& ms,
+                      const CUtensorMap& mz, const TcArgs& args, cudaStream_t s) {
+  if (bn == 64) return launch_tc_t<MODE, BF16, 64, GM1>(mx, mw, ms, mz, args, s);
+  if (bn == 128) return launch_tc_t<MODE, BF16, 128, GM1>(mx, mw, ms, mz, args, s);
+  return launch_tc_t<MODE, BF16, 256, GM1>(mx, mw, ms, mz, args, s);
 }
 
 template <int MODE>
 cudaError_t launch_mode(bool bf16, bool gm1, int bn, const CUtensorMap& mx, const CUtensorMap& mw,
-                        const TcArgs& args, cudaStream_t s) {
-  if (bf16) return gm1 ? launch_bn<MODE, true, true>(bn, mx, mw, args, s)
-                       : launch_bn<MODE, true, false>(bn, mx, mw, args, s);
-  return gm1 ? launch_bn<MODE, false, true>(bn, mx, mw, args, s)
-             : launch_bn<MODE, false, false>(bn, mx, mw, args, s);
+                        const CUtensorMap& ms, const CUtensorMap& mz, const TcArgs& args,
+                        cudaStream_t s) {
+  if (bf16) return gm1 ? launch_bn<MODE, true, true>(bn, mx, mw, ms, mz, args, s)
+                       : launch_bn<MODE, true, false>(bn, mx, mw, ms, mz, args, s);
+  return gm1 ? launch_bn<MODE, false, true>(bn, mx, mw, ms, mz, args, s)
+             : launch_bn<MODE, false, false>(bn, mx, mw, ms, mz, args, s);
 }
 
 }  // namespace
@@ -783,7 +773,27 @@ cudaError_t launch_tc(const Problem& pr, const TcPlan& plan, void* workspace,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return cudaErrorInvalidValue;
   }
+  // group scales and zero-points ([N/16][G][16] fp16) as [G 16] x [N/16]: one
+  // box = the sx slots of a k block's groups for 8 row blocks (the zero map
+  // is only read for ASYM; without zeros it repeats the scale map)
+  const int L = pr.group == -1 ? pr.K : pr.group;
+  const int G = pr.K / L;
+  const int sx = 16 * std::max(1, kKB / L);
+  CUtensorMap ms, mz;
+  for (int which = 0; which < 2; ++which) {
+    const uint16_t* src = (which == 1 && pr.mode == kASYM) ? pr.zl : pr.scales;
+    const cuuint64_t dims[2] = {(cuuint64_t)G * 16, (cuuint64_t)(pr.N / 16)};
+    const cuuint64_t strides[1] = {(cuuint64_t)G * 32};
+    const cuuint32_t box[2] = {(cuuint32_t)sx, 8};
+    const cuuint32_t es[2] = {1, 1};
+    if (encode(which ? &mz : &ms, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, const_cast<uint16_t*>(src),
+               dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
   TcArgs a{};
+  a.sx = sx;
   a.scales = pr.scales;
   a.zl = pr.zl;
   a.y = reinterpret_cast<uint16_t*>(pr.y);
@@ -808,9 +818,9 @@ cudaError_t launch_tc(const Problem& pr, const TcPlan& plan, void* workspace,
   }
   const bool gm1 = pr.group == -1;
   switch (pr.mode) {
-    case kSYM: return launch_mode<kSYM>(pr.bf16, gm1, plan.bn, mx, mw, a, stream);
-    case kASYM: return launch_mode<kASYM>(pr.bf16, gm1, plan.bn, mx, mw, a, stream);
-    default: return launch_mode<kLUT>(pr.bf16, gm1, plan.bn, mx, mw, a, stream);
+    case kSYM: return launch_mode<kSYM>(pr.bf16, gm1, plan.bn, mx, mw, ms, mz, a, stream);
+    case kASYM: return launch_mode<kASYM>(pr.bf16, gm1, plan.bn, mx, mw, ms, mz, a, stream);
+    default: return launch_mode<kLUT>(pr.bf16, gm1, plan.bn, mx, mw, ms, mz, a, stream);
   }
 }
 
