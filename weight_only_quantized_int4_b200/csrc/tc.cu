@@ -10,9 +10,11 @@
 // per 64-column K block, with A = decoded weights (fp16/bf16, written into
 // shared memory in the 128-byte-swizzled K-major layout by decode warps) and
 // B = a TMA-loaded tile of x.  Warp roles:
-//   warp 0      TMA producer: code tiles (4 KB, 8 row blocks) and x tiles
+//   warp 0      TMA producers: lane 0 code tiles (4 KB, 8 row blocks) with their
+//               group scales / zero-points, lane 1 x tiles
 //   warp 1      TMEM owner and MMA issuer (one elected thread)
-//   next kDecWarps warps   decode: codes (smem) -> (q - z) s, T[q] s -> A tile
+//   next kDecWarps warps   decode, one row block each: codes and scales (smem)
+//                          -> (q - z) s, T[q] s -> A tile
 //   last 4 warps           epilogue: TMEM -> registers -> y (or split-K partials)
 // Work is split stream-K over (tile, K block) units across a grid of one CTA
 // per SM, like the decode path; partial tiles are reduced deterministically by
@@ -33,7 +35,7 @@ __device__ unsigned g_tc_error = 0;
 
 namespace {
 
-constexpr int kDecWarps = 4;                        // decode warps (8 row blocks between them)
+constexpr int kDecWarps = 8;                        // decode warps (one of the 8 row blocks each)
 constexpr int kRbPerDec = 8 / kDecWarps;            // row blocks per decode warp
 constexpr int kTcThreads = 32 * (2 + kDecWarps + 4);
 constexpr int kEpi0 = 32 * (2 + kDecWarps);          // first epilogue thread
