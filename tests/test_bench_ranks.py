@@ -71,3 +71,21 @@ def test_reference_arm_runs_on_rank_zero_only():
                        text=True, timeout=120)
     assert p.returncode == 0, p.stderr
     assert p.stdout.strip() == ""
+
+
+def test_workload_units_and_bytes():
+    """Tensor-bound workloads (every call M >= 256) are reported in TFLOP/s,
+    the rest in GB/s; algorithmic bytes count the zero-point records and the
+    act-order permutation."""
+    assert bench.tensor_bound("prefill_m4096") and bench.tensor_bound("prefill_m256")
+    assert not bench.tensor_bound("llama7b_decode") and not bench.tensor_bound("prefill_m64")
+    assert bench.alg_flops(2, 3, 5) == 60.0
+    K, N = 4096, 14336
+    plain = bench.alg_bytes("asym", 4, -1, 1, K, N)
+    zg8 = bench.alg_bytes("asym", 4, -1, 1, K, N, zopts=(8, 4))
+    # fp16 row zero (N * 2 bytes) replaced by 4-bit zeros per 8 columns (N * K / 16)
+    assert zg8 - plain == N * K // 16 - N * 2
+    assert bench.alg_bytes("sym", 4, 128, 1, K, N, actorder=True) == \
+        bench.alg_bytes("sym", 4, 128, 1, K, N) + 4 * K
+    assert bench.alg_bytes("sym", 4, 128, 2, K, 2 * 64, gated=True) == \
+        bench.alg_bytes("sym", 4, 128, 2, K, 2 * 64) - 2 * 64 * 2
