@@ -401,7 +401,9 @@ def run_ours(args, rank, world, local_rank):
     else:
         peak, peak_kind = peaks()
         achieved = step_bytes / (ms_per_step / 1e3) / 1e9      # one GPU, the skinny kernel only
-        tpb = traffic_per_byte()
+        # DRAM bytes per algorithmic byte come from the ncu capture of the
+        # default workload; other workloads report none
+        tpb = traffic_per_byte() if args.workload == "llama7b_decode" else None
         unit = "GB/s"
         roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                     "frac": round(achieved / peak, 4), "peak_source": peak_kind,
