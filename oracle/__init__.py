@@ -292,25 +292,3 @@ def qmm_gidx(x, xdtype, qweight, scales_p, zeros_or_lut, g_idx, M, N, K, mode, b
         _p(zl), _p(_gidx(g_idx)), M, N, K, MODES[mode], bits, group, n0, n1, _p(y)),
         "oracle_qmm_gidx")
     return y
-
-
-def qmm_threaded(x, xdtype, qweight, scales_p, zeros_or_lut, M, N, K, mode, bits, group,
-                 n0, n1, threads):
-    """oracle qmm over [n0, n1) split into `threads` contiguous column ranges.
-
-    ctypes releases the GIL during the foreign call, so Python threads run the
-    ranges on separate host cores.  The arithmetic per column is unchanged.
-    """
-    bounds = np.linspace(n0, n1, threads + 1).astype(int)
-    parts = [None] * threads
-
-    def work(i):
-        parts[i] = qmm(x, xdtype, qweight, scales_p, zeros_or_lut, M, N, K, mode, bits, group,
-                       int(bounds[i]), int(bounds[i + 1]))
-
-    ts = [threading.Thread(target=work, args=(i,)) for i in range(threads)]
-    for t in ts:
-        t.start()
-    for t in ts:
-        t.join()
-    return np.concatenate(parts, axis=1)
