@@ -138,10 +138,11 @@ size_t qmm_workspace_size_for(int M, int N, int K, int bits, int group, int mode
  *   workspace     device, workspace_bytes >= qmm_workspace_size(...), zero
  *                 filled before first use (see above); may be NULL with
  *                 workspace_bytes 0, in which case no cross-CTA split-K is used.
- * The accumulation is fp32.  M <= 16 runs the bandwidth-bound decode path,
- * larger M the tcgen05 tensor-core path for 4-bit codes with fp16 activations
- * or with bf16 activations and per-row scales (group -1, SYM/ASYM); the other
- * combinations stay on the decode path.  qmm_path tells which.  The tensor path reads x through a TMA
+ * The accumulation is fp32.  M <= 32 (M <= 64 when N <= 4096) runs the
+ * bandwidth-bound decode path (16 tokens per slab), larger M the tcgen05
+ * tensor-core path for 4-bit codes with fp16 activations or with bf16
+ * activations and per-row scales (group -1, SYM/ASYM); the other combinations
+ * stay on the decode path.  qmm_path tells which.  The tensor path reads x through a TMA
  * tensor map, so x's row pitch (K * 2 bytes) must be a multiple of 16 -- true
  * for every K the packed layout allows. */
 int qmm(const void* x, int xdtype, const void* qweight, const uint16_t* scales,

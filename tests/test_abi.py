@@ -43,7 +43,13 @@ def test_sizes_and_paths(lib):
     assert q.packed_size(16, 128, "lut", 2, 64) == (16 * 32, 16 * 2 * 2, 0)
     assert q.path(1, 4096, 4096, "sym") == "skinny"
     assert q.path(16, 4096, 4096, "sym") == "skinny"
-    assert q.path(64, 4096, 4096, "sym") == "tensor"
+    # measured crossover: the decode path up to M = 32, and up to M = 64 when
+    # N <= 4096; combinations the tensor path does not take stay on it
+    assert q.path(32, 11008, 4096, "sym") == "skinny"
+    assert q.path(33, 11008, 4096, "sym") == "tensor"
+    assert q.path(64, 4096, 4096, "sym") == "skinny"
+    assert q.path(65, 4096, 4096, "sym") == "tensor"
+    assert q.path(4096, 14336, 4096, "lut", 2, 64) == "skinny"
 
 
 @pytest.mark.parametrize("N,K,bits,group,mode,status", [

@@ -63,11 +63,16 @@ void zero_mode(int K, int group, int zgroup, int zbits, int* mode, int* zg) {
 size_t round256(size_t b) { return (b + 255) / 256 * 256; }
 
 // Decode path while the product is bandwidth-bound (few tokens), tensor-core
-// path once it becomes a dense contraction.  Combinations the tensor path does
-// not cover (2-bit codes; bf16 with group scales or a table) take the decode
-// path, in slabs of 16 tokens.
-int choose_path(int M, int bits, int mode, bool bf16, int group) {
-  if (M <= 16 || !tc_supported(bits, mode, bf16, group)) return QMM_PATH_SKINNY;
+// path once it becomes a dense contraction.  The crossover was measured on
+// B200 (K = 4096, N = 4096 .. 22016, SYM / LUT, M = 17 .. 96): two 16-token
+// slabs of the decode path beat the tensor path up to M = 32 (its time has a
+// floor of about 25-40 us per call there), and up to M = 64 for N <= 4096
+// (few row tiles for 148 SMs).  Combinations the tensor path does not cover
+// (2- and 3-bit codes; bf16 with group scales or a table; zero-point options)
+// take the decode path, in slabs of 16 tokens.
+int choose_path(int M, int N, int bits, int mode, bool bf16, int group) {
+  if (!tc_supported(bits, mode, bf16, group)) return QMM_PATH_SKINNY;
+  if (M <= 32 || (M <= 64 && N <= 4096)) return QMM_PATH_SKINNY;
   return QMM_PATH_TENSOR;
 }
 
@@ -83,7 +88,7 @@ struct Plan {
 Plan make_plan(int M, int N, int K, int bits, int group, int mode, bool bf16, int path) {
   Plan p{};
   const bool streamk = path == QMM_PATH_SKINNY_STREAMK;
-  p.path = path == QMM_PATH_AUTO ? choose_path(M, bits, mode, bf16, group)
+  p.path = path == QMM_PATH_AUTO ? choose_path(M, N, bits, mode, bf16, group)
            : streamk            ? QMM_PATH_SKINNY
                                 : path;
   if (p.path == QMM_PATH_TENSOR && !tc_supported(bits, mode, bf16, group)) p.path = QMM_PATH_SKINNY;
@@ -191,7 +196,7 @@ int qmm_path(int M, int N, int K, int bits, int group, int mode) {
   if (M < 0) return QMM_ERR_ARG;
   int st = check_shape(N, K, bits, group, mode);
   if (st != QMM_OK) return st;
-  return choose_path(M, bits, mode, false, group);
+  return choose_path(M, N, bits, mode, false, group);
 }
 
 size_t qmm_workspace_size_for(int M, int N, int K, int bits, int group, int mode, int path) {
