@@ -206,3 +206,75 @@ def test_actorder_needs_workspace():
     vp = lambda t: ctypes.c_void_p(t.data_ptr())
     assert lib.qmm_actorder(vp(fake), 0, vp(fake), vp(fake), vp(fake), None, 1, 16, 1024, 4, 128,
                             0, vp(fake[2048:]), None, 0, None) == -6
+
+
+# ------------------------------------------- full-size shapes, sampled rows
+#
+# The benchmark's shapes: every weight row is packed on the GPU, the oracle
+# computes four sampled row blocks (the first, the last and two seeded ones);
+# their bytes and their outputs are compared.
+
+def _sampled_weights(N, K, sigma, seed):
+    rows = cases.row_blocks(N, 4, seed + 1)
+    W_rows = synth.weights(seed, "W", N, K, sigma, rows=rows)
+    g = torch.Generator(device="cuda").manual_seed(seed)
+    W = torch.randn(N, K, generator=g, device="cuda") * sigma
+    W[torch.from_numpy(rows).cuda()] = torch.from_numpy(W_rows).cuda()
+    return rows, W_rows, W
+
+
+def _blocks(buf, rows, per_block):
+    blocks = np.unique(rows // 16)
+    return np.concatenate([buf[b * per_block:(b + 1) * per_block] for b in blocks])
+
+
+@pytest.mark.parametrize("K,N,group,zgroup,xdtype,Ms", [
+    (4096, 14336, -1, 8, "f16", (1, 8, 32)),          # bench asym_rowscale_zg8_u4
+    (8192, 57344, 128, 128, "bf16", (1, 16)),         # bench llama70b_asym_zq4_bf16
+])
+def test_zero_options_fullsize(K, N, group, zgroup, xdtype, Ms):
+    rows, W_rows, W = _sampled_weights(N, K, 0.015, 90)
+    qw, sc, ze = q.pack_asym(W, group, zgroup, 4)
+    del W
+    torch.cuda.synchronize()
+    c, s_, z = oracle.quantize_asym(W_rows, group, zgroup)
+    qw_o, sp_o, zp_o = oracle.pack_asym(c, s_, z, group, zgroup, 4)
+    G, GZ = (1 if group == -1 else K // group), K // zgroup
+    assert np.array_equal(_blocks(qw.cpu().numpy(), rows, K * 8), qw_o)
+    assert np.array_equal(_blocks(sc.cpu().numpy().view(np.uint16), rows, 16 * G), sp_o)
+    assert np.array_equal(_blocks(ze.cpu().numpy(), rows, 8 * GZ), zp_o)
+    Wt = oracle.dequant_asym(c, s_, z, group, zgroup)
+    for M in Ms:
+        x = synth.activations(91 + M, "x", M, K, xdtype)
+        ws = q.workspace_asym(M, N, K, group, zgroup, 4)
+        y = q.qmm_asym(dev(x).view(tdtype(xdtype)), qw, sc, ze, N, K, group, zgroup, 4, ws=ws)
+        torch.cuda.synchronize()
+        y_ref = oracle.qmm_asym(x, xdtype, qw_o, sp_o, zp_o, M, len(rows), K, group, zgroup, 4)
+        y_s = y[:, torch.from_numpy(rows).cuda()].float().cpu().numpy().astype(np.float64)
+        cases.compare(y_s, y_ref, bound_of(x, xdtype, Wt), f"zero options K{K} N{N} M{M}")
+    q.check_error()
+
+
+@pytest.mark.parametrize("K,N", [(4096, 22016), (11008, 4096)])
+def test_actorder_fullsize(K, N):
+    """bench actorder_llama7b shapes, on both paths (M = 1, 16 decode; 64 tensor for N > 4096)."""
+    group = 128
+    rows, W_rows, W = _sampled_weights(N, K, 0.02, 92)
+    gidx = _gidx(K, group, 93)
+    perm = q.actorder_perm(torch.from_numpy(gidx).cuda(), group)
+    qw, sc, _ = q.pack_actorder(W, perm, "sym", 4, group)
+    del W
+    torch.cuda.synchronize()
+    c, s_, _ = oracle.quantize_gidx(W_rows, "sym", 4, group, gidx)
+    qw_o, sp_o, _ = oracle.pack_gidx(c, s_, None, gidx, "sym", 4, group)
+    assert np.array_equal(_blocks(qw.cpu().numpy(), rows, K * 8), qw_o)
+    assert np.array_equal(_blocks(sc.cpu().numpy().view(np.uint16), rows, 16 * (K // group)), sp_o)
+    Wt = oracle.dequant_gidx(c, s_, None, "sym", 4, group, gidx)
+    for M in (1, 16, 64):
+        x = synth.activations(94 + M, "x", M, K, "f16")
+        y = q.qmm_actorder(dev(x).view(torch.float16), perm, qw, sc, None, N, K, "sym", 4, group)
+        torch.cuda.synchronize()
+        y_ref = oracle.qmm_gidx(x, "f16", qw_o, sp_o, None, gidx, M, len(rows), K, "sym", 4, group)
+        y_s = y[:, torch.from_numpy(rows).cuda()].float().cpu().numpy().astype(np.float64)
+        cases.compare(y_s, y_ref, bound_of(x, "f16", Wt), f"act-order K{K} N{N} M{M}")
+    q.check_error()
