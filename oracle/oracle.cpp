@@ -52,10 +52,10 @@
 //      2-bit LUT:      word j/2 of the lane, byte 2 (j % 2) + p / 2; inside the
 //                      byte the 2-bit field 2 (p % 2) + (c % 2).
 //      3-bit LUT:      chunks of 128 columns and 768 bytes, lane l owning bytes
-//                      [24 l, 24 l + 24): words 0..3 hold the codes' two low bits
-//                      exactly as the 2-bit layout places 2-bit codes; words
-//                      4 and 5 hold the high bits, tile j's eight in byte j % 4 of
-//                      word 4 + j / 4, pair p member c % 2 at bit 2 p + (c % 2).
+//                      [24 l, 24 l + 24), read as one 192-bit little-endian
+//                      string: tile j at bits [24 j, 24 j + 24), pair p at
+//                      [24 j + 6 p, + 6), member c % 2 at + 3 (c % 2) -- a pair is
+//                      one 6-bit field.
 //    Words are little-endian uint32; nibble/field f occupies bits [b f, b f + b).
 //  * scales (and ASYM zeros): fp16, [N/16][G][16]; inside the 16 the row r of
 //    the block sits at 2 (r % 8) + r / 8.
@@ -182,7 +182,7 @@ bool shape_ok(int N, int K, int mode, int bits, int group) {
 }
 
 // Byte offset and bit shift of code (n, k) in the packed code buffer (2- and
-// 4-bit codes; for 3-bit codes, of their two low bits).
+// 4-bit codes).
 void code_place(int n, int k, int K, int mode, int bits, size_t* byte, int* shift) {
   int kc_cols = chunk_cols(bits);
   int rb = n / 16, r = n % 16;
@@ -206,8 +206,10 @@ void code_place(int n, int k, int K, int mode, int bits, size_t* byte, int* shif
   }
 }
 
-// 3-bit codes: byte offset and bit of the code's high bit.
-void code_place_high(int n, int k, int K, size_t* byte, int* shift) {
+// 3-bit codes: bit offset of code (n, k)'s lowest bit in the packed buffer.
+// The lane's 24 bytes are one 192-bit little-endian string: tile j at bits
+// [24 j, 24 j + 24), pair p at [24 j + 6 p, + 6), member c % 2 at + 3 (c % 2).
+size_t code_bit3(int n, int k, int K) {
   int rb = n / 16, r = n % 16;
   int g = r % 8, h = r / 8;
   int chunk = k / 128, kk = k % 128;
@@ -215,31 +217,32 @@ void code_place_high(int n, int k, int K, size_t* byte, int* shift) {
   int lane = 4 * g + t;
   int p = h + 2 * (c / 2);
   size_t lane_base = ((size_t)rb * (K / 128) + chunk) * 768 + (size_t)lane * 24;
-  *byte = lane_base + 16 + (size_t)(j / 4) * 4 + (j % 4);
-  *shift = 2 * p + c % 2;
+  return lane_base * 8 + 24 * j + 6 * p + 3 * (c % 2);
 }
 
 int get_code(const uint8_t* qw, int n, int k, int K, int mode, int bits) {
+  if (bits == 3) {
+    int q = 0;
+    size_t b = code_bit3(n, k, K);
+    for (int i = 0; i < 3; ++i) q |= ((qw[(b + i) / 8] >> ((b + i) % 8)) & 1) << i;
+    return q;
+  }
   size_t byte;
   int shift;
   code_place(n, k, K, mode, bits, &byte, &shift);
-  if (bits != 3) return (qw[byte] >> shift) & ((1 << bits) - 1);
-  int q = (qw[byte] >> shift) & 3;
-  code_place_high(n, k, K, &byte, &shift);
-  return q | (((qw[byte] >> shift) & 1) << 2);
+  return (qw[byte] >> shift) & ((1 << bits) - 1);
 }
 
 void put_code(uint8_t* qw, int n, int k, int K, int mode, int bits, int q) {
+  if (bits == 3) {
+    size_t b = code_bit3(n, k, K);
+    for (int i = 0; i < 3; ++i) qw[(b + i) / 8] |= (uint8_t)(((q >> i) & 1) << ((b + i) % 8));
+    return;
+  }
   size_t byte;
   int shift;
   code_place(n, k, K, mode, bits, &byte, &shift);
-  if (bits != 3) {
-    qw[byte] |= (uint8_t)((q & ((1 << bits) - 1)) << shift);
-    return;
-  }
-  qw[byte] |= (uint8_t)((q & 3) << shift);
-  code_place_high(n, k, K, &byte, &shift);
-  qw[byte] |= (uint8_t)(((q >> 2) & 1) << shift);
+  qw[byte] |= (uint8_t)((q & ((1 << bits) - 1)) << shift);
 }
 
 // Index of (row n, group gi) in the packed scale / zero buffers.

@@ -263,10 +263,10 @@ def test_layout_is_a_bijection(bits, mode):
     assert np.all(qw == 0xFF)
 
 
-def test_layout3_planes_and_bijection():
-    """3-bit codes: every code owns three bits, two adjacent ones in the low
-    plane (bytes 0..15 of its lane's 24) and one in the high plane (bytes
-    16..23); no bit is shared and all bits are used."""
+def test_layout3_fields_and_bijection():
+    """3-bit codes: every code owns three consecutive bits of its lane's 24
+    bytes; the two members of a pair are adjacent (one 6-bit field, the lower
+    column first); no bit is shared and all bits are used."""
     N, K = 32, 256
     seen = np.zeros(N * K * 3, np.int32)
     for n in range(0, N, 3):
@@ -275,11 +275,16 @@ def test_layout3_planes_and_bijection():
             codes[n, k] = 7
             qw, _, _ = oracle.pack(codes, np.zeros((N, K // 64), np.uint16), None, "lut", 3, 64)
             on = np.nonzero(np.unpackbits(qw, bitorder="little"))[0]
-            assert len(on) == 3
-            lo, hi = on[:2], on[2]
-            assert lo[1] - lo[0] == 1 and lo[0] % 2 == 0
-            assert (lo[0] // 8) % 24 < 16 and (hi // 8) % 24 >= 16
+            assert len(on) == 3 and on[1] == on[0] + 1 and on[2] == on[0] + 2
+            # the lane's string: 192 bits starting at a multiple of 192
+            assert (on[0] // 192) == (on[2] // 192)
             seen[on] += 1
+            if k % 2 == 0:   # the pair's other member (column k + 1) follows
+                codes[n, k + 1] = 7
+                qw2, _, _ = oracle.pack(codes, np.zeros((N, K // 64), np.uint16), None, "lut",
+                                        3, 64)
+                on2 = np.nonzero(np.unpackbits(qw2, bitorder="little"))[0]
+                assert list(on2) == list(range(on[0], on[0] + 6))
     assert seen.max() == 1
     qw, _, _ = oracle.pack(np.full((N, K), 7, np.uint8), np.zeros((N, 4), np.uint16), None,
                            "lut", 3, 64)
@@ -289,16 +294,14 @@ def test_layout3_planes_and_bijection():
 def test_layout3_hand_position():
     """Code 5 (binary 101) at row 9, column 21, worked out from the layout's
     definition: g = 1, h = 1, tile j = 1, t = 1, c = 1 -> lane 5 (bytes
-    120..143 of chunk 0), pair p = 1, member 1.  Low bits: word 0, byte
-    2 (j % 2) + p / 2 = 2, field 2 (p % 2) + 1 = 3 -> byte 122 bits 6-7 = 01.
-    High bit: byte 16 + j % 4 = 17 of the lane -> byte 137, bit 2 p + 1 = 3."""
+    120..143 of chunk 0, bits 960..1151), pair p = 1, member 1: bit 960 + 24 j
+    + 6 p + 3 = 993 = byte 124 bit 1, so bits 1 and 3 of byte 124 are set."""
     N, K = 16, 128
     codes = np.zeros((N, K), np.uint8)
     codes[9, 21] = 5
     qw, _, _ = oracle.pack(codes, np.zeros((N, 2), np.uint16), None, "lut", 3, 64)
     expect = np.zeros(N * K * 3 // 8, np.uint8)
-    expect[122] = 0x40
-    expect[137] = 0x08
+    expect[124] = 0x0A
     assert np.array_equal(qw, expect)
 
 
