@@ -49,10 +49,9 @@
  *    2 (p % 2) + (c % 2).  Words are little-endian; field f holds bits
  *    [bits*f, bits*f + bits).
  *    3-bit LUT (the FLUTE summary's 2/3/4-bit tables): chunks of 128 columns
- *    and 768 bytes, lane l owning bytes [24 l, 24 l + 24); words 0..3 of the
- *    lane hold the codes' two low bits placed as the 2-bit layout places 2-bit
- *    codes, words 4 and 5 the high bits: tile j's eight in byte j % 4 of word
- *    4 + j / 4, pair p member c % 2 at bit 2 p + (c % 2).
+ *    and 768 bytes, lane l owning bytes [24 l, 24 l + 24), read as one 192-bit
+ *    little-endian string: tile j at bits [24 j, 24 j + 24), pair p at
+ *    [24 j + 6 p, + 6), member c % 2 at + 3 (c % 2) -- each pair one 6-bit field.
  *  - scales (and zeros): fp16, G = K/group groups (1 for group -1), stored as
  *    [N/16][G][16] with row r of a block at position 2 (r % 8) + r / 8, i.e.
  *    rows g and g + 8 side by side.

@@ -225,9 +225,10 @@ __global__ void __launch_bounds__(256) pack_codes_kernel(CodeCtx c, uint32_t* __
 // One thread per packed word: decode its codes to (q - z) * s (or T[q] * s),
 // exact in fp32 for integer zero-points, then round once to fp16 / bf16.
 // 3-bit codes: one thread per 32-bit word, six words per lane of a 768-byte
-// chunk (128 columns).  Words 0..3 take the codes' two low bits in the 2-bit
-// layout (word w: tiles 2w, 2w + 1); words 4, 5 take the high bits (word 4 + u:
-// tiles 4u .. 4u + 3, tile j in byte j % 4, pair p member c % 2 at bit 2p + c % 2).
+// chunk (128 columns).  The lane's six words are one 192-bit little-endian
+// string: tile j at bits [24 j, 24 j + 24), pair p at [24 j + 6 p, + 6), member
+// c % 2 at + 3 (c % 2).  Word w takes the bits [32 w, 32 w + 32) of it, i.e.
+// parts of tiles 4w/3 .. (32w + 31)/24.
 __global__ void __launch_bounds__(256) pack_codes3_kernel(CodeCtx c, uint32_t* __restrict__ out,
                                                           size_t nwords) {
   const size_t wid = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
@@ -241,11 +242,9 @@ __global__ void __launch_bounds__(256) pack_codes3_kernel(CodeCtx c, uint32_t* _
   float lut[16];
   for (int e = 0; e < 16; ++e)
     lut[e] = e < c.nlut ? __half2float(__ushort_as_half(c.lut[e])) : 0.0f;
-  const bool low = w6 < 4;
-  const int ntiles = low ? 2 : 4;
+  const int lo_bit = 32 * w6;
   uint32_t v = 0;
-  for (int sub = 0; sub < ntiles; ++sub) {
-    const int j = low ? 2 * w6 + sub : 4 * (w6 - 4) + sub;   // 16-column tile
+  for (int j = (32 * w6) / 24; j <= (32 * w6 + 31) / 24 && j < 8; ++j) {   // 16-column tile
     const int k0 = chunk * 128 + 16 * j + 4 * t;
     const int gi = k0 / c.L;
     for (int h = 0; h < 2; ++h) {
@@ -258,10 +257,11 @@ __global__ void __launch_bounds__(256) pack_codes3_kernel(CodeCtx c, uint32_t* _
       for (int cc = 0; cc < 4; ++cc) {
         const uint32_t q = (uint32_t)encode(wc[cc], s, 0.0f, c, lut);
         const int p = h + 2 * (cc >> 1), hi = cc & 1;
-        if (low)
-          v |= (q & 3u) << (8 * (2 * sub + (p >> 1)) + 2 * (2 * (p & 1) + hi));
-        else
-          v |= ((q >> 2) & 1u) << (8 * sub + 2 * p + hi);
+        const int b = 24 * j + 6 * p + 3 * hi;            // the code's lowest bit
+        for (int i = 0; i < 3; ++i) {
+          const int pos = b + i - lo_bit;
+          if (pos >= 0 && pos < 32) v |= ((q >> i) & 1u) << pos;
+        }
       }
     }
   }
@@ -283,8 +283,10 @@ __global__ void __launch_bounds__(256) dequant3_kernel(const uint32_t* __restric
   const int rb = (int)(blk / nchunks);
   const int g = lane >> 2, t = lane & 3;
   const uint32_t* w = qw + blk * 192 + (size_t)lane * 6;
+  uint32_t lw[7];   // the lane's 192-bit string, one word of zero padding
+  for (int i = 0; i < 6; ++i) lw[i] = w[i];
+  lw[6] = 0;
   for (int j = 0; j < 8; ++j) {
-    const uint32_t lo = w[j >> 1], hw = w[4 + (j >> 2)];
     const int k0 = chunk * 128 + 16 * j + 4 * t;
     const int gi = k0 / L;
     for (int h = 0; h < 2; ++h) {
@@ -294,8 +296,9 @@ __global__ void __launch_bounds__(256) dequant3_kernel(const uint32_t* __restric
       float r[4];
       for (int cc = 0; cc < 4; ++cc) {
         const int p = h + 2 * (cc >> 1), hi = cc & 1;
-        const uint32_t q = ((lo >> (8 * (2 * (j & 1) + (p >> 1)) + 2 * (2 * (p & 1) + hi))) & 3u) |
-                           (((hw >> (8 * (j & 3) + 2 * p + hi)) & 1u) << 2);
+        const int b = 24 * j + 6 * p + 3 * hi;             // the code's lowest bit
+        const uint64_t win = (uint64_t)lw[b >> 5] | ((uint64_t)lw[(b >> 5) + 1] << 32);
+        const uint32_t q = (uint32_t)(win >> (b & 31)) & 7u;
         r[cc] = __fmul_rn(__half2float(__ushort_as_half(lut[q])), s);
       }
       const size_t o = (size_t)n * K + k0;

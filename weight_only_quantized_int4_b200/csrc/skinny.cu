@@ -248,8 +248,8 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1) skinny_kernel(const
         lv[i] = 0;
       }
     }
-    //  3-bit: entry[6-bit index] = the pair (low bits of both members, then
-    //  their high bits), 64 entries.
+    //  3-bit: entry[6-bit field] = the pair (member 0 in bits 0..2, member 1
+    //  in bits 3..5), 64 entries.
     constexpr int VALS = BITS == 2 ? 4 : 2;              // values per entry
     constexpr int WORDS = (BF16 ? 2 : 1) * VALS / 2;     // 32-bit words per entry copy
     constexpr int COPIES = 32 / WORDS;
@@ -258,8 +258,8 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1) skinny_kernel(const
       const int e = i / COPIES;
       uint32_t v[4];
       if constexpr (BITS == 3) {
-        v[0] = (e & 3) | (((e >> 4) & 1) << 2);
-        v[1] = ((e >> 2) & 3) | (((e >> 5) & 1) << 2);
+        v[0] = e & 7;
+        v[1] = e >> 3;
       } else {
 #pragma unroll
         for (int k = 0; k < VALS; ++k) v[k] = BITS == 4 ? ((e >> (4 * k)) & 15) : ((e >> (2 * k)) & 3);
@@ -639,23 +639,21 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1) skinny_kernel(const
                 aflo[0] = e0.y; aflo[1] = e1.y; aflo[2] = e2.y; aflo[3] = e3.y;
               }
             } else if constexpr (BITS == 3) {
-              // 3-bit LUT: pair p's two low bits at 16 (j % 2) + 4 p of word j / 2,
-              // its two high bits at 8 (j % 4) + 2 p of word 4 + j / 4; together
-              // a 6-bit index into the 64-entry pair table (entries 128 bytes apart)
-              const uint32_t lo = cw3[r][j >> 1], hw = cw3[r][4 + (j >> 2)];
+              // 3-bit LUT: pair p of tile j is the 6-bit field at bit 24 j + 6 p
+              // of the lane's 192-bit string, an index into the 64-entry pair
+              // table (entries 128 bytes apart): one funnel shift brings it to
+              // bits 7..12
 #pragma unroll
               for (int p = 0; p < 4; ++p) {
-                const int sl = 16 * (j & 1) + 4 * p, sh = 8 * (j & 3) + 2 * p;
-                const uint32_t al = sl >= 7 ? lo >> (sl - 7) : lo << (7 - sl);     // bits 7..10
-                const uint32_t ah = sh >= 11 ? hw >> (sh - 11) : hw << (11 - sh);  // bits 11..12
+                const int b = 24 * j + 6 * p, wi = b >> 5, sb = b & 31;
+                const uint32_t lo = cw3[r][wi], hi = wi + 1 < 6 ? cw3[r][wi + 1] : 0u;
+                const uint32_t f = sb >= 7 ? __funnelshift_r(lo, hi, sb - 7) : lo << (7 - sb);
                 if constexpr (!BF16) {
                   const uint32_t l4 = (uint32_t)lane << 2;
-                  af[p] = *reinterpret_cast<const uint32_t*>(
-                      tabp + lop3_and_or(al, 0x780u, lop3_and_or(ah, 0x1800u, l4)));
+                  af[p] = *reinterpret_cast<const uint32_t*>(tabp + lop3_and_or(f, 0x1F80u, l4));
                 } else {
                   const uint32_t l8 = (uint32_t)(lane & 15) << 3;
-                  const uint2 e = *reinterpret_cast<const uint2*>(
-                      tabp + lop3_and_or(al, 0x780u, lop3_and_or(ah, 0x1800u, l8)));
+                  const uint2 e = *reinterpret_cast<const uint2*>(tabp + lop3_and_or(f, 0x1F80u, l8));
                   af[p] = e.x;
                   aflo[p] = e.y;
                 }
