@@ -2,7 +2,7 @@
  *
  *   y[M, N] = x[M, K] . dequant(Wq)[N, K]^T
  *
- * x and y are fp16 or bf16; Wq holds 4-bit (or 2-bit, LUT mode) codes, decoded
+ * x and y are fp16 or bf16; Wq holds 4-bit (or 2- or 3-bit, LUT mode) codes, decoded
  * on the fly inside the kernels as
  *   QMM_SYM   (q - 8) * s           symmetric, zero-point fixed at 8
  *   QMM_ASYM  (q - z) * s           fp16 zero-point per group
@@ -16,7 +16,7 @@
  *    the zero-point fixed at 8, column-wise or groupsize 128, fp16 scales; fp16
  *    zero-points as the asymmetric extension.
  *  - FLUTE project summary (sourcepulse.org), "How It Works": lookup-table
- *    quantization, value = table entry times a scale factor; 2- and 4-bit codes.
+ *    quantization, value = table entry times a scale factor; 2-, 3- and 4-bit codes.
  *  - GPTQ-Triton project summary (sourcepulse.org), "How It Works": the
  *    quantized weights are decoded on the fly right before the multiply.
  *  - exllama discussion 24 (quoting the GPTQ paper): activations stay in
