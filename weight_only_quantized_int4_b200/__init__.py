@@ -90,12 +90,22 @@ def strerror(status: int) -> str:
     return load().qmm_strerror(status).decode()
 
 
+# Pointer arguments go to ctypes as plain ints (every entry point declares its
+# argtypes, so ctypes converts them): no c_void_p object per argument.
 def _ptr(t):
-    return None if t is None else ctypes.c_void_p(t.data_ptr())
+    return None if t is None else t.data_ptr()
+
+
+# The current device's current stream as a raw cudaStream_t.  torch's raw
+# accessor skips building a torch.cuda.Stream object on every call; the public
+# route stays for builds that lack it.
+_raw_stream = getattr(torch._C, "_cuda_getCurrentRawStream", None)
 
 
 def _stream():
-    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    if _raw_stream is not None:
+        return _raw_stream(torch.cuda.current_device())
+    return torch.cuda.current_stream().cuda_stream
 
 
 def _check(status: int, what: str):
