@@ -231,6 +231,24 @@ def whole_job_gbs(world, bytes_per_step, steps, ms):
     return world * bytes_per_step * steps / (ms / 1e3) / 1e9
 
 
+def arena_of(tensors, align=256):
+    """One uint8 buffer holding copies of `tensors` at `align`-byte offsets, and
+    views of it with each tensor's dtype and shape: (buffer, [views])."""
+    import torch
+    offs, total = [], 0
+    for t in tensors:
+        offs.append(total)
+        total += -(-t.numel() * t.element_size() // align) * align
+    device = tensors[0].device if tensors else "cpu"
+    arena = torch.empty(total, dtype=torch.uint8, device=device)
+    views = []
+    for t, o in zip(tensors, offs):
+        v = arena[o:o + t.numel() * t.element_size()].view(t.dtype).view(t.shape)
+        v.copy_(t)
+        views.append(v)
+    return arena, views
+
+
 def run_ours(args, rank, world, local_rank):
     import torch
     import weight_only_quantized_int4_b200 as q
@@ -281,21 +299,14 @@ def run_ours(args, rank, world, local_rank):
                               bits=bits, group=group, perm=perm,
                               bytes=alg_bytes(mode, bits, group, M, K, N, gated, zopts,
                                               actorder)))
-        # the set's activations and its outputs live in one buffer each (views
-        # at 256-byte offsets), so the end-to-end leg moves a step's inputs and
-        # its results with one copy each way
-        for key in ("x", "y"):
-            offs, total = [], 0
-            for c in calls:
-                offs.append(total)
-                total += -(-c[key].numel() * c[key].element_size() // 256) * 256
-            arena = torch.empty(total, dtype=torch.uint8, device=dev)
-            for c, o in zip(calls, offs):
-                t = c[key]
-                v = arena[o:o + t.numel() * t.element_size()].view(t.dtype).view(t.shape)
-                v.copy_(t)
+        # the set's activations and its outputs live in one buffer each, so the
+        # end-to-end leg moves a step's inputs and its results with one copy
+        # each way
+        for key, arenas in (("x", xarenas), ("y", yarenas)):
+            arena, views = arena_of([c[key] for c in calls])
+            for c, v in zip(calls, views):
                 c[key] = v
-            (xarenas if key == "x" else yarenas).append(arena)
+            arenas.append(arena)
         sets.append(calls)
     torch.cuda.synchronize()
     calls = sets[0]

@@ -89,3 +89,26 @@ def test_workload_units_and_bytes():
         bench.alg_bytes("sym", 4, 128, 1, K, N) + 4 * K
     assert bench.alg_bytes("sym", 4, 128, 2, K, 2 * 64, gated=True) == \
         bench.alg_bytes("sym", 4, 128, 2, K, 2 * 64) - 2 * 64 * 2
+
+
+def test_arena_views_hold_the_tensors_at_aligned_offsets():
+    # the end-to-end leg copies one buffer each way: its views must be the
+    # tensors themselves (same values, dtype, shape, contiguous) at offsets the
+    # C ABI accepts, and the copied bytes are the buffer's size
+    import torch
+    g = torch.Generator().manual_seed(0)
+    ts = [torch.randn(1, 4096, generator=g).half(),
+          torch.randn(3, 40, generator=g).to(torch.bfloat16),   # 240 bytes: padded to 256
+          torch.randn(16, 11008, generator=g).half()]
+    arena, views = bench.arena_of(ts)
+    assert arena.dtype == torch.uint8
+    assert arena.numel() == 8192 + 256 + 16 * 11008 * 2
+    base = arena.data_ptr()
+    for t, v in zip(ts, views):
+        assert v.dtype == t.dtype and v.shape == t.shape and v.is_contiguous()
+        assert torch.equal(v, t)
+        assert (v.data_ptr() - base) % 256 == 0
+        assert v.untyped_storage().data_ptr() == arena.untyped_storage().data_ptr()
+    # writing through the arena is seen by the views (one copy moves them all)
+    arena.zero_()
+    assert all(int(v.abs().sum()) == 0 for v in views)
