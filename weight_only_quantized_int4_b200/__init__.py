@@ -198,7 +198,11 @@ def path(M, N, K, mode, bits=4, group=128):
 
 def qmm(x, qweight, scales, zeros_or_lut, N, K, mode, bits=4, group=128, y=None, ws=None,
         path="auto"):
-    """y[M, N] = x[M, K] . dequant(qweight)^T on x's device and current stream."""
+    """y[M, N] = x[M, K] . dequant(qweight)^T on the current device and stream.
+
+    ws: a workspace from workspace() (split-K over all SMs; reusable by later
+    calls on the same stream), or None: then every CTA owns whole row tiles,
+    which is slower when there are few row tiles (large N / K at small M)."""
     _dev(x, "x")
     if x.dtype not in DTYPES:
         raise ValueError("x must be fp16 or bf16")
