@@ -493,3 +493,26 @@ def test_gated_gate_and_up_roles():
     assert np.all(np.abs(y[0:16]) < 1e-300 * up + 1e-200)          # silu(-1024) ~ -1024 e^-1024
     assert np.allclose(y[16:32], 7.0 * K * up, rtol=1e-12)         # silu(896) = 896 (to 1e-300)
     assert np.all(y[32:48] == 0.0)
+
+
+def test_gated_silu_at_moderate_sums():
+    """Gate sums of moderate size, exact in the codes: the output must be
+    silu(v) u with silu in its tanh form, v/2 (1 + tanh(v/2)).  The two
+    tests above hold for any v sigma(c v) (the odd-even identity and the
+    limits do not see the constant c); this one pins c = 1."""
+    import math
+    I, K, g = 80, 128, 128
+    x = oracle.round_to(np.ones((1, K)), "f16")
+    s = 1.0 / 16.0                                   # fp16 0x2C00, exact
+    codes = np.full((2 * I, K), 8, np.uint8)
+    vs = [-3.0, -1.0, 0.5, 1.0, 2.5]                 # gate sums: 16 v codes one step off 8
+    for b, v in enumerate(vs):
+        n_off = int(round(abs(v) / s))
+        codes[32 * b: 32 * b + 16, :n_off] = 9 if v > 0 else 7
+        codes[32 * b + 16: 32 * b + 32, :16] = 9     # up sum 16 s = 1
+    scales = np.full((2 * I, 1), 0x2C00, np.uint16)
+    qw, sp, _ = oracle.pack(codes, scales, None, "sym", 4, g)
+    y = oracle.qmm_gated(x, "f16", qw, sp, None, 1, I, K, "sym", 4, g)[0]
+    for b, v in enumerate(vs):
+        want = 0.5 * v * (1.0 + math.tanh(0.5 * v))
+        assert np.allclose(y[16 * b: 16 * b + 16], want, rtol=1e-12, atol=0), (v, y[16 * b], want)
