@@ -112,3 +112,23 @@ def test_arena_views_hold_the_tensors_at_aligned_offsets():
     # writing through the arena is seen by the views (one copy moves them all)
     arena.zero_()
     assert all(int(v.abs().sum()) == 0 for v in views)
+
+
+@pytest.mark.parametrize("mode,bits,group,K,N,mb", [
+    ("sym", 4, 128, 4096, 4096, 8.65), ("sym", 4, 128, 4096, 12288, 25.95),
+    ("sym", 4, 128, 4096, 22016, 46.50), ("sym", 4, 128, 11008, 4096, 23.25),
+    ("asym", 4, 128, 8192, 10240, 44.56), ("asym", 4, 128, 8192, 57344, 249.56),
+    ("asym", 4, 128, 28672, 8192, 124.78), ("lut", 4, 64, 4096, 14336, 31.20),
+    ("lut", 2, 64, 4096, 14336, 16.52), ("sym", 4, -1, 4096, 11008, 22.57),
+    ("sym", 4, 128, 4096, 11008, 23.25)])
+def test_weight_bytes_match_the_stated_figures(mode, bits, group, K, N, mb):
+    """Codes + scales (+ zeros) of each benchmark shape against the figures
+    worked out from the format: b/8 bytes per weight plus 2 bytes per group
+    (4 with ASYM zeros), i.e. 0.516 B/weight for SYM4 g128, 0.531 for ASYM4
+    g128 and LUT4 g64, 0.281 for LUT2 g64.  M = 0 leaves out x and y."""
+    got = bench.alg_bytes(mode, bits, group, 0, K, N)
+    assert round(got / 1e6, 2) == mb
+    per_weight = {("sym", 4, 128): 0.515625, ("asym", 4, 128): 0.53125,
+                  ("lut", 4, 64): 0.53125, ("lut", 2, 64): 0.28125}.get((mode, bits, group))
+    if per_weight is not None:
+        assert got == N * K * per_weight
