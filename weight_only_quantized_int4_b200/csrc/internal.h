@@ -27,6 +27,7 @@ struct Problem {
 struct SkinnyPlan {
   int nt;          // token tiles of 8 per slab (1 or 2)
   int cta_tiles;   // 1: one CTA per row tile, warps split K, no workspace
+  int deep;        // 1: one CTA per SM with a deep ring (cta_tiles and tiles <= SMs)
   int rows;        // rows per CTA tile (16 * row blocks)
   int tiles_n;     // CTA tiles along N
   int slabs;       // token slabs (ceil(M / (8 nt)))

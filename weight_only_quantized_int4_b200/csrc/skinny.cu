@@ -101,9 +101,16 @@ struct Stage {
 
 // Ring depth per warp (stages in flight = depth - 1): 3 for one token tile
 // where the 8 warps' rings still fit two CTAs per SM (228 KB, 1 KB reserved
-// per CTA), else 2.
-template <int BITS, int MODE, int NT, int TPG>
+// per CTA), else 2.  DEEP kernels run one CTA per SM (problems with at most
+// one row tile per SM): as deep a ring as fits 227 KB, at most 6, so that a
+// warp's whole share of a small matrix is requested at once.
+template <int BITS, int MODE, int NT, int TPG, bool DEEP = false>
 constexpr int ring_stages() {
+  if constexpr (DEEP) {
+    constexpr int tab = MODE == kLUT ? 256 * 32 * 4 : 0;
+    constexpr int s = (227 * 1024 - tab) / (kWarps * Stage<BITS, MODE, NT, TPG>::BYTES);
+    return s > 6 ? 6 : s;
+  }
   if (NT != 1) return 2;
   if (MODE == kSYM || MODE == kASYM) return 3;
   if ((MODE == kASYMQ || MODE == kASYMQ1) &&
@@ -176,10 +183,10 @@ __device__ __forceinline__ void mma_16816_first(float (&d)[4], const uint32_t (&
   }
 }
 
-template <int BITS, int MODE, bool BF16, int NT, int TPG>
-__global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1) skinny_kernel(const SkinnyArgs a) {
+template <int BITS, int MODE, bool BF16, int NT, int TPG, bool DEEP>
+__global__ void __launch_bounds__(kThreads, DEEP ? 1 : 2) skinny_kernel(const SkinnyArgs a) {
   using St = Stage<BITS, MODE, NT, TPG>;
-  constexpr int S = ring_stages<BITS, MODE, NT, TPG>();
+  constexpr int S = ring_stages<BITS, MODE, NT, TPG, DEEP>();
   constexpr int R = St::R;
   constexpr int TOK = St::TOK;
   constexpr int CPS = St::CPS;
@@ -744,10 +751,11 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1) skinny_kernel(const
       } else {
 #pragma unroll
         for (int i = 0; i < NACC; ++i) outv[i] = 0.0f;
-        for (int k0 = 0; k0 < nb; k0 += 4) {
-          float4 v[4][NACC / 4];
+        constexpr int KB = NT == 1 ? 4 : 2;   // contributors loaded at a time
+        for (int k0 = 0; k0 < nb; k0 += KB) {
+          float4 v[KB][NACC / 4];
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
+          for (int kk = 0; kk < KB; ++kk) {
             const int k = k0 + kk;
             if (k < nb) {
               const float4* src = reinterpret_cast<const float4*>(
@@ -757,7 +765,7 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1) skinny_kernel(const
             }
           }
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
+          for (int kk = 0; kk < KB; ++kk) {
             if (k0 + kk < nb) {
 #pragma unroll
               for (int i = 0; i < NACC / 4; ++i) {
@@ -809,24 +817,24 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 2 : 1) skinny_kernel(const
   }
 }
 
-template <int BITS, int MODE, int NT, int TPG>
+template <int BITS, int MODE, int NT, int TPG, bool DEEP>
 constexpr size_t smem_bytes() {
   using St = Stage<BITS, MODE, NT, TPG>;
-  constexpr int S = ring_stages<BITS, MODE, NT, TPG>();
+  constexpr int S = ring_stages<BITS, MODE, NT, TPG, DEEP>();
   return kTabBytes<MODE> + (size_t)kWarps * S * St::BYTES;
 }
 
 // Opts the kernel into `smem` bytes of dynamic shared memory (once per device)
 // and returns its resident CTAs per SM, or 0 if the size cannot be granted.
-template <int BITS, int MODE, bool BF16, int NT, int TPG>
+template <int BITS, int MODE, bool BF16, int NT, int TPG, bool DEEP>
 int occupancy() {
   static int occ[kMaxDevices] = {};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 0 || dev >= kMaxDevices) dev = 0;
   if (occ[dev]) return occ[dev];
-  auto k = skinny_kernel<BITS, MODE, BF16, NT, TPG>;
-  constexpr size_t smem = smem_bytes<BITS, MODE, NT, TPG>();
+  auto k = skinny_kernel<BITS, MODE, BF16, NT, TPG, DEEP>;
+  constexpr size_t smem = smem_bytes<BITS, MODE, NT, TPG, DEEP>();
   if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
       cudaSuccess) {
     cudaGetLastError();   // do not leave the failure behind as a sticky error
@@ -841,14 +849,14 @@ int occupancy() {
   return o;
 }
 
-template <int BITS, int MODE, bool BF16, int NT, int TPG>
+template <int BITS, int MODE, bool BF16, int NT, int TPG, bool DEEP>
 cudaError_t launch(const SkinnyArgs& args, int slabs, cudaStream_t stream) {
-  auto k = skinny_kernel<BITS, MODE, BF16, NT, TPG>;
-  if (occupancy<BITS, MODE, BF16, NT, TPG>() < 1) return cudaErrorInvalidConfiguration;
+  auto k = skinny_kernel<BITS, MODE, BF16, NT, TPG, DEEP>;
+  if (occupancy<BITS, MODE, BF16, NT, TPG, DEEP>() < 1) return cudaErrorInvalidConfiguration;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(args.ctas, slabs, 1);
   cfg.blockDim = dim3(kThreads, 1, 1);
-  cfg.dynamicSmemBytes = smem_bytes<BITS, MODE, NT, TPG>();
+  cfg.dynamicSmemBytes = smem_bytes<BITS, MODE, NT, TPG, DEEP>();
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -859,21 +867,30 @@ cudaError_t launch(const SkinnyArgs& args, int slabs, cudaStream_t stream) {
   if (e != cudaSuccess) cudaGetLastError();   // report it once, here
   return e;
 }
-// Calls f.template operator()<BITS, MODE, BF16, NT, TPG>() for the runtime values.
+// Calls f.template operator()<BITS, MODE, BF16, NT, TPG, DEEP>() for the
+// runtime values (the deep ring only for the plain SYM / ASYM / LUT formats).
+template <int B, int MO, bool BF, int T, int TP, class F>
+auto dispatch_deep(bool deep, F&& f) {
+  if constexpr (!zero_opts(MO)) {
+    if (deep) return f.template operator()<B, MO, BF, T, TP, true>();
+  }
+  return f.template operator()<B, MO, BF, T, TP, false>();
+}
+
 template <int B, int MO, bool BF, int T, class F>
-auto dispatch_tpg(int tpg, F&& f) {
+auto dispatch_tpg(int tpg, bool deep, F&& f) {
   switch (tpg) {
-    case 1: return f.template operator()<B, MO, BF, T, 1>();
-    case 2: return f.template operator()<B, MO, BF, T, 2>();
-    case 4: return f.template operator()<B, MO, BF, T, 4>();
-    default: return f.template operator()<B, MO, BF, T, 8>();
+    case 1: return dispatch_deep<B, MO, BF, T, 1>(deep, f);
+    case 2: return dispatch_deep<B, MO, BF, T, 2>(deep, f);
+    case 4: return dispatch_deep<B, MO, BF, T, 4>(deep, f);
+    default: return dispatch_deep<B, MO, BF, T, 8>(deep, f);
   }
 }
 
 template <class F>
-auto dispatch(int bits, int mode, bool bf16, int nt, int tpg, F&& f) {
+auto dispatch(int bits, int mode, bool bf16, int nt, int tpg, bool deep, F&& f) {
 #define QMM_CASE(B, MO, BF, T) \
-  if (bits == B && mode == MO && bf16 == BF && nt == T) return dispatch_tpg<B, MO, BF, T>(tpg, f);
+  if (bits == B && mode == MO && bf16 == BF && nt == T) return dispatch_tpg<B, MO, BF, T>(tpg, deep, f);
   QMM_CASE(4, kSYM, false, 1) QMM_CASE(4, kSYM, false, 2) QMM_CASE(4, kSYM, true, 1)
   QMM_CASE(4, kSYM, true, 2) QMM_CASE(4, kASYM, false, 1) QMM_CASE(4, kASYM, false, 2)
   QMM_CASE(4, kASYM, true, 1) QMM_CASE(4, kASYM, true, 2) QMM_CASE(4, kLUT, false, 1)
@@ -886,7 +903,7 @@ auto dispatch(int bits, int mode, bool bf16, int nt, int tpg, F&& f) {
   QMM_CASE(4, kASYMQ, true, 1) QMM_CASE(4, kASYMQ, true, 2) QMM_CASE(4, kASYMQ1, false, 1)
   QMM_CASE(4, kASYMQ1, false, 2) QMM_CASE(4, kASYMQ1, true, 1) QMM_CASE(4, kASYMQ1, true, 2)
 #undef QMM_CASE
-  return dispatch_tpg<4, kSYM, false, 1>(tpg, f);
+  return dispatch_tpg<4, kSYM, false, 1>(tpg, deep, f);
 }
 
 // Tiles (of 16 columns) per group inside a 128-column stage: 8 for groups of
@@ -907,12 +924,10 @@ SkinnyPlan plan_skinny(int M, int N, int K, int bits, int group, int mode, bool 
   const int nsc = (K + kSC - 1) / kSC;
   const long long units = (long long)p.tiles_n * nsc;
   const int tpg = tiles_per_group(group);
-  p.smem = dispatch(bits, mode, bf16, p.nt, tpg, [&]<int B, int MO, bool BF, int T, int TP>() {
-    return smem_bytes<B, MO, T, TP>();
-  });
-  const int occ = dispatch(bits, mode, bf16, p.nt, tpg, [&]<int B, int MO, bool BF, int T, int TP>() {
-    return occupancy<B, MO, BF, T, TP>();
-  });
+  p.smem = dispatch(bits, mode, bf16, p.nt, tpg, false,
+                    [&]<int B, int MO, bool BF, int T, int TP, bool D>() { return smem_bytes<B, MO, T, TP, D>(); });
+  const int occ = dispatch(bits, mode, bf16, p.nt, tpg, false,
+                           [&]<int B, int MO, bool BF, int T, int TP, bool D>() { return occupancy<B, MO, BF, T, TP, D>(); });
   // one resident wave of CTAs; every warp is a stream-K worker with >= 1 unit
   long long warps = (long long)sms * (occ > 0 ? occ : 1) * kWarps;
   const long long cap = std::max<long long>(1, units * 8 / nsc);
@@ -923,6 +938,13 @@ SkinnyPlan plan_skinny(int M, int N, int K, int bits, int group, int mode, bool 
     p.splits = p.tiles_n;
     p.warps = p.tiles_n * kWarps;
     p.ws_bytes = 0;
+    // at most one tile per SM: each CTA has an SM to itself, so it takes the
+    // deep ring (its warps' stages all requested up front on small matrices)
+    if (p.tiles_n <= sms && !zero_opts(mode)) {
+      p.deep = 1;
+      p.smem = dispatch(bits, mode, bf16, p.nt, tpg, true,
+                        [&]<int B, int MO, bool BF, int T, int TP, bool D>() { return smem_bytes<B, MO, T, TP, D>(); });
+    }
     return p;
   }
   if (warps > cap) warps = cap;
@@ -978,10 +1000,10 @@ cudaError_t launch_skinny(const Problem& pr, const SkinnyPlan& plan, void* works
     a.counters = reinterpret_cast<unsigned*>(workspace);
     a.slots = reinterpret_cast<float*>(reinterpret_cast<char*>(workspace) + counters);
   }
-  return dispatch(pr.bits, pr.mode, pr.bf16, plan.nt, tiles_per_group(pr.group),
-                  [&]<int B, int MO, bool BF, int T, int TP>() {
+  return dispatch(pr.bits, pr.mode, pr.bf16, plan.nt, tiles_per_group(pr.group), plan.deep != 0,
+                  [&]<int B, int MO, bool BF, int T, int TP, bool D>() {
                     a.stage_bytes = Stage<B, MO, T, TP>::BYTES;
-                    return launch<B, MO, BF, T, TP>(a, plan.slabs, stream);
+                    return launch<B, MO, BF, T, TP, D>(a, plan.slabs, stream);
                   });
 }
 
