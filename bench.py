@@ -49,11 +49,14 @@ WORKLOADS = {
     "prefill_m256": ("sym", 4, 128, "f16", [(4096, 11008)], [256]),
     "prefill_m1024": ("sym", 4, 128, "f16", [(4096, 11008)], [1024]),
     "prefill_m4096": ("sym", 4, 128, "f16", [(4096, 11008)], [4096]),
+    "prefill_m64_rowscale": ("sym", 4, -1, "f16", [(4096, 11008)], [64]),
+    "prefill_m256_rowscale": ("sym", 4, -1, "f16", [(4096, 11008)], [256]),
+    "prefill_m1024_rowscale": ("sym", 4, -1, "f16", [(4096, 11008)], [1024]),
     "prefill_m4096_rowscale": ("sym", 4, -1, "f16", [(4096, 11008)], [4096]),
     "llama70b_asym_bf16": ("asym", 4, 128, "bf16",
-                           [(8192, 10240), (8192, 57344), (28672, 8192)], [1, 16]),
-    "lut4_nf4": ("lut", 4, 64, "f16", [(4096, 14336)], [1, 8]),
-    "lut2": ("lut", 2, 64, "f16", [(4096, 14336)], [1, 8]),
+                           [(8192, 10240), (8192, 57344), (28672, 8192)], [1, 16, 64]),
+    "lut4_nf4": ("lut", 4, 64, "f16", [(4096, 14336)], [1, 8, 32]),
+    "lut2": ("lut", 2, 64, "f16", [(4096, 14336)], [1, 8, 32]),
     "lut3_nf3": ("lut", 3, 64, "f16", [(4096, 14336)], [1, 8]),
     # LLaMA-7B feed-forward gate fused into the matmul: gate and up (I = 11008
     # each, N = 2 I rows packed together), y[M, I] = silu(gate) * up
@@ -71,6 +74,16 @@ WORKLOADS = {
                          [1, 2, 4, 8, 16]),
 }
 GATED = {"ffn_gated"}
+# The five benchmark configurations and the workloads that time them (the
+# default run reports every one of them beside its headline, config 2).
+CONFIG_WORKLOADS = {
+    "1_4096sq_m1": ["decode_4096sq"],
+    "3_llama70b_asym_bf16": ["llama70b_asym_bf16"],
+    "4_lut_k4096_n14336": ["lut4_nf4", "lut2"],
+    "5_prefill_k4096_n11008": ["prefill_m64", "prefill_m256", "prefill_m1024", "prefill_m4096",
+                               "prefill_m64_rowscale", "prefill_m256_rowscale",
+                               "prefill_m1024_rowscale", "prefill_m4096_rowscale"],
+}
 # workload -> zero-point options (zero group, zero bits)
 ZOPTS = {"asym_rowscale_zg8_u4": (8, 4), "llama70b_asym_zq4_bf16": (128, 4)}
 ACTORDER = {"actorder_llama7b"}
@@ -249,6 +262,196 @@ def arena_of(tensors, align=256):
     return arena, views
 
 
+class Workload:
+    """Every call of one step of a workload on the device: packed weights in
+    as many copies as it takes to pass twice the L2 size (rotated step by
+    step), activations and outputs (each set in one buffer, so the end-to-end
+    leg moves a step's inputs and results with one copy each way), workspaces,
+    and one CUDA graph per weight copy; a step is one graph replay.
+
+    Inputs come from the seed-0 counter generator of `synth` (drawn on the
+    device): call c's weights are stream "W{c}.{copy}", its activations "x{c}".
+    """
+
+    def __init__(self, name, dev):
+        import torch
+        import weight_only_quantized_int4_b200 as q
+        from weight_only_quantized_int4_b200 import synth
+
+        self.name, self.dev = name, dev
+        probs = problems(name)
+        self.gated = name in GATED
+        self.zopts = ZOPTS.get(name)
+        self.actorder = name in ACTORDER
+        self.codes_per_copy = sum(N * K * bits // 8 for (_, bits, _, _, _, K, N) in probs)
+        self.copies = max(1, -(-2 * L2_BYTES // self.codes_per_copy))
+        gen = torch.Generator(device=dev).manual_seed(0)
+        self.sets, self.xarenas, self.yarenas = [], [], []
+        for cp in range(self.copies):
+            calls = []
+            for ci, (mode, bits, group, xdt, M, K, N) in enumerate(probs):
+                W = synth.weights_torch(0, f"W{ci}.{cp}", N, K, SIGMA[mode], device=dev)
+                lut = None
+                if mode == "lut":
+                    t = {4: synth.nf4_table, 3: synth.nf3_table, 2: lambda: synth.lut2_table(0)}[bits]()
+                    lut = torch.from_numpy(t.view(np.int16)).to(dev)
+                perm = None
+                if self.gated:
+                    qw, sc, ze = q.pack_gated(W[: N // 2], W[N // 2:], mode, bits, group, lut=lut)
+                elif self.zopts is not None:
+                    qw, sc, ze = q.pack_asym(W, group, self.zopts[0], self.zopts[1])
+                elif self.actorder:
+                    perm = torch.randperm(K, generator=gen, device=dev).to(torch.int32)
+                    qw, sc, ze = q.pack_actorder(W, perm, mode, bits, group, lut=lut)
+                else:
+                    qw, sc, ze = q.pack(W, mode, bits, group, lut=lut)
+                del W
+                x = synth.activations_torch(0, f"x{ci}", M, K, xdt, device=dev)
+                tdt = x.dtype
+                y = torch.empty(M, N // 2 if self.gated else N, dtype=tdt, device=dev)
+                if self.zopts is not None:
+                    ws = q.workspace_asym(M, N, K, group, self.zopts[0], self.zopts[1], device=dev)
+                elif self.actorder:
+                    ws = q.workspace_actorder(M, N, K, mode, bits, group, device=dev)
+                else:
+                    ws = q.workspace(M, N, K, mode, bits, group, device=dev)
+                zl = ze if mode == "asym" else lut
+                calls.append(dict(x=x, qw=qw, sc=sc, zl=zl, y=y, ws=ws, M=M, N=N, K=K, mode=mode,
+                                  bits=bits, group=group, perm=perm,
+                                  bytes=alg_bytes(mode, bits, group, M, K, N, self.gated,
+                                                  self.zopts, self.actorder)))
+            for key, arenas in (("x", self.xarenas), ("y", self.yarenas)):
+                arena, views = arena_of([c[key] for c in calls])
+                for c, v in zip(calls, views):
+                    c[key] = v
+                arenas.append(arena)
+            self.sets.append(calls)
+        torch.cuda.synchronize()
+        calls = self.sets[0]
+        self.n_calls = len(calls)
+        self.step_bytes = sum(c["bytes"] for c in calls)
+        self.step_flops = sum(alg_flops(c["M"], c["K"], c["N"]) for c in calls)
+        self.dtype = WORKLOADS[name][3]
+        # warm-up outside the graphs (first calls set kernel attributes), then
+        # one graph per weight copy
+        for i in range(self.copies):
+            self.step(i)
+        torch.cuda.synchronize()
+        self.stream = torch.cuda.Stream(device=dev)
+        self.graphs = []
+        with torch.cuda.stream(self.stream):
+            self.step()
+            torch.cuda.synchronize()
+            for i in range(self.copies):
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g, stream=self.stream):
+                    self.step(i)
+                self.graphs.append(g)
+        torch.cuda.synchronize()
+
+    def step(self, i=0):
+        """The step's calls through the Python API (weight copy i % copies)."""
+        import weight_only_quantized_int4_b200 as q
+        z = self.zopts
+        for c in self.sets[i % self.copies]:
+            if self.gated:
+                q.qmm_gated(c["x"], c["qw"], c["sc"], c["zl"], c["N"] // 2, c["K"], c["mode"],
+                            c["bits"], c["group"], y=c["y"], ws=c["ws"])
+            elif z is not None:
+                q.qmm_asym(c["x"], c["qw"], c["sc"], c["zl"], c["N"], c["K"], c["group"], z[0],
+                           z[1], y=c["y"], ws=c["ws"])
+            elif self.actorder:
+                q.qmm_actorder(c["x"], c["perm"], c["qw"], c["sc"], c["zl"], c["N"], c["K"],
+                               c["mode"], c["bits"], c["group"], y=c["y"], ws=c["ws"])
+            else:
+                q.qmm(c["x"], c["qw"], c["sc"], c["zl"], c["N"], c["K"], c["mode"], c["bits"],
+                      c["group"], y=c["y"], ws=c["ws"])
+
+    def time_steps(self, steps, warmup, barrier=lambda: None):
+        """Device time (ms) of `steps` graph replays after `warmup` ones, CUDA
+        events on the replay stream, synchronized and barriered on both sides."""
+        import torch
+        with torch.cuda.stream(self.stream):
+            for i in range(warmup):
+                self.graphs[i % self.copies].replay()
+            torch.cuda.synchronize()
+            barrier()
+            torch.cuda.synchronize()
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(self.stream)
+            for i in range(steps):
+                self.graphs[i % self.copies].replay()
+            e1.record(self.stream)
+            torch.cuda.synchronize()
+            barrier()
+            torch.cuda.synchronize()
+        return e0.elapsed_time(e1)
+
+    def busy(self, seconds):
+        """Replays for about `seconds` (so that clock samples see the GPU under load)."""
+        import torch
+        t_end = time.time() + seconds
+        with torch.cuda.stream(self.stream):
+            while time.time() < t_end:
+                for i in range(50):
+                    self.graphs[i % self.copies].replay()
+                torch.cuda.synchronize()
+
+    def l2_note(self):
+        return (f"inputs larger than L2: {self.copies} weight cop"
+                f"{'y' if self.copies == 1 else 'ies'} of the step rotated, "
+                f"{self.copies * self.codes_per_copy / 1e6:.0f} MB of codes in all "
+                f"(L2 {L2_BYTES / 1e6:.0f} MB)")
+
+    def result(self, ms_per_step, world=1):
+        """(value, unit, roofline) of a measured step time."""
+        if tensor_bound(self.name):
+            peak, kind = tensor_peak()
+            achieved = self.step_flops / (ms_per_step / 1e3) / 1e12
+            roof = {"bound": "tensor", "achieved": round(achieved, 1), "peak": peak,
+                    "unit": "TFLOP/s", "frac": round(achieved / peak, 4), "peak_source": kind}
+            return world * achieved, "TFLOP/s", roof
+        peak, kind = peaks()
+        achieved = self.step_bytes / (ms_per_step / 1e3) / 1e9
+        roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                "frac": round(achieved / peak, 4), "peak_source": kind}
+        return world * achieved, "GB/s", roof
+
+    def release(self):
+        del self.graphs, self.sets, self.xarenas, self.yarenas
+
+
+def steps_for(wl, seconds, lo=20, hi=5000):
+    """Timed steps worth about `seconds` of device time (from a short probe)."""
+    ms = wl.time_steps(5, 2)
+    return int(min(hi, max(lo, seconds * 1e3 / max(ms / 5, 1e-3))))
+
+
+def measure_configs(dev):
+    """Every benchmark configuration with the headline's protocol (graphs of
+    the step's calls, weights past L2, CUDA events), each with its roofline
+    fraction: value, unit, ms per step and calls per step."""
+    import torch
+    out = {}
+    for cfg, names in CONFIG_WORKLOADS.items():
+        recs = []
+        for name in names:
+            wl = Workload(name, dev)
+            steps = steps_for(wl, 0.3)
+            ms = wl.time_steps(steps, 5) / steps
+            value, unit, roof = wl.result(ms)
+            recs.append({"workload": name, "value": round(value, 1), "unit": unit,
+                         "frac": roof["frac"], "bound": roof["bound"],
+                         "ms_per_step": round(ms, 5), "calls_per_step": wl.n_calls,
+                         "steps": steps, "dtype": wl.dtype})
+            wl.release()
+            del wl
+            torch.cuda.empty_cache()
+        out[cfg] = recs
+    return out
+
+
 def run_ours(args, rank, world, local_rank):
     import torch
     import weight_only_quantized_int4_b200 as q
@@ -256,95 +459,8 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.set_device(local_rank)
     q.load()
     dev = torch.device("cuda", local_rank)
-    probs = problems(args.workload)
-    gated = args.workload in GATED
-    zopts = ZOPTS.get(args.workload)
-    actorder = args.workload in ACTORDER
-    gen = torch.Generator(device=dev).manual_seed(1234 + rank)
-    # enough weight copies that the codes of consecutive steps never fit in L2
-    codes_per_copy = sum(N * K * bits // 8 for (_, bits, _, _, _, K, N) in probs)
-    copies = max(1, -(-2 * L2_BYTES // codes_per_copy))
-    sets, xarenas, yarenas = [], [], []
-    for _ in range(copies):
-        calls = []
-        for (mode, bits, group, xdt, M, K, N) in probs:
-            W = torch.randn(N, K, generator=gen, device=dev) * SIGMA[mode]
-            lut = None
-            if mode == "lut":
-                from weight_only_quantized_int4_b200 import synth
-                t = {4: synth.nf4_table, 3: synth.nf3_table, 2: lambda: synth.lut2_table(0)}[bits]()
-                lut = torch.from_numpy(t.view(np.int16)).to(dev)
-            perm = None
-            if gated:
-                qw, sc, ze = q.pack_gated(W[: N // 2], W[N // 2:], mode, bits, group, lut=lut)
-            elif zopts is not None:
-                qw, sc, ze = q.pack_asym(W, group, zopts[0], zopts[1])
-            elif actorder:
-                perm = torch.randperm(K, generator=gen, device=dev).to(torch.int32)
-                qw, sc, ze = q.pack_actorder(W, perm, mode, bits, group, lut=lut)
-            else:
-                qw, sc, ze = q.pack(W, mode, bits, group, lut=lut)
-            del W
-            tdt = torch.float16 if xdt == "f16" else torch.bfloat16
-            x = torch.randn(M, K, generator=gen, device=dev).to(tdt)
-            y = torch.empty(M, N // 2 if gated else N, dtype=tdt, device=dev)
-            if zopts is not None:
-                ws = q.workspace_asym(M, N, K, group, zopts[0], zopts[1], device=dev)
-            elif actorder:
-                ws = q.workspace_actorder(M, N, K, mode, bits, group, device=dev)
-            else:
-                ws = q.workspace(M, N, K, mode, bits, group, device=dev)
-            zl = ze if mode == "asym" else lut
-            calls.append(dict(x=x, qw=qw, sc=sc, zl=zl, y=y, ws=ws, M=M, N=N, K=K, mode=mode,
-                              bits=bits, group=group, perm=perm,
-                              bytes=alg_bytes(mode, bits, group, M, K, N, gated, zopts,
-                                              actorder)))
-        # the set's activations and its outputs live in one buffer each, so the
-        # end-to-end leg moves a step's inputs and its results with one copy
-        # each way
-        for key, arenas in (("x", xarenas), ("y", yarenas)):
-            arena, views = arena_of([c[key] for c in calls])
-            for c, v in zip(calls, views):
-                c[key] = v
-            arenas.append(arena)
-        sets.append(calls)
-    torch.cuda.synchronize()
-    calls = sets[0]
-    step_bytes = sum(c["bytes"] for c in calls)
-    step_flops = sum(alg_flops(c["M"], c["K"], c["N"]) for c in calls)
-    tensor = tensor_bound(args.workload)
-
-    def step(i=0):
-        for c in sets[i % copies]:
-            if gated:
-                q.qmm_gated(c["x"], c["qw"], c["sc"], c["zl"], c["N"] // 2, c["K"], c["mode"],
-                            c["bits"], c["group"], y=c["y"], ws=c["ws"])
-            elif zopts is not None:
-                q.qmm_asym(c["x"], c["qw"], c["sc"], c["zl"], c["N"], c["K"], c["group"],
-                           zopts[0], zopts[1], y=c["y"], ws=c["ws"])
-            elif actorder:
-                q.qmm_actorder(c["x"], c["perm"], c["qw"], c["sc"], c["zl"], c["N"], c["K"],
-                               c["mode"], c["bits"], c["group"], y=c["y"], ws=c["ws"])
-            else:
-                q.qmm(c["x"], c["qw"], c["sc"], c["zl"], c["N"], c["K"], c["mode"], c["bits"],
-                      c["group"], y=c["y"], ws=c["ws"])
-
-    # warm-up outside the graphs (first calls set kernel attributes), then one
-    # graph per weight copy; step i replays graph i % copies
-    for i in range(copies):
-        step(i)
-    torch.cuda.synchronize()
-    stream = torch.cuda.Stream(device=dev)
-    graphs = []
-    with torch.cuda.stream(stream):
-        step()
-        torch.cuda.synchronize()
-        for i in range(copies):
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g, stream=stream):
-                step(i)
-            graphs.append(g)
-    torch.cuda.synchronize()
+    wl = Workload(args.workload, dev)
+    actorder = wl.actorder
 
     dist = None
     if world > 1:
@@ -356,109 +472,87 @@ def run_ours(args, rank, world, local_rank):
 
     clock = ClockSampler(local_rank)
     clock.start()
-    with torch.cuda.stream(stream):
-        for i in range(args.warmup):
-            graphs[i % copies].replay()
-        # keep the GPU busy ~0.3 s so the clock samples see it under load
-        t_end = time.time() + 0.3
-        while time.time() < t_end:
-            for i in range(50):
-                graphs[i % copies].replay()
-            torch.cuda.synchronize()
-        torch.cuda.synchronize()
-        barrier()
-        torch.cuda.synchronize()
-        e0 = torch.cuda.Event(enable_timing=True)
-        e1 = torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for i in range(args.steps):
-            graphs[i % copies].replay()
-        e1.record(stream)
-        torch.cuda.synchronize()
-        barrier()
-        torch.cuda.synchronize()
+    wl.busy(0.3)
+    ms = max_over_ranks(wl.time_steps(args.steps, args.warmup, barrier), dist, dev)
     clocks = clock.stop()
-    ms = max_over_ranks(e0.elapsed_time(e1), dist, dev)
     ms_per_step = ms / args.steps
-    value = whole_job_gbs(world, step_bytes, args.steps, ms)
+    value, unit, roofline = wl.result(ms_per_step, world)
 
     # ---- end to end through the public API: pinned host x in, y out, per step
-    hx = xarenas[0].cpu().pin_memory()
-    hy = torch.empty_like(yarenas[0], device="cpu").pin_memory()
-    h2d = hx.numel()
-    d2h = hy.numel()
+    # (the calls are issued from Python one by one, not replayed from a graph)
+    hx = wl.xarenas[0].cpu().pin_memory()
+    hy = torch.empty_like(wl.yarenas[0], device="cpu").pin_memory()
     e2e_steps = max(3, min(args.steps, 50))
-    with torch.cuda.stream(stream):
+    with torch.cuda.stream(wl.stream):
         for i in range(2):
-            xarenas[i % copies].copy_(hx, non_blocking=True)
-            step(i)
+            wl.xarenas[i % wl.copies].copy_(hx, non_blocking=True)
+            wl.step(i)
         torch.cuda.synchronize()
         barrier()
         torch.cuda.synchronize()
         a0 = torch.cuda.Event(enable_timing=True)
         a1 = torch.cuda.Event(enable_timing=True)
-        a0.record(stream)
+        a0.record(wl.stream)
         for i in range(e2e_steps):
-            xarenas[i % copies].copy_(hx, non_blocking=True)
-            step(i)
-            hy.copy_(yarenas[i % copies], non_blocking=True)
-        a1.record(stream)
+            wl.xarenas[i % wl.copies].copy_(hx, non_blocking=True)
+            wl.step(i)
+            hy.copy_(wl.yarenas[i % wl.copies], non_blocking=True)
+        a1.record(wl.stream)
         torch.cuda.synchronize()
         barrier()
     e2e_ms = max_over_ranks(a0.elapsed_time(a1), dist, dev)
-    e2e_value = whole_job_gbs(world, step_bytes, e2e_steps, e2e_ms)
+    e2e_value, _, _ = wl.result(e2e_ms / e2e_steps, world)
 
-    if tensor:
-        # the tensor-core kernel: flops per step over the step time (one GPU)
-        peak, peak_kind = tensor_peak()
-        achieved = step_flops / (ms_per_step / 1e3) / 1e12
-        value = world * step_flops * args.steps / (ms / 1e3) / 1e12
-        e2e_value = world * step_flops * e2e_steps / (e2e_ms / 1e3) / 1e12
-        unit = "TFLOP/s"
-        roofline = {"bound": "tensor", "achieved": round(achieved, 1), "peak": peak,
-                    "unit": "TFLOP/s", "frac": round(achieved / peak, 4), "peak_source": peak_kind,
-                    "traffic": None, "kernel": "tc_kernel (all launches of the step)",
-                    "algorithmic_flops_per_launch": step_flops / len(calls),
-                    "algorithmic_bytes_per_launch": round(step_bytes / len(calls))}
+    kernel = ("tc_kernel (all launches of the step)" if roofline["bound"] == "tensor" else
+              "permute_x_kernel + skinny_kernel (all launches of the step)" if actorder else
+              "skinny_kernel (all launches of the step)")
+    roofline["kernel"] = kernel
+    roofline["algorithmic_bytes_per_launch"] = round(wl.step_bytes / wl.n_calls)
+    if roofline["bound"] == "tensor":
+        roofline["algorithmic_flops_per_launch"] = wl.step_flops / wl.n_calls
+        roofline["traffic"] = None
     else:
-        peak, peak_kind = peaks()
-        achieved = step_bytes / (ms_per_step / 1e3) / 1e9      # one GPU, the skinny kernel only
         # DRAM bytes per algorithmic byte come from the ncu capture of the
         # default workload; other workloads report none
         tpb = traffic_per_byte() if args.workload == "llama7b_decode" else None
-        unit = "GB/s"
-        roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-                    "frac": round(achieved / peak, 4), "peak_source": peak_kind,
-                    "traffic": None if tpb is None else round(tpb * step_bytes / len(calls)),
-                    "kernel": "skinny_kernel (all launches of the step)" if not actorder else
-                              "permute_x_kernel + skinny_kernel (all launches of the step)",
-                    "algorithmic_bytes_per_launch": round(step_bytes / len(calls))}
+        roofline["traffic"] = None if tpb is None else round(tpb * wl.step_bytes / wl.n_calls)
+    w = WORKLOADS[args.workload]
     out = {"metric": METRIC, "value": round(value, 1), "unit": unit, "n_gpus": world,
            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5),
-           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f16",
-           "data": "synthetic (seeded torch.randn weights and activations)",
-           "config": {"workload": args.workload, "calls_per_step": len(calls),
-                      "shapes_KN": WORKLOADS[args.workload][4], "M": WORKLOADS[args.workload][5],
-                      "mode": WORKLOADS[args.workload][0], "group": WORKLOADS[args.workload][2],
-                      **({"zero_group": zopts[0], "zero_bits": zopts[1]} if zopts else {}),
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": wl.dtype,
+           "data": "synthetic: seed-0 counter generator (SplitMix64 + Box-Muller, drawn on the "
+                   "device), weights N(0, sigma) per the configs, activations N(0, 1)",
+           "config": {"workload": args.workload, "calls_per_step": wl.n_calls,
+                      "shapes_KN": w[4], "M": w[5], "mode": w[0], "group": w[2], "x_dtype": w[3],
+                      **({"zero_group": wl.zopts[0], "zero_bits": wl.zopts[1]} if wl.zopts else {}),
                       **({"act_order": "random column order per matrix"} if actorder else {}),
-                      "l2": f"inputs larger than L2: {copies} weight cop"
-                            f"{'y' if copies == 1 else 'ies'} of the step rotated, "
-                            f"{copies * codes_per_copy / 1e6:.0f} MB of codes in all "
-                            f"(L2 {L2_BYTES / 1e6:.0f} MB)",
+                      "l2": wl.l2_note(),
                       "launch": "CUDA graph of the step, programmatic dependent launch",
                       "parallelism": f"replicas x{world}"},
            "roofline": roofline,
-           "e2e": {"value": round(e2e_value, 1), "unit": unit, "h2d_bytes_per_step": h2d,
-                   "d2h_bytes_per_step": d2h, "steps": e2e_steps,
+           "e2e": {"value": round(e2e_value, 1), "unit": unit, "h2d_bytes_per_step": hx.numel(),
+                   "d2h_bytes_per_step": hy.numel(), "steps": e2e_steps,
                    "how": f"per step: the step's pinned x buffer -> device (one copy), the "
-                          f"{len(calls)} calls through the Python API, the y buffer -> pinned "
-                          "host (one copy); CUDA events on the stream"},
-           "gpu_launches": len(calls) * args.steps * (2 if actorder else 1),
+                          f"{wl.n_calls} calls issued one by one through the Python API (no "
+                          "graph), the y buffer -> pinned host (one copy); CUDA events on the "
+                          "stream"},
+           "gpu_launches": wl.n_calls * args.steps * (2 if actorder else 1),
            "clocks": clocks}
+    wl.release()
+    del wl
+    torch.cuda.empty_cache()
+    if rank == 0 and args.workload == "llama7b_decode" and not args.no_configs and world == 1:
+        cfgs = {"2_llama7b_decode": [{"workload": args.workload, "value": out["value"],
+                                      "unit": unit, "frac": roofline["frac"],
+                                      "bound": roofline["bound"], "ms_per_step": out["ms_per_step"],
+                                      "calls_per_step": out["config"]["calls_per_step"],
+                                      "steps": args.steps, "dtype": out["dtype"],
+                                      "note": "the headline measurement above"}]}
+        cfgs.update(measure_configs(dev))
+        out["configs"] = dict(sorted(cfgs.items()))
     if rank == 0 and not args.no_cpu_baseline:
-        out["cpu_baseline"] = cpu_baseline(args.workload, args.cpu_seconds, tensor)
-    del graphs
+        out["cpu_baseline"] = cpu_baseline(args.workload, args.cpu_seconds,
+                                           roofline["bound"] == "tensor")
     return out
 
 
@@ -476,11 +570,11 @@ def _oracle_sample(workload, rows_per_problem, seed=0):
         if gated:   # whole (gate, up) block pairs
             rows_per_problem = max(32, rows_per_problem // 32 * 32)
         rows = np.arange(rows_per_problem)
-        W = synth.weights(seed + i, "W", N, K, SIGMA[mode], rows=rows)
+        W = synth.weights(seed, f"W{i}.0", N, K, SIGMA[mode], rows=rows)
         lut = None
         if mode == "lut":
             lut = {4: synth.nf4_table, 3: synth.nf3_table, 2: lambda: synth.lut2_table(0)}[bits]()
-        x = synth.activations(seed + i, "x", M, K, xdt)
+        x = synth.activations(seed, f"x{i}", M, K, xdt)
         n = rows_per_problem
         b = n / N * alg_bytes(mode, bits, group, M, K, N, gated, zopts, actorder)
         f = alg_flops(M, K, n)
@@ -569,11 +663,25 @@ def cpu_baseline(workload, seconds, tensor=False):
         work += w
     what = (f"{work / reps / 1e9:.2f} GFLOP" if tensor
             else f"{work / reps / 1e6:.1f} MB of algorithmic bytes")
-    return {"value": round(work / dt / (1e12 if tensor else 1e9), 6),
+    scale = 1e12 if tensor else 1e9
+    # the same oracle on one host thread, on a smaller sample (16 rows per call)
+    one_items = _oracle_sample(workload, 16)
+    dt1, work1 = _run_oracle(one_items, 1, tensor)
+    reps1 = max(1, int(round(min(seconds / 2, 5.0) / max(dt1, 1e-3))))
+    for _ in range(reps1 - 1):
+        d, w = _run_oracle(one_items, 1, tensor)
+        dt1 += d
+        work1 += w
+    return {"value": round(work / dt / scale, 6),
             "unit": "TFLOP/s" if tensor else "GB/s", "cores": threads,
             "kind": "oracle", "seconds": round(dt, 2),
             "sample": f"every call of the step on its first {rows} rows of W "
-                      f"({what}), run {reps} times, columns split over {threads} threads"}
+                      f"({what}), run {reps} times, columns split over {threads} threads",
+            "single_thread": {"value": round(work1 / dt1 / scale, 6),
+                              "unit": "TFLOP/s" if tensor else "GB/s", "cores": 1,
+                              "seconds": round(dt1, 2),
+                              "sample": f"every call of the step on its first 16 rows of W, "
+                                        f"run {reps1} times on one thread"}}
 
 
 def run_reference(args):
@@ -616,6 +724,8 @@ def main():
     ap.add_argument("--workload", choices=list(WORKLOADS), default="llama7b_decode")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the other benchmark configurations after the default workload")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

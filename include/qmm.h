@@ -158,6 +158,14 @@ int qmm_with_path(const void* x, int xdtype, const void* qweight, const uint16_t
  * or QMM_PATH_TENSOR), or a negative qmm_status for an unsupported problem. */
 int qmm_path(int M, int N, int K, int bits, int group, int mode);
 
+/* The kernel a call runs (QMM_PATH_SKINNY or QMM_PATH_TENSOR) for activations
+ * of type xdtype when the caller asks for `path` (QMM_PATH_*): QMM_PATH_AUTO
+ * gives qmm's own choice, and a request for the tensor path reports
+ * QMM_PATH_SKINNY where the tensor-core kernel does not take the combination
+ * (2- and 3-bit codes; bf16 with group scales or a table; zero-point
+ * options).  A negative qmm_status for invalid arguments. */
+int qmm_path_ex(int M, int N, int K, int bits, int group, int mode, int xdtype, int path);
+
 /* qmm for callers that cannot allocate device memory.  (This entry point is
  * an addition of this library; the sources describe no counterpart.)
  *
@@ -293,8 +301,22 @@ int qmm_dequant(const void* qweight, const uint16_t* scales, const uint16_t* zer
 
 /* Synchronizes `stream`, then reads and clears the library's device error word
  * on the current device: QMM_OK, or QMM_ERR_TIMEOUT if a kernel abandoned a
- * bounded wait since the last check. */
+ * bounded wait since the last check.  The output of such a call is undefined,
+ * and a workspace it used may hold nonzero arrival counters: zero it again
+ * before reusing it. */
 int qmm_check_error(void* stream);
+
+/* Failure detection.  Every wait a kernel makes on another part of itself
+ * (a copy landing, a stage being freed, an MMA finishing) is bounded: after
+ * `cycles` SM clock cycles without progress the CTA gives up, drains the
+ * copies and MMAs it has issued (those waits have a fixed bound of about
+ * 2 s), frees its tensor memory and exits, and qmm_check_error reports
+ * QMM_ERR_TIMEOUT.  The default is about 2 s at B200 clocks; cycles <= 0
+ * restores it.  A tiny value makes a call give up on purpose, which is how the
+ * error path is tested.  Applies to calls launched afterwards, process-wide;
+ * returns the previous value.  (Waits of the tensor-core path; the decode path
+ * waits only for its own asynchronous copies, which always complete.) */
+long long qmm_set_wait_limit(long long cycles);
 
 /* Static description of a status code. */
 const char* qmm_strerror(int status);

@@ -50,6 +50,13 @@ def test_sizes_and_paths(lib):
     assert q.path(64, 4096, 4096, "sym") == "skinny"
     assert q.path(65, 4096, 4096, "sym") == "tensor"
     assert q.path(4096, 14336, 4096, "lut", 2, 64) == "skinny"
+    # the kernel a forced-path request really runs, per activation dtype
+    assert q.path(300, 272, 1024, "sym", 4, 128, "f16", "tensor") == "tensor"
+    assert q.path(300, 272, 1024, "lut", 2, 64, "f16", "tensor") == "skinny"
+    assert q.path(300, 272, 1024, "lut", 4, 64, "bf16", "tensor") == "skinny"
+    assert q.path(300, 272, 1024, "sym", 4, -1, "bf16", "tensor") == "tensor"
+    assert q.path(5, 272, 1024, "sym", 4, 128, "f16", "skinny") == "skinny"
+    assert q.path(4096, 11008, 4096, "sym", 4, 128, "f16", "auto") == "tensor"
 
 
 @pytest.mark.parametrize("N,K,bits,group,mode,status", [

@@ -28,10 +28,11 @@ PATH_NAMES = {1: "skinny", 2: "tensor"}
 
 SYMBOLS = ("qmm_packed_size", "qmm_pack", "qmm_workspace_size", "qmm_workspace_size_for", "qmm",
            "qmm_with_path",
-           "qmm_path", "qmm_dequant", "qmm_check_error", "qmm_strerror", "qmm_noalloc",
+           "qmm_path", "qmm_path_ex", "qmm_dequant", "qmm_check_error", "qmm_strerror", "qmm_noalloc",
            "qmm_pack_gated", "qmm_gated", "qmm_zeros_size", "qmm_pack_asym",
            "qmm_workspace_size_asym", "qmm_asym", "qmm_dequant_asym", "qmm_actorder_perm",
-           "qmm_pack_actorder", "qmm_workspace_size_actorder", "qmm_actorder")
+           "qmm_pack_actorder", "qmm_workspace_size_actorder", "qmm_actorder",
+           "qmm_set_wait_limit")
 
 _lib = None
 _lock = threading.Lock()
@@ -63,6 +64,7 @@ def load(path: str = LIB_PATH):
             lib.qmm.argtypes = [P, I, P, P, P, I, I, I, I, I, I, P, P, S, P]
             lib.qmm_with_path.argtypes = [P, I, P, P, P, I, I, I, I, I, I, P, P, S, P, I]
             lib.qmm_path.argtypes = [I, I, I, I, I, I]
+            lib.qmm_path_ex.argtypes = [I, I, I, I, I, I, I, I]
             lib.qmm_noalloc.argtypes = [P, I, P, P, P, I, I, I, I, I, I, P, P]
             lib.qmm_pack_gated.argtypes = [P, P, I, I, I, I, I, P, P, P, P, P]
             lib.qmm_gated.argtypes = [P, I, P, P, P, I, I, I, I, I, I, P, P, S, P]
@@ -80,6 +82,8 @@ def load(path: str = LIB_PATH):
             lib.qmm_workspace_size_actorder.restype = S
             lib.qmm_actorder.argtypes = [P, I, P, P, P, P, I, I, I, I, I, I, P, P, S, P]
             lib.qmm_check_error.argtypes = [P]
+            lib.qmm_set_wait_limit.argtypes = [ctypes.c_longlong]
+            lib.qmm_set_wait_limit.restype = ctypes.c_longlong
             lib.qmm_strerror.argtypes = [I]
             lib.qmm_strerror.restype = ctypes.c_char_p
             _lib = lib
@@ -189,10 +193,21 @@ def workspace(M, N, K, mode, bits=4, group=128, device="cuda", path="auto"):
     return torch.zeros(n, dtype=torch.uint8, device=device) if n else None
 
 
-def path(M, N, K, mode, bits=4, group=128):
-    st = load().qmm_path(M, N, K, bits, group, MODES[mode])
+def path(M, N, K, mode, bits=4, group=128, xdtype=None, request="auto"):
+    """The kernel ("skinny" or "tensor") a call runs: with xdtype None, qmm's
+    choice for fp16 activations; else for that activation dtype ("f16",
+    "bf16" or a torch dtype) when `request` (a path name) is asked for."""
+    if xdtype is None and request == "auto":
+        st = load().qmm_path(M, N, K, bits, group, MODES[mode])
+        if st < 0:
+            raise QmmError(st, "qmm_path")
+        return PATH_NAMES[st]
+    dt = {"f16": 0, "bf16": 1, None: 0}.get(xdtype, None)
+    if dt is None:
+        dt = DTYPES[xdtype]
+    st = load().qmm_path_ex(M, N, K, bits, group, MODES[mode], dt, PATHS[request])
     if st < 0:
-        raise QmmError(st, "qmm_path")
+        raise QmmError(st, "qmm_path_ex")
     return PATH_NAMES[st]
 
 
@@ -351,3 +366,9 @@ def qmm_actorder(x, perm, qweight, scales, zeros_or_lut, N, K, mode, bits=4, gro
 def check_error():
     """Raise if a kernel abandoned a bounded wait since the last check."""
     _check(load().qmm_check_error(_stream()), "qmm_check_error")
+
+
+def set_wait_limit(cycles):
+    """Clock cycles a kernel wait may take before the call gives up (<= 0: the
+    default of about 2 s); returns the previous value."""
+    return load().qmm_set_wait_limit(int(cycles))

@@ -4,6 +4,7 @@
 #include <stdint.h>
 
 #include <algorithm>
+#include <atomic>
 
 #include "common.cuh"
 #include "internal.h"
@@ -21,6 +22,12 @@ int device_sms() {
   }
   return sms[dev];
 }
+
+// About 2 s of SM clock: a wait this long means something is wrong.
+constexpr long long kDefaultWaitCycles = 4000000000ll;
+std::atomic<long long> g_wait_cycles{kDefaultWaitCycles};
+
+long long wait_limit() { return g_wait_cycles.load(std::memory_order_relaxed); }
 
 namespace {
 
@@ -145,7 +152,8 @@ static int run_qmm(const void* x, int xdtype, const void* qweight, const uint16_
       return QMM_ERR_WORKSPACE;
     }
   }
-  if (plan.path == QMM_PATH_TENSOR) return status_of(launch_tc(p, plan.tc, workspace, s));
+  if (plan.path == QMM_PATH_TENSOR)
+    return status_of(launch_tc(p, plan.tc, workspace, wait_limit(), s));
   return status_of(launch_skinny(p, plan.sk, workspace, s));
 }
 
@@ -197,6 +205,15 @@ int qmm_path(int M, int N, int K, int bits, int group, int mode) {
   int st = check_shape(N, K, bits, group, mode);
   if (st != QMM_OK) return st;
   return choose_path(M, N, bits, mode, false, group);
+}
+
+int qmm_path_ex(int M, int N, int K, int bits, int group, int mode, int xdtype, int path) {
+  if (M < 0) return QMM_ERR_ARG;
+  int st = check_shape(N, K, bits, group, mode);
+  if (st != QMM_OK) return st;
+  if (xdtype != QMM_F16 && xdtype != QMM_BF16) return QMM_ERR_ARG;
+  if (path < QMM_PATH_AUTO || path > QMM_PATH_SKINNY_STREAMK) return QMM_ERR_ARG;
+  return make_plan(std::max(M, 1), N, K, bits, group, mode, xdtype == QMM_BF16, path).path;
 }
 
 size_t qmm_workspace_size_for(int M, int N, int K, int bits, int group, int mode, int path) {
@@ -402,6 +419,11 @@ int qmm_actorder(const void* x, int xdtype, const int32_t* perm, const void* qwe
   if (st != QMM_OK) return st;
   return run_qmm(xp, xdtype, qweight, scales, zeros_or_lut, M, N, K, bits, group, mode, y,
                  workspace, plain, stream, QMM_PATH_AUTO, false);
+}
+
+long long qmm_set_wait_limit(long long cycles) {
+  const long long v = cycles > 0 ? cycles : kDefaultWaitCycles;
+  return g_wait_cycles.exchange(v, std::memory_order_relaxed);
 }
 
 int qmm_check_error(void* stream) {

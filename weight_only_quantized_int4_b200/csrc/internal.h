@@ -56,7 +56,12 @@ struct TcPlan {
 
 bool tc_supported(int bits, int mode, bool bf16, int group);
 TcPlan plan_tc(int M, int N, int K, int sms);
-cudaError_t launch_tc(const Problem& p, const TcPlan& plan, void* workspace, cudaStream_t stream);
+cudaError_t launch_tc(const Problem& p, const TcPlan& plan, void* workspace, long long wait_limit,
+                      cudaStream_t stream);
+
+// Clock cycles a kernel's barrier wait may take before the call gives up
+// (qmm_set_wait_limit).
+long long wait_limit();
 unsigned tc_read_and_clear_error();
 
 // Quantize + pack.  W2: second matrix of the gated layout (else null); perm:

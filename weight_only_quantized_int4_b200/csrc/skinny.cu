@@ -27,6 +27,7 @@
 // workspace and the last warp to finish the tile adds the partials in warp
 // order (deterministic) and stores y.  No warp waits for another.
 #include <algorithm>
+#include <atomic>
 
 #include "common.cuh"
 #include "internal.h"
@@ -1022,21 +1023,23 @@ __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
 // name is only a host-side stand-in, so the address is looked up once per
 // device (with that device current) and cached.
 cudaError_t static_scratch(void** out) {
-  static void* addr[kMaxDevices] = {};
+  // atomics: host threads making their first call on a device at the same
+  // time may both look the address up; they store the same value
+  static std::atomic<void*> addr[kMaxDevices] = {};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-  if (!addr[dev]) {
-    void* p = nullptr;
+  void* p = addr[dev].load(std::memory_order_acquire);
+  if (!p) {
     e = cudaGetSymbolAddress(&p, g_static_scratch);
     if (e != cudaSuccess) {
       cudaGetLastError();
       return e;
     }
-    addr[dev] = p;
+    addr[dev].store(p, std::memory_order_release);
   }
-  *out = addr[dev];
+  *out = p;
   return cudaSuccess;
 }
 

@@ -50,7 +50,9 @@ constexpr int kATileBytes = kRowsTile * kKB * 2;   // 16 KB
 constexpr int kMetaTile = 1024;
 template <int MODE>
 constexpr int kMetaBytes = MODE == kASYM ? 2 * kMetaTile : kMetaTile;
-constexpr long long kWaitCycles = 4000000000ll; // ~2 s at 1.9 GHz
+// Bound of the waits a CTA makes for its own copies and MMAs while draining
+// (they always complete): ~2 s at 1.9 GHz.
+constexpr long long kDrainCycles = 4000000000ll;
 
 template <int BN>
 struct TcCfg {
@@ -62,20 +64,45 @@ struct TcCfg {
 // ------------------------------------------------------------------ PTX helpers
 
 // Bounded wait for phase `parity` of `bar`.  Returns false (and raises the
-// CTA's abort flag and the device error word) if it runs out, or if another
-// thread of the CTA has already aborted.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
+// CTA's abort flag and the device error word) if `limit` clock cycles pass,
+// or at once if another thread of the CTA has already aborted.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                          long long limit) {
   if (mbar_try(bar, parity)) return true;
   const long long t0 = clock64();
   while (true) {
     if (mbar_try(bar, parity)) return true;
     if (*abort) return false;
-    if (clock64() - t0 > kWaitCycles) {
+    if (clock64() - t0 > limit) {
       *abort = 1;
       atomicOr(&g_tc_error, 1u);
       return false;
     }
   }
+}
+
+// Wait for a copy or MMA the CTA issued itself, before it frees what they
+// use: ignores the abort flag, bounded by kDrainCycles.
+__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
+  if (mbar_try(bar, parity)) return;
+  const long long t0 = clock64();
+  while (!mbar_try(bar, parity))
+    if (clock64() - t0 > kDrainCycles) return;
+}
+
+// Named barrier whose result is the AND of every participating thread's
+// predicate: a decision the warps of a role take together.
+__device__ __forceinline__ bool named_bar_and(int id, int threads, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "barrier.red.and.pred q, %2, %3, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)pred), "r"(id), "r"(threads)
+      : "memory");
+  return r != 0;
 }
 
 __device__ __forceinline__ void tc_fence_before() {
@@ -146,6 +173,7 @@ struct TcArgs {
   int tiles_n, tiles_m, tiles;
   long long units;          // tiles * nkb
   int ctas;
+  long long wait_limit;     // clock cycles a barrier wait may take before the call gives up
   float* slots;             // [2 * ctas][BN][128]: a CTA's first / last partial tile,
                             // column-major so that a warp's 32 rows are 128 contiguous bytes
   unsigned* counters;       // [tiles]
@@ -195,9 +223,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   using Cfg = TcCfg<BN>;
   constexpr int S = Cfg::STAGES;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
-  // carve: A stages | B stages | code stages | meta stages | LUT table | barriers
-  unsigned char* base = reinterpret_cast<unsigned char*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  // carve: A stages | B stages | code stages | meta stages | LUT table | barriers.
+  // The 1024-byte aligned start is an offset from the shared array itself, so
+  // the compiler keeps every access below in the shared address space (a
+  // pointer rebuilt from an integer would turn them into generic accesses).
+  unsigned char* base = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   unsigned char* sA = base;
   unsigned char* sB = sA + S * kATileBytes;
   unsigned char* sC = sB + S * Cfg::B_BYTES;
@@ -216,7 +246,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   uint64_t* ab_empty = a_full + S;
   uint64_t* acc_full = ab_empty + S;      // [2]
   uint64_t* acc_empty = acc_full + 2;     // [2]
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
+  uint64_t* mma_drain = acc_empty + 2;    // the MMA thread's last commit
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int* last_flag = const_cast<int*>(abort_flag) + 1;
   int* meta = last_flag + 1;   // [3]: first contributor, contributors, first's slot parity
@@ -240,6 +271,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       mbar_init(&acc_full[i], 1);
       mbar_init(&acc_empty[i], 4);
     }
+    mbar_init(mma_drain, 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -296,7 +328,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         bool ok = true;
         for (int kb = kb0; kb < kb1; ++kb, ++kc) {
           const int c = kc % kCodeStages;
-          if (!mbar_wait(&code_empty[c], ((kc / kCodeStages) & 1) ^ 1, abort_flag)) {
+          if (!mbar_wait(&code_empty[c], ((kc / kCodeStages) & 1) ^ 1, abort_flag, a.wait_limit)) {
             ok = false;
             break;
           }
@@ -314,6 +346,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         if (!ok) break;
         u += kb1 - kb0;
       }
+      // nothing may land after the CTA exits: the last fill of every slot
+      // (consumed already, unless the CTA is giving up)
+      for (int j = kc > kCodeStages ? kc - kCodeStages : 0; j < kc; ++j)
+        drain_wait(&code_full[j % kCodeStages], (j / kCodeStages) & 1);
     } else if (lane == 1) {
       int ks = 0;             // running k-block counter of the A/B ring
       for (long long u = u_begin; u < u_end && !*abort_flag;) {
@@ -323,7 +359,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         bool ok = true;
         for (int kb = kb0; kb < kb1; ++kb, ++ks) {
           const int s = ks % S;
-          if (!mbar_wait(&ab_empty[s], ((ks / S) & 1) ^ 1, abort_flag)) {
+          if (!mbar_wait(&ab_empty[s], ((ks / S) & 1) ^ 1, abort_flag, a.wait_limit)) {
             ok = false;
             break;
           }
@@ -333,6 +369,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         if (!ok) break;
         u += kb1 - kb0;
       }
+      for (int j = ks > S ? ks - S : 0; j < ks; ++j) drain_wait(&b_full[j % S], (j / S) & 1);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -344,14 +381,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         int tile, kb0, kb1;
         seg_of(u, tile, kb0, kb1);
         const int buf = seg & 1;
-        if (!mbar_wait(&acc_empty[buf], ((seg >> 1) & 1) ^ 1, abort_flag)) break;
+        if (!mbar_wait(&acc_empty[buf], ((seg >> 1) & 1) ^ 1, abort_flag, a.wait_limit)) break;
         tc_fence_after();
         const uint32_t d = tmem_base + (uint32_t)(buf * BN);
         bool ok = true;
         for (int kb = kb0; kb < kb1; ++kb, ++ks) {
           const int s = ks % S;
           const uint32_t ph = (ks / S) & 1;
-          if (!mbar_wait(&a_full[s], ph, abort_flag) || !mbar_wait(&b_full[s], ph, abort_flag)) {
+          if (!mbar_wait(&a_full[s], ph, abort_flag, a.wait_limit) || !mbar_wait(&b_full[s], ph, abort_flag, a.wait_limit)) {
             ok = false;
             break;
           }
@@ -368,6 +405,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         umma_commit(&acc_full[buf]);
         u += kb1 - kb0;
       }
+      // every MMA issued has finished before TMEM (and the A / B tiles) can
+      // be released: one more commit, which arrives once they all have
+      umma_commit(mma_drain);
+      drain_wait(mma_drain, 0);
     }
   } else if (warp < 2 + kDecWarps) {
     // ------------------------------------------------------------ decode warps
@@ -375,11 +416,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const int g = lane >> 2, t = lane & 3;
     const unsigned char* tabp = sT;
     int kc = 0, ks = 0;
-    for (long long u = u_begin; u < u_end && !*abort_flag; ++u, ++kc, ++ks) {
+    for (long long u = u_begin; u < u_end; ++u, ++kc, ++ks) {
       const int c = kc % kCodeStages, s = ks % S;
-      if (!mbar_wait(&code_full[c], (kc / kCodeStages) & 1, abort_flag) ||
-          !mbar_wait(&ab_empty[s], ((ks / S) & 1) ^ 1, abort_flag))
-        break;
+      // the warp stops as one (it ends each stage with a warp-wide sync)
+      const bool ok = mbar_wait(&code_full[c], (kc / kCodeStages) & 1, abort_flag, a.wait_limit) &&
+                      mbar_wait(&ab_empty[s], ((ks / S) & 1) ^ 1, abort_flag, a.wait_limit);
+      if (!__all_sync(0xffffffffu, ok)) break;
       unsigned char* At = sA + s * kATileBytes;
       // group scales (and zero-points) of the lane's rows g and g + 8, one word
       // per 16-column slice j, from the k block's meta tile (landed with the codes)
@@ -465,12 +507,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const int q = warp & 3;                  // TMEM lane quadrant of this warp
     const int row_l = q * 32 + lane;         // weight row within the tile
     int seg = 0;
-    for (long long u = u_begin; u < u_end && !*abort_flag; ++seg) {
+    for (long long u = u_begin; u < u_end; ++seg) {
       int tile, kb0, kb1;
       seg_of(u, tile, kb0, kb1);
       const int tn = tile % a.tiles_n, tm = tile / a.tiles_n;
       const int buf = seg & 1;
-      if (!mbar_wait(&acc_full[buf], (seg >> 1) & 1, abort_flag)) break;
+      // the four epilogue warps stop together (they share named barriers)
+      const bool ok = mbar_wait(&acc_full[buf], (seg >> 1) & 1, abort_flag, a.wait_limit);
+      if (!named_bar_and(1, 128, ok)) break;
       tc_fence_after();
       const int row = tn * kRowsTile + row_l;
       float s_row = 1.0f;
@@ -648,7 +692,7 @@ constexpr size_t tc_smem_bytes() {
   using Cfg = TcCfg<BN>;
   return 1024 + (size_t)Cfg::STAGES * (kATileBytes + Cfg::B_BYTES) +
          (size_t)kCodeStages * (kCodeBytes + kMetaBytes<MODE>) + (MODE == kLUT ? 256 * 32 * 4 : 0) +
-         (2 * kCodeStages + 3 * Cfg::STAGES + 4) * 8 + 32;
+         (2 * kCodeStages + 3 * Cfg::STAGES + 5) * 8 + 32;
 }
 
 template <int MODE, bool BF16, int BN, bool GM1>
@@ -748,7 +792,7 @@ TcPlan plan_tc(int M, int N, int K, int sms) {
 }
 
 cudaError_t launch_tc(const Problem& pr, const TcPlan& plan, void* workspace,
-                      cudaStream_t stream) {
+                      long long wait_limit, cudaStream_t stream) {
   auto encode = tensor_map_encoder();
   if (!encode) return cudaErrorNotSupported;
   CUtensorMap mx, mw;
@@ -813,6 +857,7 @@ cudaError_t launch_tc(const Problem& pr, const TcPlan& plan, void* workspace,
   a.tiles = plan.tiles_n * plan.tiles_m;
   a.units = (long long)a.tiles * plan.nkb;
   a.ctas = plan.ctas;
+  a.wait_limit = wait_limit;
   if (plan.ws_bytes) {
     const size_t cbytes = ((size_t)a.tiles * 4 + 255) / 256 * 256;
     a.counters = reinterpret_cast<unsigned*>(workspace);

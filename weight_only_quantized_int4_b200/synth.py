@@ -140,3 +140,76 @@ def lut2_table(seed: int = 0) -> np.ndarray:
     v = normal_at(seed, "lut2", np.arange(4, dtype=np.uint64))
     v = np.sort(v / np.max(np.abs(v)))
     return v.astype(np.float16).view(np.uint16)
+
+
+# ------------------------------------------------------------------ torch twin
+#
+# The same generator written with torch int64 tensors, for inputs too large to
+# draw on the host (the benchmark's weights): uint64 wrapping arithmetic on
+# two's-complement int64, logical right shifts by masking.  The uniforms match
+# the numpy functions above bit for bit; the Box-Muller step runs in the
+# device's float64 log / sqrt / sin / cos, whose last bits may differ from the
+# host's, so the normal deviates agree to a few ulps of float64.
+
+def _i64(u: int) -> int:
+    """uint64 constant as the int64 with the same bits."""
+    return u - (1 << 64) if u >= (1 << 63) else u
+
+
+_T_GAMMA = _i64(0x9E3779B97F4A7C15)
+_T_M1 = _i64(0xBF58476D1CE4E5B9)
+_T_M2 = _i64(0x94D049BB133111EB)
+
+
+def _srl(z, k: int):
+    """Logical right shift of an int64 tensor holding uint64 bits."""
+    return (z >> k) & ((1 << (64 - k)) - 1)
+
+
+def _mix_t(z):
+    z = (z ^ _srl(z, 30)) * _T_M1
+    z = (z ^ _srl(z, 27)) * _T_M2
+    return z ^ _srl(z, 31)
+
+
+def weights_torch(seed: int, stream: str, N: int, K: int, sigma: float, device="cpu"):
+    """weights() as an fp32 torch tensor on `device`."""
+    import torch
+
+    W = torch.empty(N, K, dtype=torch.float32, device=device)
+    rows = max(1, (1 << 24) // max(1, K))
+    for r0 in range(0, N, rows):
+        r1 = min(N, r0 + rows)
+        W[r0:r1] = (sigma * _rows_torch(seed, stream, r0, r1, K, device)).to(torch.float32)
+    return W
+
+
+def _rows_torch(seed, stream, r0, r1, K, device):
+    """Rows [r0, r1) of normal_rows(seed, stream, ., K) as float64 on `device`."""
+    import torch
+
+    key = _i64(int(stream_key(seed, stream)))
+    idx = torch.arange(r0 * K, r1 * K, dtype=torch.int64, device=device)
+    pair = idx & ~1
+
+    def uni(ctr):
+        z = _mix_t(key + (ctr + 1) * _T_GAMMA)
+        return _srl(z, 11).to(torch.float64) * (1.0 / 9007199254740992.0)
+
+    u1 = 1.0 - uni(pair)
+    u2 = uni(pair + 1)
+    r = torch.sqrt(-2.0 * torch.log(u1))
+    ang = (2.0 * math.pi) * u2
+    return torch.where((idx & 1).bool(), r * torch.sin(ang), r * torch.cos(ang)).view(r1 - r0, K)
+
+
+def activations_torch(seed: int, stream: str, M: int, K: int, dtype: str, device="cpu"):
+    """activations() as an fp16 / bf16 torch tensor on `device`."""
+    import torch
+
+    z = _rows_torch(seed, stream, 0, M, K, device)
+    if dtype == "f16":
+        return z.to(torch.float16)
+    if dtype == "bf16":
+        return z.to(torch.float32).to(torch.bfloat16)
+    raise ValueError(dtype)
