@@ -267,7 +267,9 @@ class Workload:
     as many copies as it takes to pass twice the L2 size (rotated step by
     step), activations and outputs (each set in one buffer, so the end-to-end
     leg moves a step's inputs and results with one copy each way), workspaces,
-    and one CUDA graph per weight copy; a step is one graph replay.
+    and one CUDA graph of a round of steps, one per weight copy (a graph launch
+    costs microseconds: a round keeps it off single-call steps).  The default
+    workload has one copy, so a round is one step.
 
     Inputs come from the seed-0 counter generator of `synth` (drawn on the
     device): call c's weights are stream "W{c}.{copy}", its activations "x{c}".
@@ -338,15 +340,13 @@ class Workload:
             self.step(i)
         torch.cuda.synchronize()
         self.stream = torch.cuda.Stream(device=dev)
-        self.graphs = []
         with torch.cuda.stream(self.stream):
             self.step()
             torch.cuda.synchronize()
-            for i in range(self.copies):
-                g = torch.cuda.CUDAGraph()
-                with torch.cuda.graph(g, stream=self.stream):
+            self.graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(self.graph, stream=self.stream):
+                for i in range(self.copies):
                     self.step(i)
-                self.graphs.append(g)
         torch.cuda.synchronize()
 
     def step(self, i=0):
@@ -367,26 +367,32 @@ class Workload:
                 q.qmm(c["x"], c["qw"], c["sc"], c["zl"], c["N"], c["K"], c["mode"], c["bits"],
                       c["group"], y=c["y"], ws=c["ws"])
 
+    def rounds(self, steps):
+        """Graph replays that cover at least `steps` steps."""
+        return max(1, -(-steps // self.copies))
+
     def time_steps(self, steps, warmup, barrier=lambda: None):
-        """Device time (ms) of `steps` graph replays after `warmup` ones, CUDA
+        """(device ms, steps timed): rounds covering `steps` steps (exactly
+        `steps` when a round is one step) after rounds covering `warmup`, CUDA
         events on the replay stream, synchronized and barriered on both sides."""
         import torch
         with torch.cuda.stream(self.stream):
-            for i in range(warmup):
-                self.graphs[i % self.copies].replay()
+            for _ in range(self.rounds(warmup)):
+                self.graph.replay()
             torch.cuda.synchronize()
             barrier()
             torch.cuda.synchronize()
             e0 = torch.cuda.Event(enable_timing=True)
             e1 = torch.cuda.Event(enable_timing=True)
             e0.record(self.stream)
-            for i in range(steps):
-                self.graphs[i % self.copies].replay()
+            n = self.rounds(steps)
+            for _ in range(n):
+                self.graph.replay()
             e1.record(self.stream)
             torch.cuda.synchronize()
             barrier()
             torch.cuda.synchronize()
-        return e0.elapsed_time(e1)
+        return e0.elapsed_time(e1), n * self.copies
 
     def busy(self, seconds):
         """Replays for about `seconds` (so that clock samples see the GPU under load)."""
@@ -394,8 +400,8 @@ class Workload:
         t_end = time.time() + seconds
         with torch.cuda.stream(self.stream):
             while time.time() < t_end:
-                for i in range(50):
-                    self.graphs[i % self.copies].replay()
+                for _ in range(max(1, 50 // self.copies)):
+                    self.graph.replay()
                 torch.cuda.synchronize()
 
     def l2_note(self):
@@ -419,13 +425,13 @@ class Workload:
         return world * achieved, "GB/s", roof
 
     def release(self):
-        del self.graphs, self.sets, self.xarenas, self.yarenas
+        del self.graph, self.sets, self.xarenas, self.yarenas
 
 
-def steps_for(wl, seconds, lo=20, hi=5000):
+def steps_for(wl, seconds, lo=20, hi=20000):
     """Timed steps worth about `seconds` of device time (from a short probe)."""
-    ms = wl.time_steps(5, 2)
-    return int(min(hi, max(lo, seconds * 1e3 / max(ms / 5, 1e-3))))
+    ms, n = wl.time_steps(5, 2)
+    return int(min(hi, max(lo, seconds * 1e3 / max(ms / n, 1e-4))))
 
 
 def measure_configs(dev):
@@ -438,8 +444,8 @@ def measure_configs(dev):
         recs = []
         for name in names:
             wl = Workload(name, dev)
-            steps = steps_for(wl, 0.3)
-            ms = wl.time_steps(steps, 5) / steps
+            ms, steps = wl.time_steps(steps_for(wl, 0.3), 5)
+            ms /= steps
             value, unit, roof = wl.result(ms)
             recs.append({"workload": name, "value": round(value, 1), "unit": unit,
                          "frac": roof["frac"], "bound": roof["bound"],
@@ -473,9 +479,10 @@ def run_ours(args, rank, world, local_rank):
     clock = ClockSampler(local_rank)
     clock.start()
     wl.busy(0.3)
-    ms = max_over_ranks(wl.time_steps(args.steps, args.warmup, barrier), dist, dev)
+    ms, steps = wl.time_steps(args.steps, args.warmup, barrier)
+    ms = max_over_ranks(ms, dist, dev)
     clocks = clock.stop()
-    ms_per_step = ms / args.steps
+    ms_per_step = ms / steps
     value, unit, roofline = wl.result(ms_per_step, world)
 
     # ---- end to end through the public API: pinned host x in, y out, per step
@@ -518,7 +525,7 @@ def run_ours(args, rank, world, local_rank):
         roofline["traffic"] = None if tpb is None else round(tpb * wl.step_bytes / wl.n_calls)
     w = WORKLOADS[args.workload]
     out = {"metric": METRIC, "value": round(value, 1), "unit": unit, "n_gpus": world,
-           "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5),
+           "steps": steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5),
            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": wl.dtype,
            "data": "synthetic: seed-0 counter generator (SplitMix64 + Box-Muller, drawn on the "
                    "device), weights N(0, sigma) per the configs, activations N(0, 1)",
@@ -536,7 +543,7 @@ def run_ours(args, rank, world, local_rank):
                           f"{wl.n_calls} calls issued one by one through the Python API (no "
                           "graph), the y buffer -> pinned host (one copy); CUDA events on the "
                           "stream"},
-           "gpu_launches": wl.n_calls * args.steps * (2 if actorder else 1),
+           "gpu_launches": wl.n_calls * steps * (2 if actorder else 1),
            "clocks": clocks}
     wl.release()
     del wl
@@ -546,7 +553,7 @@ def run_ours(args, rank, world, local_rank):
                                       "unit": unit, "frac": roofline["frac"],
                                       "bound": roofline["bound"], "ms_per_step": out["ms_per_step"],
                                       "calls_per_step": out["config"]["calls_per_step"],
-                                      "steps": args.steps, "dtype": out["dtype"],
+                                      "steps": out["steps"], "dtype": out["dtype"],
                                       "note": "the headline measurement above"}]}
         cfgs.update(measure_configs(dev))
         out["configs"] = dict(sorted(cfgs.items()))
