@@ -107,7 +107,7 @@ def test_dequant_bit_exact(mode, bits, group, dtype):
 
 # ------------------------------------------------------------------ matmul
 
-SMALL_M = [1, 2, 3, 8, 9, 16, 17, 40]
+SMALL_M = [1, 2, 3, 8, 9, 16, 17, 32, 33, 40, 64]
 
 
 @pytest.mark.parametrize("mode,bits,group", MODES)

@@ -185,7 +185,7 @@ __device__ __forceinline__ void mma_16816_first(float (&d)[4], const uint32_t (&
 }
 
 template <int BITS, int MODE, bool BF16, int NT, int TPG, bool DEEP>
-__global__ void __launch_bounds__(kThreads, DEEP ? 1 : 2) skinny_kernel(const SkinnyArgs a) {
+__global__ void __launch_bounds__(kThreads, (DEEP || NT > 2) ? 1 : 2) skinny_kernel(const SkinnyArgs a) {
   using St = Stage<BITS, MODE, NT, TPG>;
   constexpr int S = ring_stages<BITS, MODE, NT, TPG, DEEP>();
   constexpr int R = St::R;
@@ -291,11 +291,24 @@ __global__ void __launch_bounds__(kThreads, DEEP ? 1 : 2) skinny_kernel(const Sk
   const int xrow0 = lane >> 4, xp = lane & 15;
   const int xi_n = (mrows + 1) >> 1;                       // warp-uniform
   const uint32_t xdst0 = St::X_OFF + xrow0 * kXPitch + xp * 16;
-  const uint16_t* xsrc[(TOK + 1) / 2];
+  // the lane's x sources, one per pair of token rows (rows past M are clamped
+  // and copied with size 0); 32-token tiles recompute them instead of holding
+  // 16 pointers
+  constexpr bool kWide = NT > 2;
+  constexpr int XP = (TOK + 1) / 2;
+  const uint16_t* xsrc[kWide ? 1 : XP];
+  auto xsrc_at = [&](int i) -> const uint16_t* {
+    if constexpr (kWide)
+      return a.x + (size_t)min(m_base + xrow0 + 2 * i, a.M - 1) * a.K + xp * 8;
+    else
+      return xsrc[i];
+  };
+  if constexpr (!kWide) {
 #pragma unroll
-  for (int i = 0; i < (TOK + 1) / 2; ++i) {
-    const int m = min(m_base + xrow0 + 2 * i, a.M - 1);
-    xsrc[i] = a.x + (size_t)m * a.K + xp * 8;
+    for (int i = 0; i < XP; ++i) {
+      const int m = min(m_base + xrow0 + 2 * i, a.M - 1);
+      xsrc[i] = a.x + (size_t)m * a.K + xp * 8;
+    }
   }
   // zero-point options: bytes per zero group record (16 fp16 or 16 nibbles),
   // zero groups per stage, bytes of a row block's zeros per stage
@@ -321,9 +334,17 @@ __global__ void __launch_bounds__(kThreads, DEEP ? 1 : 2) skinny_kernel(const Sk
   // steady-state copy parameters fixed for the call: source bytes of this
   // lane's x pieces (16, or 0 for a token row past M, which reads as zeros)
   // and the shift from a stage's first column to its first group
-  uint32_t xsz[(TOK + 1) / 2];
+  uint32_t xsz[kWide ? 1 : XP];
+  if constexpr (!kWide) {
 #pragma unroll
-  for (int i = 0; i < (TOK + 1) / 2; ++i) xsz[i] = xrow0 + 2 * i < mrows ? 16u : 0u;
+    for (int i = 0; i < XP; ++i) xsz[i] = xrow0 + 2 * i < mrows ? 16u : 0u;
+  }
+  auto xsz_at = [&](int i) -> bool {
+    if constexpr (kWide)
+      return xrow0 + 2 * i < mrows;
+    else
+      return xsz[i] != 0;
+  };
   const int lgs = lg < 0 ? 31 : lg;
   const uint8_t* cbase[R];
   bool rok[R];
@@ -385,9 +406,9 @@ __global__ void __launch_bounds__(kThreads, DEEP ? 1 : 2) skinny_kernel(const Sk
           if (RB_BYTES % 512 == 0 || i * 512 + lane * 16 < RB_BYTES)
             cp_async16_all(base + r * RB_BYTES + i * 512 + lane * 16, cbase[r] + cofs + i * 512);
 #pragma unroll
-      for (int i = 0; i < (TOK + 1) / 2; ++i)
+      for (int i = 0; i < XP; ++i)
         if (i < xi_n)   // warp-uniform
-          cp_async16(base + xdst0 + 2 * i * kXPitch, xsrc[i] + k0, xsz[i] != 0);
+          cp_async16(base + xdst0 + 2 * i * kXPitch, xsrc_at(i) + k0, xsz_at(i));
       if (sq_on) {
         const int off = ((k0 >> lgs) + sq_k) << 4;
         cp_async16(base + St::S_OFF + lane * 16, sbase + off, srok);
@@ -410,10 +431,10 @@ __global__ void __launch_bounds__(kThreads, DEEP ? 1 : 2) skinny_kernel(const Sk
         }
       const bool xk = full || k0 + xp * 8 < a.K;
 #pragma unroll
-      for (int i = 0; i < (TOK + 1) / 2; ++i) {
+      for (int i = 0; i < XP; ++i) {
         if (i < xi_n) {   // warp-uniform
           const bool ok = xrow0 + 2 * i < mrows && xk;
-          cp_async16(base + xdst0 + 2 * i * kXPitch, xsrc[i] + (ok ? k0 : 0), ok);
+          cp_async16(base + xdst0 + 2 * i * kXPitch, xsrc_at(i) + (ok ? k0 : 0), ok);
         }
       }
       if (sq_on) {
@@ -538,17 +559,21 @@ __global__ void __launch_bounds__(kThreads, DEEP ? 1 : 2) skinny_kernel(const Sk
       // (g, t) the columns 4t .. 4t + 3 of each 16-column tile (the MMA's k
       // order permuted the same way for both operands), so its b0, b1 are the
       // 8 contiguous bytes at column 16 j + 4 t of token row g.
-      uint32_t xf[kTiles][NT][2];
-      {
-        const unsigned char* xa = st + St::X_OFF + g * kXPitch + 8 * t;
+      // (all eight tiles' fragments up front for 8 and 16 tokens; 32 tokens
+      // load each tile's when it is used, to keep the registers for the sums)
+      const unsigned char* xa = st + St::X_OFF + g * kXPitch + 8 * t;
+      uint32_t xf[kWide ? 1 : kTiles][NT][2];
+      auto load_xf = [&](int j, uint32_t (&f)[NT][2]) {
 #pragma unroll
-        for (int j = 0; j < kTiles; ++j)
+        for (int nt = 0; nt < NT; ++nt) {
+          const uint2 v = *reinterpret_cast<const uint2*>(xa + nt * 8 * kXPitch + 32 * j);
+          f[nt][0] = v.x;
+          f[nt][1] = v.y;
+        }
+      };
+      if constexpr (!kWide) {
 #pragma unroll
-          for (int nt = 0; nt < NT; ++nt) {
-            const uint2 v = *reinterpret_cast<const uint2*>(xa + nt * 8 * kXPitch + 32 * j);
-            xf[j][nt][0] = v.x;
-            xf[j][nt][1] = v.y;
-          }
+        for (int j = 0; j < kTiles; ++j) load_xf(j, xf[j]);
       }
       // one 4-bit zero record per stage: each row block's (z_g, z_g8) pairs once
       uint32_t zq1[MODE == kASYMQ1 ? R : 1][2];
@@ -570,6 +595,9 @@ __global__ void __launch_bounds__(kThreads, DEEP ? 1 : 2) skinny_kernel(const Sk
 #pragma unroll
       for (int j = 0; j < kTiles; ++j) {
         const int grp = j / TPG;            // group within the stage (compile-time)
+        uint32_t xfw[NT][2];
+        if constexpr (kWide) load_xf(j, xfw);
+        const uint32_t(&xj)[NT][2] = *(kWide ? &xfw : &xf[kWide ? 0 : j]);
         // the lane's 16 code bytes of chunk j / 4 (4-bit) or of the stage (2-bit)
         if constexpr (BITS == 3) {
           if (j == 0) {
@@ -689,11 +717,11 @@ __global__ void __launch_bounds__(kThreads, DEEP ? 1 : 2) skinny_kernel(const Sk
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) {
               if (j % TPG == 0)
-                mma_16816_first<BF16>(gacc[r][nt], af, xf[j][nt][0], xf[j][nt][1]);
+                mma_16816_first<BF16>(gacc[r][nt], af, xj[nt][0], xj[nt][1]);
               else
-                mma_16816<BF16>(gacc[r][nt], af, xf[j][nt][0], xf[j][nt][1]);
+                mma_16816<BF16>(gacc[r][nt], af, xj[nt][0], xj[nt][1]);
               if constexpr (MODE == kLUT && BF16)
-                mma_16816<BF16>(gacc[r][nt], aflo, xf[j][nt][0], xf[j][nt][1]);
+                mma_16816<BF16>(gacc[r][nt], aflo, xj[nt][0], xj[nt][1]);
             }
           }
         }
@@ -752,7 +780,7 @@ __global__ void __launch_bounds__(kThreads, DEEP ? 1 : 2) skinny_kernel(const Sk
       } else {
 #pragma unroll
         for (int i = 0; i < NACC; ++i) outv[i] = 0.0f;
-        constexpr int KB = NT == 1 ? 4 : 2;   // contributors loaded at a time
+        constexpr int KB = NT == 1 ? 4 : (NT == 2 ? 2 : 1);   // contributors loaded at a time
         for (int k0 = 0; k0 < nb; k0 += KB) {
           float4 v[KB][NACC / 4];
 #pragma unroll
@@ -872,7 +900,7 @@ cudaError_t launch(const SkinnyArgs& args, int slabs, cudaStream_t stream) {
 // runtime values (the deep ring only for the plain SYM / ASYM / LUT formats).
 template <int B, int MO, bool BF, int T, int TP, class F>
 auto dispatch_deep(bool deep, F&& f) {
-  if constexpr (!zero_opts(MO)) {
+  if constexpr (!zero_opts(MO) && T <= 2) {
     if (deep) return f.template operator()<B, MO, BF, T, TP, true>();
   }
   return f.template operator()<B, MO, BF, T, TP, false>();
@@ -899,6 +927,10 @@ auto dispatch(int bits, int mode, bool bf16, int nt, int tpg, bool deep, F&& f) 
   QMM_CASE(2, kLUT, false, 1) QMM_CASE(2, kLUT, false, 2) QMM_CASE(2, kLUT, true, 1)
   QMM_CASE(2, kLUT, true, 2) QMM_CASE(3, kLUT, false, 1) QMM_CASE(3, kLUT, false, 2)
   QMM_CASE(3, kLUT, true, 1) QMM_CASE(3, kLUT, true, 2)
+  QMM_CASE(4, kSYM, false, 4) QMM_CASE(4, kSYM, true, 4) QMM_CASE(4, kASYM, false, 4)
+  QMM_CASE(4, kASYM, true, 4) QMM_CASE(4, kLUT, false, 4) QMM_CASE(4, kLUT, true, 4)
+  QMM_CASE(2, kLUT, false, 4) QMM_CASE(2, kLUT, true, 4) QMM_CASE(3, kLUT, false, 4)
+  QMM_CASE(3, kLUT, true, 4)
   QMM_CASE(4, kASYMX, false, 1) QMM_CASE(4, kASYMX, false, 2) QMM_CASE(4, kASYMX, true, 1)
   QMM_CASE(4, kASYMX, true, 2) QMM_CASE(4, kASYMQ, false, 1) QMM_CASE(4, kASYMQ, false, 2)
   QMM_CASE(4, kASYMQ, true, 1) QMM_CASE(4, kASYMQ, true, 2) QMM_CASE(4, kASYMQ1, false, 1)
@@ -916,7 +948,9 @@ int tiles_per_group(int group) { return (group == -1 || group >= kSC) ? 8 : grou
 SkinnyPlan plan_skinny(int M, int N, int K, int bits, int group, int mode, bool bf16, int sms,
                        bool force_streamk) {
   SkinnyPlan p{};
-  p.nt = M <= 8 ? 1 : 2;
+  // token tiles of 8: 1 up to 8 tokens, 2 up to 16, 4 up to 32 (the plain
+  // formats; zero-point options stay at 16 tokens per slab)
+  p.nt = M <= 8 ? 1 : (M <= 16 || zero_opts(mode) ? 2 : 4);
   const int R = p.nt == 1 ? rb_per_tile<1>() : rb_per_tile<2>();
   p.rows = 16 * R;
   const int nrb = N / 16;
@@ -941,7 +975,7 @@ SkinnyPlan plan_skinny(int M, int N, int K, int bits, int group, int mode, bool 
     p.ws_bytes = 0;
     // at most one tile per SM: each CTA has an SM to itself, so it takes the
     // deep ring (its warps' stages all requested up front on small matrices)
-    if (p.tiles_n <= sms && !zero_opts(mode)) {
+    if (p.tiles_n <= sms && !zero_opts(mode) && p.nt <= 2) {
       p.deep = 1;
       p.smem = dispatch(bits, mode, bf16, p.nt, tpg, true,
                         [&]<int B, int MO, bool BF, int T, int TP, bool D>() { return smem_bytes<B, MO, T, TP, D>(); });
