@@ -53,7 +53,8 @@ def test_sizes_and_paths(lib):
     # the kernel a forced-path request really runs, per activation dtype
     assert q.path(300, 272, 1024, "sym", 4, 128, "f16", "tensor") == "tensor"
     assert q.path(300, 272, 1024, "lut", 2, 64, "f16", "tensor") == "skinny"
-    assert q.path(300, 272, 1024, "lut", 4, 64, "bf16", "tensor") == "skinny"
+    assert q.path(300, 272, 1024, "lut", 4, 64, "bf16", "tensor") == "tensor"
+    assert q.path(300, 272, 1024, "asym", 4, 128, "bf16", "tensor") == "tensor"
     assert q.path(300, 272, 1024, "sym", 4, -1, "bf16", "tensor") == "tensor"
     assert q.path(5, 272, 1024, "sym", 4, 128, "f16", "skinny") == "skinny"
     assert q.path(4096, 11008, 4096, "sym", 4, 128, "f16", "auto") == "tensor"

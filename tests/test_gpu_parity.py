@@ -152,7 +152,10 @@ def test_qmm_k_ends_mid_stage(mode, bits, group, xdtype, K):
 
 TC_CASES = [("sym", 4, 128, "f16"), ("sym", 4, -1, "f16"), ("asym", 4, 128, "f16"),
             ("lut", 4, 64, "f16"), ("lut", 4, -1, "f16"), ("sym", 4, 32, "f16"),
-            ("sym", 4, -1, "bf16"), ("asym", 4, -1, "bf16")]
+            ("sym", 4, -1, "bf16"), ("asym", 4, -1, "bf16"),
+            # bf16 with group scales or a table: each weight split into bf16 hi + lo
+            ("sym", 4, 128, "bf16"), ("asym", 4, 128, "bf16"), ("asym", 4, 64, "bf16"),
+            ("lut", 4, 64, "bf16"), ("lut", 4, -1, "bf16")]
 
 
 @pytest.mark.parametrize("mode,bits,group,xdtype", TC_CASES)

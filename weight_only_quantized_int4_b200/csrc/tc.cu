@@ -54,10 +54,19 @@ constexpr int kMetaBytes = MODE == kASYM ? 2 * kMetaTile : kMetaTile;
 // (they always complete): ~2 s at 1.9 GHz.
 constexpr long long kDrainCycles = 4000000000ll;
 
-template <int BN>
+// SPLIT: bf16 activations whose A operand is not an exact small integer
+// (group scales, or a table): each decoded weight w, exact in fp32, becomes
+// two bf16 operands hi = bf16(w) and lo = bf16(w - hi) (|w - hi - lo| <=
+// 2^-18 |w|), two A tiles per stage and two MMAs per k step into the same
+// accumulator.  A single bf16 rounding of w (2^-9) together with the bf16
+// output would use most of the error budget.
+template <int BN, bool SPLIT = false, bool TABLE = false>
 struct TcCfg {
-  static constexpr int STAGES = BN == 256 ? 3 : 4;
+  // A / B ring depth within 227 KB (the table takes 32 KB)
+  static constexpr int STAGES =
+      SPLIT ? (BN == 64 ? (TABLE ? 3 : 4) : (BN == 128 ? 3 : 2)) : (BN == 256 ? 3 : 4);
   static constexpr int B_BYTES = BN * kKB * 2;
+  static constexpr int A_BYTES = (SPLIT ? 2 : 1) * kATileBytes;   // one stage's A tile(s)
   static constexpr int TMEM_COLS = 2 * BN;     // two accumulator buffers
 };
 
@@ -220,7 +229,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_w,
               const __grid_constant__ CUtensorMap map_s, const __grid_constant__ CUtensorMap map_z,
               const TcArgs a) {
-  using Cfg = TcCfg<BN>;
+  constexpr bool SPLIT = BF16 && (!GM1 || MODE == kLUT);
+  using Cfg = TcCfg<BN, SPLIT, MODE == kLUT>;
   constexpr int S = Cfg::STAGES;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   // carve: A stages | B stages | code stages | meta stages | LUT table | barriers.
@@ -229,7 +239,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   // pointer rebuilt from an integer would turn them into generic accesses).
   unsigned char* base = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   unsigned char* sA = base;
-  unsigned char* sB = sA + S * kATileBytes;
+  unsigned char* sB = sA + S * Cfg::A_BYTES;
   unsigned char* sC = sB + S * Cfg::B_BYTES;
   unsigned char* sM = sC + kCodeStages * kCodeBytes;
   unsigned char* sT = sM + kCodeStages * kMetaBytes<MODE>;
@@ -393,12 +403,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             break;
           }
           tc_fence_after();
-          const uint32_t sa = smem_u32(sA + s * kATileBytes);
+          const uint32_t sa = smem_u32(sA + s * Cfg::A_BYTES);
           const uint32_t sb = smem_u32(sB + s * Cfg::B_BYTES);
 #pragma unroll
-          for (int k = 0; k < kKB / 16; ++k)
+          for (int k = 0; k < kKB / 16; ++k) {
             umma_f16(d, sw128_desc(sa + 32 * k), sw128_desc(sb + 32 * k), idesc,
                      (kb > kb0 || k > 0) ? 1u : 0u);
+            if constexpr (SPLIT)   // the low parts of the weights, same accumulator
+              umma_f16(d, sw128_desc(sa + kATileBytes + 32 * k), sw128_desc(sb + 32 * k), idesc, 1u);
+          }
           umma_commit(&ab_empty[s]);
         }
         if (!ok) break;
@@ -422,7 +435,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       const bool ok = mbar_wait(&code_full[c], (kc / kCodeStages) & 1, abort_flag, a.wait_limit) &&
                       mbar_wait(&ab_empty[s], ((ks / S) & 1) ^ 1, abort_flag, a.wait_limit);
       if (!__all_sync(0xffffffffu, ok)) break;
-      unsigned char* At = sA + s * kATileBytes;
+      unsigned char* At = sA + s * Cfg::A_BYTES;
       // group scales (and zero-points) of the lane's rows g and g + 8, one word
       // per 16-column slice j, from the k block's meta tile (landed with the codes)
       uint32_t sw[kRbPerDec][4], zw[kRbPerDec][4];
@@ -463,7 +476,28 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             af[2] = *reinterpret_cast<const uint32_t*>(tabp + lop3_and_or(w >> 9, 0x7F80u, l4));
             af[3] = *reinterpret_cast<const uint32_t*>(tabp + lop3_and_or(w >> 17, 0x7F80u, l4));
           }
-          if constexpr (kScales && !BF16 && MODE != kLUT) {
+          uint32_t alo[4];   // SPLIT: the low bf16 parts
+          if constexpr (SPLIT) {
+            // w exact in fp32 ((q - z) s, or T s, or T alone with per-row
+            // scales), then hi = bf16(w), lo = bf16(w - hi)
+            float2 sc = make_float2(1.f, 1.f);
+            if constexpr (kScales) sc = __half22float2(*reinterpret_cast<const __half2*>(&sw[rr][j]));
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              float2 v;
+              if constexpr (MODE == kLUT) {
+                v = __half22float2(*reinterpret_cast<const __half2*>(&af[i]));
+              } else {
+                v = make_float2(__uint_as_float(af[i] << 16), __uint_as_float(af[i] & 0xFFFF0000u));
+              }
+              const float si = (i & 1) ? sc.y : sc.x;   // registers 0, 2: row g; 1, 3: row g + 8
+              v.x *= si;
+              v.y *= si;
+              const uint32_t hi = pack2<true>(v.x, v.y);
+              alo[i] = pack2<true>(v.x - __uint_as_float(hi << 16), v.y - __uint_as_float(hi & 0xFFFF0000u));
+              af[i] = hi;
+            }
+          } else if constexpr (kScales && !BF16 && MODE != kLUT) {
             // (s_g, s_g) and (s_g8, s_g8) as fp16 pairs: one HMUL2 per register
             const uint32_t sg = __byte_perm(sw[rr][j], 0, 0x1010);
             const uint32_t sg8 = __byte_perm(sw[rr][j], 0, 0x3232);
@@ -493,6 +527,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
               make_uint2(af[0], af[2]);
           *reinterpret_cast<uint2*>(At + R1 * 128 + ((ch ^ (R1 & 7)) << 4) + off) =
               make_uint2(af[1], af[3]);
+          if constexpr (SPLIT) {
+            *reinterpret_cast<uint2*>(At + kATileBytes + R0 * 128 + ((ch ^ (R0 & 7)) << 4) + off) =
+                make_uint2(alo[0], alo[2]);
+            *reinterpret_cast<uint2*>(At + kATileBytes + R1 * 128 + ((ch ^ (R1 & 7)) << 4) + off) =
+                make_uint2(alo[1], alo[3]);
+          }
         }
       }
       fence_proxy_async();
@@ -687,10 +727,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 namespace qk {
 namespace {
 
-template <int MODE, int BN>
+template <int MODE, int BN, bool SPLIT>
 constexpr size_t tc_smem_bytes() {
-  using Cfg = TcCfg<BN>;
-  return 1024 + (size_t)Cfg::STAGES * (kATileBytes + Cfg::B_BYTES) +
+  using Cfg = TcCfg<BN, SPLIT, MODE == kLUT>;
+  return 1024 + (size_t)Cfg::STAGES * (Cfg::A_BYTES + Cfg::B_BYTES) +
          (size_t)kCodeStages * (kCodeBytes + kMetaBytes<MODE>) + (MODE == kLUT ? 256 * 32 * 4 : 0) +
          (2 * kCodeStages + 3 * Cfg::STAGES + 5) * 8 + 32;
 }
@@ -699,7 +739,8 @@ template <int MODE, bool BF16, int BN, bool GM1>
 cudaError_t launch_tc_t(const CUtensorMap& mx, const CUtensorMap& mw, const CUtensorMap& ms,
                         const CUtensorMap& mz, const TcArgs& args, cudaStream_t stream) {
   auto k = tc_kernel<MODE, BF16, BN, GM1>;
-  constexpr size_t smem = tc_smem_bytes<MODE, BN>();
+  constexpr size_t smem = tc_smem_bytes<MODE, BN, BF16 && (!GM1 || MODE == kLUT)>();
+  static_assert(smem <= 227 * 1024, "shared memory of the tensor-core kernel");
   static bool attr_set[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
@@ -761,16 +802,15 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   return fn;
 }
 
-// Combinations the tensor path computes within tolerance: 4-bit codes with
-// fp16 activations (the operand is fp16((q - z) s) or fp16(T s), one rounding
-// of 2^-11), or with bf16 activations when the scale is per row (the operand
-// is the exact integer q - z and the scale multiplies the fp32 result).  Group
-// scales with bf16 would round every weight to 8 bits, which together with the
-// bf16 output exceeds the error budget; those run on the decode path.
+// Combinations the tensor path takes: 4-bit codes without the zero-point
+// options.  fp16 activations: the operand is fp16((q - z) s) or fp16(T s), one
+// rounding of 2^-11.  bf16 activations: per-row scales keep the exact integer
+// q - z (the scale multiplies the fp32 result); group scales and tables split
+// each weight into bf16 hi + lo parts (SPLIT above).
 bool tc_supported(int bits, int mode, bool bf16, int group) {
-  if (bits != 4 || zero_opts(mode)) return false;
-  if (!bf16) return true;
-  return group == -1 && mode != kLUT;
+  (void)bf16;
+  (void)group;
+  return bits == 4 && !zero_opts(mode);
 }
 
 TcPlan plan_tc(int M, int N, int K, int sms) {
