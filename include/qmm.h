@@ -138,10 +138,12 @@ size_t qmm_workspace_size_for(int M, int N, int K, int bits, int group, int mode
  *                 filled before first use (see above); may be NULL with
  *                 workspace_bytes 0, in which case no cross-CTA split-K is used.
  * The accumulation is fp32.  M <= 32 (M <= 64 when N <= 4096) runs the
- * bandwidth-bound decode path (16 tokens per slab), larger M the tcgen05
- * tensor-core path for 4-bit codes with fp16 activations or with bf16
- * activations and per-row scales (group -1, SYM/ASYM); the other combinations
- * stay on the decode path.  qmm_path tells which.  The tensor path reads x through a TMA
+ * bandwidth-bound decode path (one slab of up to 32 tokens; larger M in slabs
+ * of 32), larger M the tcgen05 tensor-core path, which takes 4-bit codes with
+ * fp16 or bf16 activations in every mode and group (with bf16 activations and
+ * group scales or a table, each weight enters as two bf16 parts, hi + lo).
+ * Other combinations stay on the decode path.  qmm_path and qmm_path_ex tell
+ * which.  The tensor path reads x through a TMA
  * tensor map, so x's row pitch (K * 2 bytes) must be a multiple of 16 -- true
  * for every K the packed layout allows. */
 int qmm(const void* x, int xdtype, const void* qweight, const uint16_t* scales,
