@@ -53,6 +53,12 @@ constexpr int kMetaBytes = MODE == kASYM ? 2 * kMetaTile : kMetaTile;
 // Bound of the waits a CTA makes for its own copies and MMAs while draining
 // (they always complete): ~2 s at 1.9 GHz.
 constexpr long long kDrainCycles = 4000000000ll;
+// Final reduction of a CTA's last partial tile: the other contributors'
+// partial sums are brought into the (then idle) A / B ring by bulk copies,
+// 32 columns x 128 rows of fp32 (16 KB) per copy, one barrier per 32-column
+// chunk.
+constexpr int kRedChunk = 32 * kRowsTile * 4;
+constexpr int kRedSets = 9;
 
 // SPLIT: bf16 activations whose A operand is not an exact small integer
 // (group scales, or a table): each decoded weight w, exact in fp32, becomes
@@ -68,6 +74,8 @@ struct TcCfg {
   static constexpr int B_BYTES = BN * kKB * 2;
   static constexpr int A_BYTES = (SPLIT ? 2 : 1) * kATileBytes;   // one stage's A tile(s)
   static constexpr int TMEM_COLS = 2 * BN;     // two accumulator buffers
+  static constexpr int RED_BUFS = std::min(STAGES * (A_BYTES + B_BYTES) / kRedChunk, kRedSets);
+  static_assert(RED_BUFS >= 2, "staging buffers of the final reduction");
 };
 
 // ------------------------------------------------------------------ PTX helpers
@@ -257,10 +265,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   uint64_t* acc_full = ab_empty + S;      // [2]
   uint64_t* acc_empty = acc_full + 2;     // [2]
   uint64_t* mma_drain = acc_empty + 2;    // the MMA thread's last commit
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_drain + 1);
+  uint64_t* red_full = mma_drain + 1;     // [kRedSets]: staged partial sums landed
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(red_full + kRedSets);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int* last_flag = const_cast<int*>(abort_flag) + 1;
   int* meta = last_flag + 1;   // [3]: first contributor, contributors, first's slot parity
+  int* fin = meta + 3;         // [2]: the CTA's last segment is pending (1), its index
+  long long* fin_u = reinterpret_cast<long long*>(fin + 2);   // its first unit
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int b = blockIdx.x;
@@ -282,7 +293,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       mbar_init(&acc_empty[i], 4);
     }
     mbar_init(mma_drain, 1);
+    for (int i = 0; i < kRedSets; ++i) mbar_init(&red_full[i], 1);
     *abort_flag = 0;
+    fin[0] = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == 0 && lane == 0) {
@@ -316,6 +329,45 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+
+  // y for tokens c0 .. c0 + 31 of `tile` at TMEM lane row_l (weight row
+  // tn 128 + row_l), per-row scale of group -1 applied here.  Gated layout: the
+  // quadrant's 32 rows are one gate block (lanes 0-15) and its up block (lanes
+  // 16-31).  Called by whole warps.
+  auto store_y32 = [&](const float (&vals)[32], int tile, int row_l, int c0) {
+    const int tn = tile % a.tiles_n, tm = tile / a.tiles_n;
+    const int row = tn * kRowsTile + row_l;
+    float s_row = 1.0f;
+    if constexpr (GM1) {
+      if (row < a.N)
+        s_row = __half2float(__ushort_as_half(a.scales[(size_t)(row >> 4) * 16 + scale_slot(row & 15)]));
+    }
+    if (!a.gated) {
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const int m = tm * BN + c0 + i;
+        if (row < a.N && m < a.M) {
+          const float o = vals[i] * s_row;
+          a.y[(size_t)m * a.N + row] = BF16 ? __bfloat16_as_ushort(__float2bfloat16_rn(o))
+                                            : __half_as_ushort(__float2half_rn(o));
+        }
+      }
+    } else {
+      const int ny = a.N >> 1;
+      const int col = (row >> 5) * 16 + (row & 15);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const float o = vals[i] * s_row;
+        const float up = __shfl_down_sync(0xffffffffu, o, 16);
+        const int m = tm * BN + c0 + i;
+        if ((row_l & 31) < 16 && row < a.N && m < a.M) {
+          const float gv = silu(o) * up;
+          a.y[(size_t)m * ny + col] = BF16 ? __bfloat16_as_ushort(__float2bfloat16_rn(gv))
+                                           : __half_as_ushort(__float2half_rn(gv));
+        }
+      }
+    }
+  };
 
   // Segments of this CTA: [u, u + len) within one tile.
   auto seg_of = [&](long long u, int& tile, int& kb0, int& kb1) {
@@ -550,17 +602,20 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     for (long long u = u_begin; u < u_end; ++seg) {
       int tile, kb0, kb1;
       seg_of(u, tile, kb0, kb1);
-      const int tn = tile % a.tiles_n, tm = tile / a.tiles_n;
       const int buf = seg & 1;
       // the four epilogue warps stop together (they share named barriers)
       const bool ok = mbar_wait(&acc_full[buf], (seg >> 1) & 1, abort_flag, a.wait_limit);
       if (!named_bar_and(1, 128, ok)) break;
       tc_fence_after();
-      const int row = tn * kRowsTile + row_l;
-      float s_row = 1.0f;
-      if constexpr (GM1) {
-        if (row < a.N) s_row = __half2float(__ushort_as_half(a.scales[(size_t)(row >> 4) * 16 +
-                                                                      scale_slot(row & 15)]));
+      if (u + (kb1 - kb0) == u_end) {
+        // the CTA's last segment: its epilogue is shared by the decode and
+        // epilogue warps once every role has finished (after the role loops)
+        if (threadIdx.x == kEpi0) {
+          fin[0] = 1;
+          fin[1] = seg;
+          *fin_u = u;
+        }
+        break;
       }
       const long long t_first = (long long)tile * a.nkb;
       const bool whole = (u == t_first) && (kb1 == a.nkb);
@@ -578,40 +633,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           meta[2] = ((long long)first * a.units / a.ctas < t_first) ? 1 : 0;
         }
       }
-      // y for 32 tokens of this thread's row.  Gated layout: the quadrant's 32
-      // rows are one gate block (lanes 0-15) and its up block (lanes 16-31).
-      auto store32 = [&](const float (&vals)[32], int c0) {
-        if (!a.gated) {
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const int m = tm * BN + c0 + i;
-            if (row < a.N && m < a.M) {
-              const float o = vals[i] * s_row;
-              a.y[(size_t)m * a.N + row] = BF16 ? __bfloat16_as_ushort(__float2bfloat16_rn(o))
-                                                : __half_as_ushort(__float2half_rn(o));
-            }
-          }
-        } else {
-          const int ny = a.N >> 1;
-          const int col = (row >> 5) * 16 + (row & 15);
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const float o = vals[i] * s_row;
-            const float up = __shfl_down_sync(0xffffffffu, o, 16);
-            const int m = tm * BN + c0 + i;
-            if (lane < 16 && row < a.N && m < a.M) {
-              const float gv = silu(o) * up;
-              a.y[(size_t)m * ny + col] = BF16 ? __bfloat16_as_ushort(__float2bfloat16_rn(gv))
-                                               : __half_as_ushort(__float2half_rn(gv));
-            }
-          }
-        }
-      };
-      // A partial tile whose other contributors have all arrived already (the
-      // usual case for a CTA's last segment: the tile's remainder was the next
-      // CTA's first work): this CTA is certainly the last one, so it adds the
-      // others' slots to its own sums straight from TMEM, without writing its
-      // own slot.  Contributors are added in order, as in the general path.
+      auto store32 = [&](const float (&vals)[32], int c0) { store_y32(vals, tile, row_l, c0); };
+      // A partial tile whose other contributors have all arrived already:
+      // this CTA is certainly the last one, so it adds the others' slots to its
+      // own sums straight from TMEM, without writing its own slot.
+      // Contributors are added in order, as in the general path.
       if (!whole) {
         named_bar(1, 128);   // meta written
         if (threadIdx.x == kEpi0) {
@@ -669,6 +695,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           for (int i = 0; i < 32; ++i) __stcg(slot + (size_t)(c0 + i) * kRowsTile, v[i]);
         }
       }
+      // the tile's last contributor may read the slot with bulk copies (async proxy)
+      if (!whole) fence_proxy_async_global();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&acc_empty[buf]);     // the accumulator may be reused
@@ -711,6 +739,136 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
   }
 
+  // ---------------------------------------------------------- last segment
+  // Every role has finished: all MMAs are complete (the MMA thread waited for
+  // them) and no copy is in flight, so TMEM holds the last segment's sums and
+  // the A / B ring is free.  The decode and epilogue warps (three per TMEM lane
+  // quadrant) share the segment's epilogue, which a CTA's range always ends
+  // with and which no later MMA work hides: y for a whole tile; for a partial
+  // one, the slot and, if this CTA is the tile's last contributor, the sum of
+  // all contributors in order (the others' slots staged into the ring by bulk
+  // copies when they fit).
+  tc_fence_before();
+  __syncthreads();
+  const bool fin_go = __syncthreads_and(fin[0] != 0 && *abort_flag == 0);
+  if (fin_go && warp >= 2) {
+    tc_fence_after();
+    constexpr int kFinThreads = kTcThreads - 64;         // warps 2 .. 13
+    constexpr int kJ = kFinThreads / 128;                // warps per quadrant
+    constexpr int kChunks = BN / 32;
+    constexpr int kFin0 = 64;                            // bookkeeping thread
+    const int q = warp & 3, row_l = q * 32 + lane;
+    const int jw = (warp - 2) >> 2;                      // this warp's chunks: jw, jw + kJ, ...
+    const long long u = *fin_u;
+    int tile, kb0, kb1;
+    seg_of(u, tile, kb0, kb1);
+    const int buf = fin[1] & 1;
+    const uint32_t tq = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * BN);
+    const long long t_first = (long long)tile * a.nkb;
+    const bool whole = (u == t_first) && (kb1 == a.nkb);
+    if (whole) {
+#pragma unroll 1
+      for (int c = jw; c < kChunks; c += kJ) {
+        float v[32];
+        tmem_ld32(tq + (uint32_t)(c * 32), v);
+        store_y32(v, tile, row_l, c * 32);
+      }
+    } else {
+      const int first = owner_of_tc(t_first, a.units, a.ctas);
+      const int nb = owner_of_tc(t_first + a.nkb - 1, a.units, a.ctas) - first + 1;
+      const int first_e = ((long long)first * a.units / a.ctas < t_first) ? 1 : 0;
+      const int own = b - first;
+      if (threadIdx.x == kFin0) {   // have all other contributors arrived?
+        unsigned cur;
+        asm volatile("ld.acquire.gpu.u32 %0, [%1];" : "=r"(cur) : "l"(&a.counters[tile]) : "memory");
+        *last_flag = cur == (unsigned)(nb - 1) ? 1 : 0;
+      }
+      named_bar(2, kFinThreads);
+      bool last = *last_flag != 0;
+      named_bar(2, kFinThreads);   // last_flag is written again below
+      if (!last) {
+        const int e = (tile == (int)(u_begin / a.nkb)) ? 0 : 1;
+        float* slot = a.slots + (size_t)(2 * b + e) * (size_t)(BN * kRowsTile) + row_l;
+#pragma unroll 1
+        for (int c = jw; c < kChunks; c += kJ) {
+          float v[32];
+          tmem_ld32(tq + (uint32_t)(c * 32), v);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) __stcg(slot + (size_t)(c * 32 + i) * kRowsTile, v[i]);
+        }
+        fence_proxy_async_global();
+        named_bar(2, kFinThreads);   // every slot store, then one release increment
+        if (threadIdx.x == kFin0) {
+          unsigned prev;
+          asm volatile("atom.add.acq_rel.gpu.u32 %0, [%1], 1;" : "=r"(prev) : "l"(&a.counters[tile]) : "memory");
+          *last_flag = prev == (unsigned)(nb - 1) ? 1 : 0;
+        }
+        named_bar(2, kFinThreads);
+        last = *last_flag != 0;
+      }
+      if (last) {
+        // own sums from TMEM, the others' from their slots, added in order
+        const int P = nb - 1;
+        const bool staged = kChunks * P <= Cfg::RED_BUFS;
+        if (staged && threadIdx.x == kFin0) {
+          fence_proxy_async_global();   // the slots were published to this thread's acquire
+          for (int c = 0; c < kChunks; ++c) {
+            mbar_expect_tx(&red_full[c], (uint32_t)(P * kRedChunk));
+            for (int k = 0, j = 0; k < nb; ++k) {
+              if (k == own) continue;
+              const float* src = a.slots +
+                                 (size_t)(2 * (first + k) + (k == 0 ? first_e : 0)) * (BN * kRowsTile) +
+                                 (size_t)c * 32 * kRowsTile;
+              bulk_load(sA + (size_t)(c * P + j) * kRedChunk, src, kRedChunk, &red_full[c]);
+              ++j;
+            }
+          }
+        }
+#pragma unroll 1
+        for (int c = jw; c < kChunks; c += kJ) {
+          float tv[32], accv[32];
+          tmem_ld32(tq + (uint32_t)(c * 32), tv);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) accv[i] = own == 0 ? tv[i] : 0.0f;
+          // a failed wait (the call is giving up) leaves garbage in y, which
+          // the error status covers
+          if (staged) mbar_wait(&red_full[c], 0, abort_flag, a.wait_limit);
+          for (int k = 0, j = 0; k < nb; ++k) {
+            if (k == own) {
+              if (k != 0) {
+#pragma unroll
+                for (int i = 0; i < 32; ++i) accv[i] += tv[i];
+              }
+              continue;
+            }
+            float va[32];
+            if (staged) {
+              const float* pj = reinterpret_cast<const float*>(sA + (size_t)(c * P + j) * kRedChunk) + row_l;
+#pragma unroll
+              for (int i = 0; i < 32; ++i) va[i] = pj[i * kRowsTile];
+            } else {
+              const float* pa = a.slots +
+                                (size_t)(2 * (first + k) + (k == 0 ? first_e : 0)) * (BN * kRowsTile) +
+                                (size_t)c * 32 * kRowsTile + row_l;
+#pragma unroll
+              for (int i = 0; i < 32; ++i) va[i] = __ldcg(pa + (size_t)i * kRowsTile);
+            }
+#pragma unroll
+            for (int i = 0; i < 32; ++i) accv[i] += va[i];
+            ++j;
+          }
+          store_y32(accv, tile, row_l, c * 32);
+        }
+        if (threadIdx.x == kFin0) {
+          // copies still in flight (only after a failed wait) land before the CTA exits
+          if (staged)
+            for (int c = 0; c < kChunks; ++c) drain_wait(&red_full[c], 0);
+          a.counters[tile] = 0u;   // ready for the next call
+        }
+      }
+    }
+  }
+
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
@@ -732,7 +890,7 @@ constexpr size_t tc_smem_bytes() {
   using Cfg = TcCfg<BN, SPLIT, MODE == kLUT>;
   return 1024 + (size_t)Cfg::STAGES * (Cfg::A_BYTES + Cfg::B_BYTES) +
          (size_t)kCodeStages * (kCodeBytes + kMetaBytes<MODE>) + (MODE == kLUT ? 256 * 32 * 4 : 0) +
-         (2 * kCodeStages + 3 * Cfg::STAGES + 5) * 8 + 32;
+         (2 * kCodeStages + 3 * Cfg::STAGES + 5 + kRedSets) * 8 + 64;
 }
 
 template <int MODE, bool BF16, int BN, bool GM1>
