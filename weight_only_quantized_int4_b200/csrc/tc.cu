@@ -236,7 +236,7 @@ template <int MODE, bool BF16, int BN, bool GM1>
 __global__ void __launch_bounds__(kTcThreads, 1)
     tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_w,
               const __grid_constant__ CUtensorMap map_s, const __grid_constant__ CUtensorMap map_z,
-              const TcArgs a) {
+              const __grid_constant__ CUtensorMap map_y, const TcArgs a) {
   constexpr bool SPLIT = BF16 && (!GM1 || MODE == kLUT);
   using Cfg = TcCfg<BN, SPLIT, MODE == kLUT>;
   constexpr int S = Cfg::STAGES;
@@ -742,36 +742,88 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   // ---------------------------------------------------------- last segment
   // Every role has finished: all MMAs are complete (the MMA thread waited for
   // them) and no copy is in flight, so TMEM holds the last segment's sums and
-  // the A / B ring is free.  The decode and epilogue warps (three per TMEM lane
-  // quadrant) share the segment's epilogue, which a CTA's range always ends
-  // with and which no later MMA work hides: y for a whole tile; for a partial
-  // one, the slot and, if this CTA is the tile's last contributor, the sum of
-  // all contributors in order (the others' slots staged into the ring by bulk
-  // copies when they fit).
+  // the rings are free.  The decode and epilogue warps share the segment's
+  // epilogue, which a CTA's range always ends with and which no later MMA work
+  // hides: y for a whole tile; for a partial one, the slot and, if this CTA is
+  // the tile's last contributor, the sum of all contributors in order (the
+  // others' slots staged into the A / B ring by bulk copies when they fit).
+  // The twelve warps form three groups of four (one per TMEM lane quadrant);
+  // group g takes the 32-column chunks g, g + 3, ...  A group writes each
+  // chunk's y tile (32 tokens x 128 rows) or slot chunk into shared memory,
+  // and one of its threads stores it with one bulk copy.
   tc_fence_before();
   __syncthreads();
   const bool fin_go = __syncthreads_and(fin[0] != 0 && *abort_flag == 0);
   if (fin_go && warp >= 2) {
     tc_fence_after();
     constexpr int kFinThreads = kTcThreads - 64;         // warps 2 .. 13
-    constexpr int kJ = kFinThreads / 128;                // warps per quadrant
+    constexpr int kGroups = kFinThreads / 128;
     constexpr int kChunks = BN / 32;
     constexpr int kFin0 = 64;                            // bookkeeping thread
     const int q = warp & 3, row_l = q * 32 + lane;
-    const int jw = (warp - 2) >> 2;                      // this warp's chunks: jw, jw + kJ, ...
+    const int grp = (warp - 2) >> 2;
+    const bool gissuer = threadIdx.x == 64 + 128 * grp;  // the group's bulk-store thread
     const long long u = *fin_u;
     int tile, kb0, kb1;
     seg_of(u, tile, kb0, kb1);
+    const int tn = tile % a.tiles_n, tm = tile / a.tiles_n;
     const int buf = fin[1] & 1;
     const uint32_t tq = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * BN);
     const long long t_first = (long long)tile * a.nkb;
     const bool whole = (u == t_first) && (kb1 == a.nkb);
+    const int row = tn * kRowsTile + row_l;
+    float s_row = 1.0f;
+    if constexpr (GM1) {
+      if (row < a.N)
+        s_row = __half2float(__ushort_as_half(a.scales[(size_t)(row >> 4) * 16 + scale_slot(row & 15)]));
+    }
+    // staging: y tiles in the code ring, slot chunks at the start of the A / B ring
+    uint16_t* ybuf = reinterpret_cast<uint16_t*>(sC + grp * (32 * kRowsTile * 2));
+    float* sbuf = reinterpret_cast<float*>(sA + grp * kRedChunk);
+    int yput = 0;
+    // the previous bulk store of the group's buffer has read it
+    auto buffer_free = [&](int& n) {
+      if (n++ > 0) {
+        if (gissuer) bulk_wait_read_all();
+        named_bar(3 + grp, 128);
+      }
+    };
+    auto put_y = [&](const float (&vals)[32], int c) {
+      buffer_free(yput);
+      if (!a.gated) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const float o = vals[i] * s_row;
+          ybuf[i * kRowsTile + row_l] = BF16 ? __bfloat16_as_ushort(__float2bfloat16_rn(o))
+                                             : __half_as_ushort(__float2half_rn(o));
+        }
+      } else {
+        // gate rows (lanes 0-15) and up rows (lanes 16-31) of the quadrant
+        // give its 16 outputs, columns q 16 .. q 16 + 15 of the tile's 64
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const float o = vals[i] * s_row;
+          const float up = __shfl_down_sync(0xffffffffu, o, 16);
+          if (lane < 16) {
+            const float gv = silu(o) * up;
+            ybuf[i * (kRowsTile / 2) + q * 16 + lane] =
+                BF16 ? __bfloat16_as_ushort(__float2bfloat16_rn(gv)) : __half_as_ushort(__float2half_rn(gv));
+          }
+        }
+      }
+      fence_proxy_async();
+      named_bar(3 + grp, 128);
+      if (gissuer) {
+        tma_store_2d(&map_y, ybuf, a.gated ? tn * (kRowsTile / 2) : tn * kRowsTile, tm * BN + c * 32);
+        bulk_commit();
+      }
+    };
     if (whole) {
 #pragma unroll 1
-      for (int c = jw; c < kChunks; c += kJ) {
+      for (int c = grp; c < kChunks; c += kGroups) {
         float v[32];
         tmem_ld32(tq + (uint32_t)(c * 32), v);
-        store_y32(v, tile, row_l, c * 32);
+        put_y(v, c);
       }
     } else {
       const int first = owner_of_tc(t_first, a.units, a.ctas);
@@ -788,16 +840,30 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       named_bar(2, kFinThreads);   // last_flag is written again below
       if (!last) {
         const int e = (tile == (int)(u_begin / a.nkb)) ? 0 : 1;
-        float* slot = a.slots + (size_t)(2 * b + e) * (size_t)(BN * kRowsTile) + row_l;
+        float* slot = a.slots + (size_t)(2 * b + e) * (size_t)(BN * kRowsTile);
+        int sput = 0;
 #pragma unroll 1
-        for (int c = jw; c < kChunks; c += kJ) {
+        for (int c = grp; c < kChunks; c += kGroups) {
           float v[32];
           tmem_ld32(tq + (uint32_t)(c * 32), v);
+          buffer_free(sput);
+          // column-major chunk: column i's 128 rows are 512 contiguous bytes
 #pragma unroll
-          for (int i = 0; i < 32; ++i) __stcg(slot + (size_t)(c * 32 + i) * kRowsTile, v[i]);
+          for (int i = 0; i < 32; ++i) sbuf[i * kRowsTile + row_l] = v[i];
+          fence_proxy_async();
+          named_bar(3 + grp, 128);
+          if (gissuer) {
+            bulk_store(slot + (size_t)c * 32 * kRowsTile, sbuf, kRedChunk);
+            bulk_commit();
+          }
         }
-        fence_proxy_async_global();
-        named_bar(2, kFinThreads);   // every slot store, then one release increment
+        // the slot is written before the release increment (the last
+        // contributor reads it with generic loads or bulk copies)
+        if (gissuer) {
+          bulk_wait_all();
+          fence_proxy_async_global();
+        }
+        named_bar(2, kFinThreads);
         if (threadIdx.x == kFin0) {
           unsigned prev;
           asm volatile("atom.add.acq_rel.gpu.u32 %0, [%1], 1;" : "=r"(prev) : "l"(&a.counters[tile]) : "memory");
@@ -808,8 +874,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       }
       if (last) {
         // own sums from TMEM, the others' from their slots, added in order
+        // (the slot staging buffers are free again: their stores completed)
         const int P = nb - 1;
-        const bool staged = kChunks * P <= Cfg::RED_BUFS;
+        constexpr int kStage0 = 0;                       // first staging buffer
+        const bool staged = kStage0 + kChunks * P <= Cfg::RED_BUFS;
         if (staged && threadIdx.x == kFin0) {
           fence_proxy_async_global();   // the slots were published to this thread's acquire
           for (int c = 0; c < kChunks; ++c) {
@@ -819,13 +887,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
               const float* src = a.slots +
                                  (size_t)(2 * (first + k) + (k == 0 ? first_e : 0)) * (BN * kRowsTile) +
                                  (size_t)c * 32 * kRowsTile;
-              bulk_load(sA + (size_t)(c * P + j) * kRedChunk, src, kRedChunk, &red_full[c]);
+              bulk_load(sA + (size_t)(kStage0 + c * P + j) * kRedChunk, src, kRedChunk, &red_full[c]);
               ++j;
             }
           }
         }
 #pragma unroll 1
-        for (int c = jw; c < kChunks; c += kJ) {
+        for (int c = grp; c < kChunks; c += kGroups) {
           float tv[32], accv[32];
           tmem_ld32(tq + (uint32_t)(c * 32), tv);
 #pragma unroll
@@ -843,7 +911,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             }
             float va[32];
             if (staged) {
-              const float* pj = reinterpret_cast<const float*>(sA + (size_t)(c * P + j) * kRedChunk) + row_l;
+              const float* pj =
+                  reinterpret_cast<const float*>(sA + (size_t)(kStage0 + c * P + j) * kRedChunk) + row_l;
 #pragma unroll
               for (int i = 0; i < 32; ++i) va[i] = pj[i * kRowsTile];
             } else {
@@ -857,7 +926,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             for (int i = 0; i < 32; ++i) accv[i] += va[i];
             ++j;
           }
-          store_y32(accv, tile, row_l, c * 32);
+          put_y(accv, c);
         }
         if (threadIdx.x == kFin0) {
           // copies still in flight (only after a failed wait) land before the CTA exits
@@ -867,6 +936,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
       }
     }
+    if (gissuer) bulk_wait_read_all();   // the staging buffers outlive no bulk store
   }
 
   tc_fence_before();
@@ -895,7 +965,7 @@ constexpr size_t tc_smem_bytes() {
 
 template <int MODE, bool BF16, int BN, bool GM1>
 cudaError_t launch_tc_t(const CUtensorMap& mx, const CUtensorMap& mw, const CUtensorMap& ms,
-                        const CUtensorMap& mz, const TcArgs& args, cudaStream_t stream) {
+                        const CUtensorMap& mz, const CUtensorMap& my, const TcArgs& args, cudaStream_t stream) {
   auto k = tc_kernel<MODE, BF16, BN, GM1>;
   constexpr size_t smem = tc_smem_bytes<MODE, BN, BF16 && (!GM1 || MODE == kLUT)>();
   static_assert(smem <= 227 * 1024, "shared memory of the tensor-core kernel");
@@ -920,27 +990,27 @@ cudaError_t launch_tc_t(const CUtensorMap& mx, const CUtensorMap& mw, const CUte
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, k, mx, mw, ms, mz, args);
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, k, mx, mw, ms, mz, my, args);
   if (e != cudaSuccess) cudaGetLastError();   // report it once, here
   return e;
 }
 
 template <int MODE, bool BF16, bool GM1>
 cudaError_t launch_bn(int bn, const CUtensorMap& mx, const CUtensorMap& mw, const CUtensorMap& ms,
-                      const CUtensorMap& mz, const TcArgs& args, cudaStream_t s) {
-  if (bn == 64) return launch_tc_t<MODE, BF16, 64, GM1>(mx, mw, ms, mz, args, s);
-  if (bn == 128) return launch_tc_t<MODE, BF16, 128, GM1>(mx, mw, ms, mz, args, s);
-  return launch_tc_t<MODE, BF16, 256, GM1>(mx, mw, ms, mz, args, s);
+                      const CUtensorMap& mz, const CUtensorMap& my, const TcArgs& args, cudaStream_t s) {
+  if (bn == 64) return launch_tc_t<MODE, BF16, 64, GM1>(mx, mw, ms, mz, my, args, s);
+  if (bn == 128) return launch_tc_t<MODE, BF16, 128, GM1>(mx, mw, ms, mz, my, args, s);
+  return launch_tc_t<MODE, BF16, 256, GM1>(mx, mw, ms, mz, my, args, s);
 }
 
 template <int MODE>
 cudaError_t launch_mode(bool bf16, bool gm1, int bn, const CUtensorMap& mx, const CUtensorMap& mw,
-                        const CUtensorMap& ms, const CUtensorMap& mz, const TcArgs& args,
+                        const CUtensorMap& ms, const CUtensorMap& mz, const CUtensorMap& my, const TcArgs& args,
                         cudaStream_t s) {
-  if (bf16) return gm1 ? launch_bn<MODE, true, true>(bn, mx, mw, ms, mz, args, s)
-                       : launch_bn<MODE, true, false>(bn, mx, mw, ms, mz, args, s);
-  return gm1 ? launch_bn<MODE, false, true>(bn, mx, mw, ms, mz, args, s)
-             : launch_bn<MODE, false, false>(bn, mx, mw, ms, mz, args, s);
+  if (bf16) return gm1 ? launch_bn<MODE, true, true>(bn, mx, mw, ms, mz, my, args, s)
+                       : launch_bn<MODE, true, false>(bn, mx, mw, ms, mz, my, args, s);
+  return gm1 ? launch_bn<MODE, false, true>(bn, mx, mw, ms, mz, my, args, s)
+             : launch_bn<MODE, false, false>(bn, mx, mw, ms, mz, my, args, s);
 }
 
 }  // namespace
@@ -1036,6 +1106,20 @@ cudaError_t launch_tc(const Problem& pr, const TcPlan& plan, void* workspace,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return cudaErrorInvalidValue;
   }
+  // y as [M] x [N] (gated: [M] x [N/2]), one box = 32 tokens of a tile's
+  // 128 rows (gated: its 64 outputs)
+  CUtensorMap my;
+  {
+    const int ny = pr.gated ? pr.N / 2 : pr.N;
+    const cuuint64_t dims[2] = {(cuuint64_t)ny, (cuuint64_t)pr.M};
+    const cuuint64_t strides[1] = {(cuuint64_t)ny * 2};
+    const cuuint32_t box[2] = {(cuuint32_t)(pr.gated ? kRowsTile / 2 : kRowsTile), 32};
+    const cuuint32_t es[2] = {1, 1};
+    if (encode(&my, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, pr.y, dims, strides, box, es,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+               CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
   TcArgs a{};
   a.sx = sx;
   a.scales = pr.scales;
@@ -1063,9 +1147,9 @@ cudaError_t launch_tc(const Problem& pr, const TcPlan& plan, void* workspace,
   }
   const bool gm1 = pr.group == -1;
   switch (pr.mode) {
-    case kSYM: return launch_mode<kSYM>(pr.bf16, gm1, plan.bn, mx, mw, ms, mz, a, stream);
-    case kASYM: return launch_mode<kASYM>(pr.bf16, gm1, plan.bn, mx, mw, ms, mz, a, stream);
-    default: return launch_mode<kLUT>(pr.bf16, gm1, plan.bn, mx, mw, ms, mz, a, stream);
+    case kSYM: return launch_mode<kSYM>(pr.bf16, gm1, plan.bn, mx, mw, ms, mz, my, a, stream);
+    case kASYM: return launch_mode<kASYM>(pr.bf16, gm1, plan.bn, mx, mw, ms, mz, my, a, stream);
+    default: return launch_mode<kLUT>(pr.bf16, gm1, plan.bn, mx, mw, ms, mz, my, a, stream);
   }
 }
 
