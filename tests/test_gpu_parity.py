@@ -136,14 +136,17 @@ def test_qmm_small(mode, bits, group, xdtype):
 @pytest.mark.parametrize("K", [320, 704])
 def test_qmm_k_ends_mid_stage(mode, bits, group, xdtype, K):
     """K % 128 == 64: the decode path's last 128-column stage holds one valid
-    64-column chunk (the second must contribute nothing); the tensor path's
-    64-column k blocks end exactly at K."""
+    64-column chunk (the second must contribute nothing); so does the tensor
+    path's last unit where a unit is two 64-column k blocks (the codes, scales
+    and x past K are zero-filled)."""
     N = 48
     for M in (1, 5, 16, 17, 64):
         p = cases.make(mode, bits, group, M, N, K, xdtype, seed=300 + M + K)
         y_ref, bound = cases.expected(p)
         x, qw, sp, zl = upload(p)
-        for path in ("auto", "skinny", "skinny_streamk"):
+        for path in ("auto", "skinny", "skinny_streamk", "tensor"):
+            if path == "tensor" and q.path(M, N, K, mode, bits, group, xdtype, "tensor") != "tensor":
+                continue
             ws = q.workspace(M, N, K, mode, bits, group, path=path)
             y = q.qmm(x, qw, sp, zl, N, K, mode, bits, group, ws=ws, path=path)
             torch.cuda.synchronize()

@@ -99,7 +99,7 @@ Plan make_plan(int M, int N, int K, int bits, int group, int mode, bool bf16, in
            : streamk            ? QMM_PATH_SKINNY
                                 : path;
   if (p.path == QMM_PATH_TENSOR && !tc_supported(bits, mode, bf16, group)) p.path = QMM_PATH_SKINNY;
-  if (p.path == QMM_PATH_TENSOR) p.tc = plan_tc(M, N, K, device_sms());
+  if (p.path == QMM_PATH_TENSOR) p.tc = plan_tc(M, N, K, mode, bf16, group, device_sms());
   else p.sk = plan_skinny(M, N, K, bits, group, mode, bf16, device_sms(), streamk);
   return p;
 }

@@ -50,12 +50,13 @@ unsigned skinny_read_and_clear_error();
 // Stream-K plan of the tensor-core path (tcgen05, 4-bit codes).
 struct TcPlan {
   int bn;          // tokens per tile (UMMA N)
-  int tiles_n, tiles_m, nkb, ctas;
+  int ku;          // 64-column k blocks per unit of work (1 or 2)
+  int tiles_n, tiles_m, nkb, ctas;   // nkb: units per tile
   size_t ws_bytes;
 };
 
 bool tc_supported(int bits, int mode, bool bf16, int group);
-TcPlan plan_tc(int M, int N, int K, int sms);
+TcPlan plan_tc(int M, int N, int K, int mode, bool bf16, int group, int sms);
 cudaError_t launch_tc(const Problem& p, const TcPlan& plan, void* workspace, long long wait_limit,
                       cudaStream_t stream);
 

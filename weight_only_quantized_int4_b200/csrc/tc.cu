@@ -39,17 +39,14 @@ constexpr int kDecWarps = 8;                        // decode warps (one of the 
 constexpr int kRbPerDec = 8 / kDecWarps;            // row blocks per decode warp
 constexpr int kTcThreads = 32 * (2 + kDecWarps + 4);
 constexpr int kEpi0 = 32 * (2 + kDecWarps);          // first epilogue thread
-constexpr int kKB = 64;             // K columns per stage (one 128-byte swizzle row of fp16)
+constexpr int kKB = 64;             // K columns per k block (one 128-byte swizzle row of fp16)
 constexpr int kRowsTile = 128;      // weight rows per tile (UMMA M)
-constexpr int kCodeStages = 8;
-constexpr int kCodeBytes = 8 * 512; // 8 row blocks x one 512-byte chunk
+constexpr int kCodeBytes = 8 * 512; // a k block's codes: 8 row blocks x one 512-byte chunk
 constexpr int kATileBytes = kRowsTile * kKB * 2;   // 16 KB
-// Per code stage, the k block's group scales (and ASYM zero-points) of the
+// Per code stage, the unit's group scales (and ASYM zero-points) of the
 // tile's 8 row blocks, loaded by TMA with the codes: [8][sx] fp16, sx = 16
-// slots x the groups in 64 columns (at most 4), 1 KB each.
+// slots x the groups in the unit's columns, 1 KB per 64 columns.
 constexpr int kMetaTile = 1024;
-template <int MODE>
-constexpr int kMetaBytes = MODE == kASYM ? 2 * kMetaTile : kMetaTile;
 // Bound of the waits a CTA makes for its own copies and MMAs while draining
 // (they always complete): ~2 s at 1.9 GHz.
 constexpr long long kDrainCycles = 4000000000ll;
@@ -66,13 +63,25 @@ constexpr int kRedSets = 9;
 // 2^-18 |w|), two A tiles per stage and two MMAs per k step into the same
 // accumulator.  A single bf16 rounding of w (2^-9) together with the bf16
 // output would use most of the error budget.
-template <int BN, bool SPLIT = false, bool TABLE = false>
+//
+// KU: 64-column k blocks per unit of work (1 or 2).  A unit is one round of the
+// rings and barriers (one code tile, one x tile, one A tile per k block, one
+// commit); two k blocks per unit halve those rounds per column where the
+// doubled stages still fit (narrow token tiles, no table, no split).
+template <int BN, bool SPLIT = false, bool TABLE = false, int KU = 1>
 struct TcCfg {
+  static_assert(KU == 1 || (KU == 2 && BN <= 128 && !SPLIT && !TABLE), "two k blocks per unit");
   // A / B ring depth within 227 KB (the table takes 32 KB)
   static constexpr int STAGES =
-      SPLIT ? (BN == 64 ? (TABLE ? 3 : 4) : (BN == 128 ? 3 : 2)) : (BN == 256 ? 3 : 4);
-  static constexpr int B_BYTES = BN * kKB * 2;
-  static constexpr int A_BYTES = (SPLIT ? 2 : 1) * kATileBytes;   // one stage's A tile(s)
+      KU == 2 ? (BN == 64 ? 3 : 2)
+              : (SPLIT ? (BN == 64 ? (TABLE ? 3 : 4) : (BN == 128 ? 3 : 2)) : (BN == 256 ? 3 : 4));
+  static constexpr int B_BYTES = KU * BN * kKB * 2;
+  static constexpr int A_BYTES = KU * (SPLIT ? 2 : 1) * kATileBytes;   // one stage's A tile(s)
+  static constexpr int CODE_STAGES = 8 / KU;
+  static constexpr int CODE_BYTES = KU * kCodeBytes;
+  static constexpr int META_TILE = KU * kMetaTile;
+  template <int MODE>
+  static constexpr int META_BYTES = MODE == kASYM ? 2 * META_TILE : META_TILE;
   static constexpr int TMEM_COLS = 2 * BN;     // two accumulator buffers
   static constexpr int RED_BUFS = std::min(STAGES * (A_BYTES + B_BYTES) / kRedChunk, kRedSets);
   static_assert(RED_BUFS >= 2, "staging buffers of the final reduction");
@@ -232,14 +241,17 @@ __device__ __forceinline__ uint32_t lut_pair(uint32_t t16, float s) {
   }
 }
 
-template <int MODE, bool BF16, int BN, bool GM1>
+template <int MODE, bool BF16, int BN, bool GM1, int KU>
 __global__ void __launch_bounds__(kTcThreads, 1)
     tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_w,
               const __grid_constant__ CUtensorMap map_s, const __grid_constant__ CUtensorMap map_z,
               const __grid_constant__ CUtensorMap map_y, const TcArgs a) {
   constexpr bool SPLIT = BF16 && (!GM1 || MODE == kLUT);
-  using Cfg = TcCfg<BN, SPLIT, MODE == kLUT>;
+  using Cfg = TcCfg<BN, SPLIT, MODE == kLUT, KU>;
   constexpr int S = Cfg::STAGES;
+  constexpr int kCodeStages = Cfg::CODE_STAGES;
+  constexpr int kStageCode = Cfg::CODE_BYTES;
+  constexpr int kStageMeta = Cfg::template META_BYTES<MODE>;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   // carve: A stages | B stages | code stages | meta stages | LUT table | barriers.
   // The 1024-byte aligned start is an offset from the shared array itself, so
@@ -249,8 +261,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   unsigned char* sA = base;
   unsigned char* sB = sA + S * Cfg::A_BYTES;
   unsigned char* sC = sB + S * Cfg::B_BYTES;
-  unsigned char* sM = sC + kCodeStages * kCodeBytes;
-  unsigned char* sT = sM + kCodeStages * kMetaBytes<MODE>;
+  unsigned char* sM = sC + kCodeStages * kStageCode;
+  unsigned char* sT = sM + kCodeStages * kStageMeta;
   // group scales and zero-points come with the codes (per-row scales of
   // group -1 are applied in the epilogue instead)
   constexpr bool kScales = !GM1;
@@ -395,15 +407,17 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             break;
           }
           constexpr int kMetaCopies = (kScales ? 1 : 0) + (kZeros ? 1 : 0);
-          mbar_expect_tx(&code_full[c], kCodeBytes + kMetaCopies * 8 * a.sx * 2);
-          tma_load_2d(sC + c * kCodeBytes, &map_w, &code_full[c], kb * 128, tn * 8);
-          // the k block's first group, 16 slots per group (the x coordinate is
+          mbar_expect_tx(&code_full[c], kStageCode + kMetaCopies * 8 * a.sx * 2);
+          // the unit's KU chunks of each of the 8 row blocks (columns past K
+          // read as zero codes; their x columns are zero too)
+          tma_load_2d(sC + c * kStageCode, &map_w, &code_full[c], kb * 128 * KU, tn * 8);
+          // the unit's first group, 16 slots per group (the x coordinate is
           // a multiple of 16 elements: 32-byte aligned)
-          const int gx = ((kb * kKB) >> a.lg) * 16;
+          const int gx = ((kb * KU * kKB) >> a.lg) * 16;
           if constexpr (kScales)
-            tma_load_2d(sM + c * kMetaBytes<MODE>, &map_s, &code_full[c], gx, tn * 8);
+            tma_load_2d(sM + c * kStageMeta, &map_s, &code_full[c], gx, tn * 8);
           if constexpr (kZeros)
-            tma_load_2d(sM + c * kMetaBytes<MODE> + kMetaTile, &map_z, &code_full[c], gx, tn * 8);
+            tma_load_2d(sM + c * kStageMeta + Cfg::META_TILE, &map_z, &code_full[c], gx, tn * 8);
         }
         if (!ok) break;
         u += kb1 - kb0;
@@ -426,7 +440,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             break;
           }
           mbar_expect_tx(&b_full[s], Cfg::B_BYTES);
-          tma_load_2d(sB + s * Cfg::B_BYTES, &map_x, &b_full[s], kb * kKB, tm * BN);
+#pragma unroll
+          for (int kb2 = 0; kb2 < KU; ++kb2)
+            tma_load_2d(sB + s * Cfg::B_BYTES + kb2 * (BN * kKB * 2), &map_x, &b_full[s],
+                        (kb * KU + kb2) * kKB, tm * BN);
         }
         if (!ok) break;
         u += kb1 - kb0;
@@ -455,14 +472,17 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             break;
           }
           tc_fence_after();
-          const uint32_t sa = smem_u32(sA + s * Cfg::A_BYTES);
-          const uint32_t sb = smem_u32(sB + s * Cfg::B_BYTES);
 #pragma unroll
-          for (int k = 0; k < kKB / 16; ++k) {
-            umma_f16(d, sw128_desc(sa + 32 * k), sw128_desc(sb + 32 * k), idesc,
-                     (kb > kb0 || k > 0) ? 1u : 0u);
-            if constexpr (SPLIT)   // the low parts of the weights, same accumulator
-              umma_f16(d, sw128_desc(sa + kATileBytes + 32 * k), sw128_desc(sb + 32 * k), idesc, 1u);
+          for (int kb2 = 0; kb2 < KU; ++kb2) {
+            const uint32_t sa = smem_u32(sA + s * Cfg::A_BYTES + kb2 * kATileBytes);
+            const uint32_t sb = smem_u32(sB + s * Cfg::B_BYTES + kb2 * (BN * kKB * 2));
+#pragma unroll
+            for (int k = 0; k < kKB / 16; ++k) {
+              umma_f16(d, sw128_desc(sa + 32 * k), sw128_desc(sb + 32 * k), idesc,
+                       (kb > kb0 || kb2 > 0 || k > 0) ? 1u : 0u);
+              if constexpr (SPLIT)   // the low parts of the weights, same accumulator
+                umma_f16(d, sw128_desc(sa + kATileBytes + 32 * k), sw128_desc(sb + 32 * k), idesc, 1u);
+            }
           }
           umma_commit(&ab_empty[s]);
         }
@@ -487,25 +507,28 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       const bool ok = mbar_wait(&code_full[c], (kc / kCodeStages) & 1, abort_flag, a.wait_limit) &&
                       mbar_wait(&ab_empty[s], ((ks / S) & 1) ^ 1, abort_flag, a.wait_limit);
       if (!__all_sync(0xffffffffu, ok)) break;
-      unsigned char* At = sA + s * Cfg::A_BYTES;
+#pragma unroll
+      for (int kb2 = 0; kb2 < KU; ++kb2) {   // the unit's k blocks, one A tile each
+      unsigned char* At = sA + s * Cfg::A_BYTES + kb2 * kATileBytes;
       // group scales (and zero-points) of the lane's rows g and g + 8, one word
-      // per 16-column slice j, from the k block's meta tile (landed with the codes)
+      // per 16-column slice j, from the unit's meta tile (landed with the codes)
       uint32_t sw[kRbPerDec][4], zw[kRbPerDec][4];
       if constexpr (kScales || kZeros) {
-        const unsigned char* mt = sM + c * kMetaBytes<MODE>;
+        const unsigned char* mt = sM + c * kStageMeta;
 #pragma unroll
         for (int rr = 0; rr < kRbPerDec; ++rr)
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
-            const int e = (kRbPerDec * dw + rr) * a.sx + ((16 * j) >> a.lg) * 16 + 2 * g;
+            const int e = (kRbPerDec * dw + rr) * a.sx + ((16 * j + kKB * kb2) >> a.lg) * 16 + 2 * g;
             if constexpr (kScales) sw[rr][j] = *reinterpret_cast<const uint32_t*>(mt + 2 * e);
-            if constexpr (kZeros) zw[rr][j] = *reinterpret_cast<const uint32_t*>(mt + kMetaTile + 2 * e);
+            if constexpr (kZeros) zw[rr][j] = *reinterpret_cast<const uint32_t*>(mt + Cfg::META_TILE + 2 * e);
           }
       }
 #pragma unroll
       for (int rr = 0; rr < kRbPerDec; ++rr) {
         const int rbl = kRbPerDec * dw + rr;               // row block in the tile
-        const uint4 wv = *reinterpret_cast<const uint4*>(sC + c * kCodeBytes + rbl * 512 + lane * 16);
+        const uint4 wv = *reinterpret_cast<const uint4*>(sC + c * kStageCode + rbl * (KU * 512) +
+                                                         kb2 * 512 + lane * 16);
         const int R0 = rbl * 16 + g, R1 = R0 + 8;
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
@@ -587,6 +610,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           }
         }
       }
+      }   // k blocks of the unit
       fence_proxy_async();
       __syncwarp();
       if (lane == 0) {
@@ -955,19 +979,20 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 namespace qk {
 namespace {
 
-template <int MODE, int BN, bool SPLIT>
+template <int MODE, int BN, bool SPLIT, int KU>
 constexpr size_t tc_smem_bytes() {
-  using Cfg = TcCfg<BN, SPLIT, MODE == kLUT>;
+  using Cfg = TcCfg<BN, SPLIT, MODE == kLUT, KU>;
   return 1024 + (size_t)Cfg::STAGES * (Cfg::A_BYTES + Cfg::B_BYTES) +
-         (size_t)kCodeStages * (kCodeBytes + kMetaBytes<MODE>) + (MODE == kLUT ? 256 * 32 * 4 : 0) +
-         (2 * kCodeStages + 3 * Cfg::STAGES + 5 + kRedSets) * 8 + 64;
+         (size_t)Cfg::CODE_STAGES * (Cfg::CODE_BYTES + Cfg::template META_BYTES<MODE>) +
+         (MODE == kLUT ? 256 * 32 * 4 : 0) +
+         (2 * Cfg::CODE_STAGES + 3 * Cfg::STAGES + 5 + kRedSets) * 8 + 64;
 }
 
-template <int MODE, bool BF16, int BN, bool GM1>
+template <int MODE, bool BF16, int BN, bool GM1, int KU>
 cudaError_t launch_tc_t(const CUtensorMap& mx, const CUtensorMap& mw, const CUtensorMap& ms,
                         const CUtensorMap& mz, const CUtensorMap& my, const TcArgs& args, cudaStream_t stream) {
-  auto k = tc_kernel<MODE, BF16, BN, GM1>;
-  constexpr size_t smem = tc_smem_bytes<MODE, BN, BF16 && (!GM1 || MODE == kLUT)>();
+  auto k = tc_kernel<MODE, BF16, BN, GM1, KU>;
+  constexpr size_t smem = tc_smem_bytes<MODE, BN, BF16 && (!GM1 || MODE == kLUT), KU>();
   static_assert(smem <= 227 * 1024, "shared memory of the tensor-core kernel");
   static bool attr_set[64] = {};
   int dev = 0;
@@ -996,21 +1021,28 @@ cudaError_t launch_tc_t(const CUtensorMap& mx, const CUtensorMap& mw, const CUte
 }
 
 template <int MODE, bool BF16, bool GM1>
-cudaError_t launch_bn(int bn, const CUtensorMap& mx, const CUtensorMap& mw, const CUtensorMap& ms,
+cudaError_t launch_bn(int bn, int ku, const CUtensorMap& mx, const CUtensorMap& mw, const CUtensorMap& ms,
                       const CUtensorMap& mz, const CUtensorMap& my, const TcArgs& args, cudaStream_t s) {
-  if (bn == 64) return launch_tc_t<MODE, BF16, 64, GM1>(mx, mw, ms, mz, my, args, s);
-  if (bn == 128) return launch_tc_t<MODE, BF16, 128, GM1>(mx, mw, ms, mz, my, args, s);
-  return launch_tc_t<MODE, BF16, 256, GM1>(mx, mw, ms, mz, my, args, s);
+  // two k blocks per unit: narrow token tiles, no table, no hi + lo split
+  constexpr bool kTwo = MODE != kLUT && !(BF16 && !GM1);
+  if constexpr (kTwo) {
+    if (ku == 2 && bn == 64) return launch_tc_t<MODE, BF16, 64, GM1, 2>(mx, mw, ms, mz, my, args, s);
+    if (ku == 2 && bn == 128) return launch_tc_t<MODE, BF16, 128, GM1, 2>(mx, mw, ms, mz, my, args, s);
+  }
+  if (ku != 1) return cudaErrorInvalidValue;
+  if (bn == 64) return launch_tc_t<MODE, BF16, 64, GM1, 1>(mx, mw, ms, mz, my, args, s);
+  if (bn == 128) return launch_tc_t<MODE, BF16, 128, GM1, 1>(mx, mw, ms, mz, my, args, s);
+  return launch_tc_t<MODE, BF16, 256, GM1, 1>(mx, mw, ms, mz, my, args, s);
 }
 
 template <int MODE>
-cudaError_t launch_mode(bool bf16, bool gm1, int bn, const CUtensorMap& mx, const CUtensorMap& mw,
+cudaError_t launch_mode(bool bf16, bool gm1, int bn, int ku, const CUtensorMap& mx, const CUtensorMap& mw,
                         const CUtensorMap& ms, const CUtensorMap& mz, const CUtensorMap& my, const TcArgs& args,
                         cudaStream_t s) {
-  if (bf16) return gm1 ? launch_bn<MODE, true, true>(bn, mx, mw, ms, mz, my, args, s)
-                       : launch_bn<MODE, true, false>(bn, mx, mw, ms, mz, my, args, s);
-  return gm1 ? launch_bn<MODE, false, true>(bn, mx, mw, ms, mz, my, args, s)
-             : launch_bn<MODE, false, false>(bn, mx, mw, ms, mz, my, args, s);
+  if (bf16) return gm1 ? launch_bn<MODE, true, true>(bn, ku, mx, mw, ms, mz, my, args, s)
+                       : launch_bn<MODE, true, false>(bn, ku, mx, mw, ms, mz, my, args, s);
+  return gm1 ? launch_bn<MODE, false, true>(bn, ku, mx, mw, ms, mz, my, args, s)
+             : launch_bn<MODE, false, false>(bn, ku, mx, mw, ms, mz, my, args, s);
 }
 
 }  // namespace
@@ -1041,19 +1073,23 @@ bool tc_supported(int bits, int mode, bool bf16, int group) {
   return bits == 4 && !zero_opts(mode);
 }
 
-TcPlan plan_tc(int M, int N, int K, int sms) {
+TcPlan plan_tc(int M, int N, int K, int mode, bool bf16, int group, int sms) {
   TcPlan p{};
   p.bn = M <= 64 ? 64 : (M <= 128 ? 128 : 256);
+  // two k blocks per unit where the kernel has them (no table, no hi + lo
+  // split, narrow token tiles); a K that ends mid-unit is zero-filled
+  const bool split = bf16 && (group != -1 || mode == kLUT);
+  p.ku = (p.bn <= 128 && mode != kLUT && !split) ? 2 : 1;
   p.tiles_n = (N + kRowsTile - 1) / kRowsTile;
   p.tiles_m = (M + p.bn - 1) / p.bn;
-  p.nkb = K / kKB;
+  p.nkb = (K / kKB + p.ku - 1) / p.ku;
   const long long units = (long long)p.tiles_n * p.tiles_m * p.nkb;
   long long ctas = sms;   // one CTA per SM (shared memory bound)
   if (ctas > units) ctas = units;
   p.ctas = (int)ctas;
   const int tiles = p.tiles_n * p.tiles_m;
-  const bool split = !(units % ctas == 0 && (units / ctas) % p.nkb == 0);
-  p.ws_bytes = split ? ((size_t)tiles * 4 + 255) / 256 * 256 +
+  const bool partial = !(units % ctas == 0 && (units / ctas) % p.nkb == 0);
+  p.ws_bytes = partial ? ((size_t)tiles * 4 + 255) / 256 * 256 +
                            (size_t)2 * p.ctas * p.bn * kRowsTile * sizeof(float)
                      : 0;
   return p;
@@ -1079,7 +1115,7 @@ cudaError_t launch_tc(const Problem& pr, const TcPlan& plan, void* workspace,
     const int nchunks = pr.K / 64;
     const cuuint64_t dims[2] = {(cuuint64_t)nchunks * 128, (cuuint64_t)(pr.N / 16)};
     const cuuint64_t strides[1] = {(cuuint64_t)nchunks * 512};
-    const cuuint32_t box[2] = {128, 8};
+    const cuuint32_t box[2] = {(cuuint32_t)(128 * plan.ku), 8};   // the unit's chunks
     const cuuint32_t es[2] = {1, 1};
     if (encode(&mw, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<void*>(pr.qweight), dims, strides,
                box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
@@ -1088,11 +1124,11 @@ cudaError_t launch_tc(const Problem& pr, const TcPlan& plan, void* workspace,
       return cudaErrorInvalidValue;
   }
   // group scales and zero-points ([N/16][G][16] fp16) as [G 16] x [N/16]: one
-  // box = the sx slots of a k block's groups for 8 row blocks (the zero map
-  // is only read for ASYM; without zeros it repeats the scale map)
+  // box = the sx slots of a unit's groups for 8 row blocks (the zero map is
+  // only read for ASYM; without zeros it repeats the scale map)
   const int L = pr.group == -1 ? pr.K : pr.group;
   const int G = pr.K / L;
-  const int sx = 16 * std::max(1, kKB / L);
+  const int sx = 16 * std::max(1, kKB * plan.ku / L);
   CUtensorMap ms, mz;
   for (int which = 0; which < 2; ++which) {
     const uint16_t* src = (which == 1 && pr.mode == kASYM) ? pr.zl : pr.scales;
@@ -1147,9 +1183,9 @@ cudaError_t launch_tc(const Problem& pr, const TcPlan& plan, void* workspace,
   }
   const bool gm1 = pr.group == -1;
   switch (pr.mode) {
-    case kSYM: return launch_mode<kSYM>(pr.bf16, gm1, plan.bn, mx, mw, ms, mz, my, a, stream);
-    case kASYM: return launch_mode<kASYM>(pr.bf16, gm1, plan.bn, mx, mw, ms, mz, my, a, stream);
-    default: return launch_mode<kLUT>(pr.bf16, gm1, plan.bn, mx, mw, ms, mz, my, a, stream);
+    case kSYM: return launch_mode<kSYM>(pr.bf16, gm1, plan.bn, plan.ku, mx, mw, ms, mz, my, a, stream);
+    case kASYM: return launch_mode<kASYM>(pr.bf16, gm1, plan.bn, plan.ku, mx, mw, ms, mz, my, a, stream);
+    default: return launch_mode<kLUT>(pr.bf16, gm1, plan.bn, plan.ku, mx, mw, ms, mz, my, a, stream);
   }
 }
 
