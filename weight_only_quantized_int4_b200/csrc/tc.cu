@@ -67,17 +67,18 @@ constexpr int kRedSets = 9;
 // KU: 64-column k blocks per unit of work (1 or 2).  A unit is one round of the
 // rings and barriers (one code tile, one x tile, one A tile per k block, one
 // commit); two k blocks per unit halve those rounds per column where the
-// doubled stages still fit (narrow token tiles, no table, no split).
+// doubled stages still fit (no table, no split; at 256 tokens only without
+// zero-points, with two A / B stages and three code stages).
 template <int BN, bool SPLIT = false, bool TABLE = false, int KU = 1>
 struct TcCfg {
-  static_assert(KU == 1 || (KU == 2 && BN <= 128 && !SPLIT && !TABLE), "two k blocks per unit");
+  static_assert(KU == 1 || (KU == 2 && !SPLIT && !TABLE), "two k blocks per unit");
   // A / B ring depth within 227 KB (the table takes 32 KB)
   static constexpr int STAGES =
       KU == 2 ? (BN == 64 ? 3 : 2)
               : (SPLIT ? (BN == 64 ? (TABLE ? 3 : 4) : (BN == 128 ? 3 : 2)) : (BN == 256 ? 3 : 4));
   static constexpr int B_BYTES = KU * BN * kKB * 2;
   static constexpr int A_BYTES = KU * (SPLIT ? 2 : 1) * kATileBytes;   // one stage's A tile(s)
-  static constexpr int CODE_STAGES = 8 / KU;
+  static constexpr int CODE_STAGES = (KU == 2 && BN == 256) ? 3 : 8 / KU;
   static constexpr int CODE_BYTES = KU * kCodeBytes;
   static constexpr int META_TILE = KU * kMetaTile;
   template <int MODE>
@@ -1023,11 +1024,13 @@ cudaError_t launch_tc_t(const CUtensorMap& mx, const CUtensorMap& mw, const CUte
 template <int MODE, bool BF16, bool GM1>
 cudaError_t launch_bn(int bn, int ku, const CUtensorMap& mx, const CUtensorMap& mw, const CUtensorMap& ms,
                       const CUtensorMap& mz, const CUtensorMap& my, const TcArgs& args, cudaStream_t s) {
-  // two k blocks per unit: narrow token tiles, no table, no hi + lo split
+  // two k blocks per unit: no table, no hi + lo split; 256 tokens without zero-points
   constexpr bool kTwo = MODE != kLUT && !(BF16 && !GM1);
   if constexpr (kTwo) {
     if (ku == 2 && bn == 64) return launch_tc_t<MODE, BF16, 64, GM1, 2>(mx, mw, ms, mz, my, args, s);
     if (ku == 2 && bn == 128) return launch_tc_t<MODE, BF16, 128, GM1, 2>(mx, mw, ms, mz, my, args, s);
+    if constexpr (MODE == kSYM)
+      if (ku == 2 && bn == 256) return launch_tc_t<MODE, BF16, 256, GM1, 2>(mx, mw, ms, mz, my, args, s);
   }
   if (ku != 1) return cudaErrorInvalidValue;
   if (bn == 64) return launch_tc_t<MODE, BF16, 64, GM1, 1>(mx, mw, ms, mz, my, args, s);
@@ -1077,9 +1080,11 @@ TcPlan plan_tc(int M, int N, int K, int mode, bool bf16, int group, int sms) {
   TcPlan p{};
   p.bn = M <= 64 ? 64 : (M <= 128 ? 128 : 256);
   // two k blocks per unit where the kernel has them (no table, no hi + lo
-  // split, narrow token tiles); a K that ends mid-unit is zero-filled
+  // split; at 256 tokens SYM only, and only for more than one token tile:
+  // with a single one, M = 256, the two A / B stages measured 1-2.5% slower
+  // than three of 64 columns); a K that ends mid-unit is zero-filled
   const bool split = bf16 && (group != -1 || mode == kLUT);
-  p.ku = (p.bn <= 128 && mode != kLUT && !split) ? 2 : 1;
+  p.ku = (mode != kLUT && !split && (p.bn <= 128 || (mode == kSYM && M > 256))) ? 2 : 1;
   p.tiles_n = (N + kRowsTile - 1) / kRowsTile;
   p.tiles_m = (M + p.bn - 1) / p.bn;
   p.nkb = (K / kKB + p.ku - 1) / p.ku;
