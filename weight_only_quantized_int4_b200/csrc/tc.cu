@@ -67,14 +67,16 @@ constexpr int kRedSets = 9;
 // KU: 64-column k blocks per unit of work (1 or 2).  A unit is one round of the
 // rings and barriers (one code tile, one x tile, one A tile per k block, one
 // commit); two k blocks per unit halve those rounds per column where the
-// doubled stages still fit (no table, no split; at 256 tokens only without
-// zero-points, with two A / B stages and three code stages).
+// doubled stages still fit: 64 tokens in every format but a table with split
+// operands; 128 tokens without a table or a split; 256 tokens without them or
+// zero-points (two A / B stages and three code stages).
 template <int BN, bool SPLIT = false, bool TABLE = false, int KU = 1>
 struct TcCfg {
-  static_assert(KU == 1 || (KU == 2 && !SPLIT && !TABLE), "two k blocks per unit");
+  static_assert(KU == 1 || (KU == 2 && !(SPLIT && TABLE) && (BN == 64 || (!SPLIT && !TABLE))),
+                "two k blocks per unit");
   // A / B ring depth within 227 KB (the table takes 32 KB)
   static constexpr int STAGES =
-      KU == 2 ? (BN == 64 ? 3 : 2)
+      KU == 2 ? (BN == 64 ? (SPLIT ? 2 : 3) : 2)
               : (SPLIT ? (BN == 64 ? (TABLE ? 3 : 4) : (BN == 128 ? 3 : 2)) : (BN == 256 ? 3 : 4));
   static constexpr int B_BYTES = KU * BN * kKB * 2;
   static constexpr int A_BYTES = KU * (SPLIT ? 2 : 1) * kATileBytes;   // one stage's A tile(s)
@@ -475,7 +477,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           tc_fence_after();
 #pragma unroll
           for (int kb2 = 0; kb2 < KU; ++kb2) {
-            const uint32_t sa = smem_u32(sA + s * Cfg::A_BYTES + kb2 * kATileBytes);
+            const uint32_t sa = smem_u32(sA + s * Cfg::A_BYTES + kb2 * (SPLIT ? 2 : 1) * kATileBytes);
             const uint32_t sb = smem_u32(sB + s * Cfg::B_BYTES + kb2 * (BN * kKB * 2));
 #pragma unroll
             for (int k = 0; k < kKB / 16; ++k) {
@@ -510,7 +512,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       if (!__all_sync(0xffffffffu, ok)) break;
 #pragma unroll
       for (int kb2 = 0; kb2 < KU; ++kb2) {   // the unit's k blocks, one A tile each
-      unsigned char* At = sA + s * Cfg::A_BYTES + kb2 * kATileBytes;
+      unsigned char* At = sA + s * Cfg::A_BYTES + kb2 * (SPLIT ? 2 : 1) * kATileBytes;
       // group scales (and zero-points) of the lane's rows g and g + 8, one word
       // per 16-column slice j, from the unit's meta tile (landed with the codes)
       uint32_t sw[kRbPerDec][4], zw[kRbPerDec][4];
@@ -1024,10 +1026,12 @@ cudaError_t launch_tc_t(const CUtensorMap& mx, const CUtensorMap& mw, const CUte
 template <int MODE, bool BF16, bool GM1>
 cudaError_t launch_bn(int bn, int ku, const CUtensorMap& mx, const CUtensorMap& mw, const CUtensorMap& ms,
                       const CUtensorMap& mz, const CUtensorMap& my, const TcArgs& args, cudaStream_t s) {
-  // two k blocks per unit: no table, no hi + lo split; 256 tokens without zero-points
-  constexpr bool kTwo = MODE != kLUT && !(BF16 && !GM1);
-  if constexpr (kTwo) {
+  // two k blocks per unit (the combinations TcCfg allows)
+  constexpr bool kSplit = BF16 && (!GM1 || MODE == kLUT);
+  constexpr bool kTable = MODE == kLUT;
+  if constexpr (!(kSplit && kTable))
     if (ku == 2 && bn == 64) return launch_tc_t<MODE, BF16, 64, GM1, 2>(mx, mw, ms, mz, my, args, s);
+  if constexpr (!kSplit && !kTable) {
     if (ku == 2 && bn == 128) return launch_tc_t<MODE, BF16, 128, GM1, 2>(mx, mw, ms, mz, my, args, s);
     if constexpr (MODE == kSYM)
       if (ku == 2 && bn == 256) return launch_tc_t<MODE, BF16, 256, GM1, 2>(mx, mw, ms, mz, my, args, s);
@@ -1079,12 +1083,19 @@ bool tc_supported(int bits, int mode, bool bf16, int group) {
 TcPlan plan_tc(int M, int N, int K, int mode, bool bf16, int group, int sms) {
   TcPlan p{};
   p.bn = M <= 64 ? 64 : (M <= 128 ? 128 : 256);
-  // two k blocks per unit where the kernel has them (no table, no hi + lo
-  // split; at 256 tokens SYM only, and only for more than one token tile:
-  // with a single one, M = 256, the two A / B stages measured 1-2.5% slower
-  // than three of 64 columns); a K that ends mid-unit is zero-filled
+  // two k blocks per unit where the kernel has them: 64 tokens unless a
+  // table meets split operands; 128 tokens without a table or a split; 256
+  // tokens SYM only, and only for more than one token tile (with a single one,
+  // M = 256, the two A / B stages measured 1-2.5% slower than three of 64
+  // columns).  A K that ends mid-unit is zero-filled.
   const bool split = bf16 && (group != -1 || mode == kLUT);
-  p.ku = (mode != kLUT && !split && (p.bn <= 128 || (mode == kSYM && M > 256))) ? 2 : 1;
+  const bool table = mode == kLUT;
+  if (p.bn == 64)
+    p.ku = (split && table) ? 1 : 2;
+  else if (p.bn == 128)
+    p.ku = (split || table) ? 1 : 2;
+  else
+    p.ku = (!split && mode == kSYM && M > 256) ? 2 : 1;
   p.tiles_n = (N + kRowsTile - 1) / kRowsTile;
   p.tiles_m = (M + p.bn - 1) / p.bn;
   p.nkb = (K / kKB + p.ku - 1) / p.ku;
