@@ -137,9 +137,9 @@ size_t qmm_workspace_size_for(int M, int N, int K, int bits, int group, int mode
  *   workspace     device, workspace_bytes >= qmm_workspace_size(...), zero
  *                 filled before first use (see above); may be NULL with
  *                 workspace_bytes 0, in which case no cross-CTA split-K is used.
- * The accumulation is fp32.  M <= 32 (M <= 64 when N <= 4096) runs the
- * bandwidth-bound decode path (one slab of up to 32 tokens; larger M in slabs
- * of 32), larger M the tcgen05 tensor-core path, which takes 4-bit codes with
+ * The accumulation is fp32.  M <= 32 runs the bandwidth-bound decode path
+ * (one slab of up to 32 tokens; larger M in slabs of 32 where the tensor path
+ * does not apply), larger M the tcgen05 tensor-core path, which takes 4-bit codes with
  * fp16 or bf16 activations in every mode and group (with bf16 activations and
  * group scales or a table, each weight enters as two bf16 parts, hi + lo).
  * Other combinations stay on the decode path.  qmm_path and qmm_path_ex tell

@@ -43,12 +43,13 @@ def test_sizes_and_paths(lib):
     assert q.packed_size(16, 128, "lut", 2, 64) == (16 * 32, 16 * 2 * 2, 0)
     assert q.path(1, 4096, 4096, "sym") == "skinny"
     assert q.path(16, 4096, 4096, "sym") == "skinny"
-    # measured crossover: the decode path up to M = 32, and up to M = 64 when
-    # N <= 4096; combinations the tensor path does not take stay on it
+    # measured crossover: the decode path up to M = 32 (one slab reads the
+    # weights once), the tensor path above, for every N; combinations the
+    # tensor path does not take stay on the decode path
     assert q.path(32, 11008, 4096, "sym") == "skinny"
     assert q.path(33, 11008, 4096, "sym") == "tensor"
-    assert q.path(64, 4096, 4096, "sym") == "skinny"
-    assert q.path(65, 4096, 4096, "sym") == "tensor"
+    assert q.path(32, 4096, 4096, "sym") == "skinny"
+    assert q.path(33, 4096, 4096, "sym") == "tensor"
     assert q.path(4096, 14336, 4096, "lut", 2, 64) == "skinny"
     # the kernel a forced-path request really runs, per activation dtype
     assert q.path(300, 272, 1024, "sym", 4, 128, "f16", "tensor") == "tensor"

@@ -71,15 +71,16 @@ size_t round256(size_t b) { return (b + 255) / 256 * 256; }
 
 // Decode path while the product is bandwidth-bound (few tokens), tensor-core
 // path once it becomes a dense contraction.  The crossover was measured on
-// B200 (K = 4096, N = 4096 .. 22016, SYM / LUT, M = 17 .. 96): two 16-token
-// slabs of the decode path beat the tensor path up to M = 32 (its time has a
-// floor of about 25-40 us per call there), and up to M = 64 for N <= 4096
-// (few row tiles for 148 SMs).  Combinations the tensor path does not cover
-// (2- and 3-bit codes; bf16 with group scales or a table; zero-point options)
-// take the decode path, in slabs of 16 tokens.
+// B200 (K = 4096 / 8192, N = 4096 .. 14336, SYM fp16, ASYM bf16, LUT, M = 24 ..
+// 64): one 32-token slab of the decode path reads the weights once and wins or
+// ties up to M = 32; above that it needs a second slab (a second read of the
+// weights) and the tensor path, which reads them once, is 1.3-2x faster.
+// Combinations the tensor path does not cover (2- and 3-bit codes; zero-point
+// options) take the decode path, in slabs of 32 tokens.
 int choose_path(int M, int N, int bits, int mode, bool bf16, int group) {
+  (void)N;
   if (!tc_supported(bits, mode, bf16, group)) return QMM_PATH_SKINNY;
-  if (M <= 32 || (M <= 64 && N <= 4096)) return QMM_PATH_SKINNY;
+  if (M <= 32) return QMM_PATH_SKINNY;
   return QMM_PATH_TENSOR;
 }
 
