@@ -52,10 +52,10 @@ constexpr int kMetaTile = 1024;
 constexpr long long kDrainCycles = 4000000000ll;
 // Final reduction of a CTA's last partial tile: the other contributors'
 // partial sums are brought into the (then idle) A / B ring by bulk copies,
-// 32 columns x 128 rows of fp32 (16 KB) per copy, one barrier per 32-column
-// chunk.
+// 32 columns x 128 rows of fp32 (16 KB) per copy; one arrival barrier per
+// 32-column chunk (at most 8) and one release barrier per buffer set.
 constexpr int kRedChunk = 32 * kRowsTile * 4;
-constexpr int kRedSets = 9;
+constexpr int kRedSets = 9;   // >= the 8 chunks of a 256-token tile
 
 // SPLIT: bf16 activations whose A operand is not an exact small integer
 // (group scales, or a table): each decoded weight w, exact in fp32, becomes
@@ -87,7 +87,7 @@ struct TcCfg {
   static constexpr int META_BYTES = MODE == kASYM ? 2 * META_TILE : META_TILE;
   static constexpr int TMEM_COLS = 2 * BN;     // two accumulator buffers
   static constexpr int RED_BUFS = std::min(STAGES * (A_BYTES + B_BYTES) / kRedChunk, kRedSets);
-  static_assert(RED_BUFS >= 2, "staging buffers of the final reduction");
+  static_assert(RED_BUFS >= 6, "staging buffers of the final reduction (two slot chunks per group)");
 };
 
 // ------------------------------------------------------------------ PTX helpers
@@ -280,8 +280,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   uint64_t* acc_full = ab_empty + S;      // [2]
   uint64_t* acc_empty = acc_full + 2;     // [2]
   uint64_t* mma_drain = acc_empty + 2;    // the MMA thread's last commit
-  uint64_t* red_full = mma_drain + 1;     // [kRedSets]: staged partial sums landed
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(red_full + kRedSets);
+  uint64_t* red_full = mma_drain + 1;     // [kRedSets]: a chunk's staged partial sums landed
+  uint64_t* red_empty = red_full + kRedSets;   // [kRedSets]: a set read by its group
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(red_empty + kRedSets);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int* last_flag = const_cast<int*>(abort_flag) + 1;
   int* meta = last_flag + 1;   // [3]: first contributor, contributors, first's slot parity
@@ -308,7 +309,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       mbar_init(&acc_empty[i], 4);
     }
     mbar_init(mma_drain, 1);
-    for (int i = 0; i < kRedSets; ++i) mbar_init(&red_full[i], 1);
+    for (int i = 0; i < kRedSets; ++i) {
+      mbar_init(&red_full[i], 1);
+      mbar_init(&red_empty[i], 4);
+    }
     *abort_flag = 0;
     fin[0] = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -781,15 +785,18 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   tc_fence_before();
   __syncthreads();
   const bool fin_go = __syncthreads_and(fin[0] != 0 && *abort_flag == 0);
-  if (fin_go && warp >= 2) {
+  if (fin_go && warp >= 1) {
     tc_fence_after();
-    constexpr int kFinThreads = kTcThreads - 64;         // warps 2 .. 13
-    constexpr int kGroups = kFinThreads / 128;
+    constexpr int kFinThreads = kTcThreads - 32;         // warps 1 .. 13
+    constexpr int kGroups = (kTcThreads - 64) / 128;     // groups of warps 2 .. 13
     constexpr int kChunks = BN / 32;
+    static_assert(kChunks <= kRedSets, "one arrival barrier per chunk");
     constexpr int kFin0 = 64;                            // bookkeeping thread
+    const bool worker = warp >= 2;                       // warp 1 only stages slots
+    const bool copier = threadIdx.x == 32;
     const int q = warp & 3, row_l = q * 32 + lane;
-    const int grp = (warp - 2) >> 2;
-    const bool gissuer = threadIdx.x == 64 + 128 * grp;  // the group's bulk-store thread
+    const int grp = worker ? (warp - 2) >> 2 : 0;
+    const bool gissuer = worker && threadIdx.x == 64 + 128 * grp;   // the group's bulk-store thread
     const long long u = *fin_u;
     int tile, kb0, kb1;
     seg_of(u, tile, kb0, kb1);
@@ -801,22 +808,19 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const int row = tn * kRowsTile + row_l;
     float s_row = 1.0f;
     if constexpr (GM1) {
-      if (row < a.N)
+      if (worker && row < a.N)
         s_row = __half2float(__ushort_as_half(a.scales[(size_t)(row >> 4) * 16 + scale_slot(row & 15)]));
     }
-    // staging: y tiles in the code ring, slot chunks at the start of the A / B ring
+    // staging: y tiles in the code ring (one per group), slot chunks at the
+    // start of the A / B ring (two per group, so a store and the next chunk's
+    // writes overlap)
     uint16_t* ybuf = reinterpret_cast<uint16_t*>(sC + grp * (32 * kRowsTile * 2));
-    float* sbuf = reinterpret_cast<float*>(sA + grp * kRedChunk);
     int yput = 0;
-    // the previous bulk store of the group's buffer has read it
-    auto buffer_free = [&](int& n) {
-      if (n++ > 0) {
+    auto put_y = [&](const float (&vals)[32], int c) {
+      if (yput++ > 0) {   // the previous store of the group's y buffer has read it
         if (gissuer) bulk_wait_read_all();
         named_bar(3 + grp, 128);
       }
-    };
-    auto put_y = [&](const float (&vals)[32], int c) {
-      buffer_free(yput);
       if (!a.gated) {
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
@@ -846,11 +850,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       }
     };
     if (whole) {
+      if (worker) {
 #pragma unroll 1
-      for (int c = grp; c < kChunks; c += kGroups) {
-        float v[32];
-        tmem_ld32(tq + (uint32_t)(c * 32), v);
-        put_y(v, c);
+        for (int c = grp; c < kChunks; c += kGroups) {
+          float v[32];
+          tmem_ld32(tq + (uint32_t)(c * 32), v);
+          put_y(v, c);
+        }
       }
     } else {
       const int first = owner_of_tc(t_first, a.units, a.ctas);
@@ -866,29 +872,35 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       bool last = *last_flag != 0;
       named_bar(2, kFinThreads);   // last_flag is written again below
       if (!last) {
-        const int e = (tile == (int)(u_begin / a.nkb)) ? 0 : 1;
-        float* slot = a.slots + (size_t)(2 * b + e) * (size_t)(BN * kRowsTile);
-        int sput = 0;
+        if (worker) {
+          const int e = (tile == (int)(u_begin / a.nkb)) ? 0 : 1;
+          float* slot = a.slots + (size_t)(2 * b + e) * (size_t)(BN * kRowsTile);
+          int sput = 0;
 #pragma unroll 1
-        for (int c = grp; c < kChunks; c += kGroups) {
-          float v[32];
-          tmem_ld32(tq + (uint32_t)(c * 32), v);
-          buffer_free(sput);
-          // column-major chunk: column i's 128 rows are 512 contiguous bytes
+          for (int c = grp; c < kChunks; c += kGroups, ++sput) {
+            float v[32];
+            tmem_ld32(tq + (uint32_t)(c * 32), v);
+            float* sbuf = reinterpret_cast<float*>(sA + (2 * grp + (sput & 1)) * kRedChunk);
+            if (sput >= 2) {   // the store of two chunks ago has read this buffer
+              if (gissuer) bulk_wait_read_one();
+              named_bar(3 + grp, 128);
+            }
+            // column-major chunk: column i's 128 rows are 512 contiguous bytes
 #pragma unroll
-          for (int i = 0; i < 32; ++i) sbuf[i * kRowsTile + row_l] = v[i];
-          fence_proxy_async();
-          named_bar(3 + grp, 128);
-          if (gissuer) {
-            bulk_store(slot + (size_t)c * 32 * kRowsTile, sbuf, kRedChunk);
-            bulk_commit();
+            for (int i = 0; i < 32; ++i) sbuf[i * kRowsTile + row_l] = v[i];
+            fence_proxy_async();
+            named_bar(3 + grp, 128);
+            if (gissuer) {
+              bulk_store(slot + (size_t)c * 32 * kRowsTile, sbuf, kRedChunk);
+              bulk_commit();
+            }
           }
-        }
-        // the slot is written before the release increment (the last
-        // contributor reads it with generic loads or bulk copies)
-        if (gissuer) {
-          bulk_wait_all();
-          fence_proxy_async_global();
+          // the slot is written before the release increment (the last
+          // contributor reads it with generic loads or bulk copies)
+          if (gissuer) {
+            bulk_wait_all();
+            fence_proxy_async_global();
+          }
         }
         named_bar(2, kFinThreads);
         if (threadIdx.x == kFin0) {
@@ -900,66 +912,83 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         last = *last_flag != 0;
       }
       if (last) {
-        // own sums from TMEM, the others' from their slots, added in order
-        // (the slot staging buffers are free again: their stores completed)
+        // own sums from TMEM, the others' from their slots, added in order.
+        // Warp 1 stages the others' chunks into the A / B ring (free again:
+        // the slot stores above completed) with bulk copies, kSets chunks at
+        // a time: chunk c goes to buffer set c mod kSets once the chunk that
+        // used the set before has been read by its group.  Each chunk has its
+        // own arrival barrier (used once): different groups read different
+        // uses of a set, and none of them has seen the set's earlier uses, so
+        // a phase parity on a shared barrier could not tell them apart.
         const int P = nb - 1;
-        constexpr int kStage0 = 0;                       // first staging buffer
-        const bool staged = kStage0 + kChunks * P <= Cfg::RED_BUFS;
-        if (staged && threadIdx.x == kFin0) {
-          fence_proxy_async_global();   // the slots were published to this thread's acquire
+        const bool staged = P <= Cfg::RED_BUFS;
+        const int kSets = staged ? Cfg::RED_BUFS / P : 1;
+        if (staged && copier) {
+          unsigned cur;   // the slots' release, observed by this thread too
+          asm volatile("ld.acquire.gpu.u32 %0, [%1];" : "=r"(cur) : "l"(&a.counters[tile]) : "memory");
+          (void)cur;
+          fence_proxy_async_global();
+          int issued = 0;
           for (int c = 0; c < kChunks; ++c) {
+            const int set = c % kSets;
+            if (c >= kSets && !mbar_wait(&red_empty[set], ((c / kSets) - 1) & 1, abort_flag, a.wait_limit))
+              break;
             mbar_expect_tx(&red_full[c], (uint32_t)(P * kRedChunk));
             for (int k = 0, j = 0; k < nb; ++k) {
               if (k == own) continue;
               const float* src = a.slots +
                                  (size_t)(2 * (first + k) + (k == 0 ? first_e : 0)) * (BN * kRowsTile) +
                                  (size_t)c * 32 * kRowsTile;
-              bulk_load(sA + (size_t)(kStage0 + c * P + j) * kRedChunk, src, kRedChunk, &red_full[c]);
+              bulk_load(sA + (size_t)(set * P + j) * kRedChunk, src, kRedChunk, &red_full[c]);
               ++j;
             }
+            issued = c + 1;
           }
+          // every fill lands before the CTA can exit
+          for (int c = 0; c < issued; ++c) drain_wait(&red_full[c], 0);
         }
+        if (worker) {
 #pragma unroll 1
-        for (int c = grp; c < kChunks; c += kGroups) {
-          float tv[32], accv[32];
-          tmem_ld32(tq + (uint32_t)(c * 32), tv);
+          for (int c = grp; c < kChunks; c += kGroups) {
+            const int set = c % kSets;
+            float tv[32], accv[32];
+            tmem_ld32(tq + (uint32_t)(c * 32), tv);
 #pragma unroll
-          for (int i = 0; i < 32; ++i) accv[i] = own == 0 ? tv[i] : 0.0f;
-          // a failed wait (the call is giving up) leaves garbage in y, which
-          // the error status covers
-          if (staged) mbar_wait(&red_full[c], 0, abort_flag, a.wait_limit);
-          for (int k = 0, j = 0; k < nb; ++k) {
-            if (k == own) {
-              if (k != 0) {
+            for (int i = 0; i < 32; ++i) accv[i] = own == 0 ? tv[i] : 0.0f;
+            // a failed wait (the call is giving up) leaves garbage in y, which
+            // the error status covers
+            if (staged) mbar_wait(&red_full[c], 0, abort_flag, a.wait_limit);
+            for (int k = 0, j = 0; k < nb; ++k) {
+              if (k == own) {
+                if (k != 0) {
 #pragma unroll
-                for (int i = 0; i < 32; ++i) accv[i] += tv[i];
+                  for (int i = 0; i < 32; ++i) accv[i] += tv[i];
+                }
+                continue;
               }
-              continue;
+              float va[32];
+              if (staged) {
+                const float* pj = reinterpret_cast<const float*>(sA + (size_t)(set * P + j) * kRedChunk) + row_l;
+#pragma unroll
+                for (int i = 0; i < 32; ++i) va[i] = pj[i * kRowsTile];
+              } else {
+                const float* pa = a.slots +
+                                  (size_t)(2 * (first + k) + (k == 0 ? first_e : 0)) * (BN * kRowsTile) +
+                                  (size_t)c * 32 * kRowsTile + row_l;
+#pragma unroll
+                for (int i = 0; i < 32; ++i) va[i] = __ldcg(pa + (size_t)i * kRowsTile);
+              }
+#pragma unroll
+              for (int i = 0; i < 32; ++i) accv[i] += va[i];
+              ++j;
             }
-            float va[32];
-            if (staged) {
-              const float* pj =
-                  reinterpret_cast<const float*>(sA + (size_t)(kStage0 + c * P + j) * kRedChunk) + row_l;
-#pragma unroll
-              for (int i = 0; i < 32; ++i) va[i] = pj[i * kRowsTile];
-            } else {
-              const float* pa = a.slots +
-                                (size_t)(2 * (first + k) + (k == 0 ? first_e : 0)) * (BN * kRowsTile) +
-                                (size_t)c * 32 * kRowsTile + row_l;
-#pragma unroll
-              for (int i = 0; i < 32; ++i) va[i] = __ldcg(pa + (size_t)i * kRowsTile);
+            if (staged) {   // the group is done with the set
+              __syncwarp();
+              if (lane == 0) mbar_arrive(&red_empty[set]);
             }
-#pragma unroll
-            for (int i = 0; i < 32; ++i) accv[i] += va[i];
-            ++j;
+            put_y(accv, c);
           }
-          put_y(accv, c);
-        }
-        if (threadIdx.x == kFin0) {
-          // copies still in flight (only after a failed wait) land before the CTA exits
-          if (staged)
-            for (int c = 0; c < kChunks; ++c) drain_wait(&red_full[c], 0);
-          a.counters[tile] = 0u;   // ready for the next call
+          if (threadIdx.x == kFin0) a.counters[tile] = 0u;   // ready for the next call
         }
       }
     }
@@ -988,7 +1017,7 @@ constexpr size_t tc_smem_bytes() {
   return 1024 + (size_t)Cfg::STAGES * (Cfg::A_BYTES + Cfg::B_BYTES) +
          (size_t)Cfg::CODE_STAGES * (Cfg::CODE_BYTES + Cfg::template META_BYTES<MODE>) +
          (MODE == kLUT ? 256 * 32 * 4 : 0) +
-         (2 * Cfg::CODE_STAGES + 3 * Cfg::STAGES + 5 + kRedSets) * 8 + 64;
+         (2 * Cfg::CODE_STAGES + 3 * Cfg::STAGES + 5 + 2 * kRedSets) * 8 + 64;
 }
 
 template <int MODE, bool BF16, int BN, bool GM1, int KU>
