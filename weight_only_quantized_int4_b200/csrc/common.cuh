@@ -185,10 +185,6 @@ __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.comm
 __device__ __forceinline__ void bulk_wait_read_all() {
   asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
 }
-// The shared memory of all but the most recent committed bulk store has been read.
-__device__ __forceinline__ void bulk_wait_read_one() {
-  asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
-}
 // Every committed bulk store has been performed.
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 

@@ -119,6 +119,11 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
     if (clock64() - t0 > kDrainCycles) return;
 }
 
+// The shared memory of all but the most recent committed bulk store has been read.
+__device__ __forceinline__ void bulk_wait_read_one() {
+  asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+}
+
 // Named barrier whose result is the AND of every participating thread's
 // predicate: a decision the warps of a role take together.
 __device__ __forceinline__ bool named_bar_and(int id, int threads, bool pred) {
