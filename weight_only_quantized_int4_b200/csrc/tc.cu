@@ -10,17 +10,20 @@
 // per 64-column K block, with A = decoded weights (fp16/bf16, written into
 // shared memory in the 128-byte-swizzled K-major layout by decode warps) and
 // B = a TMA-loaded tile of x.  Warp roles:
-//   warp 0      TMA producers: lane 0 code tiles (4 KB, 8 row blocks) with their
-//               group scales / zero-points, lane 1 x tiles
+//   warp 0      TMA producers: lane 0 code tiles (4 KB per K block, 8 row
+//               blocks) with their group scales / zero-points, lane 1 x tiles
 //   warp 1      TMEM owner and MMA issuer (one elected thread)
 //   next kDecWarps warps   decode, one row block each: codes and scales (smem)
 //                          -> (q - z) s, T[q] s -> A tile
 //   last 4 warps           epilogue: TMEM -> registers -> y (or split-K partials)
-// Work is split stream-K over (tile, K block) units across a grid of one CTA
-// per SM, like the decode path; partial tiles are reduced deterministically by
-// the last CTA that finishes them.  Every mbarrier wait is bounded: a wait
-// that runs out sets the device error word (qmm_check_error) and the CTA
-// drains and exits instead of hanging.
+// Work is split stream-K over (tile, unit) pairs, a unit being one or two K
+// blocks (one round of the rings), across a grid of one CTA per SM, like the
+// decode path; partial tiles are reduced deterministically by the last CTA
+// that finishes them.  A CTA's last segment is finished after the role loops
+// by the decode and epilogue warps together (warp 1 staging the other
+// contributors' partial sums).  Every mbarrier wait is bounded: a wait that
+// runs out sets the device error word (qmm_check_error) and the CTA drains and
+// exits instead of hanging.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
